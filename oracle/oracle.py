@@ -1,0 +1,269 @@
+"""Python face of the CPU oracle: ctypes calls into moe_oracle.c for the
+bit-exact steps (E4M3 codes, scales, routing, bias update, permutation
+layout) and numpy FP64 for the expert matmuls and the combine.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Callable, Optional
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = [
+    "lib", "e4m3_decode_table", "e4m3_encode", "quant_act_1x128",
+    "quant_w_128x128", "dequant_act", "dequant_w", "route", "update_bias",
+    "permute_layout", "swiglu_expert", "f64_to_bf16_bits", "combine",
+    "quantized_expert", "layer_forward", "gemm_blockscaled",
+]
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e4m3_encode_array.argtypes = [P, I64, P]
+        L.orc_quant_act_1x128_bf16.argtypes = [P, I64, I64, P, P]
+        L.orc_quant_act_1x128_f32.argtypes = [P, I64, I64, P, P]
+        L.orc_quant_w_128x128.argtypes = [P, I64, I64, P, P]
+        L.orc_route.restype = I
+        L.orc_route.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
+        L.orc_update_bias.argtypes = [I, I, I, P, ctypes.c_float, P]
+        L.orc_permute_layout.argtypes = [I, I, I, P, P, P, P]
+        _LIB = L
+    return _LIB
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ------------------------------------------------------------------- E4M3
+def e4m3_decode_table() -> np.ndarray:
+    """FP64 value of each of the 256 E4M3 codes (NaN for the two NaN codes)."""
+    L = lib()
+    return np.array([L.orc_e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().orc_e4m3_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+# ------------------------------------------------------------ quantisation
+def quant_act_1x128(x: np.ndarray):
+    """1x128 tile quantisation of a [rows, cols] matrix.
+
+    ``x`` is either uint16 bf16 bits or float32.  Returns (codes uint8
+    [rows, cols], scales float32 [rows, cols/128])."""
+    rows, cols = x.shape
+    assert cols % 128 == 0
+    q = np.empty((rows, cols), dtype=np.uint8)
+    s = np.empty((rows, cols // 128), dtype=np.float32)
+    if x.dtype == np.uint16:
+        x = _c(x, np.uint16)
+        lib().orc_quant_act_1x128_bf16(_p(x), rows, cols, _p(q), _p(s))
+    else:
+        x = _c(x, np.float32)
+        lib().orc_quant_act_1x128_f32(_p(x), rows, cols, _p(q), _p(s))
+    return q, s
+
+
+def quant_w_128x128(w: np.ndarray):
+    """128x128 block quantisation of bf16 bits [rows, cols]."""
+    rows, cols = w.shape
+    assert rows % 128 == 0 and cols % 128 == 0
+    w = _c(w, np.uint16)
+    q = np.empty((rows, cols), dtype=np.uint8)
+    s = np.empty((rows // 128, cols // 128), dtype=np.float32)
+    lib().orc_quant_w_128x128(_p(w), rows, cols, _p(q), _p(s))
+    return q, s
+
+
+_TABLE = None
+
+
+def _table():
+    global _TABLE
+    if _TABLE is None:
+        _TABLE = e4m3_decode_table()
+    return _TABLE
+
+
+def dequant_act(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """code value * tile scale, in FP64 (exact)."""
+    v = _table()[q]
+    return v * np.repeat(s.astype(np.float64), 128, axis=1)
+
+
+def dequant_w(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    v = _table()[q]
+    s64 = np.repeat(np.repeat(s.astype(np.float64), 128, axis=0), 128, axis=1)
+    return v * s64
+
+
+# ----------------------------------------------------------------- routing
+def route(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarray,
+          n_groups: int, topk_groups: int, topk: int,
+          logit_offset: Optional[np.ndarray] = None, want_scores: bool = False) -> dict:
+    T, d = x_bf16.shape
+    n_routed = router_w_bf16.shape[0]
+    x = _c(x_bf16, np.uint16)
+    E = _c(router_w_bf16, np.uint16)
+    b = _c(bias, np.float32)
+    off = None if logit_offset is None else _c(logit_offset, np.float32)
+    idx = np.empty((T, topk), dtype=np.int32)
+    gate = np.empty((T, topk), dtype=np.float32)
+    counts = np.empty((n_routed,), dtype=np.int32)
+    logits = np.empty((T, n_routed), dtype=np.float32) if want_scores else None
+    scores = np.empty((T, n_routed), dtype=np.float32) if want_scores else None
+    rc = lib().orc_route(T, d, n_routed, n_groups, topk_groups, topk, _p(x), _p(E),
+                         _p(b), _p(off), _p(idx), _p(gate), _p(counts), _p(logits),
+                         _p(scores))
+    if rc != 0:
+        raise ValueError("invalid routing shape")
+    out = {"topk_idx": idx, "topk_gate": gate, "counts": counts}
+    if want_scores:
+        out["logits"] = logits
+        out["scores"] = scores
+    return out
+
+
+def update_bias(counts: np.ndarray, bias: np.ndarray, T: int, topk: int,
+                gamma: float) -> np.ndarray:
+    b = _c(bias, np.float32).copy()
+    c = _c(counts, np.int32)
+    lib().orc_update_bias(T, b.size, topk, _p(c), ctypes.c_float(gamma), _p(b))
+    return b
+
+
+def permute_layout(topk_idx: np.ndarray, counts: np.ndarray, n_routed: int):
+    T, K = topk_idx.shape
+    idx = _c(topk_idx, np.int32)
+    c = _c(counts, np.int32)
+    offsets = np.empty((n_routed + 2,), dtype=np.int32)
+    rop = np.empty((T, K), dtype=np.int32)
+    lib().orc_permute_layout(T, n_routed, K, _p(idx), _p(c), _p(offsets), _p(rop))
+    return offsets, rop
+
+
+# ----------------------------------------------------------------- experts
+def quantized_expert(w1_bf16, w3_bf16, w2_bf16):
+    """Oracle quantisation of one expert's bf16 weights (128x128 blocks)."""
+    return quant_w_128x128(w1_bf16), quant_w_128x128(w3_bf16), quant_w_128x128(w2_bf16)
+
+
+def swiglu_expert(xq: np.ndarray, xs: np.ndarray, w1, w3, w2,
+                  return_h: bool = False):
+    """One expert on FP8 rows (xq, xs = 1x128 codes and scales).
+
+    w1, w3, w2 = (codes, scales) pairs, [I,d], [I,d], [d,I].
+    a = X W1^T and c = X W3^T in FP64 over dequantised values;
+    h = silu(a) * c with silu(a) = a / (1 + exp(-a)), rounded to fp32;
+    h re-quantised 1x128 along I (every Fprop GEMM input is FP8);
+    o = H W2^T in FP64.  Returns o (FP64 [rows, d])."""
+    X = dequant_act(xq, xs)
+    W1 = dequant_w(*w1)
+    W3 = dequant_w(*w3)
+    a = X @ W1.T
+    c = X @ W3.T
+    h = (a / (1.0 + np.exp(-a))) * c
+    h32 = h.astype(np.float32)
+    hq, hs = quant_act_1x128(h32)
+    o = dequant_act(hq, hs) @ dequant_w(*w2).T
+    if return_h:
+        return o, h32, hq, hs
+    return o
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round FP64 directly to bf16 (8 significant bits), nearest-even.
+
+    Done in FP64: scale each value by a power of two so that the bf16 grid
+    step is 1, rint (ties to even), scale back; all steps are exact.
+    Values below the bf16 normal range use the subnormal step 2^-133."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    # correct floor(log2) at exact powers of two / rounding of log2
+    e = np.where(np.ldexp(1.0, e.astype(np.int32)) > a, e - 1, e)
+    e = np.where(np.ldexp(1.0, (e + 1).astype(np.int32)) <= a, e + 1, e)
+    e = np.maximum(e, -126.0)
+    step = np.ldexp(1.0, (e - 7).astype(np.int32))
+    r = np.rint(a / step) * step
+    r = np.where(a > 0, r, 0.0)
+    r32 = np.copysign(r, v).astype(np.float32)  # exact: r is on the bf16 grid
+    bits = r32.view(np.uint32) >> np.uint32(16)
+    return bits.astype(np.uint16)
+
+
+def combine(o_shared: np.ndarray, o_routed: np.ndarray, gates: np.ndarray) -> np.ndarray:
+    """y_t = o_shared_t + sum_k g_tk * o_tk in FP64, rounded once to bf16.
+
+    o_shared [T,d]; o_routed [T,K,d]; gates [T,K] fp32.  Returns bf16 bits."""
+    y = o_shared + np.einsum("tk,tkd->td", gates.astype(np.float64), o_routed)
+    return f64_to_bf16_bits(y)
+
+
+def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarray,
+                  n_groups: int, topk_groups: int, topk: int,
+                  expert_weights: Callable[[int], tuple],
+                  logit_offset: Optional[np.ndarray] = None,
+                  tokens: Optional[np.ndarray] = None) -> dict:
+    """Whole layer for all tokens (routing) and the chosen ``tokens`` (output).
+
+    expert_weights(e) returns ((w1q,w1s),(w3q,w3s),(w2q,w2s)) for expert e;
+    e = n_routed is the shared expert.  Experts are visited once each.
+    Returns routing results, x codes/scales, and y (bf16 bits) for ``tokens``."""
+    T, d = x_bf16.shape
+    n_routed = router_w_bf16.shape[0]
+    r = route(x_bf16, router_w_bf16, bias, n_groups, topk_groups, topk, logit_offset)
+    xq, xs = quant_act_1x128(x_bf16)
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    idx = r["topk_idx"][tokens]
+    o_routed = np.zeros((len(tokens), topk, d), dtype=np.float64)
+    o_shared = np.zeros((len(tokens), d), dtype=np.float64)
+    for e in range(n_routed + 1):
+        if e == n_routed:
+            sel = np.arange(len(tokens))
+            slots = None
+        else:
+            sel, slots = np.nonzero(idx == e)
+            if sel.size == 0:
+                continue
+        w = expert_weights(e)
+        o = swiglu_expert(xq[tokens[sel]], xs[tokens[sel]], *w)
+        if slots is None:
+            o_shared[sel] = o
+        else:
+            o_routed[sel, slots] = o
+    y = combine(o_shared, o_routed, r["topk_gate"][tokens])
+    r.update({"xq": xq, "xs": xs, "y": y, "tokens": tokens})
+    return r
+
+
+def gemm_blockscaled(aq, a_s, bq, b_s):
+    """C = dq(A) dq(B)^T in FP64; A [m,k] 1x128-scaled, B [n,k] 128x128-scaled."""
+    return dequant_act(aq, a_s) @ dequant_w(bq, b_s).T
