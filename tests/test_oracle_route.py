@@ -207,3 +207,20 @@ def test_route_rejects_bad_group_shape():
         oracle.route(x, E, np.zeros(10, np.float32), 3, 1, 2)
     with pytest.raises(ValueError):
         oracle.route(x, E, np.zeros(10, np.float32), 5, 1, 3)  # 1 group of 2 < K
+
+
+def test_ties_go_to_the_lower_index():
+    """Reading (pages silent on ties): equal group scores and equal biased
+    affinities resolve to the lower group / expert index.  All 8 experts get
+    the same logit, so groups 0 and 1 and experts 0, 1, 2 win (by hand)."""
+    x = np.zeros((2, 128), np.float32)
+    x[:, 0] = 1.0
+    E = np.zeros((8, 128), np.float32)
+    E[:, 0] = 0.75
+    b = np.zeros(8, np.float32)
+    r = oracle.route(S.f32_to_bf16_bits(x), S.f32_to_bf16_bits(E), b, 4, 2, 3)
+    assert r["topk_idx"].tolist() == [[0, 1, 2], [0, 1, 2]]
+    # a tie only inside the later group: experts 5 and 4 equal, above the rest
+    E[4, 0] = E[5, 0] = 2.0
+    r = oracle.route(S.f32_to_bf16_bits(x), S.f32_to_bf16_bits(E), b, 4, 2, 3)
+    assert r["topk_idx"].tolist() == [[4, 5, 0], [4, 5, 0]]
