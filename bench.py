@@ -1,0 +1,487 @@
+"""Benchmark of the DeepSeekMoE layer forward with FP8 block scaling on B200.
+
+Default workload: the full-size prefill layer (T=4096 tokens, d=7168, 256
+routed experts in 8 groups + 1 shared, top-4 groups, K=8, SwiGLU I=2048,
+FP8 E4M3 1x128 / 128x128 scales).  One step = the whole hot path over one
+batch: routing (+ load histogram), 1x128 quantisation of x, permutation,
+grouped GEMM W13 with SwiGLU + 1x128 quantisation of h, grouped GEMM W2,
+combine, bias update.  Expert weights are quantised once before timing (the
+offline weight quantisation is timed separately and reported).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  The path does not shard (one
+layer on one GPU): N > 1 runs N independent replicas, each on its own batch
+("replicas only", weak scaling); value = all ranks' tokens / max-over-ranks
+time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s and expert-GEMM FP8 TFLOPS (% of B200 FP8 dense peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0  # nominal dense ratio fp8 : bf16 (4.5 : 2.25 PFLOP/s)
+CPU_SAMPLE_TOKENS = 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- workload
+def algorithmic_counts(cfg, counts_host):
+    """Algorithmic FLOPs and bytes of one layer step."""
+    d, I, K, T = cfg.d, cfg.inter, cfg.topk, cfg.T
+    rows = T * K + T
+    touched = int((counts_host > 0).sum()) + 1  # + shared expert
+    w13_b = 2 * I * d + 4 * (2 * I // 128) * (d // 128)
+    w2_b = d * I + 4 * (d // 128) * (I // 128)
+    flops_gemm1 = 2.0 * rows * (2 * I) * d
+    flops_gemm2 = 2.0 * rows * d * I
+    gemm1_bytes = touched * w13_b + rows * (d + 4 * d // 128) + rows * (I + 4 * I // 128)
+    gemm2_bytes = touched * w2_b + rows * (I + 4 * I // 128) + rows * d * 4
+    layer_bytes = touched * (w13_b + w2_b) + 2 * T * d * 2
+    return {"rows": rows, "touched": touched, "flops_gemm1": flops_gemm1,
+            "flops_gemm2": flops_gemm2, "gemm1_bytes": gemm1_bytes, "gemm2_bytes": gemm2_bytes,
+            "layer_bytes": layer_bytes, "layer_flops": flops_gemm1 + flops_gemm2}
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "fp8_block_scaled_affinity_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_tag: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.txt")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"^source_hash:\s*(\S+)", text, re.M)
+    t = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    if not m or not t or m.group(1) != gemm_source_hash():
+        return None
+    return float(t.group(1))
+
+
+def build_layer(cfg, dev):
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    import synthetic as S
+    inp = S.make_layer_inputs_host(cfg, 0)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    shape = moe.make_shape(cfg.T, cfg.d, cfg.n_routed, cfg.n_groups, cfg.topk_groups, cfg.topk,
+                           cfg.inter, cfg.gamma)
+    layer = moe.MoeLayer(shape, bf16(inp["router_w"]), torch.from_numpy(inp["bias"]).to(dev),
+                         device=dev, host_io=True)
+    small = cfg.d * cfg.inter <= 512 * 256
+    wq_ms = 0.0
+    st = torch.cuda.current_stream()
+    for e in range(cfg.n_routed + 1):
+        if small:
+            w = tuple(bf16(m) for m in S.host_expert_weights(cfg, e))
+        else:
+            w = S.device_expert_weights(cfg, e, dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        layer.set_expert(e, *w)
+        b.record(st)
+        b.synchronize()
+        wq_ms += a.elapsed_time(b)
+    x = bf16(inp["x"])
+    off = None if inp["logit_offset"] is None else torch.from_numpy(inp["logit_offset"]).to(dev)
+    return layer, x, off, inp, wq_ms
+
+
+def stage_breakdown(layer, x, off, steps):
+    """Time each stage of the step on the launching stream with CUDA events
+    (the same kernels moe_layer_forward launches, called stage by stage)."""
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    from fp8_block_scaled_affinity_b200 import _lib
+    sh = layer.shape
+    T, d, I, N, K = sh.T, sh.d, sh.inter, sh.n_routed, sh.topk
+    R = T * K + T
+    dev = x.device
+    xq = torch.empty((T, d), dtype=torch.uint8, device=dev)
+    xs = torch.empty((T, d // 128), dtype=torch.float32, device=dev)
+    xq_p = torch.empty((R, d), dtype=torch.uint8, device=dev)
+    xs_p = torch.empty((d // 128, R), dtype=torch.float32, device=dev)
+    hq = torch.empty((R, I), dtype=torch.uint8, device=dev)
+    hs = torch.empty((I // 128, R), dtype=torch.float32, device=dev)
+    o = torch.empty((R, d), dtype=torch.float32, device=dev)
+    y = torch.empty_like(x)
+    rws = torch.empty((moe.moe_route_workspace_size(sh),), dtype=torch.uint8, device=dev)
+    pws = torch.empty((moe.moe_permute_workspace_size(sh),), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    names = ["route", "quant_x", "permute", "gemm1_swiglu", "gemm2", "combine", "update_bias"]
+    calls = [
+        lambda: moe.moe_route(sh, x, layer.router_w, layer.bias, off, layer.topk_idx,
+                              layer.topk_gate, layer.expert_counts, rws),
+        lambda: moe.fp8_quant_act_1x128(x, xq, xs),
+        lambda: moe.moe_permute(sh, layer.topk_idx, layer.expert_counts, xq, xs, xq_p, xs_p,
+                                layer.expert_offsets, layer.row_of_pair, pws),
+        lambda: moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, xq_p, xs_p, d,
+                                         layer.w13, layer.w13_scales, 2 * I,
+                                         _lib.MOE_EPI_SWIGLU_QUANT, hq, hs, layer.dev_status),
+        lambda: moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, hq, hs, I, layer.w2,
+                                         layer.w2_scales, d, _lib.MOE_EPI_F32, o, None,
+                                         layer.dev_status),
+        lambda: moe.moe_combine(sh, o, layer.expert_offsets, layer.row_of_pair,
+                                layer.topk_gate, y),
+        lambda: moe.moe_update_bias(sh, layer.expert_counts, layer.bias),
+    ]
+    tot = {n: 0.0 for n in names}
+    for it in range(steps + 2):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        ev[0].record(st)
+        for i, c in enumerate(calls):
+            c()
+            ev[i + 1].record(st)
+        ev[-1].synchronize()
+        if it >= 2:
+            for i, n in enumerate(names):
+                tot[n] += ev[i].elapsed_time(ev[i + 1])
+    return {n: tot[n] / steps for n in names}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample_time(cfg, inp, dev, n_tokens, seed=0):
+    """The oracle (as it stands) on a bounded sample: n_tokens tokens through
+    routing, quantisation, the experts they touch and the combine.  Expert
+    weights are quantised by the oracle beforehand (untimed, like the GPU
+    path's offline weight quantisation).  Returns (seconds, tokens, cores)."""
+    import numpy as np
+    import torch
+    import oracle
+    import synthetic as S
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(cfg.T, n_tokens, replace=False))
+    x = inp["x"][toks]
+    r = oracle.route(x, inp["router_w"], inp["bias"], cfg.n_groups, cfg.topk_groups, cfg.topk,
+                     logit_offset=inp["logit_offset"])
+    need = sorted(set(r["topk_idx"].ravel().tolist()) | {cfg.n_routed})
+    small = cfg.d * cfg.inter <= 512 * 256
+    W = {}
+    for e in need:
+        if small:
+            w = S.host_expert_weights(cfg, e)
+        else:
+            w = tuple(t.cpu().view(torch.int16).numpy().view(np.uint16)
+                      for t in S.device_expert_weights(cfg, e, dev))
+        W[e] = oracle.quantized_expert(*w)
+    t0 = time.perf_counter()
+    oracle.layer_forward(x, inp["router_w"], inp["bias"], cfg.n_groups, cfg.topk_groups,
+                         cfg.topk, W.__getitem__, logit_offset=inp["logit_offset"])
+    dt = time.perf_counter() - t0
+    return dt, n_tokens, os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- main
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a host float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, world, rank):
+    """The oracle timed on the host cores: each step is a bounded sample of
+    the workload (CPU_SAMPLE_TOKENS tokens)."""
+    import numpy as np
+    import torch
+    import synthetic as S
+    if rank != 0:
+        return
+    cfg = S.CONFIGS[args.workload]
+    dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
+    inp = S.make_layer_inputs_host(cfg, 0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, n, cores = oracle_sample_time(cfg, inp, dev, CPU_SAMPLE_TOKENS, seed=i)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = args.steps * CPU_SAMPLE_TOKENS / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_routed": cfg.n_routed,
+                   "n_groups": cfg.n_groups, "topk_groups": cfg.topk_groups,
+                   "topk": cfg.topk, "inter": cfg.inter,
+                   "sample_tokens_per_step": CPU_SAMPLE_TOKENS},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count() or 1,
+                         "kind": "oracle",
+                         "sample": f"{CPU_SAMPLE_TOKENS} random tokens per step of the "
+                                   f"{cfg.name} batch (routing, quantisation, touched experts,"
+                                   " combine)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    import synthetic as S
+
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.CONFIGS[args.workload]
+    peaks, peak_src = load_peaks()
+    layer, x, off, inp, wq_ms = build_layer(cfg, dev)
+    st = torch.cuda.current_stream()
+    y = torch.empty_like(x)
+
+    # ---- warm-up, then K timed steps of the whole layer (inputs in HBM)
+    for _ in range(args.warmup):
+        layer.forward(x, y, update_bias=True, logit_offset=off)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(args.steps):
+        layer.forward(x, y, update_bias=True, logit_offset=off)
+    ev1.record(st)
+    ev1.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world)
+    status = layer.status()
+    counts = layer.expert_counts.cpu().numpy()
+    tokens_total = cfg.T * args.steps * world
+    value = tokens_total / (ms / 1e3)
+
+    # ---- end to end through the host-buffer entry point (pinned memory)
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    for _ in range(max(1, args.warmup // 2)):
+        layer.forward_host(x_host, y_host, update_bias=True, logit_offset=off)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        layer.forward_host(x_host, y_host, update_bias=True, logit_offset=off)
+    e1.record(st)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    xbytes = cfg.T * cfg.d * 2
+
+    # ---- per-stage breakdown (CUDA events on the launching stream)
+    brk = stage_breakdown(layer, x, off, args.steps)
+    alg = algorithmic_counts(cfg, counts)
+    g1_ms = brk["gemm1_swiglu"]
+    achieved = alg["gemm1_bytes"] / (g1_ms / 1e3) / 1e9
+    hbm_peak = float(peaks["hbm_gbs"])
+    fp8_peak_burst = float(peaks["bf16_tflops"]) * FP8_PER_BF16
+    fp8_peak_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP8_PER_BF16
+    gemm_ms = brk["gemm1_swiglu"] + brk["gemm2"]
+    gemm_tflops = alg["layer_flops"] / (gemm_ms / 1e3) / 1e12
+    layer_tflops = alg["layer_flops"] * args.steps * world / (ms / 1e3) / 1e12
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3/f32",
+        "data": "synthetic",
+        "config": {"workload": f"moe_layer_{cfg.name}", "T": cfg.T, "d": cfg.d,
+                   "n_routed": cfg.n_routed, "n_shared": 1, "n_groups": cfg.n_groups,
+                   "topk_groups": cfg.topk_groups, "topk": cfg.topk, "inter": cfg.inter,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (FP8 expert weights "
+                         f"{(cfg.n_routed + 1) * 3 * cfg.d * cfg.inter / 1e9:.1f} GB)"},
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm_kernel<2> (W13 + SwiGLU + h quant)",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_source": peak_src,
+                     "traffic": profiled_traffic("gemm_swiglu_prefill"),
+                     "algorithmic_bytes_per_launch": alg["gemm1_bytes"],
+                     "launch_ms": g1_ms},
+        "expert_gemm": {"tflops": gemm_tflops, "fp8_peak_tflops": fp8_peak_burst,
+                        "frac_of_fp8_peak": gemm_tflops / fp8_peak_burst,
+                        "frac_of_fp8_sustained": gemm_tflops / fp8_peak_sust,
+                        "gemm1_ms": brk["gemm1_swiglu"], "gemm2_ms": brk["gemm2"],
+                        "flops_per_step": alg["layer_flops"]},
+        "layer_tflops": layer_tflops,
+        "breakdown_ms": brk,
+        "weight_quant": {"ms_total": wq_ms,
+                         "gbs": (cfg.n_routed + 1) * 3 * cfg.d * cfg.inter * 3 / (wq_ms / 1e3) / 1e9},
+        "load": {"max_over_mean": float(counts.max() / max(counts.mean(), 1e-9)),
+                 "experts_touched": alg["touched"]},
+        "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes},
+        "gpu_launches": 11 * args.steps,
+        "clocks": clk,
+        "device_status": status,
+    }
+    # CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, n, cores = oracle_sample_time(cfg, inp, dev, CPU_SAMPLE_TOKENS)
+        line["cpu_baseline"] = {
+            "value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} random tokens of the {cfg.name} batch (routing, quantisation, "
+                      "touched experts, combine); weights pre-quantised by the oracle"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill", choices=["tiny", "prefill", "decode", "skewed"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

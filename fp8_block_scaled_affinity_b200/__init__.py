@@ -1,0 +1,100 @@
+"""B200-native DeepSeekMoE layer forward with FP8 block scaling.
+
+The compute lives in libmoefp8.so (hand-written sm_100a CUDA kernels behind a
+C ABI, declared in include/moefp8.h).  This package is the thin Python side:
+the ctypes binding with the C names (``_lib``) and ``MoeLayer``, which owns
+the device buffers of one layer (allocated with torch) and calls the library.
+There is no CPU or PyTorch fallback: if the library is missing, loading it
+raises.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QUANT,  # noqa: F401
+                   MoeError, MoeRouting, MoeShape, MoeWeights, fp8_quant_act_1x128,
+                   fp8_quant_w_128x128, lib, make_routing, make_shape, make_weights,
+                   moe_combine, moe_grouped_gemm_fp8, moe_layer_forward,
+                   moe_layer_forward_host, moe_layer_host_workspace_size,
+                   moe_layer_workspace_size, moe_permute, moe_permute_workspace_size,
+                   moe_read_status, moe_route, moe_route_workspace_size, moe_update_bias,
+                   moe_version, status_string)
+
+__all__ = ["MoeLayer", "MoeShape", "MoeError", "lib", "make_shape", "moe_version"]
+
+
+class MoeLayer:
+    """Device state of one MoE layer: FP8 expert weights, router weights,
+    the balancing bias and the workspace.
+
+    shape: a MoeShape (see make_shape).  router_w: bf16 [N_r, d] on the GPU.
+    bias: fp32 [N_r] on the GPU (updated in place by forward(update_bias=True)).
+    """
+
+    def __init__(self, shape: MoeShape, router_w, bias, device=None, host_io: bool = False):
+        import torch
+        self.shape = shape
+        dev = torch.device(device) if device is not None else router_w.device
+        self.device = dev
+        N, d, I = shape.n_routed, shape.d, shape.inter
+        E = N + 1
+        self.router_w = router_w
+        self.bias = bias
+        u8 = torch.uint8
+        self.w13 = torch.empty((E, 2 * I, d), dtype=u8, device=dev)
+        self.w13_scales = torch.empty((E, 2 * I // 128, d // 128), dtype=torch.float32, device=dev)
+        self.w2 = torch.empty((E, d, I), dtype=u8, device=dev)
+        self.w2_scales = torch.empty((E, d // 128, I // 128), dtype=torch.float32, device=dev)
+        T, K = shape.T, shape.topk
+        i32 = torch.int32
+        self.topk_idx = torch.empty((T, K), dtype=i32, device=dev)
+        self.topk_gate = torch.empty((T, K), dtype=torch.float32, device=dev)
+        self.expert_counts = torch.empty((N,), dtype=i32, device=dev)
+        self.expert_offsets = torch.empty((N + 2,), dtype=i32, device=dev)
+        self.row_of_pair = torch.empty((T, K), dtype=i32, device=dev)
+        self.dev_status = torch.zeros((1,), dtype=i32, device=dev)
+        ws_bytes = (moe_layer_host_workspace_size(shape) if host_io
+                    else moe_layer_workspace_size(shape))
+        self.ws = torch.empty((max(ws_bytes, 256),), dtype=u8, device=dev)
+        self._weights = None
+        self._routing = make_routing(self.topk_idx, self.topk_gate, self.expert_counts,
+                                     self.expert_offsets, self.row_of_pair)
+
+    def set_expert(self, e: int, w1, w3, w2, stream=None) -> None:
+        """Quantise expert e's bf16 weights (W1, W3: [I, d]; W2: [d, I]) into
+        the layer's FP8 buffers with 128x128 blocks.  e = N_r is the shared
+        expert."""
+        I = self.shape.inter
+        fp8_quant_w_128x128(w1, self.w13[e, :I], self.w13_scales[e, :I // 128],
+                            stream=stream)
+        fp8_quant_w_128x128(w3, self.w13[e, I:], self.w13_scales[e, I // 128:],
+                            stream=stream)
+        fp8_quant_w_128x128(w2, self.w2[e], self.w2_scales[e], stream=stream)
+        self._weights = None
+
+    def weights(self) -> MoeWeights:
+        if self._weights is None:
+            self._weights = make_weights(self.w13, self.w13_scales, self.w2, self.w2_scales,
+                                         self.router_w)
+        return self._weights
+
+    def forward(self, x, y=None, update_bias: bool = False, logit_offset=None, stream=None):
+        """y = MoE(x) for bf16 x [T, d] on the GPU; returns y (bf16 [T, d])."""
+        import torch
+        if y is None:
+            y = torch.empty_like(x)
+        moe_layer_forward(self.shape, self.weights(), x, self.bias, logit_offset,
+                          self._routing, y, update_bias, self.ws, self.dev_status, stream)
+        return y
+
+    def forward_host(self, x_host, y_host, update_bias: bool = False, logit_offset=None,
+                     stream=None):
+        """The same with x and y in (pinned) host memory; the copies run on
+        `stream` inside the call.  Synchronise the stream before reading y."""
+        moe_layer_forward_host(self.shape, self.weights(), x_host, self.bias, logit_offset,
+                               self._routing, y_host, update_bias, self.ws, self.dev_status,
+                               stream)
+
+    def status(self, stream=None) -> int:
+        """Device status word (0 = fine); synchronises the stream."""
+        return moe_read_status(self.dev_status, stream)

@@ -1,0 +1,225 @@
+"""ctypes binding of libmoefp8.so (the C ABI declared in include/moefp8.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Functions keep the C names; tensors are torch tensors on the
+current CUDA device (their data pointers are passed), and `stream` defaults to
+torch's current stream.  A non-zero status raises MoeError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoefp8.so")
+
+MOE_OK = 0
+MOE_EPI_F32 = 0
+MOE_EPI_BF16 = 1
+MOE_EPI_SWIGLU_QUANT = 2
+MOE_DEV_TIMEOUT = 1
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("d", ctypes.c_int), ("n_routed", ctypes.c_int),
+                ("n_groups", ctypes.c_int), ("topk_groups", ctypes.c_int),
+                ("topk", ctypes.c_int), ("inter", ctypes.c_int), ("gamma", ctypes.c_float)]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [("w13", ctypes.c_void_p), ("w13_scales", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("w2_scales", ctypes.c_void_p),
+                ("router_w", ctypes.c_void_p)]
+
+
+class MoeRouting(ctypes.Structure):
+    _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_gate", ctypes.c_void_p),
+                ("expert_counts", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
+                ("row_of_pair", ctypes.c_void_p)]
+
+
+_L = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoefp8.so (built in-tree by __graft_entry__.build()).  Raises
+    if it is missing: there is no fallback implementation."""
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        SP = ctypes.POINTER(MoeShape)
+        sig = {
+            "moe_version": (I, []),
+            "moe_status_string": (ctypes.c_char_p, [I]),
+            "moe_read_status": (I, [P, P, P]),
+            "moe_route_workspace_size": (SZ, [SP]),
+            "moe_route": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "fp8_quant_act_1x128": (I, [P, I64, I64, P, P, I, P, P]),
+            "fp8_quant_w_128x128": (I, [P, I64, I64, P, P, P, P]),
+            "moe_permute_workspace_size": (SZ, [SP]),
+            "moe_permute": (I, [SP, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "moe_grouped_gemm_fp8": (I, [I, P, I, P, P, I, P, P, I, I, P, P, P, P]),
+            "moe_combine": (I, [SP, P, P, P, P, P, P, P]),
+            "moe_update_bias": (I, [SP, P, P, P, P]),
+            "moe_layer_workspace_size": (SZ, [SP]),
+            "moe_layer_forward": (I, [SP, ctypes.POINTER(MoeWeights), P, P, P,
+                                      ctypes.POINTER(MoeRouting), P, I, P, SZ, P, P]),
+            "moe_layer_host_workspace_size": (SZ, [SP]),
+            "moe_layer_forward_host": (I, [SP, ctypes.POINTER(MoeWeights), P, P, P,
+                                           ctypes.POINTER(MoeRouting), P, I, P, SZ, P, P]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _L = L
+    return _L
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(name: str, rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(name, rc)
+
+
+def make_shape(T, d, n_routed, n_groups, topk_groups, topk, inter, gamma=0.001) -> MoeShape:
+    return MoeShape(int(T), int(d), int(n_routed), int(n_groups), int(topk_groups), int(topk),
+                    int(inter), float(gamma))
+
+
+def moe_version() -> int:
+    return lib().moe_version()
+
+
+def moe_read_status(dev_status, stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check("moe_read_status", lib().moe_read_status(_ptr(dev_status), ctypes.addressof(out),
+                                                    _stream(stream)))
+    return out.value
+
+
+def moe_route_workspace_size(shape: MoeShape) -> int:
+    return lib().moe_route_workspace_size(ctypes.byref(shape))
+
+
+def moe_route(shape, x, router_w, bias, logit_offset, topk_idx, topk_gate, expert_counts,
+              ws, dev_status=None, stream=None) -> None:
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("moe_route", lib().moe_route(
+        ctypes.byref(shape), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(logit_offset),
+        _ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def fp8_quant_act_1x128(x, q, scales, scales_kb_major=False, dev_status=None, stream=None):
+    rows, cols = x.shape
+    _check("fp8_quant_act_1x128", lib().fp8_quant_act_1x128(
+        _ptr(x), rows, cols, _ptr(q), _ptr(scales), int(bool(scales_kb_major)),
+        _ptr(dev_status), _stream(stream)))
+
+
+def fp8_quant_w_128x128(w, q, scales, dev_status=None, stream=None):
+    rows, cols = w.shape
+    _check("fp8_quant_w_128x128", lib().fp8_quant_w_128x128(
+        _ptr(w), rows, cols, _ptr(q), _ptr(scales), _ptr(dev_status), _stream(stream)))
+
+
+def moe_permute_workspace_size(shape: MoeShape) -> int:
+    return lib().moe_permute_workspace_size(ctypes.byref(shape))
+
+
+def moe_permute(shape, topk_idx, expert_counts, xq, xs, xq_perm, xs_perm, expert_offsets,
+                row_of_pair, ws, dev_status=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("moe_permute", lib().moe_permute(
+        ctypes.byref(shape), _ptr(topk_idx), _ptr(expert_counts), _ptr(xq), _ptr(xs),
+        _ptr(xq_perm), _ptr(xs_perm), _ptr(expert_offsets), _ptr(row_of_pair), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_grouped_gemm_fp8(n_groups, group_offsets, max_rows, a, a_scales, k, w, w_scales, n,
+                         epilogue, out, out_scales=None, dev_status=None, stream=None):
+    _check("moe_grouped_gemm_fp8", lib().moe_grouped_gemm_fp8(
+        int(n_groups), _ptr(group_offsets), int(max_rows), _ptr(a), _ptr(a_scales), int(k),
+        _ptr(w), _ptr(w_scales), int(n), int(epilogue), _ptr(out), _ptr(out_scales),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_combine(shape, expert_out, expert_offsets, row_of_pair, topk_gate, y,
+                dev_status=None, stream=None):
+    _check("moe_combine", lib().moe_combine(
+        ctypes.byref(shape), _ptr(expert_out), _ptr(expert_offsets), _ptr(row_of_pair),
+        _ptr(topk_gate), _ptr(y), _ptr(dev_status), _stream(stream)))
+
+
+def moe_update_bias(shape, expert_counts, bias, dev_status=None, stream=None):
+    _check("moe_update_bias", lib().moe_update_bias(
+        ctypes.byref(shape), _ptr(expert_counts), _ptr(bias), _ptr(dev_status),
+        _stream(stream)))
+
+
+def moe_layer_workspace_size(shape: MoeShape) -> int:
+    return lib().moe_layer_workspace_size(ctypes.byref(shape))
+
+
+def moe_layer_host_workspace_size(shape: MoeShape) -> int:
+    return lib().moe_layer_host_workspace_size(ctypes.byref(shape))
+
+
+def make_weights(w13, w13_scales, w2, w2_scales, router_w) -> MoeWeights:
+    return MoeWeights(_ptr(w13), _ptr(w13_scales), _ptr(w2), _ptr(w2_scales), _ptr(router_w))
+
+
+def make_routing(topk_idx, topk_gate, expert_counts, expert_offsets, row_of_pair) -> MoeRouting:
+    return MoeRouting(_ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts),
+                      _ptr(expert_offsets), _ptr(row_of_pair))
+
+
+def moe_layer_forward(shape, weights: MoeWeights, x, bias, logit_offset, routing: MoeRouting,
+                      y, update_bias, ws, dev_status=None, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_layer_forward", lib().moe_layer_forward(
+        ctypes.byref(shape), ctypes.byref(weights), _ptr(x), _ptr(bias), _ptr(logit_offset),
+        ctypes.byref(routing), _ptr(y), int(bool(update_bias)), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_layer_forward_host(shape, weights: MoeWeights, x_host, bias, logit_offset,
+                           routing: MoeRouting, y_host, update_bias, ws, dev_status=None,
+                           stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_layer_forward_host", lib().moe_layer_forward_host(
+        ctypes.byref(shape), ctypes.byref(weights), _ptr(x_host), _ptr(bias),
+        _ptr(logit_offset), ctypes.byref(routing), _ptr(y_host), int(bool(update_bias)),
+        _ptr(ws), nbytes, _ptr(dev_status), _stream(stream)))

@@ -1,0 +1,311 @@
+// Single-GPU dispatch and combine of the MoE block ("DeepSeek-V3 Technical
+// Report" notes page, section "DualPipe": all-to-all dispatch / combine of
+// each chunk; section "FP8 mixed precision training": FP8 activations are
+// what is dispatched) and the bias update of section "DeepSeekMoE and
+// auxiliary-loss-free load balancing".
+//
+// moe_permute builds an expert-contiguous copy of the FP8 token rows:
+//   1. chunk_hist: per chunk of kChunk tokens, how many of its pairs go to
+//      each expert (scratch [n_chunks, N_r]);
+//   2. chunk_scan: per expert, the exclusive scan of those counts over
+//      chunks plus the expert's base offset -> first row of each
+//      (chunk, expert); block 0 also writes expert_offsets;
+//   3. chunk_rank: per chunk, one warp walks its tokens in order and hands
+//      out rows (tokens stay in ascending order inside every expert);
+//   4. copy_rows: one warp per token reads its FP8 row once (16-byte loads)
+//      and writes it K+1 times, scales transposed to the kb-major layout.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kChunk = 64;
+
+__global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ topk_idx,
+                                                         int T, int K, int n_routed,
+                                                         int32_t* __restrict__ chunk_counts,
+                                                         int* dev_status) {
+    extern __shared__ int hist_smem[];
+    for (int i = threadIdx.x; i < n_routed; i += blockDim.x) hist_smem[i] = 0;
+    __syncthreads();
+    const int t0 = blockIdx.x * kChunk;
+    const int t1 = min(T, t0 + kChunk);
+    for (int p = t0 * K + threadIdx.x; p < t1 * K; p += blockDim.x) {
+        const int e = topk_idx[p];
+        if (e < 0 || e >= n_routed) set_status(dev_status, MOE_DEV_BAD_INPUT);
+        else atomicAdd(&hist_smem[e], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_routed; i += blockDim.x)
+        chunk_counts[int64_t(blockIdx.x) * n_routed + i] = hist_smem[i];
+}
+
+// One block (256 threads) per expert e.  Exclusive scan over chunks of
+// chunk_counts[., e], plus off[e] = sum of counts of experts < e.
+__global__ void __launch_bounds__(256) chunk_scan_kernel(const int32_t* __restrict__ counts,
+                                                         int T, int K, int n_routed, int n_chunks,
+                                                         int32_t* __restrict__ chunk_counts,
+                                                         int32_t* __restrict__ expert_offsets) {
+    __shared__ int warp_sums[8];
+    __shared__ int base_s;
+    const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // base offset of expert e
+    int part = 0;
+    for (int i = tid; i < e; i += 256) part += counts[i];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) warp_sums[warp] = part;
+    __syncthreads();
+    if (tid == 0) {
+        int b = 0;
+        for (int w = 0; w < 8; ++w) b += warp_sums[w];
+        base_s = b;
+    }
+    __syncthreads();
+    int running = base_s;
+    // scan over chunks, 256 at a time
+    for (int c0 = 0; c0 < n_chunks; c0 += 256) {
+        const int c = c0 + tid;
+        const int v = c < n_chunks ? chunk_counts[int64_t(c) * n_routed + e] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        __syncthreads();
+        if (lane == 31) warp_sums[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int w = 0; w < 8; ++w) {
+            const int ws = warp_sums[w];
+            if (w < warp) before += ws;
+            total += ws;
+        }
+        if (c < n_chunks) chunk_counts[int64_t(c) * n_routed + e] = running + before + incl - v;
+        running += total;
+    }
+    if (e == 0) {
+        // expert_offsets: serial prefix by thread 0 (N_r <= 1024 values)
+        __syncthreads();
+        if (tid == 0) {
+            int acc = 0;
+            for (int i = 0; i < n_routed; ++i) {
+                expert_offsets[i] = acc;
+                acc += counts[i];
+            }
+            expert_offsets[n_routed] = acc;
+            expert_offsets[n_routed + 1] = acc + T;
+        }
+    }
+}
+
+// One warp per chunk: tokens in ascending order; lane k < K takes slot k of
+// the token (the K experts of a token are distinct, so no two lanes touch
+// the same cursor in one step).
+__global__ void __launch_bounds__(32) chunk_rank_kernel(const int32_t* __restrict__ topk_idx,
+                                                        int T, int K, int n_routed,
+                                                        const int32_t* __restrict__ chunk_base,
+                                                        const int32_t* __restrict__ offsets,
+                                                        int32_t* __restrict__ row_of_pair,
+                                                        int* dev_status) {
+    extern __shared__ int cursor[];
+    const int lane = threadIdx.x;
+    const int c = blockIdx.x;
+    for (int i = lane; i < n_routed; i += 32) cursor[i] = chunk_base[int64_t(c) * n_routed + i];
+    __syncwarp();
+    const int t1 = min(T, (c + 1) * kChunk);
+    for (int t = c * kChunk; t < t1; ++t) {
+        if (lane < K) {
+            const int e = topk_idx[int64_t(t) * K + lane];
+            int row = -1;
+            if (e >= 0 && e < n_routed) {
+                row = cursor[e];
+                cursor[e] = row + 1;
+                // expert_counts inconsistent with topk_idx: no row to give
+                if (row >= offsets[e + 1]) row = -1;
+            }
+            if (row < 0) set_status(dev_status, MOE_DEV_BAD_INPUT);
+            row_of_pair[int64_t(t) * K + lane] = row;
+        }
+        __syncwarp();
+    }
+}
+
+// One warp per token; the row is read once, 4 KB at a time (8 x 16 bytes
+// per lane), and each piece is written K+1 times.
+constexpr int kPiece = 8;
+
+__global__ void __launch_bounds__(256) copy_rows_kernel(
+    const uint4* __restrict__ xq, const float* __restrict__ xs, int T, int d, int K,
+    const int32_t* __restrict__ row_of_pair, int64_t rows_total, uint4* __restrict__ xq_perm,
+    float* __restrict__ xs_perm) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = d / 16, nkb = d / 128;
+    const int warps_total = gridDim.x * (blockDim.x / 32);
+    for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        int my_row = 0;
+        if (lane < K) my_row = row_of_pair[int64_t(t) * K + lane];
+        const int shared_row = T * K + t;
+        const uint4* src = xq + int64_t(t) * nvec;
+        for (int c0 = 0; c0 < nvec; c0 += 32 * kPiece) {
+            uint4 v[kPiece];
+#pragma unroll
+            for (int j = 0; j < kPiece; ++j) {
+                const int c = c0 + lane + 32 * j;
+                if (c < nvec) v[j] = __ldcs(src + c);
+            }
+            for (int k = 0; k <= K; ++k) {
+                const int row = (k < K) ? __shfl_sync(0xffffffffu, my_row, k) : shared_row;
+                if (row < 0) continue;
+                uint4* dst = xq_perm + int64_t(row) * nvec;
+#pragma unroll
+                for (int j = 0; j < kPiece; ++j) {
+                    const int c = c0 + lane + 32 * j;
+                    if (c < nvec) dst[c] = v[j];
+                }
+            }
+        }
+        for (int k = 0; k <= K; ++k) {
+            const int row = (k < K) ? __shfl_sync(0xffffffffu, my_row, k) : shared_row;
+            if (row < 0) continue;
+            for (int kb = lane; kb < nkb; kb += 32)
+                xs_perm[int64_t(kb) * rows_total + row] = xs[int64_t(t) * nkb + kb];
+        }
+    }
+}
+
+// y[t] = o[shared row] + sum_k g[t,k] * o[row_of_pair[t,k]] (fp32, slot
+// order), rounded once to bf16.  One warp per token, float4 per lane.
+__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ o, int T, int d,
+                                                      int K, const int32_t* __restrict__ rop,
+                                                      const float* __restrict__ gate,
+                                                      uint2* __restrict__ y, int* dev_status) {
+    const int lane = threadIdx.x & 31;
+    const int nv = d / 4;
+    const int warps_total = gridDim.x * (blockDim.x / 32);
+    for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        int my_row = 0;
+        float my_g = 0.0f;
+        if (lane < K) {
+            my_row = rop[int64_t(t) * K + lane];
+            my_g = gate[int64_t(t) * K + lane];
+            if (my_row < 0 || my_row >= T * K) {  // skipped: contributes nothing
+                set_status(dev_status, MOE_DEV_BAD_INPUT);
+                my_row = T * K + t;
+                my_g = 0.0f;
+            }
+        }
+        const int64_t shared_row = int64_t(T) * K + t;
+        for (int c = lane; c < nv; c += 32) {
+            float4 acc = __ldcs(o + shared_row * nv + c);
+            for (int k = 0; k < K; ++k) {
+                const int row = __shfl_sync(0xffffffffu, my_row, k);
+                const float g = __shfl_sync(0xffffffffu, my_g, k);
+                const float4 v = __ldcs(o + int64_t(row) * nv + c);
+                acc.x = __fmaf_rn(g, v.x, acc.x);
+                acc.y = __fmaf_rn(g, v.y, acc.y);
+                acc.z = __fmaf_rn(g, v.z, acc.z);
+                acc.w = __fmaf_rn(g, v.w, acc.w);
+            }
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            y[int64_t(t) * nv + c] =
+                make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+        }
+    }
+}
+
+__global__ void update_bias_kernel(const int32_t* __restrict__ counts, int n_routed,
+                                   int64_t total, float gamma, float* __restrict__ bias) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n_routed) return;
+    const int64_t c = int64_t(counts[i]) * n_routed;
+    if (c > total) bias[i] = __fsub_rn(bias[i], gamma);
+    else if (c < total) bias[i] = __fadd_rn(bias[i], gamma);
+}
+
+int n_chunks_of(int T) { return (T + kChunk - 1) / kChunk; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" MOE_API size_t moe_permute_workspace_size(const MoeShape* shape) {
+    if (validate_shape(shape) != MOE_OK) return 0;
+    return align_up(size_t(n_chunks_of(shape->T)) * shape->n_routed * sizeof(int32_t) + 256, 256);
+}
+
+extern "C" MOE_API int moe_permute(const MoeShape* shape, const int32_t* topk_idx,
+                                   const int32_t* expert_counts, const uint8_t* xq,
+                                   const float* xs, uint8_t* xq_perm, float* xs_perm,
+                                   int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
+                                   size_t ws_bytes, int* dev_status, void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T, d = shape->d, K = shape->topk, N = shape->n_routed;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    const int n_chunks = n_chunks_of(T);
+    if (T > 0) {
+        if (!topk_idx || !xq || !xs || !xq_perm || !xs_perm || !row_of_pair) return MOE_ERR_NULL;
+        if (!aligned16(xq) || !aligned16(xq_perm)) return MOE_ERR_ALIGN;
+        if (!ws || ws_bytes < moe_permute_workspace_size(shape)) return MOE_ERR_WORKSPACE;
+    }
+    int32_t* chunk_counts = static_cast<int32_t*>(ws);
+    const size_t hist_smem = sizeof(int) * N;
+    if (T > 0) {
+        chunk_hist_kernel<<<n_chunks, 256, hist_smem, st>>>(topk_idx, T, K, N, chunk_counts,
+                                                            dev_status);
+        if ((rc = check_launch()) != MOE_OK) return rc;
+    }
+    chunk_scan_kernel<<<N, 256, 0, st>>>(expert_counts, T, K, N, n_chunks, chunk_counts,
+                                         expert_offsets);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    chunk_rank_kernel<<<n_chunks, 32, hist_smem, st>>>(topk_idx, T, K, N, chunk_counts,
+                                                       expert_offsets, row_of_pair, dev_status);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    const int64_t rows_total = int64_t(T) * K + T;
+    int blocks = (T + 7) / 8;
+    const int cap = sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    copy_rows_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(xq), xs, T, d, K,
+                                             row_of_pair, rows_total,
+                                             reinterpret_cast<uint4*>(xq_perm), xs_perm);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_combine(const MoeShape* shape, const float* expert_out,
+                                   const int32_t* expert_offsets, const int32_t* row_of_pair,
+                                   const float* topk_gate, uint16_t* y, int* dev_status,
+                                   void* stream) {
+    (void)expert_offsets;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T;
+    if (T == 0) return MOE_OK;
+    if (!expert_out || !row_of_pair || !topk_gate || !y) return MOE_ERR_NULL;
+    if (!aligned16(expert_out) || (reinterpret_cast<uintptr_t>(y) & 7)) return MOE_ERR_ALIGN;
+    int blocks = (T + 7) / 8;
+    const int cap = sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    combine_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
+        reinterpret_cast<const float4*>(expert_out), T, shape->d, shape->topk, row_of_pair,
+        topk_gate, reinterpret_cast<uint2*>(y), dev_status);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_update_bias(const MoeShape* shape, const int32_t* expert_counts,
+                                       float* bias, int* dev_status, void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    if (!expert_counts || !bias) return MOE_ERR_NULL;
+    const int N = shape->n_routed;
+    update_bias_kernel<<<(N + 255) / 256, 256, 0, as_stream(stream)>>>(
+        expert_counts, N, int64_t(shape->T) * shape->topk, shape->gamma, bias);
+    return check_launch();
+}

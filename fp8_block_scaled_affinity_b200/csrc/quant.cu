@@ -1,0 +1,149 @@
+// Online FP8 E4M3 quantisation: 1x128 activation tiles and 128x128 weight
+// blocks ("DeepSeek-V3 Technical Report" notes page, section "FP8 mixed
+// precision training": fine-grained quantisation, online max-abs scaling,
+// E4M3 for every tensor).  Both are single coalesced HBM passes with 16-byte
+// vector loads and stores.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+// One 1x128 tile per 16 threads; each thread owns 8 consecutive bf16 values
+// (one 16-byte load, one 8-byte store).  Grid-strides over tiles.
+__global__ void __launch_bounds__(256) quant_act_1x128_kernel(
+    const uint4* __restrict__ x, int64_t rows, int64_t cols, uint2* __restrict__ q,
+    float* __restrict__ scales, int kb_major) {
+    const int64_t tiles_per_row = cols >> 7;
+    const int64_t n_tiles = rows * tiles_per_row;
+    const int sub = threadIdx.x & 15;
+    // Both half-warps iterate together (the shuffles span the full warp);
+    // a half-warp past the last tile computes on zeros and stores nothing.
+    int64_t tile = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+    const int64_t tile_stride = (int64_t(gridDim.x) * blockDim.x) >> 4;
+    for (; (tile & ~int64_t(1)) < n_tiles; tile += tile_stride) {
+        const bool valid = tile < n_tiles;
+        const int64_t r = valid ? tile / tiles_per_row : 0;
+        const int64_t t = valid ? tile - r * tiles_per_row : 0;
+        const int64_t vec = (r * cols + (t << 7)) / 8 + sub;
+        uint4 w = valid ? __ldcs(x + vec) : make_uint4(0u, 0u, 0u, 0u);
+        float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        float scale, inv;
+        scale_from_amax(amax, scale, inv);
+        uint32_t c0 = e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv));
+        uint32_t c1 = e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv));
+        uint32_t c2 = e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv));
+        uint32_t c3 = e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+        if (!valid) continue;
+        q[vec] = make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
+        if (sub == 0) {
+            if (kb_major) scales[t * rows + r] = scale;
+            else scales[r * tiles_per_row + t] = scale;
+        }
+    }
+}
+
+// One 128x128 block per CTA of 256 threads; thread i owns half a row
+// (64 values = 8 x 16-byte loads).  Block amax via warp shuffles + smem.
+__global__ void __launch_bounds__(256) quant_w_128x128_kernel(
+    const uint4* __restrict__ w, int64_t rows, int64_t cols, uint4* __restrict__ q,
+    float* __restrict__ scales) {
+    __shared__ float warp_max[8];
+    const int64_t bc = cols >> 7;
+    const int64_t n_blocks = (rows >> 7) * bc;
+    const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
+    for (int64_t b = blockIdx.x; b < n_blocks; b += gridDim.x) {
+        const int64_t bi = b / bc, bj = b - bi * bc;
+        const int64_t base = ((bi * 128 + row) * cols + bj * 128 + half * 64) / 8;
+        uint4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __ldcs(w + base + i);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            amax = fmaxf(amax, fabsf(bf16_lo(v[i].x)));
+            amax = fmaxf(amax, fabsf(bf16_hi(v[i].x)));
+            amax = fmaxf(amax, fabsf(bf16_lo(v[i].y)));
+            amax = fmaxf(amax, fabsf(bf16_hi(v[i].y)));
+            amax = fmaxf(amax, fabsf(bf16_lo(v[i].z)));
+            amax = fmaxf(amax, fabsf(bf16_hi(v[i].z)));
+            amax = fmaxf(amax, fabsf(bf16_lo(v[i].w)));
+            amax = fmaxf(amax, fabsf(bf16_hi(v[i].w)));
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+        __syncthreads();
+        amax = warp_max[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[i]);
+        __syncthreads();  // warp_max is reused by the next block
+        float scale, inv;
+        scale_from_amax(amax, scale, inv);
+        const int64_t qbase = ((bi * 128 + row) * cols + bj * 128 + half * 64) / 16;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint4 s = v[2 * i + j];
+                uint32_t a0 = e4m3x2(__fmul_rn(bf16_lo(s.x), inv), __fmul_rn(bf16_hi(s.x), inv));
+                uint32_t a1 = e4m3x2(__fmul_rn(bf16_lo(s.y), inv), __fmul_rn(bf16_hi(s.y), inv));
+                uint32_t a2 = e4m3x2(__fmul_rn(bf16_lo(s.z), inv), __fmul_rn(bf16_hi(s.z), inv));
+                uint32_t a3 = e4m3x2(__fmul_rn(bf16_lo(s.w), inv), __fmul_rn(bf16_hi(s.w), inv));
+                o[2 * j] = a0 | (a1 << 16);
+                o[2 * j + 1] = a2 | (a3 << 16);
+            }
+            q[qbase + i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (threadIdx.x == 0) scales[b] = scale;
+    }
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" MOE_API int fp8_quant_act_1x128(const uint16_t* x, int64_t rows, int64_t cols,
+                                           uint8_t* q, float* scales, int scales_kb_major,
+                                           int* dev_status, void* stream) {
+    (void)dev_status;
+    if (rows < 0 || cols < 0 || cols % 128) return MOE_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!x || !q || !scales) return MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
+        return MOE_ERR_ALIGN;
+    if (scales_kb_major != 0 && scales_kb_major != 1) return MOE_ERR_ARG;
+    const int64_t threads = rows * (cols / 128) * 16;
+    int64_t blocks = (threads + 255) / 256;
+    const int64_t cap = int64_t(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    quant_act_1x128_kernel<<<unsigned(blocks), 256, 0, as_stream(stream)>>>(
+        reinterpret_cast<const uint4*>(x), rows, cols, reinterpret_cast<uint2*>(q), scales,
+        scales_kb_major);
+    return check_launch();
+}
+
+extern "C" MOE_API int fp8_quant_w_128x128(const uint16_t* w, int64_t rows, int64_t cols,
+                                           uint8_t* q, float* scales, int* dev_status,
+                                           void* stream) {
+    (void)dev_status;
+    if (rows < 0 || cols < 0 || rows % 128 || cols % 128) return MOE_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!w || !q || !scales) return MOE_ERR_NULL;
+    if (!aligned16(w) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
+        return MOE_ERR_ALIGN;
+    const int64_t n_blocks = (rows / 128) * (cols / 128);
+    int64_t grid = n_blocks;
+    const int64_t cap = int64_t(sm_count()) * 64;
+    if (grid > cap) grid = cap;
+    quant_w_128x128_kernel<<<unsigned(grid), 256, 0, as_stream(stream)>>>(
+        reinterpret_cast<const uint4*>(w), rows, cols, reinterpret_cast<uint4*>(q), scales);
+    return check_launch();
+}

@@ -1,0 +1,284 @@
+/*
+ * moefp8 — DeepSeekMoE layer forward with FP8 block scaling, for NVIDIA B200
+ * (sm_100a).  Plain C ABI: raw pointers, sizes and a CUDA stream handle.
+ *
+ * The method is the MoE layer of "DeepSeek-V3 Technical Report" (notes page):
+ *   - section "DeepSeekMoE and auxiliary-loss-free load balancing": sigmoid
+ *     token-to-expert affinity, a per-expert bias b_i added for the routing
+ *     decision only, gates from the normalised selected (unbiased)
+ *     affinities, 1 shared + N_r routed experts, K routed experts per token,
+ *     tokens limited to M nodes (expert groups here), batch-wise expert load
+ *     monitoring with b_i -/+ gamma, no token dropping;
+ *   - section "FP8 mixed precision training": every GEMM input in E4M3 with
+ *     fine-grained scales (1x128 activation tiles, 128x128 weight blocks)
+ *     computed online from the current max |value|; FP32 accumulation;
+ *     gating kept in high precision;
+ *   - section "DualPipe": the dispatch / MLP / combine stages of a MoE
+ *     block, here on one GPU (dispatch = an expert-contiguous permutation,
+ *     combine = the gate-weighted sum).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers to caller-owned memory unless a name
+ *     ends in _host.  The library allocates no device memory; scratch space
+ *     comes from the caller (ws / ws_bytes).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL =
+ *     the legacy default stream).  No call synchronises the host, except
+ *     moe_read_status().
+ *   - The return value is a status: MOE_OK (0) or a negative MOE_ERR_*.
+ *     Argument errors are detected on the host before anything is enqueued;
+ *     MOE_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *   - dev_status (nullable) is a device int the kernels set to a positive
+ *     MOE_DEV_* code when they detect a problem at run time (a bounded wait
+ *     that ran out, an index or offset out of range).  The first code
+ *     written wins; the caller zeroes it.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  E4M3 codes are
+ *     uint8_t (OCP E4M3FN: bias 7, max 448, no infinities).
+ *   - Scale rule (online quantisation): per group of values, amax = max|v|,
+ *     scale = fp32(amax / 448), code = E4M3(fp32(v * fp32(448 / amax))),
+ *     round-to-nearest-even, saturating to +-448; amax = 0 gives scale 1.
+ *     A group whose amax is below 448 / FLT_MAX (about 1.3e-36) is outside
+ *     the supported range.
+ *   - Thread safety: the library keeps no state between calls; concurrent
+ *     calls on different buffers are independent.
+ */
+#ifndef MOEFP8_H
+#define MOEFP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_API __attribute__((visibility("default")))
+
+/* host-side status codes */
+#define MOE_OK 0
+#define MOE_ERR_NULL -1        /* a required pointer is NULL */
+#define MOE_ERR_SHAPE -2       /* a size is not a supported multiple / range */
+#define MOE_ERR_ROUTE -3       /* routing shape inconsistent (N_r % G, M*n_g < K, ...) */
+#define MOE_ERR_CUDA -4        /* a CUDA launch or runtime call failed */
+#define MOE_ERR_ALIGN -5       /* a pointer is not 16-byte aligned */
+#define MOE_ERR_WORKSPACE -6   /* ws is NULL or smaller than required */
+#define MOE_ERR_ARG -7         /* another invalid argument (epilogue, flags) */
+#define MOE_ERR_DEVICE -8      /* the current device is not sm_100 */
+
+/* device status codes (written to *dev_status by kernels) */
+#define MOE_DEV_TIMEOUT 1      /* a bounded wait inside a kernel ran out */
+#define MOE_DEV_BAD_INPUT 2    /* an index or offset array was out of range; the
+                                  offending entries were skipped */
+
+/* epilogues of moe_grouped_gemm_fp8 */
+#define MOE_EPI_F32 0           /* out: float [max_rows, n] */
+#define MOE_EPI_BF16 1          /* out: bf16  [max_rows, n] */
+#define MOE_EPI_SWIGLU_QUANT 2  /* out: E4M3 h [max_rows, n/2] + fp32 scales */
+
+/* Shape of one MoE layer.
+ *   T           tokens in the batch (>= 0)
+ *   d           hidden size (multiple of 128)
+ *   n_routed    routed experts N_r (1..1024)
+ *   n_groups    expert groups G (N_r % G == 0, G <= 32); group j holds
+ *               experts [j*N_r/G, (j+1)*N_r/G)
+ *   topk_groups M, groups a token may use (1..G)
+ *   topk        K, routed experts per token (1..32, K <= M*N_r/G)
+ *   inter       expert intermediate size I (multiple of 128)
+ *   gamma       bias update step
+ * The shared expert is expert index N_r in every per-expert array. */
+typedef struct {
+    int T, d, n_routed, n_groups, topk_groups, topk, inter;
+    float gamma;
+} MoeShape;
+
+/* Library version (major*10000 + minor*100 + patch). */
+MOE_API int moe_version(void);
+
+/* Human-readable text of a status code (static string). */
+MOE_API const char* moe_status_string(int status);
+
+/* Copy *dev_status to *host_status after synchronising `stream`.  The only
+ * call that blocks the host. */
+MOE_API int moe_read_status(const int* dev_status, int* host_status, void* stream);
+
+/* ---------------------------------------------------------------- routing
+ * moe_route: router logits, sigmoid affinity, bias, group-limited top-K,
+ * normalised gates and the load histogram ("DeepSeekMoE and
+ * auxiliary-loss-free load balancing"; gating in high precision per "FP8
+ * mixed precision training").
+ *   x            bf16 [T, d] row-major
+ *   router_w     bf16 [N_r, d] row-major (one centroid per routed expert)
+ *   bias         fp32 [N_r], read only
+ *   logit_offset fp32 [N_r] or NULL: a fixed prior added to every token's
+ *                logits (used to build skewed workloads; NULL = none)
+ *   topk_idx     int32 [T, K] out: chosen experts, by descending biased score
+ *   topk_gate    fp32 [T, K] out: gates, sum to 1 per token
+ *   expert_counts int32 [N_r] out: tokens per expert (zeroed by the call)
+ *   ws, ws_bytes scratch of at least moe_route_workspace_size(shape) bytes
+ * Definition (bit-exact contract):
+ *   u  = fp32(sum_k x[t,k]*E[i,k]) with the sum taken in FP64 in ascending k,
+ *        then u = fp32(u + logit_offset[i]) when an offset is given;
+ *   s  = fp32(1/(1+exp(-u))) evaluated in FP64;  s' = fp32(s + b_i);
+ *   group score = max s' in the group; the M best groups are kept (ties to
+ *   the lower group); the K best s' inside them are chosen (ties to the lower
+ *   expert); gate_k = fp32(s_k / S) with S the FP64 sum of the chosen s in
+ *   slot order.
+ * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE (d % 128, T < 0, N_r range),
+ * MOE_ERR_ROUTE, MOE_ERR_ALIGN (x, router_w not 16-byte aligned),
+ * MOE_ERR_WORKSPACE, MOE_ERR_CUDA. */
+MOE_API size_t moe_route_workspace_size(const MoeShape* shape);
+MOE_API int moe_route(const MoeShape* shape, const uint16_t* x, const uint16_t* router_w,
+                      const float* bias, const float* logit_offset, int32_t* topk_idx,
+                      float* topk_gate, int32_t* expert_counts, void* ws, size_t ws_bytes,
+                      int* dev_status, void* stream);
+
+/* ----------------------------------------------------------- quantisation
+ * fp8_quant_act_1x128: online 1x128 tile quantisation of activations
+ * ("FP8 mixed precision training", fine-grained quantisation).
+ *   x       bf16 [rows, cols] row-major, cols % 128 == 0, 16-byte aligned
+ *   q       uint8 [rows, cols] out, E4M3 codes
+ *   scales  fp32 out: scales_kb_major == 0 -> [rows, cols/128];
+ *           scales_kb_major == 1 -> [cols/128, rows] (the layout the
+ *           grouped GEMM reads)
+ * Bit-exact contract: the scale rule in the header comment. */
+MOE_API int fp8_quant_act_1x128(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q,
+                                float* scales, int scales_kb_major, int* dev_status,
+                                void* stream);
+
+/* fp8_quant_w_128x128: online 128x128 block quantisation of weights
+ * ("FP8 mixed precision training", block-wise 128x128 for weights).
+ *   w       bf16 [rows, cols] row-major, rows % 128 == 0, cols % 128 == 0
+ *   q       uint8 [rows, cols] out
+ *   scales  fp32 [rows/128, cols/128] out
+ * Stacked expert matrices ([E*rows_e, cols]) may be passed in one call when
+ * rows_e % 128 == 0: blocks never straddle experts. */
+MOE_API int fp8_quant_w_128x128(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,
+                                float* scales, int* dev_status, void* stream);
+
+/* ------------------------------------------------------------ permutation
+ * moe_permute: the single-GPU "dispatch": copies every token's FP8 row once
+ * per chosen expert plus once for the shared expert into an
+ * expert-contiguous buffer ("DualPipe": all-to-all dispatch of FP8
+ * activations, "FP8 mixed precision training": low-precision communication).
+ *   topk_idx, expert_counts   as produced by moe_route
+ *   xq, xs                    codes [T, d] and row-major scales [T, d/128]
+ *   xq_perm                   uint8 [T*K + T, d] out
+ *   xs_perm                   fp32 [d/128, T*K + T] out (kb-major)
+ *   expert_offsets            int32 [N_r + 2] out: expert e owns rows
+ *                             [off[e], off[e+1]); off[N_r] = T*K and the
+ *                             shared expert owns [T*K, T*K + T) in token order
+ *   row_of_pair               int32 [T, K] out: row of (token t, slot k);
+ *                             inside an expert, tokens keep ascending order
+ *   ws, ws_bytes              scratch of moe_permute_workspace_size(shape)
+ * Bit-exact contract: offsets, row_of_pair and the copied bytes/scales. */
+MOE_API size_t moe_permute_workspace_size(const MoeShape* shape);
+MOE_API int moe_permute(const MoeShape* shape, const int32_t* topk_idx,
+                        const int32_t* expert_counts, const uint8_t* xq, const float* xs,
+                        uint8_t* xq_perm, float* xs_perm, int32_t* expert_offsets,
+                        int32_t* row_of_pair, void* ws, size_t ws_bytes, int* dev_status,
+                        void* stream);
+
+/* ------------------------------------------------------------ expert GEMM
+ * moe_grouped_gemm_fp8: per group g, rows [off[g], off[g+1]) of A times the
+ * group's weight matrix, FP8 E4M3 operands with block scales applied on the
+ * FP32 accumulator once per 128-element K block ("FP8 mixed precision
+ * training": fine-grained scales, increased accumulation precision).
+ *   n_groups       number of groups (>= 1); group_offsets int32 [n_groups+1]
+ *                  on the device, non-decreasing, off[n_groups] <= max_rows
+ *   max_rows       rows allocated in a, a_scales and out
+ *   a              uint8 [max_rows, k] E4M3 codes (16-byte aligned)
+ *   a_scales       fp32 [k/128, max_rows] (kb-major 1x128 scales)
+ *   k              contraction size, multiple of 128
+ *   w              uint8 [n_groups, n, k] E4M3 codes, K-major (row j of
+ *                  group g is output feature j)
+ *   w_scales       fp32 [n_groups, n/128, k/128]
+ *   n              output features, multiple of 128 (of 256 for SwiGLU)
+ *   epilogue:
+ *     MOE_EPI_F32          out = float [max_rows, n]
+ *     MOE_EPI_BF16         out = bf16  [max_rows, n] (round to nearest even)
+ *     MOE_EPI_SWIGLU_QUANT rows [0, n/2) of each weight matrix are the gate
+ *                          projection W1 and rows [n/2, n) the up projection
+ *                          W3; h = silu(gate) * up in fp32 is quantised 1x128
+ *                          along its n/2 features: out = uint8 [max_rows, n/2],
+ *                          out_scales = fp32 [n/2/128, max_rows] (kb-major)
+ * Rows of A outside every group are neither read into results nor written.
+ * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE, MOE_ERR_ARG, MOE_ERR_ALIGN,
+ * MOE_ERR_DEVICE, MOE_ERR_CUDA; MOE_DEV_TIMEOUT on dev_status. */
+MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int max_rows,
+                                 const uint8_t* a, const float* a_scales, int k,
+                                 const uint8_t* w, const float* w_scales, int n, int epilogue,
+                                 void* out, float* out_scales, int* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- combine
+ * moe_combine: y[t] = o[shared row of t] + sum_k gate[t,k] * o[row_of_pair
+ * [t,k]], accumulated in fp32 in slot order, rounded once to bf16
+ * ("DualPipe": all-to-all combine, here a local gather).
+ *   expert_out  fp32 [T*K + T, d] (moe_grouped_gemm_fp8 with MOE_EPI_F32)
+ *   y           bf16 [T, d] out */
+MOE_API int moe_combine(const MoeShape* shape, const float* expert_out,
+                        const int32_t* expert_offsets, const int32_t* row_of_pair,
+                        const float* topk_gate, uint16_t* y, int* dev_status, void* stream);
+
+/* ------------------------------------------------------------ bias update
+ * moe_update_bias: b_i = fp32(b_i - gamma) when count_i * N_r > T*K
+ * (overloaded), fp32(b_i + gamma) when count_i * N_r < T*K (underloaded),
+ * unchanged when equal ("DeepSeekMoE and auxiliary-loss-free load
+ * balancing").  bias fp32 [N_r] is updated in place. */
+MOE_API int moe_update_bias(const MoeShape* shape, const int32_t* expert_counts, float* bias,
+                            int* dev_status, void* stream);
+
+/* ------------------------------------------------------------ whole layer
+ * Expert weights, pre-quantised with fp8_quant_w_128x128:
+ *   w13        uint8 [N_r+1, 2I, d]: rows [0,I) = W1 (gate), [I,2I) = W3 (up)
+ *   w13_scales fp32  [N_r+1, 2I/128, d/128]
+ *   w2         uint8 [N_r+1, d, I]  (down projection, K-major)
+ *   w2_scales  fp32  [N_r+1, d/128, I/128]
+ *   router_w   bf16  [N_r, d]
+ * Expert N_r is the shared expert. */
+typedef struct {
+    const uint8_t* w13;
+    const float* w13_scales;
+    const uint8_t* w2;
+    const float* w2_scales;
+    const uint16_t* router_w;
+} MoeWeights;
+
+/* Routing results of one layer call (caller-owned device buffers). */
+typedef struct {
+    int32_t* topk_idx;        /* [T, K] */
+    float* topk_gate;         /* [T, K] */
+    int32_t* expert_counts;   /* [N_r] */
+    int32_t* expert_offsets;  /* [N_r + 2] */
+    int32_t* row_of_pair;     /* [T, K] */
+} MoeRouting;
+
+/* moe_layer_forward: route -> quantise x (1x128) -> permute -> grouped GEMM
+ * (W13, SwiGLU + 1x128 quantisation of h) -> grouped GEMM (W2, fp32) ->
+ * combine -> (optionally) bias update, all on `stream`.
+ *   x            bf16 [T, d];  y bf16 [T, d] out
+ *   bias         fp32 [N_r]; updated in place after routing when
+ *                update_bias != 0 (the next call routes with the new bias)
+ *   logit_offset fp32 [N_r] or NULL (see moe_route)
+ *   ws, ws_bytes scratch of moe_layer_workspace_size(shape) bytes */
+MOE_API size_t moe_layer_workspace_size(const MoeShape* shape);
+MOE_API int moe_layer_forward(const MoeShape* shape, const MoeWeights* weights,
+                              const uint16_t* x, float* bias, const float* logit_offset,
+                              MoeRouting* routing, uint16_t* y, int update_bias, void* ws,
+                              size_t ws_bytes, int* dev_status, void* stream);
+
+/* moe_layer_forward_host: the same layer with x and y in HOST memory (pinned
+ * memory makes the copies asynchronous).  x_host is copied into the
+ * workspace, y is copied back to y_host, both on `stream`; the caller
+ * synchronises `stream` before reading y_host.
+ *   ws, ws_bytes scratch of moe_layer_host_workspace_size(shape) bytes */
+MOE_API size_t moe_layer_host_workspace_size(const MoeShape* shape);
+MOE_API int moe_layer_forward_host(const MoeShape* shape, const MoeWeights* weights,
+                                   const uint16_t* x_host, float* bias,
+                                   const float* logit_offset, MoeRouting* routing,
+                                   uint16_t* y_host, int update_bias, void* ws,
+                                   size_t ws_bytes, int* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEFP8_H */

@@ -113,14 +113,16 @@ def _table():
 
 def dequant_act(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """code value * tile scale, in FP64 (exact)."""
-    v = _table()[q]
-    return v * np.repeat(s.astype(np.float64), 128, axis=1)
+    rows, cols = q.shape
+    v = _table()[q].reshape(rows, cols // 128, 128)
+    return (v * s.astype(np.float64)[:, :, None]).reshape(rows, cols)
 
 
 def dequant_w(q: np.ndarray, s: np.ndarray) -> np.ndarray:
-    v = _table()[q]
-    s64 = np.repeat(np.repeat(s.astype(np.float64), 128, axis=0), 128, axis=1)
-    return v * s64
+    """code value * block scale, in FP64 (exact)."""
+    rows, cols = q.shape
+    v = _table()[q].reshape(rows // 128, 128, cols // 128, 128)
+    return (v * s.astype(np.float64)[:, None, :, None]).reshape(rows, cols)
 
 
 # ----------------------------------------------------------------- routing

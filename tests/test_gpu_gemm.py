@@ -1,0 +1,185 @@
+"""GPU parity of the tcgen05 grouped FP8 GEMM against the oracle's FP64
+matmul over dequantised values ("DeepSeek-V3 Technical Report" notes page,
+section "FP8 mixed precision training": FP8 GEMM inputs with 1x128 / 128x128
+scales, FP32 accumulation promoted every 128 elements of K).
+
+Tolerances: with FP32 accumulation of FP8 products and per-block promotion,
+the relative error of an output is a few fp32 rounding steps (about 1e-6);
+1e-5 relative Frobenius is used for fp32 outputs.  bf16 outputs are compared
+after both sides round to bf16 (2e-3, the layer's output bound)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+from gpu_util import DEV, bf16_dev, need_gpu, rel_frobenius, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _quant_gpu(xbits):
+    import fp8_block_scaled_affinity_b200 as moe
+    rows, cols = xbits.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=DEV)
+    s = torch.empty((cols // 128, rows), dtype=torch.float32, device=DEV)
+    moe.fp8_quant_act_1x128(bf16_dev(xbits), q, s, True)
+    return q, s
+
+
+def _quant_w_gpu(wbits):
+    import fp8_block_scaled_affinity_b200 as moe
+    rows, cols = wbits.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=DEV)
+    s = torch.empty((rows // 128, cols // 128), dtype=torch.float32, device=DEV)
+    moe.fp8_quant_w_128x128(bf16_dev(wbits), q, s)
+    return q, s
+
+
+def run_grouped(sizes, k, n, epilogue, seed, pad_rows=0, outliers=False):
+    """Random A rows split into groups of `sizes`, one weight matrix per group.
+    Returns (gpu_out, oracle_results_per_group, offsets, extras)."""
+    import fp8_block_scaled_affinity_b200 as moe
+    rng = np.random.default_rng(seed)
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R = int(off[-1]) + pad_rows
+    va = rng.standard_normal((R, k)).astype(np.float32)
+    if outliers:
+        va *= np.where(rng.random((R, k)) < 0.001, 100.0, 1.0).astype(np.float32)
+    a = S.f32_to_bf16_bits(va)
+    w = S.host_normal_bf16(rng, (G * n, k), 0.05)
+    aq, as_ = _quant_gpu(a)
+    wq, ws = _quant_w_gpu(w)
+    if epilogue == moe.MOE_EPI_SWIGLU_QUANT:
+        out = torch.full((R, n // 2), 0xEE, dtype=torch.uint8, device=DEV)
+        out_s = torch.full((n // 2 // 128, R), -1.0, dtype=torch.float32, device=DEV)
+    elif epilogue == moe.MOE_EPI_F32:
+        out = torch.full((R, n), float("nan"), dtype=torch.float32, device=DEV)
+        out_s = None
+    else:
+        out = torch.full((R, n), float("nan"), dtype=torch.bfloat16, device=DEV)
+        out_s = None
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_grouped_gemm_fp8(G, to_dev(off), R, aq, as_, k, wq, ws, n, epilogue, out, out_s,
+                             status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    # oracle, from the same bf16 inputs
+    qa_o, sa_o = oracle.quant_act_1x128(a)
+    res = []
+    for g in range(G):
+        r0, r1 = off[g], off[g + 1]
+        wg = w[g * n:(g + 1) * n]
+        if epilogue == moe.MOE_EPI_SWIGLU_QUANT:
+            I = n // 2
+            w1q, w1s = oracle.quant_w_128x128(wg[:I])
+            w3q, w3s = oracle.quant_w_128x128(wg[I:])
+            X = oracle.dequant_act(qa_o[r0:r1], sa_o[r0:r1])
+            ga = X @ oracle.dequant_w(w1q, w1s).T
+            up = X @ oracle.dequant_w(w3q, w3s).T
+            h32 = ((ga / (1.0 + np.exp(-ga))) * up).astype(np.float32)
+            res.append((h32,) + oracle.quant_act_1x128(h32) if r1 > r0 else None)
+        else:
+            wq_o, ws_o = oracle.quant_w_128x128(wg)
+            res.append(oracle.gemm_blockscaled(qa_o[r0:r1], sa_o[r0:r1], wq_o, ws_o))
+    return out, out_s, res, off
+
+
+def _check_dense(out, res, off, epilogue):
+    import fp8_block_scaled_affinity_b200 as moe
+    if epilogue == moe.MOE_EPI_F32:
+        got = out.cpu().numpy()
+    else:
+        got = S.bf16_bits_to_f32(out.cpu().view(torch.int16).numpy().view(np.uint16))
+    for g, ref in enumerate(res):
+        r0, r1 = off[g], off[g + 1]
+        if r1 == r0:
+            continue
+        if epilogue == moe.MOE_EPI_F32:
+            assert rel_frobenius(got[r0:r1], ref) <= 1e-5, g
+        else:
+            refb = S.bf16_bits_to_f32(oracle.f64_to_bf16_bits(ref))
+            assert rel_frobenius(got[r0:r1], refb) <= 2e-3, g
+    # rows outside every group stay untouched
+    if got.shape[0] > off[-1]:
+        assert np.all(np.isnan(got[off[-1]:]))
+
+
+@pytest.mark.parametrize("sizes,k,n", [([1], 128, 128), ([300], 512, 256), ([256], 256, 128),
+                                       ([257, 0, 5, 16, 17], 384, 256),
+                                       ([40] * 9 + [600], 1024, 384)])
+def test_grouped_fp32_output(sizes, k, n):
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    out, _, res, off = run_grouped(sizes, k, n, moe.MOE_EPI_F32, seed=sum(sizes) + k, pad_rows=3)
+    _check_dense(out, res, off, moe.MOE_EPI_F32)
+
+
+def test_bf16_output_with_outliers():
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    out, _, res, off = run_grouped([333], 1024, 512, moe.MOE_EPI_BF16, seed=5, outliers=True)
+    _check_dense(out, res, off, moe.MOE_EPI_BF16)
+
+
+@pytest.mark.parametrize("sizes,k,I", [([1], 128, 128), ([130, 0, 7], 256, 256),
+                                       ([128, 129, 64], 512, 128)])
+def test_swiglu_quant_epilogue(sizes, k, I):
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    out, out_s, res, off = run_grouped(sizes, k, 2 * I, moe.MOE_EPI_SWIGLU_QUANT,
+                                       seed=len(sizes) * 7 + k)
+    q = out.cpu().numpy()
+    s = out_s.cpu().numpy().T  # -> [rows, I/128]
+    table = oracle.e4m3_decode_table()
+    for g, ref in enumerate(res):
+        r0, r1 = off[g], off[g + 1]
+        if ref is None:
+            continue
+        h32, hq_ref, hs_ref = ref
+        # scales: amax of h over 128 features; fp32 accumulation order only
+        assert np.allclose(s[r0:r1], hs_ref, rtol=1e-5, atol=0)
+        # codes: equal except rare one-step flips at rounding boundaries
+        same = q[r0:r1] == hq_ref
+        assert same.mean() > 0.999
+        dq = table[q[r0:r1]] * np.repeat(s[r0:r1], 128, axis=1)
+        assert rel_frobenius(dq, h32) <= 5e-2  # E4M3 itself: about 2.4% RMS
+        dq_ref = table[hq_ref] * np.repeat(hs_ref, 128, axis=1)
+        assert rel_frobenius(dq, dq_ref) <= 2e-3
+
+
+def test_full_size_gemm_workload():
+    """A 4096x7168 (1x128 scales, 0.1% x100 outliers) times B 7168x2048
+    (128x128 scales), bf16 out: the GEMM-alone workload."""
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    cfg = S.GEMM_C2
+    a, b = S.make_gemm_inputs_host(cfg)
+    aq, as_ = _quant_gpu(a)
+    bq, bs = _quant_w_gpu(b)
+    off = to_dev(np.array([0, cfg.m], np.int32))
+    out = torch.empty((cfg.m, cfg.n), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_gemm_fp8(1, off, cfg.m, aq, as_, cfg.k, bq, bs, cfg.n, moe.MOE_EPI_BF16, out)
+    torch.cuda.synchronize()
+    got = S.bf16_bits_to_f32(out.cpu().view(torch.int16).numpy().view(np.uint16))
+    qa, sa = oracle.quant_act_1x128(a)
+    qb, sb = oracle.quant_w_128x128(b)
+    # the same quantised operands on both sides
+    assert np.array_equal(aq.cpu().numpy(), qa) and np.array_equal(bq.cpu().numpy(), qb)
+    ref = S.bf16_bits_to_f32(oracle.f64_to_bf16_bits(oracle.gemm_blockscaled(qa, sa, qb, sb)))
+    assert rel_frobenius(got, ref) <= 2e-3
+    assert np.mean(got == ref) > 0.99
+
+
+def test_gemm_rejects_bad_arguments():
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    z = torch.zeros(1024, dtype=torch.uint8, device=DEV)
+    off = to_dev(np.array([0, 1], np.int32))
+    for args, code in [((1, off, 1, z, z, 100, z, z, 128, 0, z), -2),
+                       ((1, off, 1, z, z, 128, z, z, 128, 9, z), -7),
+                       ((1, off, 1, z, z, 128, z, z, 128, 2, z, None), -1)]:
+        with pytest.raises(moe.MoeError) as e:
+            moe.moe_grouped_gemm_fp8(*args)
+        assert e.value.status == code

@@ -1,0 +1,149 @@
+"""GPU parity of routing, load histogram and bias update against the oracle,
+bit for bit ("DeepSeek-V3 Technical Report" notes page, section "DeepSeekMoE
+and auxiliary-loss-free load balancing")."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+from conftest import read_golden
+from gpu_util import DEV, bf16_dev, need_gpu, shape_of, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_route(shape, xbits, Ebits, bias, offset=None):
+    import fp8_block_scaled_affinity_b200 as moe
+    T, K, N = shape.T, shape.topk, shape.n_routed
+    idx = torch.full((max(T, 1), K), -1, dtype=torch.int32, device=DEV)
+    gate = torch.full((max(T, 1), K), -1.0, dtype=torch.float32, device=DEV)
+    counts = torch.full((N,), 77, dtype=torch.int32, device=DEV)
+    ws = torch.empty((max(moe.moe_route_workspace_size(shape), 1),), dtype=torch.uint8, device=DEV)
+    moe.moe_route(shape, bf16_dev(xbits) if T else None, bf16_dev(Ebits), to_dev(bias),
+                  None if offset is None else to_dev(offset), idx, gate, counts, ws)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy()[:T], gate.cpu().numpy()[:T], counts.cpu().numpy()
+
+
+def _compare(cfg, inp, T=None, offset=None):
+    T = cfg.T if T is None else T
+    shape = shape_of(cfg, T)
+    x = inp["x"][:T]
+    idx, gate, counts = gpu_route(shape, x, inp["router_w"], inp["bias"], offset)
+    ref = oracle.route(x, inp["router_w"], inp["bias"], cfg.n_groups, cfg.topk_groups,
+                       cfg.topk, logit_offset=offset)
+    assert np.array_equal(idx, ref["topk_idx"])
+    assert np.array_equal(gate.view(np.uint32), ref["topk_gate"].view(np.uint32))
+    assert np.array_equal(counts, ref["counts"])
+    return ref
+
+
+def test_hand_worked_example():
+    need_gpu()
+    g = {}
+    for r in read_golden("route_hand.txt"):
+        g.setdefault(r[0], []).append([float(v) for v in r[1:]])
+    x = np.zeros((2, 128), np.float32)
+    x[0, 0], x[1, 0] = 1.0, -1.0
+    E = np.zeros((8, 128), np.float32)
+    E[:, 0] = g["u"][0]
+    import fp8_block_scaled_affinity_b200 as moe
+    shape = moe.make_shape(2, 128, 8, 4, 2, 3, 128, 0.001)
+    idx, gate, counts = gpu_route(shape, S.f32_to_bf16_bits(x), S.f32_to_bf16_bits(E),
+                                  np.array(g["bias"][0], np.float32))
+    assert idx.tolist() == [[int(v) for v in row] for row in g["topk_idx"]]
+    assert counts.tolist() == [int(v) for v in g["counts"][0]]
+
+
+def test_ties_go_to_lower_index():
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    x = np.zeros((3, 128), np.float32)
+    x[:, 0] = 1.0
+    E = np.zeros((8, 128), np.float32)
+    E[:, 0] = 0.75
+    shape = moe.make_shape(3, 128, 8, 4, 2, 3, 128)
+    idx, _, _ = gpu_route(shape, S.f32_to_bf16_bits(x), S.f32_to_bf16_bits(E),
+                          np.zeros(8, np.float32))
+    assert idx.tolist() == [[0, 1, 2]] * 3
+
+
+@pytest.mark.parametrize("T", [1, 37, 256])
+def test_tiny_workload(T):
+    need_gpu()
+    cfg = S.CONFIGS["tiny"]
+    _compare(cfg, S.make_layer_inputs_host(cfg), T=T)
+
+
+@pytest.mark.parametrize("n_routed,n_groups,M,K", [(64, 8, 3, 6), (96, 32, 7, 12),
+                                                   (1024, 16, 4, 32), (48, 1, 1, 5)])
+def test_other_routing_shapes(n_routed, n_groups, M, K):
+    need_gpu()
+    rng = np.random.default_rng(n_routed + K)
+    T, d = 150, 384
+    inp = {"x": S.host_normal_bf16(rng, (T, d), 1.0),
+           "router_w": S.host_normal_bf16(rng, (n_routed, d), 0.05),
+           "bias": S.host_uniform_f32(rng, (n_routed,), 0.02)}
+    cfg = S.MoeConfig("t", T, d, n_routed, n_groups, M, K, 128, 0.05, 0.02, 0.001, 0)
+    _compare(cfg, inp)
+
+
+def test_decode_workload_full():
+    need_gpu()
+    cfg = S.CONFIGS["decode"]
+    _compare(cfg, S.make_layer_inputs_host(cfg))
+
+
+def test_prefill_workload_full():
+    need_gpu()
+    cfg = S.CONFIGS["prefill"]
+    _compare(cfg, S.make_layer_inputs_host(cfg))
+
+
+def test_skewed_workload_eight_batches_with_bias_updates():
+    """Eight successive batches of 16384 tokens with a Zipf(1.2) logit prior;
+    after each batch the bias moves by gamma.  Routing, counts and the bias
+    trajectory must match the oracle's own trajectory bit for bit."""
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    cfg = S.CONFIGS["skewed"]
+    shape = shape_of(cfg)
+    base = S.make_layer_inputs_host(cfg, 0)
+    off = base["logit_offset"]
+    b_gpu = to_dev(base["bias"])
+    b_ref = base["bias"].copy()
+    E = base["router_w"]
+    loads = []
+    for j in range(cfg.batches):
+        x = S.make_layer_inputs_host(cfg, j)["x"]
+        idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device=DEV)
+        gate = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device=DEV)
+        counts = torch.empty((cfg.n_routed,), dtype=torch.int32, device=DEV)
+        ws = torch.empty((moe.moe_route_workspace_size(shape),), dtype=torch.uint8, device=DEV)
+        moe.moe_route(shape, bf16_dev(x), bf16_dev(E), b_gpu, to_dev(off), idx, gate, counts, ws)
+        moe.moe_update_bias(shape, counts, b_gpu)
+        torch.cuda.synchronize()
+        ref = oracle.route(x, E, b_ref, cfg.n_groups, cfg.topk_groups, cfg.topk, logit_offset=off)
+        assert np.array_equal(idx.cpu().numpy(), ref["topk_idx"]), j
+        assert np.array_equal(gate.cpu().numpy().view(np.uint32),
+                              ref["topk_gate"].view(np.uint32)), j
+        assert np.array_equal(counts.cpu().numpy(), ref["counts"]), j
+        b_ref = oracle.update_bias(ref["counts"], b_ref, cfg.T, cfg.topk, cfg.gamma)
+        assert np.array_equal(b_gpu.cpu().numpy().view(np.uint32), b_ref.view(np.uint32)), j
+        c = ref["counts"]
+        loads.append(c.max() / c.mean())
+    assert loads[0] > 3.0  # the prior really skews the load
+
+
+def test_empty_batch_zeroes_counts():
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    cfg = S.CONFIGS["tiny"]
+    inp = S.make_layer_inputs_host(cfg)
+    shape = shape_of(cfg, 0)
+    _, _, counts = gpu_route(shape, inp["x"][:0], inp["router_w"], inp["bias"])
+    assert np.all(counts == 0)
+    bad = moe.make_shape(4, 128, 10, 3, 1, 2, 128)  # N_r % G != 0
+    with pytest.raises(moe.MoeError):
+        gpu_route(bad, inp["x"][:4, :128], inp["router_w"][:10, :128], inp["bias"][:10])
