@@ -179,7 +179,8 @@ def test_gemm_rejects_bad_arguments():
     off = to_dev(np.array([0, 1], np.int32))
     for args, code in [((1, off, 1, z, z, 100, z, z, 128, 0, z), -2),
                        ((1, off, 1, z, z, 128, z, z, 128, 9, z), -7),
-                       ((1, off, 1, z, z, 128, z, z, 128, 2, z, None), -1)]:
+                       ((1, off, 1, z, z, 128, z, z, 256, 2, z, None), -1),  # no out_scales
+                       ((1, off, 1, z, z, 128, z, z, 128, 2, z, z), -2)]:    # n % 256
         with pytest.raises(moe.MoeError) as e:
             moe.moe_grouped_gemm_fp8(*args)
         assert e.value.status == code
