@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "fp8_quant_w_128x128": (I, [P, I64, I64, P, P, P, P]),
             "moe_permute_workspace_size": (SZ, [SP]),
             "moe_permute": (I, [SP, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "moe_permute_static_ws": (I, [SP, P, P, P, P, P, P, P, P, P, P]),
             "moe_grouped_gemm_fp8": (I, [I, P, I, P, P, I, P, P, I, I, P, P, P, P]),
             "moe_combine": (I, [SP, P, P, P, P, P, P, P]),
             "moe_update_bias": (I, [SP, P, P, P, P]),
@@ -165,6 +166,18 @@ def moe_permute(shape, topk_idx, expert_counts, xq, xs, xq_perm, xs_perm, expert
     _check("moe_permute", lib().moe_permute(
         ctypes.byref(shape), _ptr(topk_idx), _ptr(expert_counts), _ptr(xq), _ptr(xs),
         _ptr(xq_perm), _ptr(xs_perm), _ptr(expert_offsets), _ptr(row_of_pair), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_permute_static_ws(shape, topk_idx, expert_counts, xq, xs, xq_perm, xs_perm,
+                          expert_offsets, row_of_pair, dev_status=None, stream=None):
+    """moe_permute for callers that cannot allocate device memory while they
+    run: no workspace argument; the library's own fixed 1 MiB device array
+    is used instead (ceil(T/64) * N_r <= 262144).  Calls that overlap on the
+    GPU share that array and race."""
+    _check("moe_permute_static_ws", lib().moe_permute_static_ws(
+        ctypes.byref(shape), _ptr(topk_idx), _ptr(expert_counts), _ptr(xq), _ptr(xs),
+        _ptr(xq_perm), _ptr(xs_perm), _ptr(expert_offsets), _ptr(row_of_pair),
         _ptr(dev_status), _stream(stream)))
 
 

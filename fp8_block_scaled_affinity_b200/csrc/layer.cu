@@ -131,6 +131,8 @@ extern "C" MOE_API const char* moe_status_string(int status) {
         case MOE_ERR_WORKSPACE: return "workspace missing or too small";
         case MOE_ERR_ARG: return "invalid argument";
         case MOE_ERR_DEVICE: return "device is not sm_100 (B200)";
+        case MOE_ERR_STATIC_LIMIT:
+            return "shape exceeds the fixed scratch of the no-allocation entry point";
         default: return "unknown status";
     }
 }

@@ -14,6 +14,8 @@
 //      out rows (tokens stay in ascending order inside every expert);
 //   4. copy_rows: one warp per token reads its FP8 row once (16-byte loads)
 //      and writes it K+1 times, scales transposed to the kb-major layout.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -308,4 +310,58 @@ extern "C" MOE_API int moe_update_bias(const MoeShape* shape, const int32_t* exp
     update_bias_kernel<<<(N + 255) / 256, 256, 0, as_stream(stream)>>>(
         expert_counts, N, int64_t(shape->T) * shape->topk, shape->gamma, bias);
     return check_launch();
+}
+
+// ------------------------------------------------------------------------
+// moe_permute_static_ws: moe_permute without a caller workspace.
+//
+// Some callers cannot call cudaMalloc once they are running: a serving loop
+// whose device-memory budget is fixed when it starts, or a host framework
+// that owns all device memory through its own pool and forbids allocations
+// behind its back (cudaMalloc may also synchronise the whole device, which
+// latency-bound loops avoid).  This entry point lets them run the
+// permutation without sizing or passing a workspace: the per-chunk counts
+// live in the array below, which every GPU that loads the library keeps
+// until the process exits.
+namespace moe {
+namespace {
+
+constexpr int64_t kStaticChunkEntries = 262144;  // int32 entries = 1 MiB
+// + 64 entries: moe_permute asks for 256 bytes of headroom on top of the counts
+__device__ __align__(256) int32_t g_permute_scratch[kStaticChunkEntries + 64];
+
+// Device address of g_permute_scratch, looked up once per device.  In host
+// code the symbol only names a host-side stand-in, never a device address.
+int32_t* static_scratch_ptr() {
+    static std::mutex mu;
+    static int32_t* ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int32_t*>(p);
+    }
+    return ptrs[dev];
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" MOE_API int moe_permute_static_ws(const MoeShape* shape, const int32_t* topk_idx,
+                                             const int32_t* expert_counts, const uint8_t* xq,
+                                             const float* xs, uint8_t* xq_perm, float* xs_perm,
+                                             int32_t* expert_offsets, int32_t* row_of_pair,
+                                             int* dev_status, void* stream) {
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    if (int64_t(n_chunks_of(shape->T)) * shape->n_routed > kStaticChunkEntries)
+        return MOE_ERR_STATIC_LIMIT;
+    int32_t* scratch = static_scratch_ptr();
+    if (!scratch) return MOE_ERR_CUDA;
+    // The scratch needs no clearing: chunk_hist writes every entry that the
+    // later kernels of this call read.
+    return moe_permute(shape, topk_idx, expert_counts, xq, xs, xq_perm, xs_perm, expert_offsets,
+                       row_of_pair, scratch, sizeof(g_permute_scratch), dev_status, stream);
 }

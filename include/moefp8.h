@@ -63,6 +63,7 @@ extern "C" {
 #define MOE_ERR_WORKSPACE -6   /* ws is NULL or smaller than required */
 #define MOE_ERR_ARG -7         /* another invalid argument (epilogue, flags) */
 #define MOE_ERR_DEVICE -8      /* the current device is not sm_100 */
+#define MOE_ERR_STATIC_LIMIT -9 /* shape too large for moe_permute_static_ws */
 
 /* device status codes (written to *dev_status by kernels) */
 #define MOE_DEV_TIMEOUT 1      /* a bounded wait inside a kernel ran out */
@@ -176,6 +177,29 @@ MOE_API int moe_permute(const MoeShape* shape, const int32_t* topk_idx,
                         uint8_t* xq_perm, float* xs_perm, int32_t* expert_offsets,
                         int32_t* row_of_pair, void* ws, size_t ws_bytes, int* dev_status,
                         void* stream);
+
+/* moe_permute_static_ws: moe_permute for callers that cannot allocate
+ * device memory while they run (a serving loop whose memory budget is fixed
+ * at start-up, a host framework that owns all device memory through its own
+ * pool); it needs no workspace argument.  The pages have no counterpart:
+ * this is a property of the library, not of the method.
+ *   Arguments, layouts and results are those of moe_permute, without ws.
+ *   Scratch: a 1 MiB array of device memory inside the library, held by every
+ *   GPU that loads the library until the process exits.  Limit:
+ *   ceil(T / 64) * N_r <= 262144 (e.g. T <= 65536 with N_r = 256); larger
+ *   shapes return MOE_ERR_STATIC_LIMIT without doing anything.
+ *   The first call on a device looks the array's device address up (once
+ *   per device, with that device current), so make that first call before
+ *   any stream capture.
+ *   All calls share the one array: two calls whose work overlaps on the GPU
+ *   (different streams, or different host threads, on one device) race and
+ *   give wrong results.  Each call overwrites every scratch entry it reads,
+ *   so nothing carries over from the previous call. */
+MOE_API int moe_permute_static_ws(const MoeShape* shape, const int32_t* topk_idx,
+                                  const int32_t* expert_counts, const uint8_t* xq,
+                                  const float* xs, uint8_t* xq_perm, float* xs_perm,
+                                  int32_t* expert_offsets, int32_t* row_of_pair,
+                                  int* dev_status, void* stream);
 
 /* ------------------------------------------------------------ expert GEMM
  * moe_grouped_gemm_fp8: per group g, rows [off[g], off[g+1]) of A times the
