@@ -466,7 +466,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill", choices=["tiny", "prefill", "decode", "skewed"])
+    ap.add_argument("--workload", default="prefill", choices=["tiny", "prefill", "decode", "skewed", "prefill_e16"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -7,23 +7,22 @@
 // into a fresh TMEM buffer, and promotion warps fold it into register FP32
 // accumulators with the block's combined scale sa[token] * sb[weight block].
 //
-// Layout ("swap AB"): the weight tile is the MMA's M side (128 rows = one
-// 128x128 quantisation block row), the tokens are the N side (16..256,
-// rounded up to 16), so small expert groups waste no tensor work and a
-// weight tile is streamed once per token tile.
+// Tile: 128 tokens (the MMA's M side, one token per TMEM lane, so a thread's
+// token scale is one register) x 256 weight columns (N: two 128-row weight
+// blocks, each with one scale per K block) x 128 K.  For the SwiGLU epilogue
+// the two weight blocks are the gate (W1) and up (W3) rows of the same 128
+// features, so a thread holds gate and up of the same (token, feature).
 //
 // Roles (384 threads, one CTA per SM, persistent over work items):
-//   warp 0       TMA producer: weight tiles + token tiles into a 4-stage
-//                smem ring; combined scales into a small smem ring
+//   warp 0       TMA producer: token tile (16 KB) + two weight tiles (32 KB)
+//                per K block into a 4-stage smem ring
 //   warp 1       TMEM owner and MMA issuer (one thread)
-//   warps 2-3    idle (they give their registers to the promoters)
-//   warps 4-11   promotion + epilogue: warp w reads TMEM lanes
-//                32*(w%4)..+31 (weight rows) and one half of the columns
-//
-// Work item = (group g, feature tile f, token tile): NUM_ACC = 2 (SwiGLU)
-// computes gate and up rows of the same 128 features into two accumulators
-// of up to 128 tokens; NUM_ACC = 1 computes 128 output features for up to
-// 256 tokens.  TMEM: 2 partial buffers x 256 columns = all 512 columns.
+//   warp 2       scale loader: cp.async of the K block's 128 token scales and
+//                2 weight-block scales into a small smem ring
+//   warp 3       idle (its registers go to the promoters)
+//   warps 4-11   promotion + epilogue: warp w reads TMEM lanes 32*(w%4)..+31
+//                (its 32 tokens) and one half of the 256 columns
+// TMEM: 2 partial buffers x 256 columns = all 512 columns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <mutex>
@@ -35,10 +34,12 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kStages = 4;
-constexpr int kStageBytes = 48 * 1024;
-constexpr int kCombSlots = 8;
+constexpr int kTileBytes = 128 * 128;            // one 128 x 128 FP8 tile
+constexpr int kStageBytes = 3 * kTileBytes;      // token tile + 2 weight tiles
+constexpr int kScaleSlots = 8;
 constexpr int kMaxGroups = 1040;
-constexpr int kTileBytes = 128 * 128;  // one 128 x 128 FP8 tile
+constexpr int kBM = 128;                         // tokens per tile
+constexpr int kPromoters = 8;                    // promotion warps
 
 struct GemmParams {
     const int32_t* group_offsets;
@@ -49,7 +50,7 @@ struct GemmParams {
     int nkb;
     const float* w_scales;  // [n_groups, n/128, nkb]
     int n;                  // weight rows per group
-    int n_feat;             // feature tiles per group
+    int n_ftiles;           // 256-column tiles per group
     int epilogue;
     void* out;
     float* out_scales;
@@ -61,20 +62,21 @@ struct SharedState {
     uint64_t empty[kStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
-    uint64_t cfull[kCombSlots];
-    uint64_t cempty[kCombSlots];
+    uint64_t sfull[kScaleSlots];
+    uint64_t sempty[kScaleSlots];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
     int total_items;
     int goff[kMaxGroups + 1];
     int gstart[kMaxGroups + 1];
-    alignas(16) float red[2][4][64];
-    alignas(16) float inv[2][64];
-    alignas(16) float comb[kCombSlots][256];
+    alignas(16) float sa[kScaleSlots][kBM];   // token scales of one K block
+    alignas(16) float sb[kScaleSlots][2];     // the two weight-block scales
+    alignas(16) float red[2][2][kBM];         // [item parity][half][token] amax of h
 };
 
 constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + sizeof(SharedState) + 1024;
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 limit per CTA");
 
 // ------------------------------------------------------------- PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -94,14 +96,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// The waiting thread is suspended until the phase completes or about
+// kSuspendNs pass, so waiting warps do not take issue slots from the others.
+constexpr uint32_t kSuspendNs = 50000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -115,7 +121,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, SharedS
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255) == 0) {
+        if ((it & 15) == 0) {
             if (*reinterpret_cast<volatile int*>(&ss->abort_flag)) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 atomicExch(&ss->abort_flag, 1);
@@ -133,6 +139,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
         : "memory");
+}
+
+// 4-byte asynchronous copy global -> shared; src_bytes = 0 writes a zero.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// Arrive on `bar` once this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -174,14 +192,13 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         : "memory");
 }
 
-// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers,
-// waiting for the load to finish.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers.  The
+// load is asynchronous: tmem_wait2() must follow before the values are used.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
@@ -192,20 +209,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
-__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
-    uint64_t v;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
-    return v;
-}
-__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
-    uint32_t a, b;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
-    lo = __uint_as_float(a);
-    hi = __uint_as_float(b);
-}
-// acc(2 lanes) += p(2 lanes) * c(2 lanes), one instruction for two floats.
-__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t p, uint64_t c) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(p), "l"(c));
+#define MOE_R32(x)                                                                            \
+    "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),        \
+        "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]),            \
+        "+r"(x[13]), "+r"(x[14]), "+r"(x[15]), "+r"(x[16]), "+r"(x[17]), "+r"(x[18]),         \
+        "+r"(x[19]), "+r"(x[20]), "+r"(x[21]), "+r"(x[22]), "+r"(x[23]), "+r"(x[24]),         \
+        "+r"(x[25]), "+r"(x[26]), "+r"(x[27]), "+r"(x[28]), "+r"(x[29]), "+r"(x[30]),         \
+        "+r"(x[31])
+
+// Wait for this thread's TMEM loads; the two register sets are tied to the
+// wait so that no use of them is scheduled before it.
+__device__ __forceinline__ void tmem_wait2(uint32_t (&a)[32], uint32_t (&b)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MOE_R32(a), MOE_R32(b)::"memory");
 }
 
 __device__ __forceinline__ void named_bar(int id, int count) {
@@ -236,12 +251,15 @@ __device__ __forceinline__ void set_max_regs_dec() {
 
 // ------------------------------------------------------------- schedule
 struct Item {
-    int g, f, row0, ntok, nmma;
+    int g;      // group
+    int f;      // 256-column tile
+    int row0;   // first token row
+    int ntok;   // valid tokens (<= 128)
+    int ncols;  // MMA N: 256, or 128 for a last half-width tile
 };
 
-template <int NMAX>
-__device__ __forceinline__ Item decode_item(const SharedState* ss, int n_groups, int item) {
-    int lo = 0, hi = n_groups;
+__device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmParams& p, int item) {
+    int lo = 0, hi = p.n_groups;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (ss->gstart[mid] <= item) lo = mid;
@@ -251,40 +269,45 @@ __device__ __forceinline__ Item decode_item(const SharedState* ss, int n_groups,
     it.g = lo;
     const int local = item - ss->gstart[lo];
     const int rows = ss->goff[lo + 1] - ss->goff[lo];
-    const int ntiles = (rows + NMAX - 1) / NMAX;
-    it.f = local / ntiles;
-    const int tt = local - it.f * ntiles;
-    const int base = rows / ntiles, rem = rows - base * ntiles;
-    it.ntok = base + (tt < rem ? 1 : 0);
-    it.row0 = ss->goff[lo] + tt * base + min(tt, rem);
-    it.nmma = max(16, (it.ntok + 15) & ~15);
+    const int mtiles = (rows + kBM - 1) / kBM;
+    it.f = local / mtiles;
+    const int mt = local - it.f * mtiles;
+    it.row0 = ss->goff[lo] + mt * kBM;
+    it.ntok = min(kBM, rows - mt * kBM);
+    it.ncols = (p.epilogue == MOE_EPI_SWIGLU_QUANT) ? 256 : min(256, p.n - it.f * 256);
     return it;
 }
 
+// Weight rows of the two 128-row blocks of a tile (first row inside the
+// stacked [n_groups * n, k] matrix) and their block-row indices.
+__device__ __forceinline__ void weight_blocks(const GemmParams& p, const Item& w, int& r0, int& r1,
+                                              int& b0, int& b1) {
+    if (p.epilogue == MOE_EPI_SWIGLU_QUANT) {
+        b0 = w.f;                   // gate rows f*128 .. of W1
+        b1 = p.n / 256 + w.f;       // up rows (n/2 + f*128) .. of W3
+    } else {
+        b0 = 2 * w.f;
+        b1 = 2 * w.f + 1;
+    }
+    r0 = w.g * p.n + b0 * 128;
+    r1 = w.g * p.n + b1 * 128;
+}
+
 // ================================================= TMA producer (warp 0)
-template <int NUM_ACC>
 __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap& map_w,
-                                         const CUtensorMap& map_a64, const CUtensorMap& map_a16,
-                                         uint8_t* smem, SharedState* ss) {
-    constexpr int NMAX = 256 / NUM_ACC;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    (void)warp;
-    (void)lane;
-    const int G = p.n_groups;
+                                         const CUtensorMap& map_a, uint8_t* smem,
+                                         SharedState* ss) {
+    const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
-    // ================================================= TMA producer
-    uint32_t it = 0, cit = 0;
+    uint32_t it = 0;
     uint32_t issued_mask = 0, issued_parity = 0;
     bool ok = true;
-    const int nfw = p.n / 128;  // weight block rows per group
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item<NMAX>(ss, G, item);
-        const int wrow0 = w.g * p.n + w.f * 128;
-        const int wrow1 = wrow0 + p.n / 2;  // up projection (NUM_ACC == 2)
-        const uint32_t tx = uint32_t(NUM_ACC * kTileBytes + w.nmma * 128);
-        const float* sbw = p.w_scales + (size_t(w.g) * nfw + w.f) * p.nkb;
-        const float* sbw1 = p.w_scales + (size_t(w.g) * nfw + w.f + nfw / 2) * p.nkb;
-        for (int kb = 0; kb < p.nkb; ++kb, ++it, ++cit) {
+        const Item w = decode_item(ss, p, item);
+        int wr0, wr1, b0, b1;
+        weight_blocks(p, w, wr0, wr1, b0, b1);
+        const uint32_t tx = uint32_t(kTileBytes + w.ncols * 128);
+        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
             const int s = it % kStages;
             const uint32_t par = ((it / kStages) & 1u);
             if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
@@ -294,32 +317,13 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap&
                 uint8_t* st = smem + size_t(s) * kStageBytes;
                 const uint32_t fb = smem_u32(&ss->full[s]);
                 mbar_arrive_expect_tx(fb, tx);
-                tma_load_2d(smem_u32(st), &map_w, fb, kb * 128, wrow0);
-                if (NUM_ACC == 2) tma_load_2d(smem_u32(st + kTileBytes), &map_w, fb, kb * 128, wrow1);
-                uint8_t* bt = st + NUM_ACC * kTileBytes;
-                int r = 0;
-                for (; r + 64 <= w.nmma; r += 64)
-                    tma_load_2d(smem_u32(bt + r * 128), &map_a64, fb, kb * 128, w.row0 + r);
-                for (; r < w.nmma; r += 16)
-                    tma_load_2d(smem_u32(bt + r * 128), &map_a16, fb, kb * 128, w.row0 + r);
+                tma_load_2d(smem_u32(st), &map_a, fb, kb * 128, w.row0);
+                tma_load_2d(smem_u32(st + kTileBytes), &map_w, fb, kb * 128, wr0);
+                if (w.ncols == 256)
+                    tma_load_2d(smem_u32(st + 2 * kTileBytes), &map_w, fb, kb * 128, wr1);
                 issued_mask |= 1u << s;
                 issued_parity = (issued_parity & ~(1u << s)) | (par << s);
             }
-            // combined scales sa[token] * sb[weight block] for this K block
-            const int c = cit % kCombSlots;
-            const uint32_t cpar = ((cit / kCombSlots) & 1u);
-            if (lane == 0) ok = mbar_wait(smem_u32(&ss->cempty[c]), cpar ^ 1u, ss, p.dev_status);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            const float sb0 = __ldg(sbw + kb);
-            const float sb1 = NUM_ACC == 2 ? __ldg(sbw1 + kb) : 0.0f;
-            const float* sa = p.a_scales + size_t(kb) * p.max_rows + w.row0;
-            for (int j = lane; j < w.nmma; j += 32) {
-                const float a = j < w.ntok ? __ldg(sa + j) : 0.0f;
-                ss->comb[c][j] = a * sb0;
-                if (NUM_ACC == 2) ss->comb[c][128 + j] = a * sb1;
-            }
-            mbar_arrive(smem_u32(&ss->cfull[c]));
         }
     }
     if (!ok && lane == 0) {
@@ -331,23 +335,58 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap&
     __syncwarp();
 }
 
+// ================================================= scale loader (warp 2)
+// cp.async of each K block's 128 token scales (kb-major, so they are
+// contiguous) and the tile's two weight-block scales; the copies arrive on
+// sfull when they land.
+__device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* ss) {
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    const int nbr = p.n / 128;  // weight block rows per group
+    uint32_t cit = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        const Item w = decode_item(ss, p, item);
+        int wr0, wr1, b0, b1;
+        weight_blocks(p, w, wr0, wr1, b0, b1);
+        const float* sb0 = p.w_scales + (size_t(w.g) * nbr + b0) * p.nkb;
+        const float* sb1 = p.w_scales + (size_t(w.g) * nbr + (w.ncols == 256 ? b1 : b0)) * p.nkb;
+        for (int kb = 0; kb < p.nkb; ++kb, ++cit) {
+            const int c = cit % kScaleSlots;
+            if (lane == 0)
+                ok = mbar_wait(smem_u32(&ss->sempty[c]), ((cit / kScaleSlots) & 1u) ^ 1u, ss,
+                               p.dev_status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const float* sa = p.a_scales + size_t(kb) * p.max_rows + w.row0;
+#pragma unroll
+            for (int i = 0; i < kBM / 32; ++i) {
+                const int j = lane + 32 * i;
+                const bool real = j < w.ntok;  // rows past the group get 0
+                cp_async4(&ss->sa[c][j], real ? sa + j : sa, real ? 4u : 0u);
+            }
+            if (lane == 0) {
+                cp_async4(&ss->sb[c][0], sb0 + kb, 4u);
+                cp_async4(&ss->sb[c][1], sb1 + kb, 4u);
+            }
+            cp_async_arrive(smem_u32(&ss->sfull[c]));
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncwarp();
+}
+
 // ================================================= MMA issuer (warp 1)
-template <int NUM_ACC>
 __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, SharedState* ss,
                                            uint32_t tmem_base) {
-    constexpr int NMAX = 256 / NUM_ACC;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    (void)warp;
-    (void)lane;
-    const int G = p.n_groups;
+    const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
-    // ================================================= MMA issuer
     if (lane == 0) {
         uint32_t it = 0, tb = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-            const Item w = decode_item<NMAX>(ss, G, item);
-            const uint32_t idesc = idesc_e4m3(128, w.nmma);
+            const Item w = decode_item(ss, p, item);
+            const uint32_t idesc = idesc_e4m3(128, w.ncols);
             for (int kb = 0; kb < p.nkb; ++kb, ++it, ++tb) {
                 const int s = it % kStages;
                 const uint32_t buf = tb & 1u;
@@ -357,15 +396,11 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + size_t(s) * kStageBytes);
-                const uint32_t bt = st + NUM_ACC * kTileBytes;
+                const uint32_t d = tmem_base + buf * 256;
 #pragma unroll
-                for (int a = 0; a < NUM_ACC; ++a) {
-                    const uint32_t d = tmem_base + buf * 256 + a * 128;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_e4m3(d, sw128_desc(st + a * kTileBytes + kk * 32),
-                                 sw128_desc(bt + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_e4m3(d, sw128_desc(st + kk * 32), sw128_desc(st + kTileBytes + kk * 32),
+                             idesc, kk > 0 ? 1u : 0u);
                 mma_commit(smem_u32(&ss->empty[s]));
                 mma_commit(smem_u32(&ss->tfull[buf]));
             }
@@ -378,156 +413,142 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
 }
 
 // ================================================= promotion + epilogue (warps 4-11)
-template <int NUM_ACC>
+// Thread (warp w, lane l) owns token row r = 32*(w%4) + l of the tile and
+// 128 of its 256 columns: half h = (w-4)/4.
+//   SwiGLU: gate columns [64h, 64h+64) and up columns [128+64h, 128+64h+64)
+//           (the same 64 features of W1 and W3), scales s0 and s1;
+//   F32/BF16: columns [128h, 128h+128), scale s_h.
 __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
                                          uint32_t tmem_base) {
-    constexpr int NMAX = 256 / NUM_ACC;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    (void)warp;
-    (void)lane;
-    const int G = p.n_groups;
     const int total_items = ss->total_items;
-    // ================================================= promotion + epilogue
-    const int q = warp & 3;          // TMEM lane quadrant = weight rows 32q..32q+31
-    const int half = (warp - 4) >> 2;  // column half
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int r = q * 32 + lane;  // token row inside the tile
+    const bool swiglu = p.epilogue == MOE_EPI_SWIGLU_QUANT;
     const uint32_t lane_addr = tmem_base + (uint32_t(q * 32) << 16);
-    uint32_t tb = 0, cit = 0;
+    uint32_t tb = 0, cit = 0, parity = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
-        const Item w = decode_item<NMAX>(ss, G, item);
-        uint64_t acc[64];
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x, parity ^= 1u) {
+        const Item w = decode_item(ss, p, item);
+        // columns of this thread's four 32-column chunks
+        int col[4];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0;
+        for (int ch = 0; ch < 4; ++ch)
+            col[ch] = swiglu ? ((ch >> 1) * 128 + half * 64 + (ch & 1) * 32) : (half * 128 + ch * 32);
+        const bool active = swiglu || col[0] < w.ncols;
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
         for (int kb = 0; ok && kb < p.nkb; ++kb, ++tb, ++cit) {
             const uint32_t buf = tb & 1u;
-            const int c = cit % kCombSlots;
+            const int c = cit % kScaleSlots;
             if (lane == 0) {
                 ok = mbar_wait(smem_u32(&ss->tfull[buf]), (tb >> 1) & 1u, ss, p.dev_status);
-                if (ok) ok = mbar_wait(smem_u32(&ss->cfull[c]), (cit / kCombSlots) & 1u, ss,
+                if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (cit / kScaleSlots) & 1u, ss,
                                        p.dev_status);
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
+            __syncwarp();
             tc_fence_after();
+            if (active) {
+                const float sa = ss->sa[c][r];
+                const float s0 = sa * ss->sb[c][swiglu ? 0 : half];
+                const float s1 = swiglu ? sa * ss->sb[c][1] : s0;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                // column (token) offset of this 32-column chunk inside its accumulator
-                const int rc = NUM_ACC == 2 ? half * 64 + (ch & 1) * 32 : half * 128 + ch * 32;
-                const int a = NUM_ACC == 2 ? (ch >> 1) : 0;
-                if (rc >= w.nmma) continue;
-                uint32_t r[32];
-                tmem_ld32(lane_addr + buf * 256 + a * 128 + rc, r);
-                const float4* cs = reinterpret_cast<const float4*>(&ss->comb[c][a * 128 + rc]);
+                for (int pr = 0; pr < 2; ++pr) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32_async(lane_addr + buf * 256 + col[2 * pr], v0);
+                    tmem_ld32_async(lane_addr + buf * 256 + col[2 * pr + 1], v1);
+                    tmem_wait2(v0, v1);
+                    const float sc = pr == 0 ? s0 : s1;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 cv = cs[i];
-                    ffma2(acc[ch * 16 + 2 * i], pack2(r[4 * i], r[4 * i + 1]),
-                          pack2(__float_as_uint(cv.x), __float_as_uint(cv.y)));
-                    ffma2(acc[ch * 16 + 2 * i + 1], pack2(r[4 * i + 2], r[4 * i + 3]),
-                          pack2(__float_as_uint(cv.z), __float_as_uint(cv.w)));
+                    for (int i = 0; i < 32; ++i) {
+                        acc[64 * pr + i] = fmaf(__uint_as_float(v0[i]), sc, acc[64 * pr + i]);
+                        acc[64 * pr + 32 + i] = fmaf(__uint_as_float(v1[i]), sc, acc[64 * pr + 32 + i]);
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(smem_u32(&ss->tempty[buf]));
-                mbar_arrive(smem_u32(&ss->cempty[c]));
+                mbar_arrive(smem_u32(&ss->sempty[c]));
             }
         }
         // ---------------- epilogue
-        const int feat = q * 32 + lane;  // row inside the 128-row weight tile
-        if (NUM_ACC == 1) {
-            const size_t ld = size_t(p.n);
-            const int col0 = w.f * 128 + feat;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                float v0, v1;
-                unpack2(acc[i], v0, v1);
-                const int j = half * 128 + 2 * i;
+        const bool row_ok = r < w.ntok;
+        const size_t row = size_t(w.row0) + r;
+        if (!swiglu) {
+            if (active && row_ok) {
+                const size_t c0 = size_t(w.f) * 256 + half * 128;
                 if (p.epilogue == MOE_EPI_F32) {
-                    float* o = static_cast<float*>(p.out);
-                    if (j < w.ntok) o[size_t(w.row0 + j) * ld + col0] = v0;
-                    if (j + 1 < w.ntok) o[size_t(w.row0 + j + 1) * ld + col0] = v1;
+                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.n + c0);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
                 } else {
-                    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out);
-                    if (j < w.ntok) o[size_t(w.row0 + j) * ld + col0] = __float2bfloat16_rn(v0);
-                    if (j + 1 < w.ntok)
-                        o[size_t(w.row0 + j + 1) * ld + col0] = __float2bfloat16_rn(v1);
+                    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row * p.n + c0);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * i + 2 * j], acc[8 * i + 2 * j + 1]);
+                            u[j] = *reinterpret_cast<uint32_t*>(&b);
+                        }
+                        o[i] = make_uint4(u[0], u[1], u[2], u[3]);
+                    }
                 }
             }
         } else {
-            // h = silu(gate) * up for 64 tokens (this half), then 1x128
-            // quantisation over the tile's 128 features (4 quadrant warps).
-            float h[64];
+            // h = silu(gate) * up for this thread's 64 features, then the
+            // 1x128 scale of the token's 128 features (both halves).
+            float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float g0, g1, u0, u1;
-                unpack2(acc[i], g0, g1);
-                unpack2(acc[32 + i], u0, u1);
-                h[2 * i] = __fmul_rn(__fdiv_rn(g0, 1.0f + expf(-g0)), u0);
-                h[2 * i + 1] = __fmul_rn(__fdiv_rn(g1, 1.0f + expf(-g1)), u1);
+            for (int i = 0; i < 64; ++i) {
+                const float g = acc[i];
+                const float hv = __fmul_rn(__fmul_rn(g, __frcp_rn(__fadd_rn(1.0f, expf(-g)))),
+                                           acc[64 + i]);
+                acc[i] = hv;
+                amax = fmaxf(amax, fabsf(hv));
             }
-            // column maxima of |h| over this warp's 32 lanes: after the
-            // butterfly, lane l holds the max of column (32*b + l).
+            ss->red[parity][half][r] = amax;
+            named_bar(1, kPromoters * 32);
+            amax = fmaxf(amax, ss->red[parity][half ^ 1][r]);
+            float scale, inv;
+            scale_from_amax(amax, scale, inv);
+            if (row_ok) {
+                uint4* o = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + row * (p.n / 2) +
+                                                    size_t(w.f) * 128 + half * 64);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                float v[32];
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t u[4];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = fabsf(h[32 * b + i]);
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    const bool upper = (lane & o) != 0;
-#pragma unroll
-                    for (int i = 0; i < o; ++i) {
-                        const float send = upper ? v[i] : v[i + o];
-                        const float keep = upper ? v[i + o] : v[i];
-                        v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                    for (int j = 0; j < 4; ++j) {
+                        const int b = 16 * i + 4 * j;
+                        const uint32_t lo = e4m3x2(__fmul_rn(acc[b], inv), __fmul_rn(acc[b + 1], inv));
+                        const uint32_t hi = e4m3x2(__fmul_rn(acc[b + 2], inv), __fmul_rn(acc[b + 3], inv));
+                        u[j] = lo | (hi << 16);
                     }
+                    o[i] = make_uint4(u[0], u[1], u[2], u[3]);
                 }
-                ss->red[half][q][32 * b + lane] = v[0];
-            }
-            named_bar(1 + half, 128);
-            if (q == 0) {
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    const int jj = 32 * b + lane;
-                    float amax = fmaxf(fmaxf(ss->red[half][0][jj], ss->red[half][1][jj]),
-                                       fmaxf(ss->red[half][2][jj], ss->red[half][3][jj]));
-                    float scale, inv;
-                    scale_from_amax(amax, scale, inv);
-                    ss->inv[half][jj] = inv;
-                    const int j = half * 64 + jj;
-                    if (j < w.ntok) p.out_scales[size_t(w.f) * p.max_rows + w.row0 + j] = scale;
-                }
-            }
-            named_bar(1 + half, 128);
-            uint8_t* o = static_cast<uint8_t*>(p.out);
-            const size_t ld = size_t(p.n / 2);
-            const int col0 = w.f * 128 + feat;
-#pragma unroll
-            for (int i = 0; i < 64; i += 2) {
-                const int j = half * 64 + i;
-                const uint16_t c2 = e4m3x2(__fmul_rn(h[i], ss->inv[half][i]),
-                                           __fmul_rn(h[i + 1], ss->inv[half][i + 1]));
-                if (j < w.ntok) o[size_t(w.row0 + j) * ld + col0] = uint8_t(c2 & 0xFF);
-                if (j + 1 < w.ntok) o[size_t(w.row0 + j + 1) * ld + col0] = uint8_t(c2 >> 8);
+                if (half == 0) p.out_scales[size_t(w.f) * p.max_rows + row] = scale;
             }
         }
-        // all warps of this half agree on whether to go on
-        const bool any_abort =
-            named_bar_or(3 + half, 128, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
+        // all promotion warps agree on whether to go on
+        const bool any_abort = named_bar_or(
+            2, kPromoters * 32, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
         if (any_abort) break;
     }
     tc_fence_before();
 }
 
 // ----------------------------------------------------------------- kernel
-template <int NUM_ACC>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
-                        const __grid_constant__ CUtensorMap map_a64,
-                        const __grid_constant__ CUtensorMap map_a16, const GemmParams p) {
-    constexpr int NMAX = 256 / NUM_ACC;
+                        const __grid_constant__ CUtensorMap map_a, const GemmParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -542,11 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ss->tfull[b]), 1);
-            mbar_init(smem_u32(&ss->tempty[b]), 8);
+            mbar_init(smem_u32(&ss->tempty[b]), kPromoters);
         }
-        for (int c = 0; c < kCombSlots; ++c) {
-            mbar_init(smem_u32(&ss->cfull[c]), 32);
-            mbar_init(smem_u32(&ss->cempty[c]), 8);
+        for (int c = 0; c < kScaleSlots; ++c) {
+            mbar_init(smem_u32(&ss->sfull[c]), 32);
+            mbar_init(smem_u32(&ss->sempty[c]), kPromoters);
         }
         mbar_init(smem_u32(&ss->drain), 1);
         ss->abort_flag = 0;
@@ -558,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // group offsets and an exclusive scan of work items per group
+    // group offsets (validated) and an exclusive scan of work items per group
     const int G = p.n_groups;
     int bad = 0;
     for (int i = threadIdx.x; i <= G; i += kThreads) {
@@ -582,12 +603,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             int v = 0;
             if (g < G) {
                 const int rows = ss->goff[g + 1] - ss->goff[g];
-                v = rows > 0 ? ((rows + NMAX - 1) / NMAX) * p.n_feat : 0;
+                v = ((rows + kBM - 1) / kBM) * p.n_ftiles;
             }
             vals[j] = v;
             sum += v;
         }
-        // block exclusive scan of per-thread sums (reuse gstart as scratch)
         int incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -618,11 +638,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 4) {
         set_max_regs_dec<56>();
-        if (warp == 0) producer<NUM_ACC>(p, map_w, map_a64, map_a16, smem, ss);
-        else if (warp == 1) mma_issuer<NUM_ACC>(p, smem, ss, tmem_base);
+        if (warp == 0) producer(p, map_w, map_a, smem, ss);
+        else if (warp == 1) mma_issuer(p, smem, ss, tmem_base);
+        else if (warp == 2) scale_loader(p, ss);
     } else {
         set_max_regs_inc<224>();
-        promoter<NUM_ACC>(p, ss, tmem_base);
+        promoter(p, ss, tmem_base);
     }
 
     __syncthreads();
@@ -632,7 +653,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
     }
 }
-
 
 // ------------------------------------------------------------------ host
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -677,14 +697,11 @@ bool device_is_sm100() {
     return major == 10;
 }
 
-template <int NUM_ACC>
-int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& m64,
-           const CUtensorMap& m16, cudaStream_t st) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<NUM_ACC>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma, cudaStream_t st) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kSmemBytes)) != cudaSuccess)
         return MOE_ERR_CUDA;
-    grouped_gemm_kernel<NUM_ACC><<<sm_count(), kThreads, kSmemBytes, st>>>(mw, m64, m16, p);
+    grouped_gemm_kernel<<<sm_count(), kThreads, kSmemBytes, st>>>(mw, ma, p);
     return check_launch();
 }
 
@@ -722,18 +739,15 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     p.nkb = k / 128;
     p.w_scales = w_scales;
     p.n = n;
-    p.n_feat = epilogue == MOE_EPI_SWIGLU_QUANT ? n / 256 : n / 128;
+    p.n_ftiles = (n + 255) / 256;
     p.epilogue = epilogue;
     p.out = out;
     p.out_scales = out_scales;
     p.dev_status = dev_status;
 
-    CUtensorMap mw, m64, m16;
+    CUtensorMap mw, ma;
     if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128) ||
-        !make_map(&m64, a, uint64_t(max_rows), uint64_t(k), 64) ||
-        !make_map(&m16, a, uint64_t(max_rows), uint64_t(k), 16))
+        !make_map(&ma, a, uint64_t(max_rows), uint64_t(k), 128))
         return MOE_ERR_CUDA;
-    cudaStream_t st = as_stream(stream);
-    if (epilogue == MOE_EPI_SWIGLU_QUANT) return launch<2>(p, mw, m64, m16, st);
-    return launch<1>(p, mw, m64, m16, st);
+    return launch(p, mw, ma, as_stream(stream));
 }

@@ -78,6 +78,11 @@ CONFIGS = {
     "decode": MoeConfig("decode", T=128, d=7168, n_routed=256, n_groups=8,
                         topk_groups=4, topk=8, inter=2048, sigma_w=0.006,
                         beta=0.05, gamma=0.001, seed=3),
+    # profiling case: the prefill layer's per-expert shapes (about 128 rows per
+    # expert, d=7168, I=2048) with 16 routed experts, 0.75 GB of FP8 weights
+    "prefill_e16": MoeConfig("prefill_e16", T=256, d=7168, n_routed=16, n_groups=8,
+                             topk_groups=4, topk=8, inter=2048, sigma_w=0.006,
+                             beta=0.05, gamma=0.001, seed=5),
     "skewed": MoeConfig("skewed", T=16384, d=7168, n_routed=256, n_groups=8,
                         topk_groups=4, topk=8, inter=2048, sigma_w=0.006,
                         beta=0.05, gamma=0.001, seed=4, zipf=1.2, batches=8),
