@@ -36,7 +36,7 @@ constexpr int kThreads = 384;
 constexpr int kStages = 4;
 constexpr int kTileBytes = 128 * 128;            // one 128 x 128 FP8 tile
 constexpr int kStageBytes = 3 * kTileBytes;      // token tile + 2 weight tiles
-constexpr int kScaleSlots = 8;
+constexpr int kScaleSlots = 16;
 constexpr int kMaxGroups = 1040;
 constexpr int kBM = 128;                         // tokens per tile
 constexpr int kPromoters = 8;                    // promotion warps

@@ -15,60 +15,91 @@ namespace {
 
 constexpr int kLT = 64;   // tokens per logits tile
 constexpr int kLE = 64;   // experts per logits tile
-constexpr int kLK = 32;   // k per smem stage
+constexpr int kLK = 16;   // k per smem stage (double-buffered)
+constexpr int kLV = kLK / 8;  // 16-byte vectors per row and stage
+constexpr int kLThreads = 64;
 
 // u[t, i] = fp32(sum_k x[t,k] * E[i,k]) with an FP64 accumulator updated in
 // ascending k (each bf16*bf16 product is exact in FP64, so fma == mul+add).
-// 256 threads; thread (ty, tx) owns tokens 4ty..4ty+3 and experts 4tx..4tx+3.
-__global__ void __launch_bounds__(256) route_logits_kernel(
+// 64 threads; thread (ty, tx) owns tokens 8ty..8ty+7 and experts 8tx..8tx+7
+// of the 64 x 64 tile (64 FP64 accumulators).  Shared memory holds the tile's
+// K chunk as doubles; the experts are stored interleaved (expert 8tx+j at
+// column 8j+tx) so that the 8 threads of a row read consecutive doubles.
+// Chunks are double-buffered and the next one is fetched into registers
+// while the current one is multiplied.
+__global__ void __launch_bounds__(kLThreads) route_logits_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int d, int n_routed,
     float* __restrict__ u) {
-    __shared__ __align__(16) double xs[kLK][kLT];
-    __shared__ __align__(16) double es[kLK][kLE];
+    __shared__ __align__(16) double xs[2][kLK][kLT];
+    __shared__ __align__(16) double es[2][kLK][kLE];
     const int t0 = blockIdx.x * kLT, e0 = blockIdx.y * kLE;
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-    const int lrow = tid >> 2, lk = (tid & 3) * 8;
-    const bool xrow_ok = t0 + lrow < T, erow_ok = e0 + lrow < n_routed;
-    const uint4* xp = reinterpret_cast<const uint4*>(x + int64_t(t0 + lrow) * d + lk);
-    const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e0 + lrow) * d + lk);
-    double acc[4][4];
+    const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+    // loader: thread tid stages row tid of the x tile and row tid of the E
+    // tile, kLK k values of each per chunk
+    const bool xrow_ok = t0 + tid < T, erow_ok = e0 + tid < n_routed;
+    const uint4* xp = reinterpret_cast<const uint4*>(x + int64_t(t0 + tid) * d);
+    const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e0 + tid) * d);
+    const int ecol = (tid & 7) * 8 + (tid >> 3);  // interleaved column of expert tid
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    uint4 xv[kLV], ev[kLV];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kLV; ++i) {
+        xv[i] = xrow_ok ? __ldg(xp + i) : zero;
+        ev[i] = erow_ok ? __ldg(ep + i) : zero;
+    }
+    double acc[8][8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int k0 = 0; k0 < d; k0 += kLK) {
-        const uint4 xv = xrow_ok ? __ldg(xp + k0 / 8) : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 ev = erow_ok ? __ldg(ep + k0 / 8) : make_uint4(0u, 0u, 0u, 0u);
-        __syncthreads();
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, ew[4] = {ev.x, ev.y, ev.z, ev.w};
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            xs[lk + 2 * j][lrow] = (double)bf16_lo(xw[j]);
-            xs[lk + 2 * j + 1][lrow] = (double)bf16_hi(xw[j]);
-            es[lk + 2 * j][lrow] = (double)bf16_lo(ew[j]);
-            es[lk + 2 * j + 1][lrow] = (double)bf16_hi(ew[j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    int buf = 0;
+    for (int k0 = 0; k0 < d; k0 += kLK, buf ^= 1) {
+#pragma unroll
+        for (int i = 0; i < kLV; ++i) {
+            const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+            const uint32_t ew[4] = {ev[i].x, ev[i].y, ev[i].z, ev[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int kk = 8 * i + 2 * j;
+                xs[buf][kk][tid] = (double)bf16_lo(xw[j]);
+                xs[buf][kk + 1][tid] = (double)bf16_hi(xw[j]);
+                es[buf][kk][ecol] = (double)bf16_lo(ew[j]);
+                es[buf][kk + 1][ecol] = (double)bf16_hi(ew[j]);
+            }
         }
-        __syncthreads();
-#pragma unroll 8
+        __syncthreads();  // this chunk is staged; the other buffer is free again
+        if (k0 + kLK < d) {
+            const int v = (k0 + kLK) / 8;
+#pragma unroll
+            for (int i = 0; i < kLV; ++i) {
+                xv[i] = xrow_ok ? __ldg(xp + v + i) : zero;
+                ev[i] = erow_ok ? __ldg(ep + v + i) : zero;
+            }
+        }
+#pragma unroll 4
         for (int k = 0; k < kLK; ++k) {
-            const double2 xa = *reinterpret_cast<const double2*>(&xs[k][ty * 4]);
-            const double2 xb = *reinterpret_cast<const double2*>(&xs[k][ty * 4 + 2]);
-            const double2 ea = *reinterpret_cast<const double2*>(&es[k][tx * 4]);
-            const double2 eb = *reinterpret_cast<const double2*>(&es[k][tx * 4 + 2]);
-            const double xv4[4] = {xa.x, xa.y, xb.x, xb.y}, ev4[4] = {ea.x, ea.y, eb.x, eb.y};
+            double xr[8], er[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i) {
+                const double2 v2 = *reinterpret_cast<const double2*>(&xs[buf][k][ty * 8 + 2 * i]);
+                xr[2 * i] = v2.x;
+                xr[2 * i + 1] = v2.y;
+            }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv4[i], ev4[j], acc[i][j]);
+            for (int j = 0; j < 8; ++j) er[j] = es[buf][k][8 * j + tx];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fma(xr[i], er[j], acc[i][j]);
         }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + ty * 8 + i;
         if (t >= T) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = e0 + tx * 4 + j;
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + tx * 8 + j;
             if (e < n_routed) u[int64_t(t) * n_routed + e] = __double2float_rn(acc[i][j]);
         }
     }
@@ -218,7 +249,7 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
     if (!ws || ws_bytes < moe_route_workspace_size(shape)) return MOE_ERR_WORKSPACE;
     float* u = static_cast<float*>(ws);
     dim3 g1((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
-    route_logits_kernel<<<g1, 256, 0, st>>>(x, router_w, T, d, N, u);
+    route_logits_kernel<<<g1, kLThreads, 0, st>>>(x, router_w, T, d, N, u);
     if ((rc = check_launch()) != MOE_OK) return rc;
     const size_t smem = sizeof(float) * size_t(N) * (1 + 2 * kSelWarps);
     if (smem > 48 * 1024 &&
