@@ -192,35 +192,29 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         : "memory");
 }
 
-// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers.  The
-// load is asynchronous: tmem_wait2() must follow before the values are used.
-__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+// 64 consecutive TMEM columns of this warp's 32 lanes -> 64 registers; the
+// wait for the load is part of the same statement.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
           "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
+          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+          "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
-}
-
-#define MOE_R32(x)                                                                            \
-    "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),        \
-        "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]),            \
-        "+r"(x[13]), "+r"(x[14]), "+r"(x[15]), "+r"(x[16]), "+r"(x[17]), "+r"(x[18]),         \
-        "+r"(x[19]), "+r"(x[20]), "+r"(x[21]), "+r"(x[22]), "+r"(x[23]), "+r"(x[24]),         \
-        "+r"(x[25]), "+r"(x[26]), "+r"(x[27]), "+r"(x[28]), "+r"(x[29]), "+r"(x[30]),         \
-        "+r"(x[31])
-
-// Wait for this thread's TMEM loads; the two register sets are tied to the
-// wait so that no use of them is scheduled before it.
-__device__ __forceinline__ void tmem_wait2(uint32_t (&a)[32], uint32_t (&b)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : MOE_R32(a), MOE_R32(b)::"memory");
 }
 
 __device__ __forceinline__ void named_bar(int id, int count) {
@@ -456,25 +450,27 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
                 const float sa = ss->sa[c][r];
                 const float s0 = sa * ss->sb[c][swiglu ? 0 : half];
                 const float s1 = swiglu ? sa * ss->sb[c][1] : s0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
+                uint32_t v[64];
+                tmem_ld64(lane_addr + buf * 256 + col[0], v);  // columns col[0], col[1]
 #pragma unroll
-                for (int pr = 0; pr < 2; ++pr) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32_async(lane_addr + buf * 256 + col[2 * pr], v0);
-                    tmem_ld32_async(lane_addr + buf * 256 + col[2 * pr + 1], v1);
-                    tmem_wait2(v0, v1);
-                    const float sc = pr == 0 ? s0 : s1;
+                for (int i = 0; i < 64; ++i) acc[i] = fmaf(__uint_as_float(v[i]), s0, acc[i]);
+                tmem_ld64(lane_addr + buf * 256 + col[2], v);  // columns col[2], col[3]
+                // the partial is in registers: hand the TMEM buffer back to
+                // the MMA before the last FMAs
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        acc[64 * pr + i] = fmaf(__uint_as_float(v0[i]), sc, acc[64 * pr + i]);
-                        acc[64 * pr + 32 + i] = fmaf(__uint_as_float(v1[i]), sc, acc[64 * pr + 32 + i]);
-                    }
+                for (int i = 0; i < 64; ++i) acc[64 + i] = fmaf(__uint_as_float(v[i]), s1, acc[64 + i]);
+            } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&ss->sempty[c]));
+                    mbar_arrive(smem_u32(&ss->tempty[buf]));
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&ss->tempty[buf]));
-                mbar_arrive(smem_u32(&ss->sempty[c]));
             }
         }
         // ---------------- epilogue
@@ -509,8 +505,8 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 const float g = acc[i];
-                const float hv = __fmul_rn(__fmul_rn(g, __frcp_rn(__fadd_rn(1.0f, expf(-g)))),
-                                           acc[64 + i]);
+                // silu(g) = g / (1 + e^-g); fast exp and divide (~1e-6 relative)
+                const float hv = __fdividef(g, 1.0f + __expf(-g)) * acc[64 + i];
                 acc[i] = hv;
                 amax = fmaxf(amax, fabsf(hv));
             }
