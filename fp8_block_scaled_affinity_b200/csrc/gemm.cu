@@ -217,6 +217,21 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
         : "memory");
 }
 
+__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+    return v;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+    return f;
+}
+// acc (two fp32 lanes) += p * s, one instruction for two values.
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t p, uint64_t s) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(p), "l"(s));
+}
+
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -431,9 +446,9 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
         for (int ch = 0; ch < 4; ++ch)
             col[ch] = swiglu ? ((ch >> 1) * 128 + half * 64 + (ch & 1) * 32) : (half * 128 + ch * 32);
         const bool active = swiglu || col[0] < w.ncols;
-        float acc[128];
+        uint64_t acc2[64];  // fp32 accumulator pairs (columns 2i, 2i+1 of the thread)
 #pragma unroll
-        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < 64; ++i) acc2[i] = 0;
         for (int kb = 0; ok && kb < p.nkb; ++kb, ++tb, ++cit) {
             const uint32_t buf = tb & 1u;
             const int c = cit % kScaleSlots;
@@ -450,12 +465,14 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
                 const float sa = ss->sa[c][r];
                 const float s0 = sa * ss->sb[c][swiglu ? 0 : half];
                 const float s1 = swiglu ? sa * ss->sb[c][1] : s0;
+                const uint64_t s0x2 = pack2(__float_as_uint(s0), __float_as_uint(s0));
+                const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
                 uint32_t v[64];
                 tmem_ld64(lane_addr + buf * 256 + col[0], v);  // columns col[0], col[1]
 #pragma unroll
-                for (int i = 0; i < 64; ++i) acc[i] = fmaf(__uint_as_float(v[i]), s0, acc[i]);
+                for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
                 tmem_ld64(lane_addr + buf * 256 + col[2], v);  // columns col[2], col[3]
                 // the partial is in registers: hand the TMEM buffer back to
                 // the MMA before the last FMAs
@@ -463,7 +480,7 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
 #pragma unroll
-                for (int i = 0; i < 64; ++i) acc[64 + i] = fmaf(__uint_as_float(v[i]), s1, acc[64 + i]);
+                for (int i = 0; i < 32; ++i) ffma2(acc2[32 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
             } else {
                 tc_fence_before();
                 __syncwarp();
@@ -474,6 +491,13 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
             }
         }
         // ---------------- epilogue
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const float2 f = unpack2(acc2[i]);
+            acc[2 * i] = f.x;
+            acc[2 * i + 1] = f.y;
+        }
         const bool row_ok = r < w.ntok;
         const size_t row = size_t(w.row0) + r;
         if (!swiglu) {
