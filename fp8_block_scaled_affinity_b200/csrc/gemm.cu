@@ -8,21 +8,24 @@
 // accumulators with the block's combined scale sa[token] * sb[weight block].
 //
 // Tile: 128 tokens (the MMA's M side, one token per TMEM lane, so a thread's
-// token scale is one register) x 256 weight columns (N: two 128-row weight
-// blocks, each with one scale per K block) x 128 K.  For the SwiGLU epilogue
-// the two weight blocks are the gate (W1) and up (W3) rows of the same 128
-// features, so a thread holds gate and up of the same (token, feature).
+// token scale is one register) x BN weight columns (N) x 128 K.
+//   BN = 256 (SwiGLU epilogue): the gate (W1) and up (W3) blocks of the same
+//     128 features, so a thread holds gate and up of the same (token,
+//     feature); 2 TMEM partial buffers, 4 smem stages of 48 KB.
+//   BN = 128 (fp32 / bf16 output): one 128-row weight block; 4 TMEM partial
+//     buffers (more slack between MMA and promotion), 4 stages of 32 KB; a
+//     tile's output row segment is parked in shared memory and stored during
+//     the next tile's K loop, one 16-byte store per K block, so the stores
+//     overlap compute instead of stalling the promotion warps.
 //
 // Roles (384 threads, one CTA per SM, persistent over work items):
-//   warp 0       TMA producer: token tile (16 KB) + two weight tiles (32 KB)
-//                per K block into a 4-stage smem ring
+//   warp 0       TMA producer: token tile (16 KB) + weight tile(s) per K block
 //   warp 1       TMEM owner and MMA issuer (one thread)
 //   warp 2       scale loader: cp.async of the K block's 128 token scales and
-//                2 weight-block scales into a small smem ring
+//                the weight-block scales into a small smem ring
 //   warp 3       idle (its registers go to the promoters)
 //   warps 4-11   promotion + epilogue: warp w reads TMEM lanes 32*(w%4)..+31
-//                (its 32 tokens) and one half of the 256 columns
-// TMEM: 2 partial buffers x 256 columns = all 512 columns.
+//                (its 32 tokens) and one half of the BN columns
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <mutex>
@@ -33,13 +36,25 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kStages = 4;
 constexpr int kTileBytes = 128 * 128;            // one 128 x 128 FP8 tile
-constexpr int kStageBytes = 3 * kTileBytes;      // token tile + 2 weight tiles
+constexpr int kStages = 4;                       // smem ring of operand stages
+constexpr int kParkStride = 272;                 // bytes per parked row segment (256 + pad)
+constexpr int kMaxBufs = 4;
 constexpr int kScaleSlots = 16;
 constexpr int kMaxGroups = 1040;
 constexpr int kBM = 128;                         // tokens per tile
 constexpr int kPromoters = 8;                    // promotion warps
+
+template <int BN>
+struct Cfg {
+    static constexpr int kStageBytes = kTileBytes + BN * 128;  // tokens + weights
+    static constexpr int kStages = moe::kStages;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kParkBytes = BN == 128 ? kPromoters * 32 * kParkStride : 0;
+    static constexpr int kBufs = 512 / BN;                     // TMEM partial buffers
+    static constexpr int kPairs = BN / 4;                      // fp32 pairs per promoter thread
+    static_assert(kBufs <= kMaxBufs, "TMEM buffers");
+};
 
 struct GemmParams {
     const int32_t* group_offsets;
@@ -50,7 +65,7 @@ struct GemmParams {
     int nkb;
     const float* w_scales;  // [n_groups, n/128, nkb]
     int n;                  // weight rows per group
-    int n_ftiles;           // 256-column tiles per group
+    int n_ftiles;           // BN-column tiles per group
     int epilogue;
     void* out;
     float* out_scales;
@@ -60,8 +75,8 @@ struct GemmParams {
 struct SharedState {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t tfull[kMaxBufs];
+    uint64_t tempty[kMaxBufs];
     uint64_t sfull[kScaleSlots];
     uint64_t sempty[kScaleSlots];
     uint64_t drain;
@@ -71,12 +86,16 @@ struct SharedState {
     int goff[kMaxGroups + 1];
     int gstart[kMaxGroups + 1];
     alignas(16) float sa[kScaleSlots][kBM];   // token scales of one K block
-    alignas(16) float sb[kScaleSlots][2];     // the two weight-block scales
+    alignas(16) float sb[kScaleSlots][2];     // the weight-block scale(s)
     alignas(16) float red[2][2][kBM];         // [item parity][half][token] amax of h
 };
 
-constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + sizeof(SharedState) + 1024;
-static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 limit per CTA");
+template <int BN>
+constexpr size_t smem_bytes() {
+    return size_t(Cfg<BN>::kRingBytes) + Cfg<BN>::kParkBytes + sizeof(SharedState) + 1024;
+}
+static_assert(smem_bytes<256>() <= 232448 && smem_bytes<128>() <= 232448,
+              "dynamic shared memory above the sm_100 limit per CTA");
 
 // ------------------------------------------------------------- PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -192,6 +211,24 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         : "memory");
 }
 
+// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers; the
+// wait for the load is part of the same statement.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
 // 64 consecutive TMEM columns of this warp's 32 lanes -> 64 registers; the
 // wait for the load is part of the same statement.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
@@ -261,10 +298,9 @@ __device__ __forceinline__ void set_max_regs_dec() {
 // ------------------------------------------------------------- schedule
 struct Item {
     int g;      // group
-    int f;      // 256-column tile
+    int f;      // BN-column tile
     int row0;   // first token row
     int ntok;   // valid tokens (<= 128)
-    int ncols;  // MMA N: 256, or 128 for a last half-width tile
 };
 
 __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmParams& p, int item) {
@@ -283,29 +319,31 @@ __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmPar
     const int mt = local - it.f * mtiles;
     it.row0 = ss->goff[lo] + mt * kBM;
     it.ntok = min(kBM, rows - mt * kBM);
-    it.ncols = (p.epilogue == MOE_EPI_SWIGLU_QUANT) ? 256 : min(256, p.n - it.f * 256);
     return it;
 }
 
-// Weight rows of the two 128-row blocks of a tile (first row inside the
-// stacked [n_groups * n, k] matrix) and their block-row indices.
+// 128-row weight block(s) of a tile: first row inside the stacked
+// [n_groups * n, k] matrix and block-row index (for its scales).
+template <int BN>
 __device__ __forceinline__ void weight_blocks(const GemmParams& p, const Item& w, int& r0, int& r1,
                                               int& b0, int& b1) {
-    if (p.epilogue == MOE_EPI_SWIGLU_QUANT) {
+    if (BN == 256) {
         b0 = w.f;                   // gate rows f*128 .. of W1
         b1 = p.n / 256 + w.f;       // up rows (n/2 + f*128) .. of W3
     } else {
-        b0 = 2 * w.f;
-        b1 = 2 * w.f + 1;
+        b0 = w.f;
+        b1 = w.f;
     }
     r0 = w.g * p.n + b0 * 128;
     r1 = w.g * p.n + b1 * 128;
 }
 
 // ================================================= TMA producer (warp 0)
+template <int BN>
 __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap& map_w,
                                          const CUtensorMap& map_a, uint8_t* smem,
                                          SharedState* ss) {
+    using C = Cfg<BN>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     uint32_t it = 0;
@@ -314,21 +352,20 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap&
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
         const Item w = decode_item(ss, p, item);
         int wr0, wr1, b0, b1;
-        weight_blocks(p, w, wr0, wr1, b0, b1);
-        const uint32_t tx = uint32_t(kTileBytes + w.ncols * 128);
+        weight_blocks<BN>(p, w, wr0, wr1, b0, b1);
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
-            const int s = it % kStages;
-            const uint32_t par = ((it / kStages) & 1u);
+            const int s = it % C::kStages;
+            const uint32_t par = ((it / C::kStages) & 1u);
             if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             if (lane == 0) {
-                uint8_t* st = smem + size_t(s) * kStageBytes;
+                uint8_t* st = smem + size_t(s) * C::kStageBytes;
                 const uint32_t fb = smem_u32(&ss->full[s]);
-                mbar_arrive_expect_tx(fb, tx);
+                mbar_arrive_expect_tx(fb, uint32_t(C::kStageBytes));
                 tma_load_2d(smem_u32(st), &map_a, fb, kb * 128, w.row0);
                 tma_load_2d(smem_u32(st + kTileBytes), &map_w, fb, kb * 128, wr0);
-                if (w.ncols == 256)
+                if (BN == 256)
                     tma_load_2d(smem_u32(st + 2 * kTileBytes), &map_w, fb, kb * 128, wr1);
                 issued_mask |= 1u << s;
                 issued_parity = (issued_parity & ~(1u << s)) | (par << s);
@@ -337,7 +374,7 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap&
     }
     if (!ok && lane == 0) {
         // let loads already in flight land before the CTA leaves
-        for (int s = 0; s < kStages; ++s)
+        for (int s = 0; s < C::kStages; ++s)
             if ((issued_mask >> s) & 1u)
                 mbar_wait(smem_u32(&ss->full[s]), (issued_parity >> s) & 1u, ss, nullptr);
     }
@@ -346,8 +383,9 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap&
 
 // ================================================= scale loader (warp 2)
 // cp.async of each K block's 128 token scales (kb-major, so they are
-// contiguous) and the tile's two weight-block scales; the copies arrive on
+// contiguous) and the tile's weight-block scale(s); the copies arrive on
 // sfull when they land.
+template <int BN>
 __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* ss) {
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
@@ -357,9 +395,9 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
     for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
         const Item w = decode_item(ss, p, item);
         int wr0, wr1, b0, b1;
-        weight_blocks(p, w, wr0, wr1, b0, b1);
+        weight_blocks<BN>(p, w, wr0, wr1, b0, b1);
         const float* sb0 = p.w_scales + (size_t(w.g) * nbr + b0) * p.nkb;
-        const float* sb1 = p.w_scales + (size_t(w.g) * nbr + (w.ncols == 256 ? b1 : b0)) * p.nkb;
+        const float* sb1 = p.w_scales + (size_t(w.g) * nbr + b1) * p.nkb;
         for (int kb = 0; kb < p.nkb; ++kb, ++cit) {
             const int c = cit % kScaleSlots;
             if (lane == 0)
@@ -386,26 +424,28 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
 }
 
 // ================================================= MMA issuer (warp 1)
+template <int BN>
 __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, SharedState* ss,
                                            uint32_t tmem_base) {
+    using C = Cfg<BN>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     if (lane == 0) {
         uint32_t it = 0, tb = 0;
         bool ok = true;
+        const uint32_t idesc = idesc_e4m3(128, BN);
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-            const Item w = decode_item(ss, p, item);
-            const uint32_t idesc = idesc_e4m3(128, w.ncols);
             for (int kb = 0; kb < p.nkb; ++kb, ++it, ++tb) {
-                const int s = it % kStages;
-                const uint32_t buf = tb & 1u;
-                ok = mbar_wait(smem_u32(&ss->tempty[buf]), ((tb >> 1) & 1u) ^ 1u, ss, p.dev_status);
+                const int s = it % C::kStages;
+                const uint32_t buf = tb % C::kBufs;
+                const uint32_t tpar = (tb / C::kBufs) & 1u;
+                ok = mbar_wait(smem_u32(&ss->tempty[buf]), tpar ^ 1u, ss, p.dev_status);
                 if (!ok) break;
-                ok = mbar_wait(smem_u32(&ss->full[s]), (it / kStages) & 1u, ss, p.dev_status);
+                ok = mbar_wait(smem_u32(&ss->full[s]), (it / C::kStages) & 1u, ss, p.dev_status);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t st = smem_u32(smem + size_t(s) * kStageBytes);
-                const uint32_t d = tmem_base + buf * 256;
+                const uint32_t st = smem_u32(smem + size_t(s) * C::kStageBytes);
+                const uint32_t d = tmem_base + buf * BN;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_e4m3(d, sw128_desc(st + kk * 32), sw128_desc(st + kTileBytes + kk * 32),
@@ -421,39 +461,58 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
     __syncwarp();
 }
 
+// Parked output of the fp32 / bf16 epilogue: a promoter thread's 64 values
+// (256 bytes) wait in shared memory and move to global memory 16 bytes per K
+// block of the next tile.  Vector j of the parked row -> its global segment.
+__device__ __forceinline__ void unpark_vec(const char* park, char* dst, bool bf16, int j) {
+    if (bf16) {
+        const float4 a = *reinterpret_cast<const float4*>(park + 32 * j);
+        const float4 b = *reinterpret_cast<const float4*>(park + 32 * j + 16);
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y), h1 = __floats2bfloat162_rn(a.z, a.w);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y), h3 = __floats2bfloat162_rn(b.z, b.w);
+        reinterpret_cast<uint4*>(dst)[j] =
+            make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                       *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+    } else {
+        reinterpret_cast<float4*>(dst)[j] = *reinterpret_cast<const float4*>(park + 16 * j);
+    }
+}
+
 // ================================================= promotion + epilogue (warps 4-11)
 // Thread (warp w, lane l) owns token row r = 32*(w%4) + l of the tile and
-// 128 of its 256 columns: half h = (w-4)/4.
-//   SwiGLU: gate columns [64h, 64h+64) and up columns [128+64h, 128+64h+64)
-//           (the same 64 features of W1 and W3), scales s0 and s1;
-//   F32/BF16: columns [128h, 128h+128), scale s_h.
-__device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
+// half h = (w-4)/4 of its columns:
+//   BN = 256 (SwiGLU): gate columns [64h, 64h+64) and up columns
+//     [128+64h, 128+64h+64) (the same 64 features of W1 and W3);
+//   BN = 128: columns [64h, 64h+64) of the single weight block.
+template <int BN>
+__device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, char* park_area,
                                          uint32_t tmem_base) {
+    using C = Cfg<BN>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     const int q = warp & 3;
     const int half = (warp - 4) >> 2;
     const int r = q * 32 + lane;  // token row inside the tile
-    const bool swiglu = p.epilogue == MOE_EPI_SWIGLU_QUANT;
     const uint32_t lane_addr = tmem_base + (uint32_t(q * 32) << 16);
+    const bool bf16_out = p.epilogue == MOE_EPI_BF16;
+    const int c0 = BN == 256 ? half * 64 : half * 64;        // first column of chunk 0
+    const int c1 = BN == 256 ? 128 + half * 64 : half * 64;  // first column of chunk 1
     uint32_t tb = 0, cit = 0, parity = 0;
     bool ok = true;
+    // this thread's parking slot and the global segment it belongs to
+    char* const park = park_area + (threadIdx.x - 128) * kParkStride;
+    char* park_dst = nullptr;
+    const int nvec = bf16_out ? 8 : 16;  // 16-byte global stores per parked segment
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, parity ^= 1u) {
         const Item w = decode_item(ss, p, item);
-        // columns of this thread's four 32-column chunks
-        int col[4];
+        uint64_t acc2[C::kPairs];  // fp32 accumulator pairs
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-            col[ch] = swiglu ? ((ch >> 1) * 128 + half * 64 + (ch & 1) * 32) : (half * 128 + ch * 32);
-        const bool active = swiglu || col[0] < w.ncols;
-        uint64_t acc2[64];  // fp32 accumulator pairs (columns 2i, 2i+1 of the thread)
-#pragma unroll
-        for (int i = 0; i < 64; ++i) acc2[i] = 0;
+        for (int i = 0; i < C::kPairs; ++i) acc2[i] = 0;
         for (int kb = 0; ok && kb < p.nkb; ++kb, ++tb, ++cit) {
-            const uint32_t buf = tb & 1u;
+            const uint32_t buf = tb % C::kBufs;
             const int c = cit % kScaleSlots;
             if (lane == 0) {
-                ok = mbar_wait(smem_u32(&ss->tfull[buf]), (tb >> 1) & 1u, ss, p.dev_status);
+                ok = mbar_wait(smem_u32(&ss->tfull[buf]), (tb / C::kBufs) & 1u, ss, p.dev_status);
                 if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (cit / kScaleSlots) & 1u, ss,
                                        p.dev_status);
             }
@@ -461,70 +520,69 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
             if (!ok) break;
             __syncwarp();
             tc_fence_after();
-            if (active) {
-                const float sa = ss->sa[c][r];
-                const float s0 = sa * ss->sb[c][swiglu ? 0 : half];
-                const float s1 = swiglu ? sa * ss->sb[c][1] : s0;
-                const uint64_t s0x2 = pack2(__float_as_uint(s0), __float_as_uint(s0));
-                const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
+            const float sa = ss->sa[c][r];
+            const float s0 = sa * ss->sb[c][0];
+            const float s1 = sa * ss->sb[c][1];
+            const uint64_t s0x2 = pack2(__float_as_uint(s0), __float_as_uint(s0));
+            const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
+            if (BN == 256) {
                 uint32_t v[64];
-                tmem_ld64(lane_addr + buf * 256 + col[0], v);  // columns col[0], col[1]
+                tmem_ld64(lane_addr + buf * BN + c0, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
-                tmem_ld64(lane_addr + buf * 256 + col[2], v);  // columns col[2], col[3]
+                tmem_ld64(lane_addr + buf * BN + c1, v);
                 // the partial is in registers: hand the TMEM buffer back to
                 // the MMA before the last FMAs
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ffma2(acc2[32 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
+                for (int i = 0; i < 32; ++i)
+                    ffma2(acc2[32 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
             } else {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + buf * BN + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
+                tmem_ld32(lane_addr + buf * BN + c0 + 32, v);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_u32(&ss->sempty[c]));
-                    mbar_arrive(smem_u32(&ss->tempty[buf]));
-                }
+                if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    ffma2(acc2[16 + i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
+                // one 16-byte store of the previous tile's output per K block
+                if (park_dst && kb < nvec) unpark_vec(park, park_dst, bf16_out, kb);
             }
         }
         // ---------------- epilogue
-        float acc[128];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const float2 f = unpack2(acc2[i]);
-            acc[2 * i] = f.x;
-            acc[2 * i + 1] = f.y;
-        }
         const bool row_ok = r < w.ntok;
         const size_t row = size_t(w.row0) + r;
-        if (!swiglu) {
-            if (active && row_ok) {
-                const size_t c0 = size_t(w.f) * 256 + half * 128;
-                if (p.epilogue == MOE_EPI_F32) {
-                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.n + c0);
+        if (BN == 128) {
+            // finish the previous tile's segment, then park this one
+            if (park_dst)
+                for (int j = min(p.nkb, nvec); j < nvec; ++j) unpark_vec(park, park_dst, bf16_out, j);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-                } else {
-                    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row * p.n + c0);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        uint32_t u[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            __nv_bfloat162 b = __floats2bfloat162_rn(acc[8 * i + 2 * j], acc[8 * i + 2 * j + 1]);
-                            u[j] = *reinterpret_cast<uint32_t*>(&b);
-                        }
-                        o[i] = make_uint4(u[0], u[1], u[2], u[3]);
-                    }
-                }
+            for (int i = 0; i < 16; ++i) {
+                const float2 a = unpack2(acc2[2 * i]), b = unpack2(acc2[2 * i + 1]);
+                *reinterpret_cast<float4*>(park + 16 * i) = make_float4(a.x, a.y, b.x, b.y);
             }
+            const size_t col = size_t(w.f) * 128 + half * 64;
+            park_dst = !row_ok ? nullptr
+                      : bf16_out ? reinterpret_cast<char*>(static_cast<__nv_bfloat16*>(p.out) + row * p.n + col)
+                                 : reinterpret_cast<char*>(static_cast<float*>(p.out) + row * p.n + col);
         } else {
             // h = silu(gate) * up for this thread's 64 features, then the
             // 1x128 scale of the token's 128 features (both halves).
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float2 f = unpack2(acc2[i]);
+                acc[2 * i] = f.x;
+                acc[2 * i + 1] = f.y;
+            }
             float amax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
@@ -562,26 +620,31 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss,
             2, kPromoters * 32, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
         if (any_abort) break;
     }
+    if (BN == 128 && park_dst)
+        for (int j = 0; j < nvec; ++j) unpark_vec(park, park_dst, bf16_out, j);
     tc_fence_before();
 }
 
 // ----------------------------------------------------------------- kernel
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                         const __grid_constant__ CUtensorMap map_a, const GemmParams p) {
+    using C = Cfg<BN>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    SharedState* ss = reinterpret_cast<SharedState*>(smem + size_t(kStages) * kStageBytes);
+    SharedState* ss =
+        reinterpret_cast<SharedState*>(smem + size_t(C::kRingBytes) + C::kParkBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // ---- prologue: barriers, TMEM, schedule
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_u32(&ss->full[s]), 1);
             mbar_init(smem_u32(&ss->empty[s]), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::kBufs; ++b) {
             mbar_init(smem_u32(&ss->tfull[b]), 1);
             mbar_init(smem_u32(&ss->tempty[b]), kPromoters);
         }
@@ -657,13 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = ss->tmem_base;
 
     if (warp < 4) {
-        set_max_regs_dec<56>();
-        if (warp == 0) producer(p, map_w, map_a, smem, ss);
-        else if (warp == 1) mma_issuer(p, smem, ss, tmem_base);
-        else if (warp == 2) scale_loader(p, ss);
+        set_max_regs_dec<72>();
+        if (warp == 0) producer<BN>(p, map_w, map_a, smem, ss);
+        else if (warp == 1) mma_issuer<BN>(p, smem, ss, tmem_base);
+        else if (warp == 2) scale_loader<BN>(p, ss);
     } else {
-        set_max_regs_inc<224>();
-        promoter(p, ss, tmem_base);
+        set_max_regs_inc<208>();
+        promoter<BN>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base);
     }
 
     __syncthreads();
@@ -717,11 +780,12 @@ bool device_is_sm100() {
     return major == 10;
 }
 
+template <int BN>
 int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma, cudaStream_t st) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kSmemBytes)) != cudaSuccess)
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem_bytes<BN>())) != cudaSuccess)
         return MOE_ERR_CUDA;
-    grouped_gemm_kernel<<<sm_count(), kThreads, kSmemBytes, st>>>(mw, ma, p);
+    grouped_gemm_kernel<BN><<<sm_count(), kThreads, smem_bytes<BN>(), st>>>(mw, ma, p);
     return check_launch();
 }
 
@@ -759,7 +823,8 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     p.nkb = k / 128;
     p.w_scales = w_scales;
     p.n = n;
-    p.n_ftiles = (n + 255) / 256;
+    const bool swiglu = epilogue == MOE_EPI_SWIGLU_QUANT;
+    p.n_ftiles = swiglu ? n / 256 : n / 128;
     p.epilogue = epilogue;
     p.out = out;
     p.out_scales = out_scales;
@@ -769,5 +834,6 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128) ||
         !make_map(&ma, a, uint64_t(max_rows), uint64_t(k), 128))
         return MOE_ERR_CUDA;
-    return launch(p, mw, ma, as_stream(stream));
+    return swiglu ? launch<256>(p, mw, ma, as_stream(stream))
+                  : launch<128>(p, mw, ma, as_stream(stream));
 }
