@@ -194,8 +194,6 @@ def stage_breakdown(layer, x, off, steps):
     T, d, I, N, K = sh.T, sh.d, sh.inter, sh.n_routed, sh.topk
     R = T * K + T
     dev = x.device
-    xq = torch.empty((T, d), dtype=torch.uint8, device=dev)
-    xs = torch.empty((T, d // 128), dtype=torch.float32, device=dev)
     xq_p = torch.empty((R, d), dtype=torch.uint8, device=dev)
     xs_p = torch.empty((d // 128, R), dtype=torch.float32, device=dev)
     hq = torch.empty((R, I), dtype=torch.uint8, device=dev)
@@ -205,13 +203,12 @@ def stage_breakdown(layer, x, off, steps):
     rws = torch.empty((moe.moe_route_workspace_size(sh),), dtype=torch.uint8, device=dev)
     pws = torch.empty((moe.moe_permute_workspace_size(sh),), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
-    names = ["route", "quant_x", "permute", "gemm1_swiglu", "gemm2", "combine", "update_bias"]
+    names = ["route", "quant_permute", "gemm1_swiglu", "gemm2", "combine", "update_bias"]
     calls = [
         lambda: moe.moe_route(sh, x, layer.router_w, layer.bias, off, layer.topk_idx,
                               layer.topk_gate, layer.expert_counts, rws),
-        lambda: moe.fp8_quant_act_1x128(x, xq, xs),
-        lambda: moe.moe_permute(sh, layer.topk_idx, layer.expert_counts, xq, xs, xq_p, xs_p,
-                                layer.expert_offsets, layer.row_of_pair, pws),
+        lambda: moe.moe_quant_permute(sh, x, layer.topk_idx, layer.expert_counts, xq_p, xs_p,
+                                      layer.expert_offsets, layer.row_of_pair, pws),
         lambda: moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, xq_p, xs_p, d,
                                          layer.w13, layer.w13_scales, 2 * I,
                                          _lib.MOE_EPI_SWIGLU_QUANT, hq, hs, layer.dev_status),
@@ -268,6 +265,276 @@ def oracle_sample_time(cfg, inp, dev, n_tokens, seed=0):
     return dt, n_tokens, os.cpu_count() or 1
 
 
+# ------------------------------------------------------ memory-bound passes
+def memory_passes(cfg, brk, alg, hbm_peak):
+    """Algorithmic bytes / event time of the HBM-bound passes of one step."""
+    T, d, K = cfg.T, cfg.d, cfg.topk
+    nkb = d // 128
+    rows = T * K + T
+    passes = {
+        # bf16 row read once, E4M3 row + 1x128 scales written to K+1 rows
+        "quant_permute": (brk["quant_permute"], T * d * 2 + rows * (d + 4 * nkb)),
+        # fp32 expert rows read (K routed + shared) and gates, bf16 y written
+        "combine": (brk["combine"], rows * d * 4 + T * K * 8 + T * d * 2),
+    }
+    out = {}
+    for name, (ms, nbytes) in passes.items():
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
+    return out
+
+
+def weight_quant_pass(dev, hbm_peak, rows=32768, cols=7168, reps=5):
+    """fp8_quant_w_128x128 timed alone on one [rows, cols] bf16 matrix (the
+    stacked W1/W3 of 8 experts; 0.7 GB moved, above L2)."""
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    w = (torch.randn((rows, cols), generator=g, device=dev) * 0.006).to(torch.bfloat16)
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    sc = torch.empty((rows // 128, cols // 128), dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+    for _ in range(2):
+        moe.fp8_quant_w_128x128(w, q, sc)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(st)
+    for _ in range(reps):
+        moe.fp8_quant_w_128x128(w, q, sc)
+    ev[1].record(st)
+    ev[1].synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / reps
+    nbytes = rows * cols * 3 + 4 * (rows // 128) * (cols // 128)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del w, q, sc
+    return {"ms": ms, "shape": [rows, cols], "bytes": nbytes, "gbs": gbs,
+            "frac_of_hbm": gbs / hbm_peak}
+
+
+# ------------------------------------------------------------ router alone
+FP64_FMA_PER_CLK_SM = 64  # B200 FP64 FMA lanes per SM (37 TFLOP/s at 1965 MHz, 148 SMs)
+
+
+def run_route(args, world, rank, local):
+    """moe_route alone on the prefill batch (T=4096, d=7168, 256 experts):
+    logits, sigmoid, group-limited top-K, gates and histogram.  The logits
+    are T*N_r*d FP64 multiply-adds; the roofline is the FP64 FMA rate from
+    the unit count and the SM clock."""
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    import synthetic as S
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.CONFIGS["prefill"]
+    inp = S.make_layer_inputs_host(cfg, 0)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    x, rw = bf16(inp["x"]), bf16(inp["router_w"])
+    bias = torch.from_numpy(inp["bias"]).to(dev)
+    shape = moe.make_shape(cfg.T, cfg.d, cfg.n_routed, cfg.n_groups, cfg.topk_groups, cfg.topk,
+                           cfg.inter, cfg.gamma)
+    idx = torch.empty((cfg.T, cfg.topk), dtype=torch.int32, device=dev)
+    gate = torch.empty((cfg.T, cfg.topk), dtype=torch.float32, device=dev)
+    counts = torch.empty((cfg.n_routed,), dtype=torch.int32, device=dev)
+    ws = torch.empty((moe.moe_route_workspace_size(shape),), dtype=torch.uint8, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def route(xx=x):
+        moe.moe_route(shape, xx, rw, bias, None, idx, gate, counts, ws, status)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        route()
+    torch.cuda.synchronize()
+    barrier(world)
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(st)
+        route()
+        e1.record(st)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs), world)
+    fma = float(cfg.T) * cfg.n_routed * cfg.d
+    tflops = 2.0 * fma * args.steps * world / (ms / 1e3) / 1e12
+    mhz = (clk or {}).get("sm_mhz") or 1965.0
+    peak = 2.0 * FP64_FMA_PER_CLK_SM * props.multi_processor_count * mhz * 1e6 / 1e12
+    x_h = x.cpu().pin_memory()
+    x_d = torch.empty_like(x)
+    idx_h = torch.empty((cfg.T, cfg.topk), dtype=torch.int32).pin_memory()
+    gate_h = torch.empty((cfg.T, cfg.topk), dtype=torch.float32).pin_memory()
+    e2e_ms = 0.0
+    for it in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        x_d.copy_(x_h, non_blocking=True)
+        route(x_d)
+        idx_h.copy_(idx, non_blocking=True)
+        gate_h.copy_(gate, non_blocking=True)
+        e1.record(st)
+        e1.synchronize()
+        if it >= args.warmup:
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    tok = cfg.T * args.steps * world
+    line = {
+        "metric": METRIC, "value": tok / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "moe_route_prefill", "T": cfg.T, "d": cfg.d,
+                   "n_routed": cfg.n_routed, "n_groups": cfg.n_groups,
+                   "topk_groups": cfg.topk_groups, "topk": cfg.topk,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "256 MB buffer written between timed launches"},
+        "roofline": {"bound": "alu", "kernel": "router logits (FP64 FMA, ascending k)",
+                     "achieved": tflops / world, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / world / peak,
+                     "peak_source": f"{FP64_FMA_PER_CLK_SM} FP64 FMA/clk/SM x "
+                                    f"{props.multi_processor_count} SMs x {mhz:.0f} MHz",
+                     "traffic": None, "algorithmic_fma_per_launch": fma},
+        "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": x.numel() * 2,
+                "d2h_bytes_per_step": idx.numel() * 4 + gate.numel() * 4},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "device_status": int(status.item()),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------- GEMM-alone workload
+def run_gemm(args, world, rank, local):
+    """The FP8 block-scaled GEMM alone: A [4096, 7168] (1x128 scales) times B
+    [7168, 2048] (128x128 scales, stored K-major as [2048, 7168]), bf16 out.
+    One step = one moe_grouped_gemm_fp8 launch (one group); a 256 MB buffer
+    is written between steps (outside the timed events) so each launch reads
+    its operands from HBM."""
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    import synthetic as S
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.GEMM_C2
+    peaks, peak_src = load_peaks()
+    a_bits, b_bits = S.make_gemm_inputs_host(cfg)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    a, b = bf16(a_bits), bf16(b_bits)
+    aq = torch.empty((cfg.m, cfg.k), dtype=torch.uint8, device=dev)
+    as_ = torch.empty((cfg.k // 128, cfg.m), dtype=torch.float32, device=dev)
+    bq = torch.empty((cfg.n, cfg.k), dtype=torch.uint8, device=dev)
+    bs = torch.empty((cfg.n // 128, cfg.k // 128), dtype=torch.float32, device=dev)
+    moe.fp8_quant_act_1x128(a, aq, as_, scales_kb_major=True)
+    moe.fp8_quant_w_128x128(b, bq, bs)
+    off = torch.tensor([0, cfg.m], dtype=torch.int32, device=dev)
+    out = torch.empty((cfg.m, cfg.n), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def gemm(a_codes=aq, a_scales=as_, c=out):
+        moe.moe_grouped_gemm_fp8(1, off, cfg.m, a_codes, a_scales, cfg.k, bq, bs, cfg.n,
+                                 moe.MOE_EPI_BF16, c, None, status)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        gemm()
+    torch.cuda.synchronize()
+    barrier(world)
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(st)
+        gemm()
+        e1.record(st)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs), world)
+    flops = 2.0 * cfg.m * cfg.n * cfg.k
+    tflops = flops * args.steps * world / (ms / 1e3) / 1e12
+    fp8_peak = float(peaks["bf16_tflops"]) * FP8_PER_BF16
+
+    # end to end: A's codes and scales from pinned host memory, C back to it
+    aq_h, as_h = aq.cpu().pin_memory(), as_.cpu().pin_memory()
+    c_h = torch.empty((cfg.m, cfg.n), dtype=torch.bfloat16).pin_memory()
+    aq_d, as_d = torch.empty_like(aq), torch.empty_like(as_)
+    e2e_ms = 0.0
+    for it in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        aq_d.copy_(aq_h, non_blocking=True)
+        as_d.copy_(as_h, non_blocking=True)
+        gemm(aq_d, as_d, out)
+        c_h.copy_(out, non_blocking=True)
+        e1.record(st)
+        e1.synchronize()
+        if it >= args.warmup:
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8e4m3/f32", "data": "synthetic",
+        "config": {"workload": "fp8_blockscaled_gemm", "m": cfg.m, "n": cfg.n, "k": cfg.k,
+                   "out": "bf16", "parallelism": f"replicas x{world}",
+                   "l2": "256 MB buffer written between timed launches"},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<1> (one group, bf16 out)",
+                     "achieved": tflops / world, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": tflops / world / fp8_peak,
+                     "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g} (nominal fp8:bf16)",
+                     "traffic": profiled_traffic("gemm_blockscaled_4096x7168x2048"),
+                     "algorithmic_flops_per_launch": flops, "launch_ms": ms / args.steps},
+        "e2e": {"value": flops * args.steps * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": aq.numel() + as_.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "device_status": int(status.item()),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n_rows = 16
+        qa, sa = oracle.quant_act_1x128(a_bits[:n_rows])
+        qb, sb = oracle.quant_w_128x128(b_bits)
+        t0 = time.perf_counter()
+        oracle.gemm_blockscaled(qa, sa, qb, sb)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {
+            "value": 2.0 * n_rows * cfg.n * cfg.k / dt / 1e12, "unit": "TFLOP/s",
+            "cores": os.cpu_count() or 1, "kind": "oracle",
+            "sample": f"{n_rows} rows of A times all of B (operands pre-quantised by the oracle)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------- main
 def dist_setup():
     import torch
@@ -310,6 +577,10 @@ def run_reference(args, world, rank):
     import synthetic as S
     if rank != 0:
         return
+    if args.workload == "gemm":
+        return run_reference_gemm(args)
+    if args.workload == "route":
+        return run_reference_route(args)
     cfg = S.CONFIGS[args.workload]
     dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
     inp = S.make_layer_inputs_host(cfg, 0)
@@ -340,6 +611,71 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_route(args, n_tok=64):
+    """The oracle's routing on n_tok tokens of the prefill batch per step."""
+    import oracle
+    import synthetic as S
+    cfg = S.CONFIGS["prefill"]
+    inp = S.make_layer_inputs_host(cfg, 0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0_ = (i * n_tok) % cfg.T
+        xs = inp["x"][t0_:t0_ + n_tok]
+        t0 = time.perf_counter()
+        oracle.route(xs, inp["router_w"], inp["bias"], cfg.n_groups, cfg.topk_groups, cfg.topk)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = n_tok * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "moe_route_prefill", "T": cfg.T, "d": cfg.d,
+                   "n_routed": cfg.n_routed, "sample_tokens_per_step": n_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count() or 1,
+                         "kind": "oracle", "sample": f"{n_tok} tokens per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_gemm(args, n_rows=16):
+    """The oracle's block-scaled GEMM on n_rows rows of A per step (operands
+    quantised by the oracle beforehand, untimed)."""
+    import oracle
+    import synthetic as S
+    cfg = S.GEMM_C2
+    a_bits, b_bits = S.make_gemm_inputs_host(cfg)
+    qb, sb = oracle.quant_w_128x128(b_bits)
+    times = []
+    for i in range(args.warmup + args.steps):
+        r0 = (i * n_rows) % cfg.m
+        qa, sa = oracle.quant_act_1x128(a_bits[r0:r0 + n_rows])
+        t0 = time.perf_counter()
+        oracle.gemm_blockscaled(qa, sa, qb, sb)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = 2.0 * n_rows * cfg.n * cfg.k * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "fp8_blockscaled_gemm", "m": cfg.m, "n": cfg.n, "k": cfg.k,
+                   "out": "bf16", "sample_rows_per_step": n_rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count() or 1,
+                         "kind": "oracle",
+                         "sample": f"{n_rows} rows of A per step times all of B"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     import numpy as np
     import torch
@@ -353,10 +689,17 @@ def run_ours(args, world, rank, local):
     layer, x, off, inp, wq_ms = build_layer(cfg, dev)
     st = torch.cuda.current_stream()
     y = torch.empty_like(x)
+    bias0 = layer.bias.clone()
+    # successive batches (the skewed workload has 8; step i routes batch
+    # i mod 8 with the bias left by step i-1)
+    batches = [x] + [torch.from_numpy(np.ascontiguousarray(
+        S.make_layer_inputs_host(cfg, j)["x"]).view(np.int16)).view(torch.bfloat16).to(dev)
+        for j in range(1, cfg.batches)]
+    nb = len(batches)
 
     # ---- warm-up, then K timed steps of the whole layer (inputs in HBM)
-    for _ in range(args.warmup):
-        layer.forward(x, y, update_bias=True, logit_offset=off)
+    for i in range(args.warmup):
+        layer.forward(batches[i % nb], y, update_bias=True, logit_offset=off)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -366,8 +709,8 @@ def run_ours(args, world, rank, local):
     clocks.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(st)
-    for _ in range(args.steps):
-        layer.forward(x, y, update_bias=True, logit_offset=off)
+    for i in range(args.steps):
+        layer.forward(batches[i % nb], y, update_bias=True, logit_offset=off)
     ev1.record(st)
     ev1.synchronize()
     clk = clocks.stop()
@@ -380,20 +723,29 @@ def run_ours(args, world, rank, local):
     value = tokens_total / (ms / 1e3)
 
     # ---- end to end through the host-buffer entry point (pinned memory)
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty_like(x_host).pin_memory()
-    for _ in range(max(1, args.warmup // 2)):
-        layer.forward_host(x_host, y_host, update_bias=True, logit_offset=off)
+    hosts = [b.cpu().pin_memory() for b in batches]
+    y_host = torch.empty_like(hosts[0]).pin_memory()
+    for i in range(max(1, args.warmup // 2)):
+        layer.forward_host(hosts[i % nb], y_host, update_bias=True, logit_offset=off)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
-    for _ in range(args.steps):
-        layer.forward_host(x_host, y_host, update_bias=True, logit_offset=off)
+    for i in range(args.steps):
+        layer.forward_host(hosts[i % nb], y_host, update_bias=True, logit_offset=off)
     e1.record(st)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     xbytes = cfg.T * cfg.d * 2
+
+    # ---- per-batch expert load from the initial bias, batches in order
+    # (untimed): max / mean of the counts each batch is routed with
+    layer.bias.copy_(bias0)
+    per_batch = []
+    for j in range(nb):
+        layer.forward(batches[j], y, update_bias=True, logit_offset=off)
+        c = layer.expert_counts.cpu().numpy()
+        per_batch.append(round(float(c.max() / max(c.mean(), 1e-9)), 4))
 
     # ---- per-stage breakdown (CUDA events on the launching stream)
     brk = stage_breakdown(layer, x, off, args.steps)
@@ -439,13 +791,15 @@ def run_ours(args, world, rank, local):
                         "flops_per_step": alg["layer_flops"]},
         "layer_tflops": layer_tflops,
         "breakdown_ms": brk,
-        "weight_quant": {"ms_total": wq_ms,
-                         "gbs": (cfg.n_routed + 1) * 3 * cfg.d * cfg.inter * 3 / (wq_ms / 1e3) / 1e9},
+        "weight_quant": weight_quant_pass(dev, hbm_peak),
+        "memory_passes": memory_passes(cfg, brk, alg, hbm_peak),
         "load": {"max_over_mean": float(counts.max() / max(counts.mean(), 1e-9)),
+                 "max_over_mean_per_batch": per_batch,
                  "experts_touched": alg["touched"]},
         "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes},
-        "gpu_launches": 11 * args.steps,
+        # route 2, quant+permute 4, GEMMs 2, combine 1, bias update 1
+        "gpu_launches": 10 * args.steps,
         "clocks": clk,
         "device_status": status,
     }
@@ -466,7 +820,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill", choices=["tiny", "prefill", "decode", "skewed", "prefill_e16"])
+    ap.add_argument("--workload", default="prefill",
+                    choices=["tiny", "prefill", "decode", "skewed", "prefill_e16", "gemm",
+                             "route"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -475,6 +831,10 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.workload == "gemm":
+            run_gemm(args, world, rank, local)
+        elif args.workload == "route":
+            run_route(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "moe_permute_workspace_size": (SZ, [SP]),
             "moe_permute": (I, [SP, P, P, P, P, P, P, P, P, P, SZ, P, P]),
             "moe_permute_static_ws": (I, [SP, P, P, P, P, P, P, P, P, P, P]),
+            "moe_quant_permute": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
             "moe_grouped_gemm_fp8": (I, [I, P, I, P, P, I, P, P, I, I, P, P, P, P]),
             "moe_combine": (I, [SP, P, P, P, P, P, P, P]),
             "moe_update_bias": (I, [SP, P, P, P, P]),
@@ -166,6 +167,16 @@ def moe_permute(shape, topk_idx, expert_counts, xq, xs, xq_perm, xs_perm, expert
     _check("moe_permute", lib().moe_permute(
         ctypes.byref(shape), _ptr(topk_idx), _ptr(expert_counts), _ptr(xq), _ptr(xs),
         _ptr(xq_perm), _ptr(xs_perm), _ptr(expert_offsets), _ptr(row_of_pair), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_quant_permute(shape, x, topk_idx, expert_counts, xq_perm, xs_perm, expert_offsets,
+                      row_of_pair, ws, dev_status=None, stream=None):
+    """fp8_quant_act_1x128 of x (bf16 [T, d]) fused with moe_permute."""
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("moe_quant_permute", lib().moe_quant_permute(
+        ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(expert_counts), _ptr(xq_perm),
+        _ptr(xs_perm), _ptr(expert_offsets), _ptr(row_of_pair), _ptr(ws), nbytes,
         _ptr(dev_status), _stream(stream)))
 
 

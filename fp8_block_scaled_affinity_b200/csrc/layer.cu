@@ -27,8 +27,6 @@ namespace {
 
 // Workspace of the layer: every piece starts on a 256-byte boundary.
 struct LayerWs {
-    uint8_t* xq;       // [T, d]
-    float* xs;         // [T, d/128]
     uint8_t* xq_perm;  // [R, d]      R = T*K + T
     float* xs_perm;    // [d/128, R]
     uint8_t* hq;       // [R, I]
@@ -52,8 +50,6 @@ LayerWs carve(const MoeShape* s, void* base, bool host_io) {
         off = align_up(off + bytes, 256);
         return reinterpret_cast<void*>(p + at);
     };
-    w.xq = static_cast<uint8_t*>(take(T * d));
-    w.xs = static_cast<float*>(take(T * (d / 128) * 4));
     w.xq_perm = static_cast<uint8_t*>(take(R * d));
     w.xs_perm = static_cast<float*>(take((d / 128) * R * 4));
     w.hq = static_cast<uint8_t*>(take(R * I));
@@ -78,11 +74,9 @@ int run_layer(const MoeShape* s, const MoeWeights* wt, const uint16_t* x, float*
                        rt->expert_counts, w.route_ws, moe_route_workspace_size(s), dev_status,
                        stream);
     if (rc != MOE_OK) return rc;
-    rc = fp8_quant_act_1x128(x, T, d, w.xq, w.xs, 0, dev_status, stream);
-    if (rc != MOE_OK) return rc;
-    rc = moe_permute(s, rt->topk_idx, rt->expert_counts, w.xq, w.xs, w.xq_perm, w.xs_perm,
-                     rt->expert_offsets, rt->row_of_pair, w.perm_ws,
-                     moe_permute_workspace_size(s), dev_status, stream);
+    rc = moe_quant_permute(s, x, rt->topk_idx, rt->expert_counts, w.xq_perm, w.xs_perm,
+                           rt->expert_offsets, rt->row_of_pair, w.perm_ws,
+                           moe_permute_workspace_size(s), dev_status, stream);
     if (rc != MOE_OK) return rc;
     if (T > 0) {
         rc = moe_grouped_gemm_fp8(N + 1, rt->expert_offsets, R, w.xq_perm, w.xs_perm, d,

@@ -104,34 +104,45 @@ __global__ void __launch_bounds__(256) chunk_scan_kernel(const int32_t* __restri
 
 // One warp per chunk: tokens in ascending order; lane k < K takes slot k of
 // the token (the K experts of a token are distinct, so no two lanes touch
-// the same cursor in one step).
+// the same cursor in one step).  The chunk's expert ids and the experts' row
+// limits are staged in shared memory first, so the serial walk touches no
+// global memory except the row_of_pair stores.
 __global__ void __launch_bounds__(32) chunk_rank_kernel(const int32_t* __restrict__ topk_idx,
                                                         int T, int K, int n_routed,
                                                         const int32_t* __restrict__ chunk_base,
                                                         const int32_t* __restrict__ offsets,
                                                         int32_t* __restrict__ row_of_pair,
                                                         int* dev_status) {
-    extern __shared__ int cursor[];
+    extern __shared__ int rank_smem[];
+    int* cursor = rank_smem;              // [n_routed]
+    int* limit = rank_smem + n_routed;    // [n_routed]
+    int* ids = rank_smem + 2 * n_routed;  // [kChunk * K]
     const int lane = threadIdx.x;
     const int c = blockIdx.x;
-    for (int i = lane; i < n_routed; i += 32) cursor[i] = chunk_base[int64_t(c) * n_routed + i];
+    const int t0 = c * kChunk, t1 = min(T, t0 + kChunk);
+    for (int i = lane; i < n_routed; i += 32) {
+        cursor[i] = chunk_base[int64_t(c) * n_routed + i];
+        limit[i] = offsets[i + 1];
+    }
+    for (int p = lane; p < (t1 - t0) * K; p += 32) ids[p] = topk_idx[int64_t(t0) * K + p];
     __syncwarp();
-    const int t1 = min(T, (c + 1) * kChunk);
-    for (int t = c * kChunk; t < t1; ++t) {
+    bool bad = false;
+    for (int t = t0; t < t1; ++t) {
         if (lane < K) {
-            const int e = topk_idx[int64_t(t) * K + lane];
+            const int e = ids[(t - t0) * K + lane];
             int row = -1;
             if (e >= 0 && e < n_routed) {
                 row = cursor[e];
                 cursor[e] = row + 1;
                 // expert_counts inconsistent with topk_idx: no row to give
-                if (row >= offsets[e + 1]) row = -1;
+                if (row >= limit[e]) row = -1;
             }
-            if (row < 0) set_status(dev_status, MOE_DEV_BAD_INPUT);
+            bad |= row < 0;
             row_of_pair[int64_t(t) * K + lane] = row;
         }
         __syncwarp();
     }
+    if (bad) set_status(dev_status, MOE_DEV_BAD_INPUT);
 }
 
 // One warp per token; the row is read once, 4 KB at a time (8 x 16 bytes
@@ -173,6 +184,69 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(
             if (row < 0) continue;
             for (int kb = lane; kb < nkb; kb += 32)
                 xs_perm[int64_t(kb) * rows_total + row] = xs[int64_t(t) * nkb + kb];
+        }
+    }
+}
+
+// moe_quant_permute's copy: one warp per token reads the token's bf16 row
+// once (16-byte loads, kPiece per lane in flight), quantises each 1x128 tile
+// exactly as fp8_quant_act_1x128 does (a half-warp owns one tile: amax by
+// shuffles, scale rule of quant.cu, RN products, satfinite E4M3) and writes
+// the codes and the scale K+1 times (routed rows and the shared row).
+__global__ void __launch_bounds__(256) quant_copy_rows_kernel(
+    const uint4* __restrict__ x, int T, int d, int K, const int32_t* __restrict__ row_of_pair,
+    int64_t rows_total, uint2* __restrict__ xq_perm, float* __restrict__ xs_perm) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = d / 8, nkb = d / 128;  // 8 bf16 in, 8 codes out per vector
+    const int warps_total = gridDim.x * (blockDim.x / 32);
+    for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        int my_row = 0;
+        if (lane < K) my_row = row_of_pair[int64_t(t) * K + lane];
+        const int shared_row = T * K + t;
+        const uint4* src = x + int64_t(t) * nvec;
+        for (int c0 = 0; c0 < nvec; c0 += 32 * kPiece) {
+            uint4 v[kPiece];
+#pragma unroll
+            for (int j = 0; j < kPiece; ++j) {
+                const int c = c0 + lane + 32 * j;
+                v[j] = c < nvec ? __ldcs(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            uint2 code[kPiece];
+            float tile_scale = 1.0f;  // lane L < 16: scale of tile c0/16 + L
+#pragma unroll
+            for (int j = 0; j < kPiece; ++j) {
+                const uint4 w = v[j];
+                const float f[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                    bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                float scale, inv;
+                scale_from_amax(amax, scale, inv);
+                const uint32_t c0_ = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv));
+                const uint32_t c1_ = e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
+                const uint32_t c2_ = e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv));
+                const uint32_t c3_ = e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv));
+                code[j] = make_uint2(c0_ | (c1_ << 16), c2_ | (c3_ << 16));
+                // piece j holds tiles 2j (lanes 0-15) and 2j+1 (lanes 16-31)
+                const float sj = __shfl_sync(0xffffffffu, scale, (lane & 1) * 16);
+                if ((lane >> 1) == j) tile_scale = sj;
+            }
+            const int tile = c0 / 16 + lane;
+            for (int k = 0; k <= K; ++k) {
+                const int row = (k < K) ? __shfl_sync(0xffffffffu, my_row, k) : shared_row;
+                if (row < 0) continue;
+                uint2* dst = xq_perm + int64_t(row) * nvec;
+#pragma unroll
+                for (int j = 0; j < kPiece; ++j) {
+                    const int c = c0 + lane + 32 * j;
+                    if (c < nvec) dst[c] = code[j];
+                }
+                if (lane < 16 && tile < nkb) xs_perm[int64_t(tile) * rows_total + row] = tile_scale;
+            }
         }
     }
 }
@@ -239,44 +313,87 @@ extern "C" MOE_API size_t moe_permute_workspace_size(const MoeShape* shape) {
     return align_up(size_t(n_chunks_of(shape->T)) * shape->n_routed * sizeof(int32_t) + 256, 256);
 }
 
-extern "C" MOE_API int moe_permute(const MoeShape* shape, const int32_t* topk_idx,
-                                   const int32_t* expert_counts, const uint8_t* xq,
-                                   const float* xs, uint8_t* xq_perm, float* xs_perm,
-                                   int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
-                                   size_t ws_bytes, int* dev_status, void* stream) {
-    (void)dev_status;
-    int rc = validate_shape(shape);
-    if (rc != MOE_OK) return rc;
-    const int T = shape->T, d = shape->d, K = shape->topk, N = shape->n_routed;
-    if (!expert_counts || !expert_offsets) return MOE_ERR_NULL;
-    cudaStream_t st = as_stream(stream);
+namespace moe {
+namespace {
+
+// Steps 1-3 of the permutation (offsets and row_of_pair); returns the
+// status.  T > 0 is checked by the caller.
+int build_rows(const MoeShape* shape, const int32_t* topk_idx, const int32_t* expert_counts,
+               int32_t* expert_offsets, int32_t* row_of_pair, int32_t* chunk_counts,
+               int* dev_status, cudaStream_t st) {
+    const int T = shape->T, K = shape->topk, N = shape->n_routed;
     const int n_chunks = n_chunks_of(T);
+    int rc;
     if (T > 0) {
-        if (!topk_idx || !xq || !xs || !xq_perm || !xs_perm || !row_of_pair) return MOE_ERR_NULL;
-        if (!aligned16(xq) || !aligned16(xq_perm)) return MOE_ERR_ALIGN;
-        if (!ws || ws_bytes < moe_permute_workspace_size(shape)) return MOE_ERR_WORKSPACE;
-    }
-    int32_t* chunk_counts = static_cast<int32_t*>(ws);
-    const size_t hist_smem = sizeof(int) * N;
-    if (T > 0) {
-        chunk_hist_kernel<<<n_chunks, 256, hist_smem, st>>>(topk_idx, T, K, N, chunk_counts,
-                                                            dev_status);
+        chunk_hist_kernel<<<n_chunks, 256, sizeof(int) * N, st>>>(topk_idx, T, K, N,
+                                                                   chunk_counts, dev_status);
         if ((rc = check_launch()) != MOE_OK) return rc;
     }
     chunk_scan_kernel<<<N, 256, 0, st>>>(expert_counts, T, K, N, n_chunks, chunk_counts,
                                          expert_offsets);
     if ((rc = check_launch()) != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
-    chunk_rank_kernel<<<n_chunks, 32, hist_smem, st>>>(topk_idx, T, K, N, chunk_counts,
+    const size_t rank_smem = sizeof(int) * (2 * size_t(N) + size_t(kChunk) * K);
+    chunk_rank_kernel<<<n_chunks, 32, rank_smem, st>>>(topk_idx, T, K, N, chunk_counts,
                                                        expert_offsets, row_of_pair, dev_status);
-    if ((rc = check_launch()) != MOE_OK) return rc;
-    const int64_t rows_total = int64_t(T) * K + T;
+    return check_launch();
+}
+
+int copy_grid(int T) {
     int blocks = (T + 7) / 8;
     const int cap = sm_count() * 8;
-    if (blocks > cap) blocks = cap;
-    copy_rows_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(xq), xs, T, d, K,
-                                             row_of_pair, rows_total,
-                                             reinterpret_cast<uint4*>(xq_perm), xs_perm);
+    return blocks > cap ? cap : blocks;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" MOE_API int moe_permute(const MoeShape* shape, const int32_t* topk_idx,
+                                   const int32_t* expert_counts, const uint8_t* xq,
+                                   const float* xs, uint8_t* xq_perm, float* xs_perm,
+                                   int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
+                                   size_t ws_bytes, int* dev_status, void* stream) {
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T, d = shape->d, K = shape->topk;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_NULL;
+    if (T > 0) {
+        if (!topk_idx || !xq || !xs || !xq_perm || !xs_perm || !row_of_pair) return MOE_ERR_NULL;
+        if (!aligned16(xq) || !aligned16(xq_perm)) return MOE_ERR_ALIGN;
+        if (!ws || ws_bytes < moe_permute_workspace_size(shape)) return MOE_ERR_WORKSPACE;
+    }
+    cudaStream_t st = as_stream(stream);
+    rc = build_rows(shape, topk_idx, expert_counts, expert_offsets, row_of_pair,
+                    static_cast<int32_t*>(ws), dev_status, st);
+    if (rc != MOE_OK || T == 0) return rc;
+    copy_rows_kernel<<<copy_grid(T), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(xq), xs, T, d, K, row_of_pair, int64_t(T) * K + T,
+        reinterpret_cast<uint4*>(xq_perm), xs_perm);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_quant_permute(const MoeShape* shape, const uint16_t* x,
+                                         const int32_t* topk_idx, const int32_t* expert_counts,
+                                         uint8_t* xq_perm, float* xs_perm,
+                                         int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
+                                         size_t ws_bytes, int* dev_status, void* stream) {
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T, d = shape->d, K = shape->topk;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_NULL;
+    if (T > 0) {
+        if (!topk_idx || !x || !xq_perm || !xs_perm || !row_of_pair) return MOE_ERR_NULL;
+        if (!aligned16(x) || !aligned16(xq_perm) || (reinterpret_cast<uintptr_t>(xs_perm) & 3))
+            return MOE_ERR_ALIGN;
+        if (!ws || ws_bytes < moe_permute_workspace_size(shape)) return MOE_ERR_WORKSPACE;
+    }
+    cudaStream_t st = as_stream(stream);
+    rc = build_rows(shape, topk_idx, expert_counts, expert_offsets, row_of_pair,
+                    static_cast<int32_t*>(ws), dev_status, st);
+    if (rc != MOE_OK || T == 0) return rc;
+    quant_copy_rows_kernel<<<copy_grid(T), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(x), T, d, K, row_of_pair, int64_t(T) * K + T,
+        reinterpret_cast<uint2*>(xq_perm), xs_perm);
     return check_launch();
 }
 

@@ -9,41 +9,56 @@ namespace moe {
 namespace {
 
 // One 1x128 tile per 16 threads; each thread owns 8 consecutive bf16 values
-// (one 16-byte load, one 8-byte store).  Grid-strides over tiles.
+// (one 16-byte load, one 8-byte store) of kActUnroll tiles at a time, whose
+// loads are all issued before any is used, so each thread keeps several
+// loads in flight.  Grid-strides over tiles.
+constexpr int kActUnroll = 4;
+
 __global__ void __launch_bounds__(256) quant_act_1x128_kernel(
     const uint4* __restrict__ x, int64_t rows, int64_t cols, uint2* __restrict__ q,
     float* __restrict__ scales, int kb_major) {
     const int64_t tiles_per_row = cols >> 7;
     const int64_t n_tiles = rows * tiles_per_row;
     const int sub = threadIdx.x & 15;
-    // Both half-warps iterate together (the shuffles span the full warp);
-    // a half-warp past the last tile computes on zeros and stores nothing.
+    // Both half-warps iterate together (the shuffles span the full warp; the
+    // stride is even, so the two tiles of a warp stay a pair); a half-warp
+    // past the last tile computes on zeros and stores nothing.
     int64_t tile = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
     const int64_t tile_stride = (int64_t(gridDim.x) * blockDim.x) >> 4;
-    for (; (tile & ~int64_t(1)) < n_tiles; tile += tile_stride) {
-        const bool valid = tile < n_tiles;
-        const int64_t r = valid ? tile / tiles_per_row : 0;
-        const int64_t t = valid ? tile - r * tiles_per_row : 0;
-        const int64_t vec = (r * cols + (t << 7)) / 8 + sub;
-        uint4 w = valid ? __ldcs(x + vec) : make_uint4(0u, 0u, 0u, 0u);
-        float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-        float amax = 0.0f;
+    for (; (tile & ~int64_t(1)) < n_tiles; tile += kActUnroll * tile_stride) {
+        uint4 w[kActUnroll];
+        int64_t vec[kActUnroll], r[kActUnroll], t[kActUnroll];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        for (int u = 0; u < kActUnroll; ++u) {
+            const int64_t tt = tile + u * tile_stride;
+            const bool valid = tt < n_tiles;
+            r[u] = valid ? tt / tiles_per_row : -1;
+            t[u] = valid ? tt - r[u] * tiles_per_row : 0;
+            vec[u] = valid ? (r[u] * cols + (t[u] << 7)) / 8 + sub : 0;
+            w[u] = valid ? __ldcs(x + vec[u]) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        float scale, inv;
-        scale_from_amax(amax, scale, inv);
-        uint32_t c0 = e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv));
-        uint32_t c1 = e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv));
-        uint32_t c2 = e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv));
-        uint32_t c3 = e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
-        if (!valid) continue;
-        q[vec] = make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
-        if (sub == 0) {
-            if (kb_major) scales[t * rows + r] = scale;
-            else scales[r * tiles_per_row + t] = scale;
+        for (int u = 0; u < kActUnroll; ++u) {
+            float v[8] = {bf16_lo(w[u].x), bf16_hi(w[u].x), bf16_lo(w[u].y), bf16_hi(w[u].y),
+                          bf16_lo(w[u].z), bf16_hi(w[u].z), bf16_lo(w[u].w), bf16_hi(w[u].w)};
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            float scale, inv;
+            scale_from_amax(amax, scale, inv);
+            uint32_t c0 = e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv));
+            uint32_t c1 = e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv));
+            uint32_t c2 = e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv));
+            uint32_t c3 = e4m3x2(__fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+            if (r[u] < 0) continue;
+            q[vec[u]] = make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
+            if (sub == 0) {
+                if (kb_major) scales[t[u] * rows + r[u]] = scale;
+                else scales[r[u] * tiles_per_row + t[u]] = scale;
+            }
         }
     }
 }
@@ -121,7 +136,7 @@ extern "C" MOE_API int fp8_quant_act_1x128(const uint16_t* x, int64_t rows, int6
         return MOE_ERR_ALIGN;
     if (scales_kb_major != 0 && scales_kb_major != 1) return MOE_ERR_ARG;
     const int64_t threads = rows * (cols / 128) * 16;
-    int64_t blocks = (threads + 255) / 256;
+    int64_t blocks = (threads + 256 * kActUnroll - 1) / (256 * kActUnroll);
     const int64_t cap = int64_t(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
     quant_act_1x128_kernel<<<unsigned(blocks), 256, 0, as_stream(stream)>>>(

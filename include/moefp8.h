@@ -178,6 +178,21 @@ MOE_API int moe_permute(const MoeShape* shape, const int32_t* topk_idx,
                         int32_t* row_of_pair, void* ws, size_t ws_bytes, int* dev_status,
                         void* stream);
 
+/* moe_quant_permute: fp8_quant_act_1x128 of x fused with moe_permute.  The
+ * token rows are read once in bf16 and each 1x128 tile is quantised (same
+ * scale rule and rounding as fp8_quant_act_1x128) straight into the K + 1
+ * destination rows, so the unpermuted codes are never written to memory
+ * ("FP8 mixed precision training": activations are quantised online, per
+ * 1x128 tile, before they are dispatched).
+ *   x                         bf16 [T, d] (16-byte aligned)
+ *   other arguments           as moe_permute (ws of moe_permute_workspace_size)
+ * Bit-exact contract: equal to fp8_quant_act_1x128 followed by moe_permute.
+ * Errors: as moe_permute. */
+MOE_API int moe_quant_permute(const MoeShape* shape, const uint16_t* x, const int32_t* topk_idx,
+                              const int32_t* expert_counts, uint8_t* xq_perm, float* xs_perm,
+                              int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
+                              size_t ws_bytes, int* dev_status, void* stream);
+
 /* moe_permute_static_ws: moe_permute for callers that cannot allocate
  * device memory while they run (a serving loop whose memory budget is fixed
  * at start-up, a host framework that owns all device memory through its own
@@ -275,7 +290,8 @@ typedef struct {
     int32_t* row_of_pair;     /* [T, K] */
 } MoeRouting;
 
-/* moe_layer_forward: route -> quantise x (1x128) -> permute -> grouped GEMM
+/* moe_layer_forward: route -> quantise x (1x128) + permute (one pass,
+ * moe_quant_permute) -> grouped GEMM
  * (W13, SwiGLU + 1x128 quantisation of h) -> grouped GEMM (W2, fp32) ->
  * combine -> (optionally) bias update, all on `stream`.
  *   x            bf16 [T, d];  y bf16 [T, d] out

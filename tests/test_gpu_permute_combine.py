@@ -67,6 +67,52 @@ def test_permute_bit_exact(T, N, K, d, skew):
     assert np.array_equal(ps.view(np.uint32), exp_s.view(np.uint32))
 
 
+def gpu_quant_permute(shape, idx, counts, x_bits):
+    import fp8_block_scaled_affinity_b200 as moe
+    T, K, N, d = shape.T, shape.topk, shape.n_routed, shape.d
+    R = T * K + T
+    xq_perm = torch.full((max(R, 1), d), 0xEE, dtype=torch.uint8, device=DEV)
+    xs_perm = torch.full((d // 128, max(R, 1)), -1.0, dtype=torch.float32, device=DEV)
+    off = torch.full((N + 2,), -1, dtype=torch.int32, device=DEV)
+    rop = torch.full((max(T, 1), K), -1, dtype=torch.int32, device=DEV)
+    ws = torch.empty((moe.moe_permute_workspace_size(shape),), dtype=torch.uint8, device=DEV)
+    x = torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).to(DEV)
+    moe.moe_quant_permute(shape, x, to_dev(idx), to_dev(counts), xq_perm, xs_perm, off, rop, ws)
+    torch.cuda.synchronize()
+    return (xq_perm.cpu().numpy()[:R], xs_perm.cpu().numpy()[:, :R], off.cpu().numpy(),
+            rop.cpu().numpy()[:T])
+
+
+@pytest.mark.parametrize("T,N,K,d,skew", [(1, 16, 4, 128, False), (257, 16, 4, 512, False),
+                                          (1000, 256, 8, 7168, True), (130, 64, 1, 2176, False),
+                                          (64, 32, 32, 128, False)])
+def test_quant_permute_bit_exact(T, N, K, d, skew):
+    """The fused pass (bf16 rows quantised 1x128 straight into their K + 1
+    destinations) against the oracle's quantiser and permutation: codes,
+    scales, offsets and row_of_pair bit for bit.  d = 2176 (17 tiles) leaves a
+    ragged last group of tiles in every row."""
+    need_gpu()
+    rng = np.random.default_rng(T * 7 + N + K)
+    idx, counts = _routing(T, N, K, rng, skew)
+    x = S.host_normal_bf16(rng, (T, d), 1.0)
+    x[0, :128] = 0  # an all-zero tile: scale 1, codes 0
+    xq, xs = oracle.quant_act_1x128(x)
+    import fp8_block_scaled_affinity_b200 as moe
+    shape = moe.make_shape(T, d, N, 1, 1, K, 128)
+    pq, ps, off, rop = gpu_quant_permute(shape, idx, counts, x)
+    off_ref, rop_ref = oracle.permute_layout(idx, counts, N)
+    assert np.array_equal(off, off_ref)
+    assert np.array_equal(rop, rop_ref)
+    src = np.concatenate([np.repeat(np.arange(T), K), np.arange(T)])
+    rows = np.concatenate([rop_ref.ravel(), T * K + np.arange(T)])
+    exp_q = np.empty_like(pq)
+    exp_q[rows] = xq[src]
+    exp_s = np.empty_like(ps)
+    exp_s[:, rows] = xs[src].T
+    assert np.array_equal(pq, exp_q)
+    assert np.array_equal(ps.view(np.uint32), exp_s.view(np.uint32))
+
+
 def test_permute_empty_batch():
     import fp8_block_scaled_affinity_b200 as moe
     need_gpu()

@@ -69,6 +69,66 @@ def test_ties_go_to_lower_index():
     assert idx.tolist() == [[0, 1, 2]] * 3
 
 
+def _compare_arrays(x, E, bias, G, M, K, offset=None):
+    import fp8_block_scaled_affinity_b200 as moe
+    T, d = x.shape
+    N = E.shape[0]
+    shape = moe.make_shape(T, d, N, G, M, K, 128)
+    idx, gate, counts = gpu_route(shape, x, E, bias, offset)
+    ref = oracle.route(x, E, bias, G, M, K, logit_offset=offset)
+    assert np.array_equal(idx, ref["topk_idx"])
+    assert np.array_equal(gate.view(np.uint32), ref["topk_gate"].view(np.uint32))
+    assert np.array_equal(counts, ref["counts"])
+    return ref
+
+
+@pytest.mark.parametrize("T", [200, 700])
+def test_fully_tied_router(T):
+    """A zero router: every logit is 0 and every biased score ties, so no
+    token's choice can be decided from bounds; every token gets all of its
+    logits from the defining FP64 sums (one sum per thread for a short list,
+    FP64 tiles for a long one) and the ties go to the lower indices."""
+    need_gpu()
+    rng = np.random.default_rng(T)
+    x = S.host_normal_bf16(rng, (T, 256), 1.0)
+    E = np.zeros((64, 256), np.uint16)
+    ref = _compare_arrays(x, E, np.zeros(64, np.float32), 8, 2, 6)
+    assert (ref["topk_idx"] == np.arange(6)).all()
+
+
+def test_duplicated_router_rows():
+    """Pairs of identical router rows with equal biases tie exactly; tokens
+    whose K-th and (K+1)-th choices are such a pair need the exact path,
+    the others are decided from bounds."""
+    need_gpu()
+    rng = np.random.default_rng(11)
+    T, d, N = 512, 384, 64
+    x = S.host_normal_bf16(rng, (T, d), 1.0)
+    E = S.host_normal_bf16(rng, (N, d), 0.05)
+    E[1::2] = E[0::2]
+    bias = S.host_uniform_f32(rng, (N,), 0.02)
+    bias[1::2] = bias[0::2]
+    _compare_arrays(x, E, bias, 4, 2, 5)
+
+
+def test_huge_cancelling_entries():
+    """Entries near 1e30 times router entries near 3e8: the products reach
+    the top of the fp32 range (their fp32 bound is useless, so the tokens go
+    to the exact path) and cancel exactly in the FP64 sum, which must widen
+    both factors to FP64 before multiplying."""
+    need_gpu()
+    rng = np.random.default_rng(5)
+    T, d, N = 64, 256, 32
+    xf = rng.standard_normal((T, d)).astype(np.float32)
+    xf[:, 0], xf[:, 1] = 1e30, -1e30
+    Ef = (rng.standard_normal((N, d)) * 0.05).astype(np.float32)
+    c = rng.uniform(1.7e8, 3.0e8, N).astype(np.float32)
+    Ef[:, 0] = c
+    Ef[:, 1] = c
+    x, E = S.f32_to_bf16_bits(xf), S.f32_to_bf16_bits(Ef)
+    _compare_arrays(x, E, S.host_uniform_f32(rng, (N,), 0.02), 4, 2, 4)
+
+
 @pytest.mark.parametrize("T", [1, 37, 256])
 def test_tiny_workload(T):
     need_gpu()

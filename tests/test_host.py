@@ -72,6 +72,12 @@ def test_validation_before_any_cuda_call(moe):
     assert L.moe_grouped_gemm_fp8(1, 1, 1, 1, 1, 128, 1, 1, 128, 2, 1, None, None, None) == -2
     assert L.moe_grouped_gemm_fp8(0, 1, 1, 1, 1, 128, 1, 1, 128, 0, 1, None, None, None) == -2
     assert L.moe_grouped_gemm_fp8(1, None, 1, 1, 1, 128, 1, 1, 128, 0, 1, None, None, None) == -1
+    # fused quantise + permute: missing x, misaligned x, missing workspace
+    s = moe.make_shape(4, 128, 16, 4, 2, 4, 128)
+    sp = ctypes.byref(s)
+    assert L.moe_quant_permute(sp, None, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None, None) == -1
+    assert L.moe_quant_permute(sp, 8, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None, None) == -5
+    assert L.moe_quant_permute(sp, 16, 16, 16, 16, 16, 16, 16, None, 0, None, None) == -6
 
 
 def test_workspace_sizes(moe):
@@ -81,8 +87,11 @@ def test_workspace_sizes(moe):
     assert moe.moe_route_workspace_size(s) >= T * N * 4
     assert moe.moe_permute_workspace_size(s) >= (T // 64) * N * 4
     ws = moe.moe_layer_workspace_size(s)
-    need = T * d + T * d // 32 + R * d + R * d // 32 + R * I + R * I // 32 + R * d * 4
-    assert need <= ws <= need + 64 * 1024 + T * N * 4 + (T // 64 + 1) * N * 4 + 4096
+    # permuted codes + scales, h codes + scales, fp32 expert outputs (x is
+    # quantised straight into its permuted rows: no unpermuted copy)
+    need = R * d + R * d // 32 + R * I + R * I // 32 + R * d * 4
+    scratch = moe.moe_route_workspace_size(s) + moe.moe_permute_workspace_size(s)
+    assert need + scratch <= ws <= need + scratch + 64 * 1024
     assert moe.moe_layer_host_workspace_size(s) >= ws + 2 * T * d * 2
     assert moe.moe_layer_workspace_size(moe.make_shape(4, 128, 10, 3, 1, 2, 128)) == 0
 
