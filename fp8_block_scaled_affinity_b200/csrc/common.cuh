@@ -30,6 +30,9 @@ int sm_count();
 // Validates a MoE shape; returns MOE_OK or an error code.
 int validate_shape(const MoeShape* s);
 
+// True when the current device is an sm_100 part.
+bool device_is_sm100();
+
 // --------------------------------------------------------------- device
 __device__ __forceinline__ void set_status(int* st, int code) {
     if (st) atomicCAS(st, 0, code);

@@ -737,7 +737,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+template <int BN>
+int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma, cudaStream_t st) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem_bytes<BN>())) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    grouped_gemm_kernel<BN><<<sm_count(), kThreads, smem_bytes<BN>(), st>>>(mw, ma, p);
+    return check_launch();
+}
+
+}  // namespace
+
 // ------------------------------------------------------------------ host
+// Tensor maps and the device check (declared in common.cuh; the router uses
+// them too).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -780,16 +793,6 @@ bool device_is_sm100() {
     return major == 10;
 }
 
-template <int BN>
-int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma, cudaStream_t st) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem_bytes<BN>())) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    grouped_gemm_kernel<BN><<<sm_count(), kThreads, smem_bytes<BN>(), st>>>(mw, ma, p);
-    return check_launch();
-}
-
-}  // namespace
 }  // namespace moe
 
 using namespace moe;

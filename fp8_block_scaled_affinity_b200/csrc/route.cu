@@ -7,56 +7,54 @@
 // training"): a logit is the FP64 dot product summed in ascending k, rounded
 // to fp32, so the result is reproducible bit for bit.
 //
-// Computing all T*N_r logits that way is FP64-bound.  The path here
-// computes them cheaply with a rigorous error bound, decides the routing
-// from the bounds wherever they decide it, and evaluates the defining FP64
-// sum only where it is needed:
-//   1. route_norms_kernel: ||x_t||_2, ||E_i||_2 and the range of |values| of
-//      every row;
-//   2. route_approx_kernel: u~ = fp32 sums over blocks of 32 k (packed fp32
-//      FMA), the block sums added in FP64.  Each product of two bf16 values
-//      is exact in fp32, so |u~ - u_def| <= c * ||x_t|| * ||E_i|| + tiny,
-//      c = gamma_31 (fp32) + FP64 terms (Cauchy-Schwarz on sum |x_k E_k|);
-//   3. route_certify_kernel (warp per token): intervals for every biased
-//      score s' from that bound (sigmoid is 1/4-Lipschitz; fp32 roundings
-//      are bounded), the group / top-K choice on the interval centres, and
-//      a check that every chosen interval lies strictly above every rejected
-//      one.  Then the chosen set equals the set the definition chooses.
-//      Tokens that fail the check go on a list;
-//   4. route_exact_pairs_kernel: the defining FP64 sum for the K chosen
-//      logits of every certified token and, when the list is short, for all
-//      N_r logits of every listed token (one sum per thread);
-//      route_logits_list_kernel does the listed tokens in 64x64 FP64 tiles
-//      when the list is long;
+// Computing all T*N_r logits that way is FP64-bound.  The path here gets
+// them from exact integer arithmetic on the tensor cores, decides the
+// routing from the result wherever a rigorous bound allows, and evaluates
+// the defining FP64 sum only where it is still needed:
+//   1. route_slice_kernel: every row v (of x and of E) is written as
+//      v = 2^(sigma-28) * (X0*2^21 + X1*2^14 + X2*2^7 + X3) + r with signed
+//      7-bit digits X0..X3 (int8 planes), sigma the exponent of max |v|;
+//      r = 0 unless the row has values below 2^(sigma-21) of its maximum.
+//      Also ||v||_1, ||v||_2 and the exactness of the row;
+//   2. route_imma_kernel: tcgen05.mma kind::i8 over the digit planes, the
+//      16 plane products summed per level L = s + r into seven exact int32
+//      TMEM accumulators; sum_k X_k E_k = sum_L 2^(7(6-L)) acc_L;
+//   3. route_certify_kernel (warp per token): u~ from the levels (exact up to
+//      one FP64 rounding when both rows are exact); a bound B on the distance
+//      to the defining FP64 sum (the rows' remainders, gamma_d(FP64) *
+//      ||x|| ||E||, the FP64 roundings); intervals for every biased score s'
+//      (sigmoid is 1/4-Lipschitz; fp32 roundings are bounded); the group /
+//      top-K choice on the interval centres and a check that every chosen
+//      interval lies strictly above every rejected one.  Certified tokens get
+//      their chosen logits as fp32(u~) when [u~-B, u~+B] holds no fp32
+//      rounding boundary; others go on a list;
+//   4. route_exact_pairs_kernel: the defining FP64 sum for the chosen
+//      logits that were not settled in 3 and, when the list is short, for
+//      all N_r logits of every listed token (one sum per thread);
+//      route_logits_list_kernel does listed tokens in 64x64 FP64 tiles when
+//      the list is long;
 //   5. route_select_kernel (warp per token): exact s and s' of the chosen
 //      experts, slot order, gates and histogram for certified tokens; the
 //      full selection on the exact logits for listed ones.
 #include <float.h>
 #include <math.h>
 
-#include "common.cuh"
+#include "tc.cuh"
 
 namespace moe {
 namespace {
 
 // --------------------------------------------------------------- helpers
-// bf16 pair (one 32-bit word) -> fp32 values
-__device__ __forceinline__ uint64_t pack2f(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void unpack2f(uint64_t v, float& a, float& b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ void fma2(uint64_t& d, uint64_t a, uint64_t b) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    const uint64_t zero = 0;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(zero));
-    return d;
+// Index checks of the routing kernels: an out-of-range index is skipped and
+// reported (dev_status = MOE_DEV_BAD_INPUT; check[2*site] = 1 and
+// check[2*site+1] = the offending value).  Sites: 0 list overflow, 1 list
+// length, 2 pair index, 3 listed token, 4 chosen expert (certified path),
+// 5 chosen expert (full path).
+constexpr int kCheckWords = 16;
+
+__device__ __forceinline__ void route_bad(int* dev_status, int32_t* check, int site, int value) {
+    set_status(dev_status, MOE_DEV_BAD_INPUT);
+    if (atomicCAS(&check[2 * site], 0, 1) == 0) check[2 * site + 1] = value;
 }
 
 // bf16 word pair -> doubles (exact)
@@ -95,185 +93,292 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// ------------------------------------------------------------ 1. row norms
-// One warp per row; rows [0, T) are tokens, [T, T+N) router rows.
-//   norm[r] = sqrt(sum v^2) in FP64, raised by the factor (1 + nmargin) that
-//             covers its rounding;
-//   vmax[r] = max |v| (+inf if the row holds a non-finite value);
-//   vmin[r] = min |v| over v != 0 (FLT_MAX for an all-zero row).
-// Block 0 also clears the list counter of this call.
-__global__ void __launch_bounds__(256) route_norms_kernel(const uint16_t* __restrict__ x,
-                                                          const uint16_t* __restrict__ E, int T,
-                                                          int N, int d, double nmargin,
-                                                          double* __restrict__ norm,
-                                                          float* __restrict__ vmax,
-                                                          float* __restrict__ vmin,
-                                                          int32_t* __restrict__ list_count) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) *list_count = 0;
+// ------------------------------------------------------ 1. digit planes
+// One warp per row; rows [0, T) are tokens (planes xp), [T, T+N) router rows
+// (planes ep).  Plane s of a row set holds digit X_s of every value, planes
+// stacked as [4][rows][d] int8.  Per row r:
+//   rsc[r] = 2^(sigma-28), the unit of the integer X;
+//   rex[r] = 1 when every value is exactly 2^(sigma-28) * X, 0 when some
+//            value has bits below that unit, -1 when the row holds a
+//            non-finite value;
+//   r1[r] = sum |v - 2^(sigma-28) X| (the truncated remainders), l2[r] =
+//            ||v||_2 (FP64, raised by 1 + nmargin to cover their rounding);
+//   vmax[r], vmin[r] = max |v| (+inf for a non-finite row) and min |v| over
+//            v != 0 (FLT_MAX for an all-zero row).
+// Block 0 also clears the two list counters and the check words of this call.
+__global__ void __launch_bounds__(256) route_slice_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d,
+    double nmargin, int8_t* __restrict__ xp, int8_t* __restrict__ ep, double* __restrict__ rsc,
+    int32_t* __restrict__ rex, double* __restrict__ r1, double* __restrict__ l2,
+    float* __restrict__ vmax, float* __restrict__ vmin, int32_t* __restrict__ list_count,
+    int32_t* __restrict__ pair_count, int32_t* __restrict__ check) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *list_count = 0;
+        *pair_count = 0;
+    }
+    if (blockIdx.x == 0 && threadIdx.x < kCheckWords) check[threadIdx.x] = 0;
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (blockDim.x >> 5);
     for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T + N; r += warps) {
-        const uint4* row = reinterpret_cast<const uint4*>(r < T ? x + int64_t(r) * d
-                                                                : E + int64_t(r - T) * d);
-        double ss = 0.0;
+        const bool is_x = r < T;
+        const int rr = is_x ? r : r - T;
+        const int nrows = is_x ? T : N;
+        const uint4* row = reinterpret_cast<const uint4*>((is_x ? x : E) + int64_t(rr) * d);
+        int8_t* planes = is_x ? xp : ep;
         float mx = 0.0f, mn = FLT_MAX;
+        bool finite = true;
         for (int v = lane; v < d / 8; v += 32) {
             const uint4 w = __ldg(row + v);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float f = h ? bf16_hi(ws[q]) : bf16_lo(ws[q]);
-                    const float a = fabsf(f);
-                    mx = (a <= FLT_MAX) ? fmaxf(mx, a) : INFINITY;
-                    if (a > 0.0f) mn = fminf(mn, a);
-                    ss = fma((double)f, (double)f, ss);
-                }
+                const float a = fabsf(bf16_lo(ws[q])), b = fabsf(bf16_hi(ws[q]));
+                finite = finite && a <= FLT_MAX && b <= FLT_MAX;
+                mx = fmaxf(mx, fmaxf(a, b));
+                if (a > 0.0f) mn = fminf(mn, a);
+                if (b > 0.0f) mn = fminf(mn, b);
             }
+        }
+        mx = warp_max(mx);
+        mn = warp_min(mn);
+        finite = __all_sync(0xffffffffu, finite);
+        int sigma = 0;
+        if (finite && mx > 0.0f) frexpf(mx, &sigma);  // mx < 2^sigma
+        const double unit_inv = ldexp(1.0, 28 - sigma);
+        bool exact = finite;
+        double s1 = 0.0, s2 = 0.0;
+        for (int v = lane; v < d / 8; v += 32) {
+            const uint4 w = __ldg(row + v);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            uint32_t dg[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float f = (q & 1) ? bf16_hi(ws[q >> 1]) : bf16_lo(ws[q >> 1]);
+                s2 = fma((double)f, (double)f, s2);
+                const double xd = finite ? (double)f * unit_inv : 0.0;
+                const int X = __double2int_rz(xd);  // |X| < 2^28
+                exact = exact && (double)X == xd;
+                s1 += fabs(xd - (double)X);  // exact: a remainder below one unit
+                const int x0 = X / (1 << 21);
+                int rem = X - x0 * (1 << 21);
+                const int x1 = rem / (1 << 14);
+                rem -= x1 * (1 << 14);
+                const int x2 = rem / (1 << 7);
+                const int x3 = rem - x2 * (1 << 7);
+                const int digit[4] = {x0, x1, x2, x3};
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    dg[s][q >> 2] |= (uint32_t(digit[s]) & 0xFFu) << (8 * (q & 3));
+            }
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                reinterpret_cast<uint2*>(planes + (int64_t(s) * nrows + rr) * d)[v] =
+                    make_uint2(dg[s][0], dg[s][1]);
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
-            ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, o);
         }
+        exact = __all_sync(0xffffffffu, exact);
         if (lane == 0) {
-            norm[r] = sqrt(ss) * (1.0 + nmargin);
-            vmax[r] = mx;
+            vmax[r] = finite ? mx : INFINITY;
             vmin[r] = mn;
+            rsc[r] = ldexp(1.0, sigma - 28);
+            rex[r] = finite ? (exact ? 1 : 0) : -1;
+            r1[r] = ldexp(s1, sigma - 28) * (1.0 + nmargin);
+            l2[r] = sqrt(s2) * (1.0 + nmargin);
         }
     }
 }
 
-// -------------------------------------------------------- 2. approx logits
-// Tile of 32 tokens x 32 experts per CTA of one warp; lane (ty, tx) =
-// (lane / 4, lane % 4) owns tokens 4ty..4ty+3 and experts 8tx..8tx+7.  K is
-// walked in blocks of 32: the block's x and E slices are staged in shared
-// memory as fp32 (x duplicated into pairs for the packed FMA), the block
-// sum starts from the exact first product and takes 31 packed fp32 FMAs,
-// and is then added to an FP64 accumulator.  blockIdx.z splits K into
-// gridDim.z ranges of whole blocks; with more than one range the partial
-// sums are added atomically (any order: only the bound matters here).
-constexpr int kAT = 32, kAE = 32, kAK = 32;
+// --------------------------------------------------- 2. integer logits
+// One CTA per (128 tokens, 64 experts, K range): the four digit planes of
+// both operands are streamed by TMA in 128-k stages (two stages in flight);
+// one thread issues 16 plane products x 4 MMAs (M=128, N=64, K=32) per
+// stage into seven TMEM accumulators (level L = s + r at columns 64L), and
+// the four warps move the levels out: stored, or added atomically when K is
+// split (integer addition: exact in any order).  Rows past T or N read other
+// rows' digits or zeros and are never stored.
+constexpr int kIM = 128, kIN = 64, kIK = 128, kIStages = 2, kLevels = 7;
+constexpr int kIPlaneA = kIM * kIK, kIPlaneB = kIN * kIK;   // bytes per plane tile
+constexpr int kIStageBytes = 4 * kIPlaneA + 4 * kIPlaneB;   // 96 KB
 
-__global__ void __launch_bounds__(32) route_approx_kernel(const uint16_t* __restrict__ x,
-                                                          const uint16_t* __restrict__ E, int T,
-                                                          int N, int d, int blocks_per_split,
-                                                          double* __restrict__ uhat) {
-    __shared__ __align__(16) uint64_t xs[kAK][kAT];  // (x, x) pairs
-    __shared__ __align__(16) float es[kAK][kAE];
-    const int lane = threadIdx.x, ty = lane >> 2, tx = lane & 3;
-    const int t0 = blockIdx.x * kAT, e0 = blockIdx.y * kAE;
-    const int nblk = d / kAK;
-    const int b0 = blockIdx.z * blocks_per_split;
-    const int b1 = min(nblk, b0 + blocks_per_split);
-    if (b0 >= b1) return;
-    // loader: lane stages x row t0 + lane and router row e0 + lane
-    const bool xrow_ok = t0 + lane < T, erow_ok = e0 + lane < N;
-    const uint4* xp = reinterpret_cast<const uint4*>(x + int64_t(t0 + lane) * d);
-    const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e0 + lane) * d);
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    uint4 xv[4], ev[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        xv[i] = xrow_ok ? __ldg(xp + b0 * 4 + i) : zero;
-        ev[i] = erow_ok ? __ldg(ep + b0 * 4 + i) : zero;
+struct ImmaShared {
+    uint64_t full[kIStages];
+    uint64_t empty[kIStages];
+    uint64_t done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kImmaSmem = size_t(kIStages) * kIStageBytes + 1024 + sizeof(ImmaShared) + 64;
+
+__global__ void __launch_bounds__(128, 1) route_imma_kernel(
+    const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_e, int T,
+    int N, int nchunks, int chunks_per_split, int32_t* __restrict__ acc, int* dev_status) {
+    extern __shared__ __align__(1024) uint8_t imma_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(imma_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    ImmaShared* ss = reinterpret_cast<ImmaShared*>(smem + size_t(kIStages) * kIStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kIM, e0 = blockIdx.y * kIN;
+    const int c0 = blockIdx.z * chunks_per_split;
+    const int c1 = min(nchunks, c0 + chunks_per_split);
+    if (c0 >= c1) return;  // uniform over the CTA
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kIStages; ++i) {
+            tc::mbar_init(tc::smem_u32(&ss->full[i]), 1);
+            tc::mbar_init(tc::smem_u32(&ss->empty[i]), 1);
+        }
+        tc::mbar_init(tc::smem_u32(&ss->done), 1);
+        ss->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    double acc64[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc64[i][j] = 0.0;
-    for (int b = b0; b < b1; ++b) {
-        __syncwarp();  // the previous block's reads of the tile are done
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
-            const uint32_t ew[4] = {ev[i].x, ev[i].y, ev[i].z, ev[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int kk = 8 * i + 2 * j;
-                const float xl = bf16_lo(xw[j]), xh = bf16_hi(xw[j]);
-                xs[kk][lane] = pack2f(xl, xl);
-                xs[kk + 1][lane] = pack2f(xh, xh);
-                es[kk][lane] = bf16_lo(ew[j]);
-                es[kk + 1][lane] = bf16_hi(ew[j]);
-            }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                         tc::smem_u32(&ss->tmem_base))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = ss->tmem_base;
+    if (warp == 0 && lane == 0) {
+        // producer
+        int issued = 0;
+        for (int c = c0; c < c1; ++c, ++issued) {
+            const int st = issued % kIStages;
+            if (issued >= kIStages &&
+                !tc::mbar_wait(tc::smem_u32(&ss->empty[st]), ((issued / kIStages) - 1) & 1,
+                               &ss->abort, dev_status))
+                break;
+            const uint32_t bar = tc::smem_u32(&ss->full[st]);
+            tc::mbar_arrive_expect_tx(bar, kIStageBytes);
+            uint8_t* stage = smem + size_t(st) * kIStageBytes;
+            for (int s = 0; s < 4; ++s)
+                tc::tma_load_2d(tc::smem_u32(stage + s * kIPlaneA), &map_x, bar, c * kIK,
+                                s * T + t0);
+            for (int r = 0; r < 4; ++r)
+                tc::tma_load_2d(tc::smem_u32(stage + 4 * kIPlaneA + r * kIPlaneB), &map_e, bar,
+                                c * kIK, r * N + e0);
         }
-        __syncwarp();
-        if (b + 1 < b1) {
+        // the copies of the last stages have landed before the CTA moves on
+        for (int i = max(0, issued - kIStages); i < issued; ++i)
+            tc::mbar_wait(tc::smem_u32(&ss->full[i % kIStages]), (i / kIStages) & 1, &ss->abort,
+                          dev_status);
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer
+        const uint32_t idesc = tc::idesc_s8(kIM, kIN);
+        for (int c = c0, i = 0; c < c1; ++c, ++i) {
+            const int st = i % kIStages;
+            if (!tc::mbar_wait(tc::smem_u32(&ss->full[st]), (i / kIStages) & 1, &ss->abort,
+                               dev_status))
+                break;
+            tc::fence_after();
+            const uint32_t a0 = tc::smem_u32(smem + size_t(st) * kIStageBytes);
+            const uint32_t b0 = a0 + 4 * kIPlaneA;
+            for (int s = 0; s < 4; ++s)
+                for (int r = 0; r < 4; ++r) {
+                    const int L = s + r;
+                    const bool first_of_level = (s == (L > 3 ? L - 3 : 0));
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                xv[i] = xrow_ok ? __ldg(xp + (b + 1) * 4 + i) : zero;
-                ev[i] = erow_ok ? __ldg(ep + (b + 1) * 4 + i) : zero;
-            }
-        }
-        uint64_t acc[4][4];
-#pragma unroll
-        for (int k = 0; k < kAK; ++k) {
-            const ulonglong2 xa = *reinterpret_cast<const ulonglong2*>(&xs[k][4 * ty]);
-            const ulonglong2 xb = *reinterpret_cast<const ulonglong2*>(&xs[k][4 * ty + 2]);
-            const ulonglong2 ea = *reinterpret_cast<const ulonglong2*>(&es[k][8 * tx]);
-            const ulonglong2 eb = *reinterpret_cast<const ulonglong2*>(&es[k][8 * tx + 4]);
-            const uint64_t xr[4] = {xa.x, xa.y, xb.x, xb.y};
-            const uint64_t er[4] = {ea.x, ea.y, eb.x, eb.y};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (k == 0) acc[i][j] = mul2(xr[i], er[j]);
-                    else fma2(acc[i][j], xr[i], er[j]);
+                    for (int kk = 0; kk < kIK / 32; ++kk) {
+                        const uint32_t accumulate = (i == 0 && kk == 0 && first_of_level) ? 0u : 1u;
+                        tc::mma_s8(tmem + uint32_t(L * kIN),
+                                   tc::sw128_desc(a0 + s * kIPlaneA + kk * 32),
+                                   tc::sw128_desc(b0 + r * kIPlaneB + kk * 32), idesc, accumulate);
+                    }
                 }
+            tc::commit(tc::smem_u32(&ss->empty[st]));
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float a, c;
-                unpack2f(acc[i][j], a, c);
-                acc64[i][2 * j] += (double)a;
-                acc64[i][2 * j + 1] += (double)c;
-            }
+        tc::commit(tc::smem_u32(&ss->done));  // after every MMA issued above
     }
-    const bool split = gridDim.z > 1;
+    __syncwarp();
+    // levels out: warp w holds TMEM lanes (tokens) 32w .. 32w+31
+    bool ok = tc::mbar_wait(tc::smem_u32(&ss->done), 0, &ss->abort, dev_status) &&
+              !*reinterpret_cast<volatile int*>(&ss->abort);
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+    tc::fence_after();
+    if (ok) {
+        const int t = t0 + warp * 32 + lane;
+        const bool split = gridDim.z > 1;
+        for (int L = 0; L < kLevels; ++L) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t0 + 4 * ty + i;
-        if (t >= T) continue;
+            for (int c = 0; c < kIN; c += 16) {
+                uint32_t v[16];
+                tc::tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + uint32_t(L * kIN + c), v);
+                if (t < T) {
+                    int32_t* dst = acc + (int64_t(L) * T + t) * N + e0 + c;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = e0 + 8 * tx + j;
-            if (e >= N) continue;
-            double* dst = uhat + int64_t(t) * N + e;
-            if (split) atomicAdd(dst, acc64[i][j]);
-            else *dst = acc64[i][j];
+                    for (int j = 0; j < 16; ++j) {
+                        if (e0 + c + j >= N) break;
+                        if (split) atomicAdd(dst + j, int32_t(v[j]));
+                        else dst[j] = int32_t(v[j]);
+                    }
+                }
+            }
         }
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem)
+                     : "memory");
     }
 }
 
 // ---------------------------------------------------------- 3. certify
-// One warp per token.  For expert i, with u~ the approximation and
-//   B  = cbound * ||x_t|| * ||E_i|| + 2^-23 |u~| + tiny   (>= |u~ - u_def|),
-// the biased score s'_i of the definition lies within delta_i of
+// One warp per token.  u~ = 2^(sigma_t + sigma_i - 56) * sum_L 2^(7(6-L)) acc_L
+// is the exact sum of the rows' integer parts up to one FP64 rounding;
+//   B = r1(x_t) max|E_i| + r1(E_i) max|x_t| + gamma_d(FP64) ||x_t||_2 ||E_i||_2
+//       + 2^-52 |u~| + tiny
+// bounds |u~ - u_def| before u_def's fp32 rounding (the slicing remainders:
+// sum |r_k E_k| + sum |X_k rho_k| with r1 the remainder sums; the error of
+// the defining FP64 sum; the roundings of u~ and of u~ +- B).  The biased score s'_i of the definition lies within delta_i of
 // centre_i = sigma(u~ + off_i) + b_i, where
 //   delta_i = B'/4 + 2^-23 + 2^-24 |b_i| + 1e-14,
 //   B' = B + 2^-23 (|u~| + |off_i| + B)
-// (B' covers the two fp32 roundings of u and of u + off; sigma is
-// 1/4-Lipschitz; 2^-23 + 2^-24 |b_i| covers the fp32 roundings of s and
-// s + b; 1e-14 the FP64 evaluation of sigma).  The interval ends are stored
-// rounded outwards to fp32.  Groups and experts are chosen on the centres;
-// the choice is certified when the lowest chosen lower end is strictly above
-// the highest rejected upper end, for the groups and then for the experts
-// inside the chosen groups.
+// (B' adds the fp32 roundings of u and of u + off; sigma is 1/4-Lipschitz;
+// 2^-23 + 2^-24 |b_i| covers the fp32 roundings of s and s + b; 1e-14 the
+// FP64 evaluation of sigma).  The interval ends are stored rounded outwards
+// to fp32.  Groups and experts are chosen on the centres; the choice is
+// certified when the lowest chosen lower end is strictly above the highest
+// rejected upper end, for the groups and then for the experts inside the
+// chosen groups.  A certified token's chosen logit is fp32(u~) when
+// u~ - B and u~ + B round to the same fp32 value; otherwise (t, slot) goes
+// on the pair list, to be summed.
 constexpr int kCertWarps = 8;
 
+__device__ __forceinline__ double level_sum(const int32_t* __restrict__ acc, int64_t plane,
+                                            int64_t at) {
+    const int64_t hi = int64_t(acc[at]) * (1 << 14) + int64_t(acc[plane + at]) * (1 << 7) +
+                       int64_t(acc[2 * plane + at]);
+    const int64_t lo = int64_t(acc[3 * plane + at]) * (1 << 21) +
+                       int64_t(acc[4 * plane + at]) * (1 << 14) +
+                       int64_t(acc[5 * plane + at]) * (1 << 7) + int64_t(acc[6 * plane + at]);
+    return (double)hi * 0x1p28 + (double)lo;
+}
+
+__device__ __forceinline__ double logit_bound(double u, int t, int i, int T,
+                                              const double* __restrict__ r1,
+                                              const double* __restrict__ l2,
+                                              const float* __restrict__ vmax, double gamma64) {
+    return r1[t] * (double)vmax[T + i] + r1[T + i] * (double)vmax[t] +
+           gamma64 * l2[t] * l2[T + i] + 0x1p-52 * fabs(u) + 1e-300;
+}
+
 __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
-    const double* __restrict__ uhat, const double* __restrict__ norm,
-    const float* __restrict__ bias, const float* __restrict__ logit_offset, int T, int N,
-    int n_groups, int topk_groups, int topk, double cbound, double tiny,
-    int32_t* __restrict__ cand, int32_t* __restrict__ cert, int32_t* __restrict__ list,
-    int32_t* __restrict__ list_count) {
+    const int32_t* __restrict__ acc, const double* __restrict__ rsc,
+    const int32_t* __restrict__ rex, const double* __restrict__ r1,
+    const double* __restrict__ l2, const float* __restrict__ vmax, const float* __restrict__ bias,
+    const float* __restrict__ logit_offset, int T, int N, int n_groups, int topk_groups,
+    int topk, double gamma64, int32_t* __restrict__ cand, int32_t* __restrict__ cert,
+    float* __restrict__ u_exact, int32_t* __restrict__ list, int32_t* __restrict__ list_count,
+    int32_t* __restrict__ pair_list, int32_t* __restrict__ pair_count, int* dev_status,
+    int32_t* __restrict__ check) {
     extern __shared__ __align__(16) float cert_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float* cen = cert_smem + warp * 3 * N;
@@ -281,17 +386,17 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
     float* hi = lo + N;
     const int t = blockIdx.x * kCertWarps + warp;
     if (t >= T) return;  // no block-wide barrier below
-    const double nx = norm[t];
-    bool fin = true;
+    const int64_t plane = int64_t(T) * N;
+    bool fin = rex[t] >= 0;
     for (int i = lane; i < N; i += 32) {
-        const double u = uhat[int64_t(t) * N + i];
+        const double u = level_sum(acc, plane, int64_t(t) * N + i) * rsc[t] * rsc[T + i];
         const double off = logit_offset ? (double)logit_offset[i] : 0.0;
         const double b = (double)bias[i];
-        const double B = cbound * nx * norm[T + i] + 0x1p-23 * fabs(u) + tiny;
+        const double B = logit_bound(u, t, i, T, r1, l2, vmax, gamma64);
         const double Bp = B + 0x1p-23 * (fabs(u) + fabs(off) + B);
         const double c = 1.0 / (1.0 + exp(-(u + off))) + b;
         const double delta = 0.25 * Bp + 0x1p-23 + 0x1p-24 * fabs(b) + 1e-14;
-        fin = fin && isfinite(c) && isfinite(delta);
+        fin = fin && rex[T + i] >= 0 && isfinite(c) && isfinite(delta);
         cen[i] = __double2float_rn(c);
         lo[i] = __double2float_rd(c - delta);
         hi[i] = __double2float_ru(c + delta);
@@ -363,10 +468,29 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
         const bool all_chosen = __all_sync(0xffffffffu, lane >= topk || my_idx < N);
         ok = ok && all_chosen && (chosen_lo > rej_hi);
     }
-    if (lane < topk) cand[int64_t(t) * topk + lane] = ok ? my_idx : -1;
+    if (lane < topk) {
+        cand[int64_t(t) * topk + lane] = ok ? my_idx : -1;
+        if (ok) {
+            const double u =
+                level_sum(acc, plane, int64_t(t) * N + my_idx) * rsc[t] * rsc[T + my_idx];
+            const double B = logit_bound(u, t, my_idx, T, r1, l2, vmax, gamma64);
+            const float a = __double2float_rn(u - B), z = __double2float_rn(u + B);
+            if (a == z) {
+                u_exact[int64_t(t) * topk + lane] = a;
+            } else {  // to be summed: job (t, slot) on the pair list
+                const int pos = atomicAdd(pair_count, 1);
+                if (pos < T * topk) pair_list[pos] = t * topk + lane;
+                else route_bad(dev_status, check, 0, pos);
+            }
+        }
+    }
     if (lane == 0) {
         cert[t] = ok ? 1 : 0;
-        if (!ok) list[atomicAdd(list_count, 1)] = t;
+        if (!ok) {
+            const int pos = atomicAdd(list_count, 1);
+            if (pos < T) list[pos] = t;
+            else route_bad(dev_status, check, 0, pos);
+        }
     }
 }
 
@@ -377,71 +501,109 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
 // [2^-133, 2^127) (checked from the rows' ranges) every product is exact in
 // fp32, is formed there and added in FP64, which equals the FP64 fma of the
 // definition.  Otherwise both factors are widened to FP64 first.
+// Products of one 16-byte vector pair (8 k), widened to FP64.
+__device__ __forceinline__ void vec_products(const uint4& xv, const uint4& ev, bool fp32_products,
+                                             double (&p)[8]) {
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+    if (fp32_products) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            p[2 * q] = (double)__fmul_rn(bf16_lo(xw[q]), bf16_lo(ew[q]));
+            p[2 * q + 1] = (double)__fmul_rn(bf16_hi(xw[q]), bf16_hi(ew[q]));
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            p[2 * q] = __dmul_rn(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]));
+            p[2 * q + 1] = __dmul_rn(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]));
+        }
+    }
+}
+
 __device__ __forceinline__ float exact_logit(const uint16_t* __restrict__ xr,
                                              const uint16_t* __restrict__ er, int d,
                                              bool fp32_products) {
+    // 16-byte vectors (8 k) of both rows stream through an 8-deep register
+    // ring: slot i is consumed, then refilled with the vector 8 further on.
+    // The products of the next vector are formed and widened before the
+    // FP64 adds of the current one, so the conversions overlap the add
+    // chain.  Each product of two bf16 values is exact in FP64 (and in fp32
+    // under fp32_products), so adding it equals the FP64 fma of the
+    // definition.
+    constexpr int kRing = 8;
     const uint4* xp = reinterpret_cast<const uint4*>(xr);
     const uint4* ep = reinterpret_cast<const uint4*>(er);
-    const int nv = d / 8;
+    const int nv = d / 8;  // a multiple of 16
+    uint4 xv[kRing], ev[kRing];
+#pragma unroll
+    for (int i = 0; i < kRing; ++i) {
+        xv[i] = __ldg(xp + i);
+        ev[i] = __ldg(ep + i);
+    }
     double acc = 0.0;
-    uint4 xa = __ldg(xp), ea = __ldg(ep);
-    for (int v = 0; v < nv; ++v) {
-        uint4 xb = xa, eb = ea;
-        if (v + 1 < nv) {
-            xb = __ldg(xp + v + 1);
-            eb = __ldg(ep + v + 1);
-        }
-        const uint32_t xw[4] = {xa.x, xa.y, xa.z, xa.w};
-        const uint32_t ew[4] = {ea.x, ea.y, ea.z, ea.w};
-        if (fp32_products) {
+    double p[8];
+    vec_products(xv[0], ev[0], fp32_products, p);
+    for (int v0 = 0; v0 < nv; v0 += kRing) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc = __dadd_rn(acc, (double)__fmul_rn(bf16_lo(xw[q]), bf16_lo(ew[q])));
-                acc = __dadd_rn(acc, (double)__fmul_rn(bf16_hi(xw[q]), bf16_hi(ew[q])));
+        for (int i = 0; i < kRing; ++i) {
+            if (v0 + kRing + i < nv) {
+                xv[i] = __ldg(xp + v0 + kRing + i);
+                ev[i] = __ldg(ep + v0 + kRing + i);
             }
-        } else {
+            double pn[8];
+            const int ni = (i + 1) % kRing;
+            if (v0 + i + 1 < nv) vec_products(xv[ni], ev[ni], fp32_products, pn);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc = __fma_rn(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]), acc);
-                acc = __fma_rn(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]), acc);
-            }
+            for (int q = 0; q < 8; ++q) acc = __dadd_rn(acc, p[q]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) p[q] = pn[q];
         }
-        xa = xb;
-        ea = eb;
     }
     return __double2float_rn(acc);
 }
 
-// Tokens on the uncertified list get every logit from one sum per thread
+// Chosen logits that the bound did not settle, and every logit of the
+// tokens on the uncertified list, come from one sum per thread
 // while the list holds at most kPairList tokens; longer lists go to the
 // tiled kernel below.
 constexpr int kPairList = 256;
 
-__global__ void __launch_bounds__(256) route_exact_pairs_kernel(
+__global__ void __launch_bounds__(64) route_exact_pairs_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d, int K,
-    const int32_t* __restrict__ cand, const int32_t* __restrict__ cert,
-    const int32_t* __restrict__ list, const int32_t* __restrict__ list_count,
-    const float* __restrict__ vmax, const float* __restrict__ vmin,
-    float* __restrict__ u_exact, double* __restrict__ uhat) {
-    const int64_t nA = int64_t(T) * K;
-    const int nl = *list_count;
+    const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
+    const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
+    const int32_t* __restrict__ list_count, const float* __restrict__ vmax,
+    const float* __restrict__ vmin, float* __restrict__ u_exact, double* __restrict__ uhat,
+    int* dev_status, int32_t* __restrict__ check) {
+    int np = *pair_count, nl = *list_count;
+    if (np > T * K || nl > T) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) route_bad(dev_status, check, 1, max(np, nl));
+        np = min(np, T * K);
+        nl = min(nl, T);
+    }
+    const int64_t nA = np;
     const int64_t nB = nl <= kPairList ? int64_t(nl) * N : 0;
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j < nA + nB; j += stride) {
-        int t, e;
+        int t, e, pj = -1;
         if (j < nA) {
-            t = int(j / K);
-            if (!cert[t]) continue;
-            e = cand[j];
+            pj = pair_list[j];
+            t = pj / K;
+            e = (pj >= 0 && pj < T * K) ? cand[pj] : -1;
         } else {
             const int64_t jj = j - nA;
             t = list[jj / N];
             e = int(jj % N);
         }
+        if (t < 0 || t >= T || e < 0 || e >= N) {
+            route_bad(dev_status, check, 2, int(j));
+            continue;
+        }
         const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
                                    double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
         const float u = exact_logit(x + int64_t(t) * d, E + int64_t(e) * d, d, fp32_products);
-        if (j < nA) u_exact[j] = u;
+        if (pj >= 0) u_exact[pj] = u;
         else uhat[int64_t(t) * N + e] = (double)u;
     }
 }
@@ -462,17 +624,21 @@ constexpr int kLThreads = 64;
 __global__ void __launch_bounds__(kLThreads) route_logits_list_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int d, int n_routed,
     const int32_t* __restrict__ list, const int32_t* __restrict__ list_count,
-    double* __restrict__ uhat) {
+    double* __restrict__ uhat, int* dev_status, int32_t* __restrict__ check) {
     __shared__ __align__(16) double xs[2][kLK][kLT];
     __shared__ __align__(16) double es[2][kLK][kLE];
-    const int nl = *list_count;
+    const int nl = min(*list_count, T);
     const int l0 = blockIdx.x * kLT, e0 = blockIdx.y * kLE;
     if (nl <= kPairList || l0 >= nl) return;
     const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
     // loader: thread tid stages row tid of the x tile (listed token l0 + tid)
     // and row tid of the E tile, kLK k values of each per chunk
     const bool xrow_ok = l0 + tid < nl, erow_ok = e0 + tid < n_routed;
-    const int xt = xrow_ok ? list[l0 + tid] : 0;
+    int xt = xrow_ok ? list[l0 + tid] : 0;
+    if (xt < 0 || xt >= T) {
+        route_bad(dev_status, check, 3, xt);
+        xt = 0;
+    }
     const uint4* xp = reinterpret_cast<const uint4*>(x + int64_t(xt) * d);
     const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e0 + tid) * d);
     const int ecol = (tid & 7) * 8 + (tid >> 3);  // interleaved column of expert tid
@@ -534,6 +700,7 @@ __global__ void __launch_bounds__(kLThreads) route_logits_list_kernel(
         const int l = l0 + ty * 8 + i;
         if (l >= nl) continue;
         const int t = list[l];
+        if (t < 0 || t >= T) continue;  // reported above
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = e0 + tx * 8 + j;
@@ -556,7 +723,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(
     const int32_t* __restrict__ cand, const float* __restrict__ u_exact, int T, int n_routed,
     int n_groups, int topk_groups, int topk, const float* __restrict__ bias,
     const float* __restrict__ logit_offset, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_gate, int32_t* __restrict__ counts) {
+    float* __restrict__ topk_gate, int32_t* __restrict__ counts, int* dev_status,
+    int32_t* __restrict__ check) {
     extern __shared__ __align__(16) float sel_smem[];
     int* hist = reinterpret_cast<int*>(sel_smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -573,6 +741,10 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(
             float sbv = 0.0f, s_own = 0.0f;
             if (lane < topk) {
                 idx = cand[int64_t(t) * topk + lane];
+                if (idx < 0 || idx >= n_routed) {
+                    route_bad(dev_status, check, 4, idx);
+                    idx = 0;
+                }
                 float ui = u_exact[int64_t(t) * topk + lane];
                 if (logit_offset) ui = __fadd_rn(ui, logit_offset[idx]);
                 s_own = __double2float_rn(1.0 / (1.0 + exp(-(double)ui)));
@@ -639,11 +811,21 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(
                 if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
                 if (lane == r) my_idx = bi;
             }
-            if (lane < topk) sv = s[my_idx];
+            if (lane < topk) {
+                if (my_idx < 0 || my_idx >= n_routed) {
+                    route_bad(dev_status, check, 5, my_idx);
+                    my_idx = 0;
+                }
+                sv = s[my_idx];
+            }
         }
         // gates: S = FP64 sum of the chosen unbiased s in slot order
         double S = 0.0;
         for (int r = 0; r < topk; ++r) S += (double)__shfl_sync(0xffffffffu, sv, r);
+        if (lane < topk && (my_idx < 0 || my_idx >= n_routed)) {
+            route_bad(dev_status, check, 4, my_idx);
+            my_idx = 0;
+        }
         if (lane < topk) {
             topk_idx[int64_t(t) * topk + lane] = my_idx;
             topk_gate[int64_t(t) * topk + lane] = __double2float_rn((double)sv / S);
@@ -672,21 +854,30 @@ int validate_shape(const MoeShape* s) {
 
 // Workspace of moe_route: every piece starts on a 256-byte boundary.
 struct RouteWs {
-    double* uhat;        // [T, N]  approximate, then exact for listed tokens
-    double* norm;        // [T + N]
+    int8_t* xp;          // [4, T, d]  digit planes of x
+    int8_t* ep;          // [4, N, d]  digit planes of E
+    int32_t* acc;        // [7, T, N]  integer levels
+    double* rsc;         // [T + N]
+    int32_t* rex;        // [T + N]
+    double* r1;          // [T + N]
+    double* l2;          // [T + N]
     float* vmax;         // [T + N]
     float* vmin;         // [T + N]
+    double* uhat;        // [T, N]  exact logits of listed tokens
     int32_t* cand;       // [T, K]
     float* u_exact;      // [T, K]
     int32_t* cert;       // [T]
     int32_t* list;       // [T]
     int32_t* list_count; // [1]
+    int32_t* pair_list;  // [T * K]
+    int32_t* pair_count; // [1]
+    int32_t* check;      // [kCheckWords]
     size_t bytes;
 };
 
 RouteWs route_carve(const MoeShape* s, void* base) {
     RouteWs w{};
-    const size_t T = s->T, N = s->n_routed, K = s->topk;
+    const size_t T = s->T, N = s->n_routed, K = s->topk, d = s->d;
     uintptr_t p = reinterpret_cast<uintptr_t>(base);
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -694,15 +885,24 @@ RouteWs route_carve(const MoeShape* s, void* base) {
         off = align_up(off + bytes, 256);
         return reinterpret_cast<void*>(p + at);
     };
-    w.uhat = static_cast<double*>(take(T * N * 8));
-    w.norm = static_cast<double*>(take((T + N) * 8));
+    w.xp = static_cast<int8_t*>(take(4 * T * d));
+    w.ep = static_cast<int8_t*>(take(4 * N * d));
+    w.acc = static_cast<int32_t*>(take(size_t(kLevels) * T * N * 4));
+    w.rsc = static_cast<double*>(take((T + N) * 8));
+    w.rex = static_cast<int32_t*>(take((T + N) * 4));
+    w.r1 = static_cast<double*>(take((T + N) * 8));
+    w.l2 = static_cast<double*>(take((T + N) * 8));
     w.vmax = static_cast<float*>(take((T + N) * 4));
     w.vmin = static_cast<float*>(take((T + N) * 4));
+    w.uhat = static_cast<double*>(take(T * N * 8));
     w.cand = static_cast<int32_t*>(take(T * K * 4));
     w.u_exact = static_cast<float*>(take(T * K * 4));
     w.cert = static_cast<int32_t*>(take(T * 4));
     w.list = static_cast<int32_t*>(take(T * 4));
     w.list_count = static_cast<int32_t*>(take(4));
+    w.pair_list = static_cast<int32_t*>(take(T * K * 4));
+    w.pair_count = static_cast<int32_t*>(take(4));
+    w.check = static_cast<int32_t*>(take(4 * kCheckWords));
     w.bytes = off;
     return w;
 }
@@ -721,7 +921,6 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
                                  const float* logit_offset, int32_t* topk_idx, float* topk_gate,
                                  int32_t* expert_counts, void* ws, size_t ws_bytes,
                                  int* dev_status, void* stream) {
-    (void)dev_status;
     int rc = validate_shape(shape);
     if (rc != MOE_OK) return rc;
     if (!router_w || !bias || !expert_counts) return MOE_ERR_NULL;
@@ -735,57 +934,62 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
     if (!ws || ws_bytes < moe_route_workspace_size(shape)) return MOE_ERR_WORKSPACE;
     const RouteWs w = route_carve(shape, ws);
     const int sms = sm_count();
+    if (!device_is_sm100()) return MOE_ERR_DEVICE;
 
-    // 1. norms and ranges of every row (also clears the list counter)
+    // 1. digit planes and row statistics (also clears the list counter)
     const double nmargin = 4.0 * (d + 64) * 0x1p-53 + 0x1p-50;
-    route_norms_kernel<<<(T + N + 7) / 8, 256, 0, st>>>(x, router_w, T, N, d, nmargin, w.norm,
-                                                        w.vmax, w.vmin, w.list_count);
+    route_slice_kernel<<<(T + N + 7) / 8, 256, 0, st>>>(x, router_w, T, N, d, nmargin, w.xp,
+                                                        w.ep, w.rsc, w.rex, w.r1, w.l2, w.vmax,
+                                                        w.vmin, w.list_count, w.pair_count,
+                                                        w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
-    // 2. approximate logits; K is split when the tiles alone fill few SMs
-    const int tiles = ((T + kAT - 1) / kAT) * ((N + kAE - 1) / kAE);
-    const int nblk = d / kAK;
-    int splits = (4 * sms + tiles - 1) / tiles;
-    if (splits > nblk) splits = nblk;
+    // 2. integer logits; K is split when the tiles alone leave SMs idle
+    const int tiles = ((T + kIM - 1) / kIM) * ((N + kIN - 1) / kIN);
+    const int nchunks = d / kIK;
+    int splits = sms / tiles;
+    if (splits > nchunks) splits = nchunks;
     if (splits < 1) splits = 1;
-    const int per_split = (nblk + splits - 1) / splits;
-    splits = (nblk + per_split - 1) / per_split;
+    const int per_split = (nchunks + splits - 1) / splits;
+    splits = (nchunks + per_split - 1) / per_split;
     if (splits > 1 &&
-        cudaMemsetAsync(w.uhat, 0, sizeof(double) * size_t(T) * N, st) != cudaSuccess)
+        cudaMemsetAsync(w.acc, 0, sizeof(int32_t) * kLevels * size_t(T) * N, st) != cudaSuccess)
         return MOE_ERR_CUDA;
-    dim3 ga((T + kAT - 1) / kAT, (N + kAE - 1) / kAE, splits);
-    route_approx_kernel<<<ga, 32, 0, st>>>(x, router_w, T, N, d, per_split, w.uhat);
+    CUtensorMap mx, me;
+    if (!make_map(&mx, w.xp, 4 * uint64_t(T), uint64_t(d), kIM) ||
+        !make_map(&me, w.ep, 4 * uint64_t(N), uint64_t(d), kIN))
+        return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(route_imma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kImmaSmem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dim3 gi((T + kIM - 1) / kIM, (N + kIN - 1) / kIN, splits);
+    route_imma_kernel<<<gi, 128, kImmaSmem, st>>>(mx, me, T, N, nchunks, per_split, w.acc,
+                                                  dev_status);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
-    // 3. certify the choice of every token
-    // |u~ - u_def| <= cbound * ||x|| ||E|| + tiny: gamma_31 of fp32 for the
-    // block sums, FP64 terms for the sum of block sums and for the defining
-    // FP64 sum, products below 2^-126 (at most 2^-150 off each) in tiny.
-    const double u32 = 0x1p-24;
-    const double cbound = (31.0 * u32 / (1.0 - 31.0 * u32)) * (1.0 + 0x1p-20) +
-                          4.0 * (d + nblk + 64) * 0x1p-53;
-    const double tiny = double(d) * 0x1p-148;
+    // 3. certify the choice of every token; gamma_d of FP64 bounds the
+    // defining sum's rounding: |u_def - sum| <= gamma_d ||x|| ||E||
+    const double gamma64 = (double(d) * 0x1p-53 / (1.0 - double(d) * 0x1p-53)) * (1.0 + 0x1p-20);
     const size_t csmem = sizeof(float) * 3 * size_t(N) * kCertWarps;
     if (csmem > 48 * 1024 &&
         cudaFuncSetAttribute(route_certify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(csmem)) != cudaSuccess)
         return MOE_ERR_CUDA;
     route_certify_kernel<<<(T + kCertWarps - 1) / kCertWarps, kCertWarps * 32, csmem, st>>>(
-        w.uhat, w.norm, bias, logit_offset, T, N, shape->n_groups, shape->topk_groups, K,
-        cbound, tiny, w.cand, w.cert, w.list, w.list_count);
+        w.acc, w.rsc, w.rex, w.r1, w.l2, w.vmax, bias, logit_offset, T, N, shape->n_groups,
+        shape->topk_groups, K, gamma64, w.cand, w.cert, w.u_exact, w.list, w.list_count,
+        w.pair_list, w.pair_count, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
     // 4. the defining FP64 sums where they are needed
-    int64_t pair_threads = int64_t(T) * K + int64_t(kPairList) * N;
-    int64_t pblocks = (pair_threads + 255) / 256;
-    if (pblocks > int64_t(sms) * 16) pblocks = int64_t(sms) * 16;
-    route_exact_pairs_kernel<<<unsigned(pblocks), 256, 0, st>>>(
-        x, router_w, T, N, d, K, w.cand, w.cert, w.list, w.list_count, w.vmax, w.vmin,
-        w.u_exact, w.uhat);
+    // one sum per thread (grid-stride over the jobs the lists hold)
+    route_exact_pairs_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
+        x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
+        w.vmax, w.vmin, w.u_exact, w.uhat, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
     dim3 gl((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
     route_logits_list_kernel<<<gl, kLThreads, 0, st>>>(x, router_w, T, d, N, w.list,
-                                                       w.list_count, w.uhat);
+                                                       w.list_count, w.uhat, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
     // 5. slot order, gates, histogram
@@ -796,6 +1000,6 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
         return MOE_ERR_CUDA;
     route_select_kernel<<<(T + kSelWarps - 1) / kSelWarps, kSelWarps * 32, smem, st>>>(
         w.uhat, w.cert, w.cand, w.u_exact, T, N, shape->n_groups, shape->topk_groups, K, bias,
-        logit_offset, topk_idx, topk_gate, expert_counts);
+        logit_offset, topk_idx, topk_gate, expert_counts, dev_status, w.check);
     return check_launch();
 }

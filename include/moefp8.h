@@ -125,7 +125,11 @@ MOE_API int moe_read_status(const int* dev_status, int* host_status, void* strea
  *   slot order.
  * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE (d % 128, T < 0, N_r range),
  * MOE_ERR_ROUTE, MOE_ERR_ALIGN (x, router_w not 16-byte aligned),
- * MOE_ERR_WORKSPACE, MOE_ERR_CUDA. */
+ * MOE_ERR_WORKSPACE, MOE_ERR_DEVICE (not sm_100), MOE_ERR_CUDA;
+ * MOE_DEV_TIMEOUT or MOE_DEV_BAD_INPUT on dev_status (may be NULL).
+ * The logits are computed exactly on the tensor cores from int8 digit
+ * planes of x and E wherever a rigorous bound settles the result, and with
+ * the defining FP64 sum elsewhere; the outputs equal the definition. */
 MOE_API size_t moe_route_workspace_size(const MoeShape* shape);
 MOE_API int moe_route(const MoeShape* shape, const uint16_t* x, const uint16_t* router_w,
                       const float* bias, const float* logit_offset, int32_t* topk_idx,
