@@ -104,14 +104,17 @@ __device__ __forceinline__ float warp_max(float v) {
 //   r1[r] = sum |v - 2^(sigma-28) X| (the truncated remainders), l2[r] =
 //            ||v||_2 (FP64, raised by 1 + nmargin to cover their rounding);
 //   vmax[r], vmin[r] = max |v| (+inf for a non-finite row) and min |v| over
-//            v != 0 (FLT_MAX for an all-zero row).
+//            v != 0 (FLT_MAX for an all-zero row);
+//   lb[r]  = the lowest bit any value of the row can carry: a bf16 value
+//            in [2^e, 2^(e+1)) has no bit below 2^(e-7) (2^-133 below 2^-126).
 // Block 0 also clears the two list counters and the check words of this call.
 __global__ void __launch_bounds__(256) route_slice_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d,
     double nmargin, int8_t* __restrict__ xp, int8_t* __restrict__ ep, double* __restrict__ rsc,
     int32_t* __restrict__ rex, double* __restrict__ r1, double* __restrict__ l2,
-    float* __restrict__ vmax, float* __restrict__ vmin, int32_t* __restrict__ list_count,
-    int32_t* __restrict__ pair_count, int32_t* __restrict__ check) {
+    float* __restrict__ vmax, float* __restrict__ vmin, double* __restrict__ lb,
+    int32_t* __restrict__ list_count, int32_t* __restrict__ pair_count,
+    int32_t* __restrict__ check) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *list_count = 0;
         *pair_count = 0;
@@ -184,6 +187,9 @@ __global__ void __launch_bounds__(256) route_slice_kernel(
         if (lane == 0) {
             vmax[r] = finite ? mx : INFINITY;
             vmin[r] = mn;
+            int emin = 0;
+            frexpf(mn < FLT_MAX ? mn : 1.0f, &emin);  // mn in [2^(emin-1), 2^emin)
+            lb[r] = ldexp(1.0, max(emin - 1, -126) - 7);
             rsc[r] = ldexp(1.0, sigma - 28);
             rex[r] = finite ? (exact ? 1 : 0) : -1;
             r1[r] = ldexp(s1, sigma - 28) * (1.0 + nmargin);
@@ -347,19 +353,54 @@ __global__ void __launch_bounds__(128, 1) route_imma_kernel(
 // to fp32.  Groups and experts are chosen on the centres; the choice is
 // certified when the lowest chosen lower end is strictly above the highest
 // rejected upper end, for the groups and then for the experts inside the
-// chosen groups.  A certified token's chosen logit is fp32(u~) when
+// chosen groups.  A certified token's chosen logit is the exact fp32
+// rounding of the level sum when both rows are sliced exactly and the
+// defining sum provably does not round (sum_is_exact), else fp32(u~) when
 // u~ - B and u~ + B round to the same fp32 value; otherwise (t, slot) goes
 // on the pair list, to be summed.
 constexpr int kCertWarps = 8;
 
+// sum_L 2^(7(6-L)) acc_L = hi * 2^28 + lo, both parts exact in int64.
+__device__ __forceinline__ void level_parts(const int32_t* __restrict__ acc, int64_t plane,
+                                            int64_t at, int64_t& hi, int64_t& lo) {
+    hi = int64_t(acc[at]) * (1 << 14) + int64_t(acc[plane + at]) * (1 << 7) +
+         int64_t(acc[2 * plane + at]);
+    lo = int64_t(acc[3 * plane + at]) * (1 << 21) + int64_t(acc[4 * plane + at]) * (1 << 14) +
+         int64_t(acc[5 * plane + at]) * (1 << 7) + int64_t(acc[6 * plane + at]);
+}
+
 __device__ __forceinline__ double level_sum(const int32_t* __restrict__ acc, int64_t plane,
                                             int64_t at) {
-    const int64_t hi = int64_t(acc[at]) * (1 << 14) + int64_t(acc[plane + at]) * (1 << 7) +
-                       int64_t(acc[2 * plane + at]);
-    const int64_t lo = int64_t(acc[3 * plane + at]) * (1 << 21) +
-                       int64_t(acc[4 * plane + at]) * (1 << 14) +
-                       int64_t(acc[5 * plane + at]) * (1 << 7) + int64_t(acc[6 * plane + at]);
+    int64_t hi, lo;
+    level_parts(acc, plane, at, hi, lo);
     return (double)hi * 0x1p28 + (double)lo;
+}
+
+// Every product x_k E_k is a multiple of Q = lb(x_t) lb(E_i) and every
+// partial sum of the defining FP64 sum is at most ||x_t||_2 ||E_i||_2 in
+// magnitude; below 2^53 Q each partial sum is a double, so no addition
+// rounds and the defining sum equals the exact sum, in any order.
+__device__ __forceinline__ bool sum_is_exact(int t, int i, int T, const double* __restrict__ l2,
+                                             const double* __restrict__ lb) {
+    return l2[t] * l2[T + i] < 0x1p53 * (lb[t] * lb[T + i]);
+}
+
+// fp32(round-to-nearest-even) of (hi * 2^28 + lo) * scale, exactly: the sum
+// is split into s = fl(hi*2^28 + lo) and its exact error e (TwoSum); s + e
+// rounds like s unless s is the midpoint of two fp32 values, where e (if
+// not zero) decides.  scale is a power of two.
+__device__ __forceinline__ float exact_level_fp32(int64_t hi, int64_t lo, double scale) {
+    const double a = (double)hi * 0x1p28, b = (double)lo;  // both exact
+    const double sum = a + b;
+    const double bb = sum - a;
+    const double e = (a - (sum - bb)) + (b - bb);
+    const double sv = sum * scale, ev = e * scale;
+    const float r = __double2float_rn(sv);
+    if (ev == 0.0 || (double)r == sv) return r;
+    const float dn = __double2float_rd(sv), up = __double2float_ru(sv);
+    const double mid = 0.5 * ((double)dn + (double)up);
+    if (sv != mid) return r;
+    return ev > 0.0 ? up : dn;
 }
 
 __device__ __forceinline__ double logit_bound(double u, int t, int i, int T,
@@ -373,7 +414,8 @@ __device__ __forceinline__ double logit_bound(double u, int t, int i, int T,
 __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
     const int32_t* __restrict__ acc, const double* __restrict__ rsc,
     const int32_t* __restrict__ rex, const double* __restrict__ r1,
-    const double* __restrict__ l2, const float* __restrict__ vmax, const float* __restrict__ bias,
+    const double* __restrict__ l2, const float* __restrict__ vmax,
+    const double* __restrict__ lb, const float* __restrict__ bias,
     const float* __restrict__ logit_offset, int T, int N, int n_groups, int topk_groups,
     int topk, double gamma64, int32_t* __restrict__ cand, int32_t* __restrict__ cert,
     float* __restrict__ u_exact, int32_t* __restrict__ list, int32_t* __restrict__ list_count,
@@ -471,11 +513,16 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
     if (lane < topk) {
         cand[int64_t(t) * topk + lane] = ok ? my_idx : -1;
         if (ok) {
-            const double u =
-                level_sum(acc, plane, int64_t(t) * N + my_idx) * rsc[t] * rsc[T + my_idx];
+            int64_t hi, lo;
+            level_parts(acc, plane, int64_t(t) * N + my_idx, hi, lo);
+            const double scale = rsc[t] * rsc[T + my_idx];
+            const double u = ((double)hi * 0x1p28 + (double)lo) * scale;
             const double B = logit_bound(u, t, my_idx, T, r1, l2, vmax, gamma64);
             const float a = __double2float_rn(u - B), z = __double2float_rn(u + B);
-            if (a == z) {
+            if (rex[t] == 1 && rex[T + my_idx] == 1 && sum_is_exact(t, my_idx, T, l2, lb)) {
+                // the levels hold the exact sum and the defining sum equals it
+                u_exact[int64_t(t) * topk + lane] = exact_level_fp32(hi, lo, scale);
+            } else if (a == z) {
                 u_exact[int64_t(t) * topk + lane] = a;
             } else {  // to be summed: job (t, slot) on the pair list
                 const int pos = atomicAdd(pair_count, 1);
@@ -519,6 +566,29 @@ __device__ __forceinline__ void vec_products(const uint4& xv, const uint4& ev, b
             p[2 * q + 1] = __dmul_rn(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]));
         }
     }
+}
+
+// The defining sum when no addition of it can round (sum_is_exact): any
+// order gives the same double, so eight interleaved accumulators shorten
+// the dependent chain eightfold.
+__device__ __forceinline__ float exact_logit_unordered(const uint16_t* __restrict__ xr,
+                                                       const uint16_t* __restrict__ er, int d) {
+    const uint4* xp = reinterpret_cast<const uint4*>(xr);
+    const uint4* ep = reinterpret_cast<const uint4*>(er);
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+    for (int v = 0; v < d / 8; ++v) {
+        const uint4 xv = __ldg(xp + v), ev = __ldg(ep + v);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = __fma_rn(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]), acc[2 * q]);
+            acc[2 * q + 1] = __fma_rn(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]), acc[2 * q + 1]);
+        }
+    }
+    const double s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    return __double2float_rn(s);
 }
 
 __device__ __forceinline__ float exact_logit(const uint16_t* __restrict__ xr,
@@ -574,8 +644,9 @@ __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
     const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
     const int32_t* __restrict__ list_count, const float* __restrict__ vmax,
-    const float* __restrict__ vmin, float* __restrict__ u_exact, double* __restrict__ uhat,
-    int* dev_status, int32_t* __restrict__ check) {
+    const float* __restrict__ vmin, const double* __restrict__ l2, const double* __restrict__ lb,
+    float* __restrict__ u_exact, double* __restrict__ uhat, int* dev_status,
+    int32_t* __restrict__ check) {
     int np = *pair_count, nl = *list_count;
     if (np > T * K || nl > T) {
         if (blockIdx.x == 0 && threadIdx.x == 0) route_bad(dev_status, check, 1, max(np, nl));
@@ -602,7 +673,10 @@ __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
         }
         const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
                                    double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
-        const float u = exact_logit(x + int64_t(t) * d, E + int64_t(e) * d, d, fp32_products);
+        const float u =
+            sum_is_exact(t, e, T, l2, lb)
+                ? exact_logit_unordered(x + int64_t(t) * d, E + int64_t(e) * d, d)
+                : exact_logit(x + int64_t(t) * d, E + int64_t(e) * d, d, fp32_products);
         if (pj >= 0) u_exact[pj] = u;
         else uhat[int64_t(t) * N + e] = (double)u;
     }
@@ -863,6 +937,7 @@ struct RouteWs {
     double* l2;          // [T + N]
     float* vmax;         // [T + N]
     float* vmin;         // [T + N]
+    double* lb;          // [T + N]
     double* uhat;        // [T, N]  exact logits of listed tokens
     int32_t* cand;       // [T, K]
     float* u_exact;      // [T, K]
@@ -894,6 +969,7 @@ RouteWs route_carve(const MoeShape* s, void* base) {
     w.l2 = static_cast<double*>(take((T + N) * 8));
     w.vmax = static_cast<float*>(take((T + N) * 4));
     w.vmin = static_cast<float*>(take((T + N) * 4));
+    w.lb = static_cast<double*>(take((T + N) * 8));
     w.uhat = static_cast<double*>(take(T * N * 8));
     w.cand = static_cast<int32_t*>(take(T * K * 4));
     w.u_exact = static_cast<float*>(take(T * K * 4));
@@ -940,7 +1016,7 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
     const double nmargin = 4.0 * (d + 64) * 0x1p-53 + 0x1p-50;
     route_slice_kernel<<<(T + N + 7) / 8, 256, 0, st>>>(x, router_w, T, N, d, nmargin, w.xp,
                                                         w.ep, w.rsc, w.rex, w.r1, w.l2, w.vmax,
-                                                        w.vmin, w.list_count, w.pair_count,
+                                                        w.vmin, w.lb, w.list_count, w.pair_count,
                                                         w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
@@ -976,7 +1052,7 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
                              int(csmem)) != cudaSuccess)
         return MOE_ERR_CUDA;
     route_certify_kernel<<<(T + kCertWarps - 1) / kCertWarps, kCertWarps * 32, csmem, st>>>(
-        w.acc, w.rsc, w.rex, w.r1, w.l2, w.vmax, bias, logit_offset, T, N, shape->n_groups,
+        w.acc, w.rsc, w.rex, w.r1, w.l2, w.vmax, w.lb, bias, logit_offset, T, N, shape->n_groups,
         shape->topk_groups, K, gamma64, w.cand, w.cert, w.u_exact, w.list, w.list_count,
         w.pair_list, w.pair_count, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
@@ -985,7 +1061,7 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
     // one sum per thread (grid-stride over the jobs the lists hold)
     route_exact_pairs_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
         x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
-        w.vmax, w.vmin, w.u_exact, w.uhat, dev_status, w.check);
+        w.vmax, w.vmin, w.l2, w.lb, w.u_exact, w.uhat, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
     dim3 gl((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
     route_logits_list_kernel<<<gl, kLThreads, 0, st>>>(x, router_w, T, d, N, w.list,
