@@ -14,9 +14,10 @@
 //     feature); 2 TMEM partial buffers, 4 smem stages of 48 KB.
 //   BN = 128 (fp32 / bf16 output): one 128-row weight block; 4 TMEM partial
 //     buffers (more slack between MMA and promotion), 4 stages of 32 KB; a
-//     tile's output row segment is parked in shared memory and stored during
-//     the next tile's K loop, one 16-byte store per K block, so the stores
-//     overlap compute instead of stalling the promotion warps.
+//     warp's 32 finished row segments go to a swizzled tile in shared memory
+//     and leave as TMA bulk tensor stores (full 128-byte lines, written by
+//     the copy engine while the next tile's K loop runs); the rows of a
+//     group's ragged last warp are stored directly.
 //
 // Roles (384 threads, one CTA per SM, persistent over work items):
 //   warp 0       TMA producer: token tile (16 KB) + weight tile(s) per K block
@@ -38,7 +39,7 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kTileBytes = 128 * 128;            // one 128 x 128 FP8 tile
 constexpr int kStages = 4;                       // smem ring of operand stages
-constexpr int kParkStride = 272;                 // bytes per parked row segment (256 + pad)
+constexpr int kParkWarpBytes = 32 * 256;         // one warp's 32 parked rows (fp32 halves)
 constexpr int kMaxBufs = 4;
 constexpr int kScaleSlots = 16;
 constexpr int kMaxGroups = 1040;
@@ -50,7 +51,7 @@ struct Cfg {
     static constexpr int kStageBytes = kTileBytes + BN * 128;  // tokens + weights
     static constexpr int kStages = moe::kStages;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kParkBytes = BN == 128 ? kPromoters * 32 * kParkStride : 0;
+    static constexpr int kParkBytes = BN == 128 ? kPromoters * kParkWarpBytes : 0;
     static constexpr int kBufs = 512 / BN;                     // TMEM partial buffers
     static constexpr int kPairs = BN / 4;                      // fp32 pairs per promoter thread
     static_assert(kBufs <= kMaxBufs, "TMEM buffers");
@@ -461,21 +462,29 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
     __syncwarp();
 }
 
-// Parked output of the fp32 / bf16 epilogue: a promoter thread's 64 values
-// (256 bytes) wait in shared memory and move to global memory 16 bytes per K
-// block of the next tile.  Vector j of the parked row -> its global segment.
-__device__ __forceinline__ void unpark_vec(const char* park, char* dst, bool bf16, int j) {
-    if (bf16) {
-        const float4 a = *reinterpret_cast<const float4*>(park + 32 * j);
-        const float4 b = *reinterpret_cast<const float4*>(park + 32 * j + 16);
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y), h1 = __floats2bfloat162_rn(a.z, a.w);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y), h3 = __floats2bfloat162_rn(b.z, b.w);
-        reinterpret_cast<uint4*>(dst)[j] =
-            make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                       *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
-    } else {
-        reinterpret_cast<float4*>(dst)[j] = *reinterpret_cast<const float4*>(park + 16 * j);
-    }
+// fp32 / bf16 epilogue: a warp's 32 finished row segments (64 values each)
+// are written into its parking tile in shared memory in the 128-byte swizzle
+// layout of the output tensor map (16-byte chunk c of row r at c ^ (r % 8)),
+// then one lane hands the tile to the TMA engine as bulk tensor stores.  The
+// next tile waits until the engine has read the parking tile.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ================================================= promotion + epilogue (warps 4-11)
@@ -486,7 +495,7 @@ __device__ __forceinline__ void unpark_vec(const char* park, char* dst, bool bf1
 //   BN = 128: columns [64h, 64h+64) of the single weight block.
 template <int BN>
 __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, char* park_area,
-                                         uint32_t tmem_base) {
+                                         uint32_t tmem_base, const CUtensorMap* map_o) {
     using C = Cfg<BN>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
@@ -499,10 +508,8 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
     const int c1 = BN == 256 ? 128 + half * 64 : half * 64;  // first column of chunk 1
     uint32_t tb = 0, cit = 0, parity = 0;
     bool ok = true;
-    // this thread's parking slot and the global segment it belongs to
-    char* const park = park_area + (threadIdx.x - 128) * kParkStride;
-    char* park_dst = nullptr;
-    const int nvec = bf16_out ? 8 : 16;  // 16-byte global stores per parked segment
+    // this warp's parking tile (swizzled, 1024-byte aligned)
+    char* const wpark = park_area + (warp - 4) * kParkWarpBytes;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x, parity ^= 1u) {
         const Item w = decode_item(ss, p, item);
         uint64_t acc2[C::kPairs];  // fp32 accumulator pairs
@@ -553,26 +560,79 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     ffma2(acc2[16 + i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
-                // one 16-byte store of the previous tile's output per K block
-                if (park_dst && kb < nvec) unpark_vec(park, park_dst, bf16_out, kb);
             }
         }
         // ---------------- epilogue
         const bool row_ok = r < w.ntok;
         const size_t row = size_t(w.row0) + r;
         if (BN == 128) {
-            // finish the previous tile's segment, then park this one
-            if (park_dst)
-                for (int j = min(p.nkb, nvec); j < nvec; ++j) unpark_vec(park, park_dst, bf16_out, j);
+            const int rows_here = w.ntok - q * 32;  // valid rows of this warp's 32
+            const int col = w.f * 128 + half * 64;
+            if (rows_here >= 32) {
+                // the engine has read the previous tile out of the parking tile
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+                if (bf16_out) {
+                    // one 128-byte box: 64 bf16 per row
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float2 a = unpack2(acc2[2 * i]), b = unpack2(acc2[2 * i + 1]);
-                *reinterpret_cast<float4*>(park + 16 * i) = make_float4(a.x, a.y, b.x, b.y);
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const float2 f = unpack2(acc2[4 * j + h]);
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x, f.y);
+                            u[h] = *reinterpret_cast<uint32_t*>(&b2);
+                        }
+                        *reinterpret_cast<uint4*>(wpark + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                            make_uint4(u[0], u[1], u[2], u[3]);
+                    }
+                } else {
+                    // two 128-byte boxes: columns [0, 32) and [32, 64) of the half
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 a = unpack2(acc2[2 * i]), b = unpack2(acc2[2 * i + 1]);
+                        char* box = wpark + (i >> 3) * 4096;
+                        *reinterpret_cast<float4*>(box + lane * 128 + (((i & 7) ^ (lane & 7)) * 16)) =
+                            make_float4(a.x, a.y, b.x, b.y);
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int y = w.row0 + q * 32;
+                    if (bf16_out) {
+                        tma_store_2d(map_o, smem_u32(wpark), col, y);
+                    } else {
+                        tma_store_2d(map_o, smem_u32(wpark), col, y);
+                        tma_store_2d(map_o, smem_u32(wpark + 4096), col + 32, y);
+                    }
+                    bulk_commit();
+                }
+            } else if (row_ok) {
+                // the group's ragged last rows: plain stores, only the valid rows
+                if (bf16_out) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                          row * p.n + col);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t u[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const float2 f = unpack2(acc2[4 * j + h]);
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x, f.y);
+                            u[h] = *reinterpret_cast<uint32_t*>(&b2);
+                        }
+                        dst[j] = make_uint4(u[0], u[1], u[2], u[3]);
+                    }
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.n + col);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 a = unpack2(acc2[2 * i]), b = unpack2(acc2[2 * i + 1]);
+                        dst[i] = make_float4(a.x, a.y, b.x, b.y);
+                    }
+                }
             }
-            const size_t col = size_t(w.f) * 128 + half * 64;
-            park_dst = !row_ok ? nullptr
-                      : bf16_out ? reinterpret_cast<char*>(static_cast<__nv_bfloat16*>(p.out) + row * p.n + col)
-                                 : reinterpret_cast<char*>(static_cast<float*>(p.out) + row * p.n + col);
         } else {
             // h = silu(gate) * up for this thread's 64 features, then the
             // 1x128 scale of the token's 128 features (both halves).
@@ -620,8 +680,9 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
             2, kPromoters * 32, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
         if (any_abort) break;
     }
-    if (BN == 128 && park_dst)
-        for (int j = 0; j < nvec; ++j) unpark_vec(park, park_dst, bf16_out, j);
+    // every bulk store of this warp has completed before the CTA moves on
+    if (BN == 128 && lane == 0) bulk_wait_all();
+    __syncwarp();
     tc_fence_before();
 }
 
@@ -629,7 +690,8 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
-                        const __grid_constant__ CUtensorMap map_a, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap map_a,
+                        const __grid_constant__ CUtensorMap map_o, const GemmParams p) {
     using C = Cfg<BN>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -726,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (warp == 2) scale_loader<BN>(p, ss);
     } else {
         set_max_regs_inc<208>();
-        promoter<BN>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base);
+        promoter<BN>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base, &map_o);
     }
 
     __syncthreads();
@@ -738,11 +800,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int BN>
-int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma, cudaStream_t st) {
+int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma,
+           const CUtensorMap& mo, cudaStream_t st) {
     if (cudaFuncSetAttribute(grouped_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem_bytes<BN>())) != cudaSuccess)
         return MOE_ERR_CUDA;
-    grouped_gemm_kernel<BN><<<sm_count(), kThreads, smem_bytes<BN>(), st>>>(mw, ma, p);
+    grouped_gemm_kernel<BN><<<sm_count(), kThreads, smem_bytes<BN>(), st>>>(mw, ma, mo, p);
     return check_launch();
 }
 
@@ -782,6 +845,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
+}
+
+// 2D output map over [rows, cols] of fp32 or bf16 (cols contiguous): box = 32 rows x
+// 128 bytes, 128-byte swizzle (the layout of the epilogue's parking tiles).
+bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const uint32_t esize = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * esize};
+    cuuint32_t box[2] = {128 / esize, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base,
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool device_is_sm100() {
@@ -833,10 +911,13 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     p.out_scales = out_scales;
     p.dev_status = dev_status;
 
-    CUtensorMap mw, ma;
+    CUtensorMap mw, ma, mo;
     if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128) ||
         !make_map(&ma, a, uint64_t(max_rows), uint64_t(k), 128))
         return MOE_ERR_CUDA;
-    return swiglu ? launch<256>(p, mw, ma, as_stream(stream))
-                  : launch<128>(p, mw, ma, as_stream(stream));
+    if (swiglu) mo = mw;  // unused by the SwiGLU epilogue
+    else if (!make_out_map(&mo, out, uint64_t(max_rows), uint64_t(n), epilogue == MOE_EPI_BF16))
+        return MOE_ERR_CUDA;
+    return swiglu ? launch<256>(p, mw, ma, mo, as_stream(stream))
+                  : launch<128>(p, mw, ma, mo, as_stream(stream));
 }

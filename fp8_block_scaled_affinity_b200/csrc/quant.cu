@@ -63,24 +63,42 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(
     }
 }
 
-// One 128x128 block per CTA of 256 threads; thread i owns half a row
-// (64 values = 8 x 16-byte loads).  Block amax via warp shuffles + smem.
-__global__ void __launch_bounds__(256) quant_w_128x128_kernel(
+// One 128x128 block per CTA iteration, 512 threads; thread i owns a quarter
+// row (32 values = 4 x 16-byte loads).  Block amax via warp shuffles + smem.
+// The next block's vectors are loaded into registers before the current
+// block is reduced and stored, so every thread keeps its loads in flight.
+constexpr int kWThreads = 512;
+
+__global__ void __launch_bounds__(kWThreads) quant_w_128x128_kernel(
     const uint4* __restrict__ w, int64_t rows, int64_t cols, uint4* __restrict__ q,
     float* __restrict__ scales) {
-    __shared__ float warp_max[8];
+    constexpr int kWarps = kWThreads / 32;
+    __shared__ float warp_max[2][kWarps];
     const int64_t bc = cols >> 7;
     const int64_t n_blocks = (rows >> 7) * bc;
-    const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
-    for (int64_t b = blockIdx.x; b < n_blocks; b += gridDim.x) {
+    const int row = threadIdx.x >> 2, quarter = threadIdx.x & 3;
+    auto base_of = [&](int64_t b) {  // in 16-byte vectors (8 values)
         const int64_t bi = b / bc, bj = b - bi * bc;
-        const int64_t base = ((bi * 128 + row) * cols + bj * 128 + half * 64) / 8;
-        uint4 v[8];
+        return ((bi * 128 + row) * cols + bj * 128 + quarter * 32) / 8;
+    };
+    int64_t b = blockIdx.x;
+    uint4 v[4];
+    if (b < n_blocks) {
+        const int64_t base = base_of(b);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __ldcs(w + base + i);
+        for (int i = 0; i < 4; ++i) v[i] = __ldcs(w + base + i);
+    }
+    for (int it = 0; b < n_blocks; b += gridDim.x, ++it) {
+        const int64_t bn = b + gridDim.x;
+        uint4 nv[4];
+        if (bn < n_blocks) {
+            const int64_t base = base_of(bn);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) nv[i] = __ldcs(w + base + i);
+        }
         float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             amax = fmaxf(amax, fabsf(bf16_lo(v[i].x)));
             amax = fmaxf(amax, fabsf(bf16_hi(v[i].x)));
             amax = fmaxf(amax, fabsf(bf16_lo(v[i].y)));
@@ -92,17 +110,19 @@ __global__ void __launch_bounds__(256) quant_w_128x128_kernel(
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+        // two slots alternate, so one barrier per block suffices
+        float* wm = warp_max[it & 1];
+        if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = amax;
         __syncthreads();
-        amax = warp_max[0];
+        amax = wm[0];
 #pragma unroll
-        for (int i = 1; i < 8; ++i) amax = fmaxf(amax, warp_max[i]);
-        __syncthreads();  // warp_max is reused by the next block
+        for (int i = 1; i < kWarps; ++i) amax = fmaxf(amax, wm[i]);
         float scale, inv;
         scale_from_amax(amax, scale, inv);
-        const int64_t qbase = ((bi * 128 + row) * cols + bj * 128 + half * 64) / 16;
+        const int64_t bi = b / bc, bj = b - bi * bc;
+        const int64_t qbase = ((bi * 128 + row) * cols + bj * 128 + quarter * 32) / 16;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
             uint32_t o[4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -114,9 +134,11 @@ __global__ void __launch_bounds__(256) quant_w_128x128_kernel(
                 o[2 * j] = a0 | (a1 << 16);
                 o[2 * j + 1] = a2 | (a3 << 16);
             }
-            q[qbase + i] = make_uint4(o[0], o[1], o[2], o[3]);
+            __stcs(q + qbase + i, make_uint4(o[0], o[1], o[2], o[3]));
         }
         if (threadIdx.x == 0) scales[b] = scale;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = nv[i];
     }
 }
 
@@ -156,9 +178,9 @@ extern "C" MOE_API int fp8_quant_w_128x128(const uint16_t* w, int64_t rows, int6
         return MOE_ERR_ALIGN;
     const int64_t n_blocks = (rows / 128) * (cols / 128);
     int64_t grid = n_blocks;
-    const int64_t cap = int64_t(sm_count()) * 64;
+    const int64_t cap = int64_t(sm_count()) * 4;  // 4 CTAs of 512 threads per SM
     if (grid > cap) grid = cap;
-    quant_w_128x128_kernel<<<unsigned(grid), 256, 0, as_stream(stream)>>>(
+    quant_w_128x128_kernel<<<unsigned(grid), kWThreads, 0, as_stream(stream)>>>(
         reinterpret_cast<const uint4*>(w), rows, cols, reinterpret_cast<uint4*>(q), scales);
     return check_launch();
 }
