@@ -16,6 +16,8 @@
 //      and writes it K+1 times, scales transposed to the kb-major layout.
 #include <mutex>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -252,15 +254,26 @@ __global__ void __launch_bounds__(256) quant_copy_rows_kernel(
 }
 
 // y[t] = o[shared row] + sum_k g[t,k] * o[row_of_pair[t,k]] (fp32, slot
-// order), rounded once to bf16.  One warp per token, float4 per lane.
+// order), rounded once to bf16.  A work unit is one token's 64-float4 slice
+// of the row (a warp, two float4 per lane), so a small batch still spreads
+// over every SM; the rows of four slots are loaded before their FMAs, which
+// keeps eight 16-byte loads in flight per lane.
+constexpr int kCombineU = 2;      // float4 per lane per unit
+constexpr int kCombineSlots = 4;  // slots whose loads are issued together
+
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ o, int T, int d,
                                                       int K, const int32_t* __restrict__ rop,
                                                       const float* __restrict__ gate,
                                                       uint2* __restrict__ y, int* dev_status) {
     const int lane = threadIdx.x & 31;
-    const int nv = d / 4;
-    const int warps_total = gridDim.x * (blockDim.x / 32);
-    for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps_total) {
+    const int nv = d / 4;  // float4 per row, a multiple of 32
+    const int chunks = (nv + 32 * kCombineU - 1) / (32 * kCombineU);
+    const int64_t units = int64_t(T) * chunks;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t u = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); u < units;
+         u += warps_total) {
+        const int t = int(u / chunks);
+        const int c0 = int(u - int64_t(t) * chunks) * (32 * kCombineU) + lane;
         int my_row = 0;
         float my_g = 0.0f;
         if (lane < K) {
@@ -273,20 +286,44 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
             }
         }
         const int64_t shared_row = int64_t(T) * K + t;
-        for (int c = lane; c < nv; c += 32) {
-            float4 acc = __ldcs(o + shared_row * nv + c);
-            for (int k = 0; k < K; ++k) {
+        bool on[kCombineU];
+        float4 acc[kCombineU];
+#pragma unroll
+        for (int j = 0; j < kCombineU; ++j) {
+            on[j] = c0 + 32 * j < nv;
+            acc[j] = on[j] ? __ldcs(o + shared_row * nv + c0 + 32 * j) : make_float4(0, 0, 0, 0);
+        }
+        for (int k0 = 0; k0 < K; k0 += kCombineSlots) {
+            float4 v[kCombineSlots][kCombineU];
+            float g[kCombineSlots];
+#pragma unroll
+            for (int s = 0; s < kCombineSlots; ++s) {
+                const int k = min(k0 + s, K - 1);
                 const int row = __shfl_sync(0xffffffffu, my_row, k);
-                const float g = __shfl_sync(0xffffffffu, my_g, k);
-                const float4 v = __ldcs(o + int64_t(row) * nv + c);
-                acc.x = __fmaf_rn(g, v.x, acc.x);
-                acc.y = __fmaf_rn(g, v.y, acc.y);
-                acc.z = __fmaf_rn(g, v.z, acc.z);
-                acc.w = __fmaf_rn(g, v.w, acc.w);
+                g[s] = __shfl_sync(0xffffffffu, my_g, k);
+#pragma unroll
+                for (int j = 0; j < kCombineU; ++j)
+                    v[s][j] = (on[j] && k0 + s < K) ? __ldcs(o + int64_t(row) * nv + c0 + 32 * j)
+                                                    : make_float4(0, 0, 0, 0);
             }
-            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-            y[int64_t(t) * nv + c] =
+#pragma unroll
+            for (int s = 0; s < kCombineSlots; ++s) {
+                if (k0 + s >= K) break;
+#pragma unroll
+                for (int j = 0; j < kCombineU; ++j) {
+                    acc[j].x = __fmaf_rn(g[s], v[s][j].x, acc[j].x);
+                    acc[j].y = __fmaf_rn(g[s], v[s][j].y, acc[j].y);
+                    acc[j].z = __fmaf_rn(g[s], v[s][j].z, acc[j].z);
+                    acc[j].w = __fmaf_rn(g[s], v[s][j].w, acc[j].w);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kCombineU; ++j) {
+            if (!on[j]) continue;
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x, acc[j].y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z, acc[j].w);
+            y[int64_t(t) * nv + c0 + 32 * j] =
                 make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
         }
     }
@@ -408,9 +445,10 @@ extern "C" MOE_API int moe_combine(const MoeShape* shape, const float* expert_ou
     if (T == 0) return MOE_OK;
     if (!expert_out || !row_of_pair || !topk_gate || !y) return MOE_ERR_NULL;
     if (!aligned16(expert_out) || (reinterpret_cast<uintptr_t>(y) & 7)) return MOE_ERR_ALIGN;
-    int blocks = (T + 7) / 8;
-    const int cap = sm_count() * 8;
-    if (blocks > cap) blocks = cap;
+    const int64_t chunks = (shape->d / 4 + 32 * kCombineU - 1) / (32 * kCombineU);
+    const int64_t units = int64_t(T) * chunks;  // one warp each, 8 per block
+    const int64_t cap = int64_t(sm_count()) * 8;
+    const int blocks = int(std::min<int64_t>((units + 7) / 8, cap));
     combine_kernel<<<blocks, 256, 0, as_stream(stream)>>>(
         reinterpret_cast<const float4*>(expert_out), T, shape->d, shape->topk, row_of_pair,
         topk_gate, reinterpret_cast<uint2*>(y), dev_status);
