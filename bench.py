@@ -455,6 +455,8 @@ def run_gemm(args, world, rank, local):
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
 
+    form = moe.moe_grouped_gemm_form(1, cfg.m, cfg.n, moe.MOE_EPI_BF16)
+
     def gemm(a_codes=aq, a_scales=as_, c=out):
         moe.moe_grouped_gemm_fp8(1, off, cfg.m, a_codes, a_scales, cfg.k, bq, bs, cfg.n,
                                  moe.MOE_EPI_BF16, c, None, status)
@@ -509,7 +511,9 @@ def run_gemm(args, world, rank, local):
         "config": {"workload": "fp8_blockscaled_gemm", "m": cfg.m, "n": cfg.n, "k": cfg.k,
                    "out": "bf16", "parallelism": f"replicas x{world}",
                    "l2": "256 MB buffer written between timed launches"},
-        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<1> (one group, bf16 out)",
+        "roofline": {"bound": "tensor",
+                     "kernel": f"grouped_gemm_kernel<{int(form == 2)}, 0> "
+                               f"({'CTA pairs' if form == 2 else 'single CTAs'}; one group, bf16 out)",
                      "achieved": tflops / world, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": tflops / world / fp8_peak,
                      "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g} (nominal fp8:bf16)",
@@ -762,7 +766,14 @@ def run_ours(args, world, rank, local):
     # tensor-bound above it (the skewed batch: 147,456 rows on 94 experts)
     intensity = alg["flops_gemm1"] / alg["gemm1_bytes"]
     ridge = fp8_peak_burst * 1e12 / (hbm_peak * 1e9)
-    label = "grouped_gemm_kernel<256> (W13 + SwiGLU + h quant)"
+    rows_total = cfg.T * cfg.topk + cfg.T
+    form = moe.moe_grouped_gemm_form(cfg.n_routed + 1, rows_total, 2 * cfg.inter,
+                                      moe.MOE_EPI_SWIGLU_QUANT)
+    label = (f"grouped_gemm_kernel<{int(form == 2)}, 1> "
+             f"({'CTA pairs' if form == 2 else 'single CTAs'}; W13 + SwiGLU + h quant)")
+    gemm_forms = {"w13": form,
+                  "w2": moe.moe_grouped_gemm_form(cfg.n_routed + 1, rows_total, cfg.d,
+                                                  moe.MOE_EPI_F32)}
     if intensity < ridge:
         roofline = {"bound": "hbm", "kernel": label, "achieved": achieved, "peak": hbm_peak,
                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": peak_src,
@@ -803,6 +814,7 @@ def run_ours(args, world, rank, local):
                          f"{(cfg.n_routed + 1) * 3 * cfg.d * cfg.inter / 1e9:.1f} GB)"},
         "roofline": roofline,
         "expert_gemm": {"tflops": gemm_tflops, "fp8_peak_tflops": fp8_peak_burst,
+                        "ctas_per_tile": gemm_forms,
                         "frac_of_fp8_peak": gemm_tflops / fp8_peak_burst,
                         "frac_of_fp8_sustained": gemm_tflops / fp8_peak_sust,
                         "gemm1_ms": brk["gemm1_swiglu"], "gemm2_ms": brk["gemm2"],

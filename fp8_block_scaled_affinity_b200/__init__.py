@@ -14,7 +14,8 @@ from typing import Optional
 from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QUANT,  # noqa: F401
                    MoeError, MoeRouting, MoeShape, MoeWeights, fp8_quant_act_1x128,
                    fp8_quant_w_128x128, lib, make_routing, make_shape, make_weights,
-                   moe_combine, moe_grouped_gemm_fp8, moe_layer_forward,
+                   moe_combine, moe_grouped_gemm_form, moe_grouped_gemm_fp8,
+                   moe_layer_forward,
                    moe_layer_forward_host, moe_layer_host_workspace_size,
                    moe_layer_workspace_size, moe_permute, moe_permute_workspace_size, moe_quant_permute,
                    moe_read_status, moe_route, moe_route_workspace_size, moe_update_bias,

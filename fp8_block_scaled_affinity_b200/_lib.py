@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "moe_permute_static_ws": (I, [SP, P, P, P, P, P, P, P, P, P, P]),
             "moe_quant_permute": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
             "moe_grouped_gemm_fp8": (I, [I, P, I, P, P, I, P, P, I, I, P, P, P, P]),
+            "moe_grouped_gemm_form": (I, [I, I, I, I]),
             "moe_combine": (I, [SP, P, P, P, P, P, P, P]),
             "moe_update_bias": (I, [SP, P, P, P, P]),
             "moe_layer_workspace_size": (SZ, [SP]),
@@ -198,6 +199,12 @@ def moe_grouped_gemm_fp8(n_groups, group_offsets, max_rows, a, a_scales, k, w, w
         int(n_groups), _ptr(group_offsets), int(max_rows), _ptr(a), _ptr(a_scales), int(k),
         _ptr(w), _ptr(w_scales), int(n), int(epilogue), _ptr(out), _ptr(out_scales),
         _ptr(dev_status), _stream(stream)))
+
+
+def moe_grouped_gemm_form(n_groups, max_rows, n, epilogue) -> int:
+    """CTAs per tile moe_grouped_gemm_fp8 uses for these arguments on the
+    current device: 1 (single CTAs), 2 (CTA pairs), 0 (invalid arguments)."""
+    return int(lib().moe_grouped_gemm_form(int(n_groups), int(max_rows), int(n), int(epilogue)))
 
 
 def moe_combine(shape, expert_out, expert_offsets, row_of_pair, topk_gate, y,

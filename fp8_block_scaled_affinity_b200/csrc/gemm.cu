@@ -7,28 +7,40 @@
 // into a fresh TMEM buffer, and promotion warps fold it into register FP32
 // accumulators with the block's combined scale sa[token] * sb[weight block].
 //
-// Tile: 128 tokens (the MMA's M side, one token per TMEM lane, so a thread's
-// token scale is one register) x BN weight columns (N) x 128 K.
-//   BN = 256 (SwiGLU epilogue): the gate (W1) and up (W3) blocks of the same
-//     128 features, so a thread holds gate and up of the same (token,
-//     feature); 2 TMEM partial buffers, 4 smem stages of 48 KB.
-//   BN = 128 (fp32 / bf16 output): one 128-row weight block; 4 TMEM partial
-//     buffers (more slack between MMA and promotion), 4 stages of 32 KB; a
-//     warp's 32 finished row segments go to a swizzled tile in shared memory
-//     and leave as TMA bulk tensor stores (full 128-byte lines, written by
-//     the copy engine while the next tile's K loop runs); the rows of a
-//     group's ragged last warp are stored directly.
+// Each CTA owns 128 tokens (the MMA's M side, one token per TMEM lane, so a
+// thread's token scale is one register) and, per K block, a TMEM partial of
+// 128 x C columns (C = 256, or 128 for the single-CTA fp32/bf16 form).  The
+// C columns are two 128-row weight blocks: the gate (W1) and up (W3) blocks
+// of the same 128 features for the SwiGLU epilogue, two neighbouring blocks
+// of the output otherwise.
+//
+// CTA pairs (cta_group::2, the default): a cluster of two CTAs on two SMs
+// runs one M = 256, N = 256 MMA per 32-deep K step; each CTA loads its own
+// 128 tokens and ONE of the two weight blocks, so every weight byte crosses
+// L2 -> SM once per 256 tokens instead of once per 128.  The leader (rank 0)
+// issues the MMAs; both CTAs' TMA loads complete on the leader's stage
+// barrier, and the MMA commits arrive on both CTAs' barriers.  The
+// single-CTA form (cta_group::1) serves output widths that are not a
+// multiple of 256 and can be forced with MOEFP8_GEMM_PAIR=0.
+//
+// Token boxes: the TMA box of a CTA's tokens is 128, 64, 32 or 16 rows (the
+// smallest that holds its valid rows; none when it has none), so ragged
+// tails and tiny groups do not pull 128 rows through L2.  Shared-memory rows
+// past the box hold stale codes; they feed only TMEM lanes whose tokens are
+// discarded.
 //
 // Roles (384 threads, one CTA per SM, persistent over work items):
-//   warp 0       TMA producer: token tile (16 KB) + weight tile(s) per K block
-//   warp 1       TMEM owner and MMA issuer (one thread)
+//   warp 0       TMA producer
+//   warp 1       TMEM owner; in the leader, the MMA issuer (one thread)
 //   warp 2       scale loader: cp.async of the K block's 128 token scales and
-//                the weight-block scales into a small smem ring
+//                the two weight-block scales into a small smem ring
 //   warp 3       idle (its registers go to the promoters)
 //   warps 4-11   promotion + epilogue: warp w reads TMEM lanes 32*(w%4)..+31
-//                (its 32 tokens) and one half of the BN columns
+//                (its 32 tokens) and one half of the C columns
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -38,23 +50,29 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kTileBytes = 128 * 128;            // one 128 x 128 FP8 tile
-constexpr int kStages = 4;                       // smem ring of operand stages
-constexpr int kParkWarpBytes = 32 * 256;         // one warp's 32 parked rows (fp32 halves)
+constexpr int kParkWarpBytes = 2 * 4096;         // two 32-row x 128-byte output boxes
 constexpr int kMaxBufs = 4;
+constexpr int kMaxStages = 6;
 constexpr int kScaleSlots = 16;
 constexpr int kMaxGroups = 1040;
-constexpr int kBM = 128;                         // tokens per tile
+constexpr int kBM = 128;                         // tokens per CTA tile
 constexpr int kPromoters = 8;                    // promotion warps
+constexpr int kABoxes = 4;                       // token boxes of 128, 64, 32, 16 rows
 
-template <int BN>
+template <bool PAIR, bool SWIGLU>
 struct Cfg {
-    static constexpr int kStageBytes = kTileBytes + BN * 128;  // tokens + weights
-    static constexpr int kStages = moe::kStages;
+    static constexpr int kAccCols = (PAIR || SWIGLU) ? 256 : 128;  // TMEM columns per partial
+    static constexpr int kBufs = 512 / kAccCols;                   // TMEM partial buffers
+    static constexpr int kWRows = PAIR ? 128 : kAccCols;           // weight rows this CTA loads
+    static constexpr int kStageBytes = kTileBytes + kWRows * 128;  // tokens + weights
+    static constexpr int kStages = (PAIR && SWIGLU) ? 6 : 4;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kParkBytes = BN == 128 ? kPromoters * kParkWarpBytes : 0;
-    static constexpr int kBufs = 512 / BN;                     // TMEM partial buffers
-    static constexpr int kPairs = BN / 4;                      // fp32 pairs per promoter thread
-    static_assert(kBufs <= kMaxBufs, "TMEM buffers");
+    static constexpr int kParkBytes = SWIGLU ? 0 : kPromoters * kParkWarpBytes;
+    static constexpr int kPairs = kAccCols / 4;                    // fp32 pairs per promoter thread
+    static constexpr int kItemRows = PAIR ? 2 * kBM : kBM;         // tokens per work item
+    static constexpr int kMmaM = PAIR ? 256 : 128;
+    static constexpr int kCtas = PAIR ? 2 : 1;
+    static_assert(kBufs <= kMaxBufs && kStages <= kMaxStages, "ring sizes");
 };
 
 struct GemmParams {
@@ -66,16 +84,21 @@ struct GemmParams {
     int nkb;
     const float* w_scales;  // [n_groups, n/128, nkb]
     int n;                  // weight rows per group
-    int n_ftiles;           // BN-column tiles per group
+    int n_ftiles;           // column tiles per group
     int epilogue;
     void* out;
     float* out_scales;
     int* dev_status;
 };
 
+// Token tensor maps, one per box height (128, 64, 32, 16 rows).
+struct AMaps {
+    CUtensorMap m[kABoxes];
+};
+
 struct SharedState {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[kMaxBufs];
     uint64_t tempty[kMaxBufs];
     uint64_t sfull[kScaleSlots];
@@ -83,24 +106,54 @@ struct SharedState {
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
+    uint32_t peer_abort;     // cluster address of the peer CTA's abort_flag (0: no peer)
     int total_items;
     int goff[kMaxGroups + 1];
     int gstart[kMaxGroups + 1];
     alignas(16) float sa[kScaleSlots][kBM];   // token scales of one K block
-    alignas(16) float sb[kScaleSlots][2];     // the weight-block scale(s)
+    alignas(16) float sb[kScaleSlots][2];     // the two weight-block scales
     alignas(16) float red[2][2][kBM];         // [item parity][half][token] amax of h
 };
 
-template <int BN>
+template <bool PAIR, bool SWIGLU>
 constexpr size_t smem_bytes() {
-    return size_t(Cfg<BN>::kRingBytes) + Cfg<BN>::kParkBytes + sizeof(SharedState) + 1024;
+    using C = Cfg<PAIR, SWIGLU>;
+    return size_t(C::kRingBytes) + C::kParkBytes + sizeof(SharedState) + 1024;
 }
-static_assert(smem_bytes<256>() <= 232448 && smem_bytes<128>() <= 232448,
+static_assert(smem_bytes<false, false>() <= 232448 && smem_bytes<false, true>() <= 232448 &&
+                  smem_bytes<true, false>() <= 232448 && smem_bytes<true, true>() <= 232448,
               "dynamic shared memory above the sm_100 limit per CTA");
 
 // ------------------------------------------------------------- PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// Every thread of both CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -115,36 +168,77 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Arrive on a barrier of any CTA of the cluster (cluster address).  The
+// data it guards is TMEM, ordered by tcgen05 fences, so CTA-scope release
+// semantics suffice.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+}
 
-// The waiting thread is suspended until the phase completes or about
-// kSuspendNs pass, so waiting warps do not take issue slots from the others.
+// Wait forms.  kSuspend: the waiting thread is suspended until the phase
+// completes or about kSuspendNs pass, so waiting warps do not take issue
+// slots from the others (single CTAs: every arrival is local).  kPoll: the
+// same without the time hint; kSpin: test_wait, never suspends (the MMA
+// issuer of a CTA pair, whose barriers also receive the peer's arrivals).
 constexpr uint32_t kSuspendNs = 50000;
+enum WaitForm { kSuspend = 0, kPoll = 1, kSpin = 2 };
+// waits on barriers that a peer CTA also signals
+template <bool PAIR> constexpr int kRemoteWait = PAIR ? kPoll : kSuspend;
+template <bool PAIR> constexpr int kIssuerWait = PAIR ? kSpin : kSuspend;
 
+template <int FORM>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "n"(kSuspendNs)
-        : "memory");
+    if (FORM == kSuspend)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "n"(kSuspendNs)
+            : "memory");
+    else if (FORM == kPoll)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 
-// Bounded wait: returns false (and raises the CTA's abort flag and the
-// device status) when the phase does not complete within kWaitLimitNs, or
-// when another role of the CTA has already aborted.
+// Raise this CTA's abort flag (and the peer's, for a CTA pair).
+__device__ __forceinline__ void raise_abort(SharedState* ss) {
+    atomicExch(&ss->abort_flag, 1);
+    if (ss->peer_abort)
+        asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(ss->peer_abort),
+                     "r"(1)
+                     : "memory");
+}
+
+// Bounded wait: returns false (and raises the abort flags and the device
+// status) when the phase does not complete within kWaitLimitNs, or when
+// another role of the CTA (or of its peer) has already aborted.
+template <int FORM = kSuspend>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, SharedState* ss,
-                                       int* dev_status) {
-    if (mbar_try_wait(bar, parity)) return true;
+                                          int* dev_status) {
+    if (mbar_try_wait<FORM>(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<FORM>(bar, parity)) return true;
         if ((it & 15) == 0) {
             if (*reinterpret_cast<volatile int*>(&ss->abort_flag)) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                atomicExch(&ss->abort_flag, 1);
+                raise_abort(ss);
                 set_status(dev_status, MOE_DEV_TIMEOUT);
                 return false;
             }
@@ -152,13 +246,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, SharedS
     }
 }
 
+// 2D tile load global -> this CTA's shared memory, completing on `bar`.
+// PAIR: the .cta_group::2 form, whose barrier may be the leader CTA's
+// (a cluster address).  No multicast.
+template <bool PAIR>
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
+    if (PAIR)
+        asm volatile(
+            "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+            "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+            "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+            : "memory");
 }
 
 // 4-byte asynchronous copy global -> shared; src_bytes = 0 writes a zero.
@@ -180,6 +285,31 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// TMEM allocation of all 512 columns (both CTAs of a pair allocate together).
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc_all(uint32_t dst_smem) {
+    if (PAIR) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                         dst_smem)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                         dst_smem)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_free_all(uint32_t base) {
+    if (PAIR)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(base)
+                     : "memory");
+    else
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(base)
+                     : "memory");
+}
+
 // K-major operand tile in shared memory, 128-byte swizzle: rows of 128 bytes
 // (one 128-deep K block of E4M3), 8-row atoms 1024 bytes apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -197,19 +327,49 @@ __device__ __forceinline__ uint32_t idesc_e4m3(int m, int n) {
     return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
 }
 
+// PAIR: one M = 256 MMA over both CTAs (A rows 0-127 and B rows 0-127 from
+// the leader's shared memory, rows 128-255 from the peer's, same offsets).
+template <bool PAIR>
 __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+    if (PAIR)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// Arrive on `bar` of this CTA once the MMAs issued so far have completed.
+template <bool PAIR>
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
+    if (PAIR)
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+            : "memory");
+    else
+        asm volatile(
+            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+            : "memory");
+}
+// As mma_commit, arriving on the barrier at the same offset in both CTAs of
+// a pair.
+template <bool PAIR>
+__device__ __forceinline__ void mma_commit_both(uint32_t bar) {
+    if (PAIR)
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+            " [%0], %1;" ::"r"(bar),
+            "h"(uint16_t(3))
+            : "memory");
+    else
+        mma_commit<false>(bar);
 }
 
 // 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers; the
@@ -299,11 +459,12 @@ __device__ __forceinline__ void set_max_regs_dec() {
 // ------------------------------------------------------------- schedule
 struct Item {
     int g;      // group
-    int f;      // BN-column tile
-    int row0;   // first token row
-    int ntok;   // valid tokens (<= 128)
+    int f;      // column tile
+    int row0;   // first token row of the item (of the pair's 256 for a CTA pair)
+    int rows;   // rows of the group from row0 on (may exceed the item)
 };
 
+template <int ITEM_ROWS>
 __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmParams& p, int item) {
     int lo = 0, hi = p.n_groups;
     while (hi - lo > 1) {
@@ -315,66 +476,96 @@ __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmPar
     it.g = lo;
     const int local = item - ss->gstart[lo];
     const int rows = ss->goff[lo + 1] - ss->goff[lo];
-    const int mtiles = (rows + kBM - 1) / kBM;
+    const int mtiles = (rows + ITEM_ROWS - 1) / ITEM_ROWS;
     it.f = local / mtiles;
     const int mt = local - it.f * mtiles;
-    it.row0 = ss->goff[lo] + mt * kBM;
-    it.ntok = min(kBM, rows - mt * kBM);
+    it.row0 = ss->goff[lo] + mt * ITEM_ROWS;
+    it.rows = rows - mt * ITEM_ROWS;
     return it;
 }
 
-// 128-row weight block(s) of a tile: first row inside the stacked
-// [n_groups * n, k] matrix and block-row index (for its scales).
-template <int BN>
-__device__ __forceinline__ void weight_blocks(const GemmParams& p, const Item& w, int& r0, int& r1,
-                                              int& b0, int& b1) {
-    if (BN == 256) {
-        b0 = w.f;                   // gate rows f*128 .. of W1
-        b1 = p.n / 256 + w.f;       // up rows (n/2 + f*128) .. of W3
+// Valid tokens of CTA `rank` in an item (0..128).
+__device__ __forceinline__ int cta_tokens(const Item& w, int rank) {
+    return max(0, min(kBM, w.rows - kBM * rank));
+}
+
+// Token box for n valid rows: index into AMaps (128, 64, 32, 16 rows) and
+// its bytes; n == 0 loads nothing.
+__device__ __forceinline__ int box_index(int n) {
+    return n > 64 ? 0 : n > 32 ? 1 : n > 16 ? 2 : 3;
+}
+__device__ __forceinline__ uint32_t box_bytes(int n) {
+    return n == 0 ? 0u : uint32_t(kTileBytes >> box_index(n));
+}
+
+// The two 128-row weight blocks of a column tile (block-row indices inside
+// one group's [n, k] matrix): their scales go to sb[0] and sb[1], and a CTA
+// of a pair loads block b[rank].
+template <bool PAIR, bool SWIGLU>
+__device__ __forceinline__ void weight_blocks(const GemmParams& p, const Item& w, int& b0,
+                                              int& b1) {
+    if (SWIGLU) {
+        b0 = w.f;                // gate rows f*128 .. of W1
+        b1 = p.n / 256 + w.f;    // up rows (n/2 + f*128) .. of W3
+    } else if (PAIR) {
+        b0 = 2 * w.f;
+        b1 = 2 * w.f + 1;
     } else {
         b0 = w.f;
         b1 = w.f;
     }
-    r0 = w.g * p.n + b0 * 128;
-    r1 = w.g * p.n + b1 * 128;
 }
 
 // ================================================= TMA producer (warp 0)
-template <int BN>
-__device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap& map_w,
-                                         const CUtensorMap& map_a, uint8_t* smem,
-                                         SharedState* ss) {
-    using C = Cfg<BN>;
+template <bool PAIR, bool SWIGLU>
+__device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap* map_w,
+                                         const AMaps& maps_a, uint8_t* smem, SharedState* ss,
+                                         int rank, int unit, int units) {
+    using C = Cfg<PAIR, SWIGLU>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     uint32_t it = 0;
     uint32_t issued_mask = 0, issued_parity = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(ss, p, item);
-        int wr0, wr1, b0, b1;
-        weight_blocks<BN>(p, w, wr0, wr1, b0, b1);
+    for (int item = unit; ok && item < total_items; item += units) {
+        const Item w = decode_item<C::kItemRows>(ss, p, item);
+        int b0, b1;
+        weight_blocks<PAIR, SWIGLU>(p, w, b0, b1);
+        const int n0 = cta_tokens(w, 0);
+        const int n1 = PAIR ? cta_tokens(w, 1) : 0;
+        const int my_n = rank ? n1 : n0;
+        const CUtensorMap* map_a = &maps_a.m[box_index(my_n)];
+        const int a_y = w.row0 + kBM * rank;
+        // bytes landing on the stage barrier: every CTA's tokens and weights
+        const uint32_t tx = box_bytes(n0) + box_bytes(n1) + uint32_t(C::kCtas * C::kWRows * 128);
+        const int wr_mine = w.g * p.n + (rank ? b1 : b0) * 128;
+        const int wr_second = w.g * p.n + b1 * 128;  // single-CTA SwiGLU: the up block
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
             const int s = it % C::kStages;
             const uint32_t par = ((it / C::kStages) & 1u);
-            if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
+            if (lane == 0)
+                ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->empty[s]), par ^ 1u, ss,
+                                                  p.dev_status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             if (lane == 0) {
                 uint8_t* st = smem + size_t(s) * C::kStageBytes;
-                const uint32_t fb = smem_u32(&ss->full[s]);
-                mbar_arrive_expect_tx(fb, uint32_t(C::kStageBytes));
-                tma_load_2d(smem_u32(st), &map_a, fb, kb * 128, w.row0);
-                tma_load_2d(smem_u32(st + kTileBytes), &map_w, fb, kb * 128, wr0);
-                if (BN == 256)
-                    tma_load_2d(smem_u32(st + 2 * kTileBytes), &map_w, fb, kb * 128, wr1);
+                const uint32_t local_full = smem_u32(&ss->full[s]);
+                const uint32_t fb = PAIR ? mapa(local_full, 0) : local_full;
+                if (rank == 0) mbar_arrive_expect_tx(local_full, tx);
+                if (my_n > 0) tma_load_2d<PAIR>(smem_u32(st), map_a, fb, kb * 128, a_y);
+                tma_load_2d<PAIR>(smem_u32(st + kTileBytes), map_w, fb, kb * 128, wr_mine);
+                if (!PAIR && SWIGLU)
+                    tma_load_2d<PAIR>(smem_u32(st + 2 * kTileBytes), map_w, fb, kb * 128,
+                                      wr_second);
                 issued_mask |= 1u << s;
                 issued_parity = (issued_parity & ~(1u << s)) | (par << s);
             }
         }
     }
-    if (!ok && lane == 0) {
-        // let loads already in flight land before the CTA leaves
+    if (!ok && lane == 0 && rank == 0) {
+        // let loads already in flight land before the CTA leaves (the stage
+        // barriers of a pair are the leader's)
         for (int s = 0; s < C::kStages; ++s)
             if ((issued_mask >> s) & 1u)
                 mbar_wait(smem_u32(&ss->full[s]), (issued_parity >> s) & 1u, ss, nullptr);
@@ -384,19 +575,23 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap&
 
 // ================================================= scale loader (warp 2)
 // cp.async of each K block's 128 token scales (kb-major, so they are
-// contiguous) and the tile's weight-block scale(s); the copies arrive on
+// contiguous) and the tile's two weight-block scales; the copies arrive on
 // sfull when they land.
-template <int BN>
-__device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* ss) {
+template <bool PAIR, bool SWIGLU>
+__device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* ss, int rank,
+                                             int unit, int units) {
+    using C = Cfg<PAIR, SWIGLU>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     const int nbr = p.n / 128;  // weight block rows per group
     uint32_t cit = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-        const Item w = decode_item(ss, p, item);
-        int wr0, wr1, b0, b1;
-        weight_blocks<BN>(p, w, wr0, wr1, b0, b1);
+    for (int item = unit; ok && item < total_items; item += units) {
+        const Item w = decode_item<C::kItemRows>(ss, p, item);
+        int b0, b1;
+        weight_blocks<PAIR, SWIGLU>(p, w, b0, b1);
+        const int my_n = cta_tokens(w, rank);
+        const int my_row0 = w.row0 + kBM * rank;
         const float* sb0 = p.w_scales + (size_t(w.g) * nbr + b0) * p.nkb;
         const float* sb1 = p.w_scales + (size_t(w.g) * nbr + b1) * p.nkb;
         for (int kb = 0; kb < p.nkb; ++kb, ++cit) {
@@ -406,12 +601,12 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
                                p.dev_status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            const float* sa = p.a_scales + size_t(kb) * p.max_rows + w.row0;
+            const float* sa = p.a_scales + size_t(kb) * p.max_rows + my_row0;
 #pragma unroll
             for (int i = 0; i < kBM / 32; ++i) {
                 const int j = lane + 32 * i;
-                const bool real = j < w.ntok;  // rows past the group get 0
-                cp_async4(&ss->sa[c][j], real ? sa + j : sa, real ? 4u : 0u);
+                const bool real = j < my_n;  // rows past the group get 0
+                cp_async4(&ss->sa[c][j], real ? sa + j : p.a_scales, real ? 4u : 0u);
             }
             if (lane == 0) {
                 cp_async4(&ss->sb[c][0], sb0 + kb, 4u);
@@ -424,49 +619,51 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
     __syncwarp();
 }
 
-// ================================================= MMA issuer (warp 1)
-template <int BN>
+// ================================================= MMA issuer (warp 1 of the leader)
+template <bool PAIR, bool SWIGLU>
 __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, SharedState* ss,
-                                           uint32_t tmem_base) {
-    using C = Cfg<BN>;
+                                           uint32_t tmem_base, int unit, int units) {
+    using C = Cfg<PAIR, SWIGLU>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     if (lane == 0) {
         uint32_t it = 0, tb = 0;
         bool ok = true;
-        const uint32_t idesc = idesc_e4m3(128, BN);
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        const uint32_t idesc = idesc_e4m3(C::kMmaM, C::kAccCols);
+        for (int item = unit; ok && item < total_items; item += units) {
             for (int kb = 0; kb < p.nkb; ++kb, ++it, ++tb) {
                 const int s = it % C::kStages;
                 const uint32_t buf = tb % C::kBufs;
                 const uint32_t tpar = (tb / C::kBufs) & 1u;
-                ok = mbar_wait(smem_u32(&ss->tempty[buf]), tpar ^ 1u, ss, p.dev_status);
+                ok = mbar_wait<kIssuerWait<PAIR>>(smem_u32(&ss->tempty[buf]), tpar ^ 1u, ss,
+                                                   p.dev_status);
                 if (!ok) break;
-                ok = mbar_wait(smem_u32(&ss->full[s]), (it / C::kStages) & 1u, ss, p.dev_status);
+                ok = mbar_wait<kIssuerWait<PAIR>>(smem_u32(&ss->full[s]), (it / C::kStages) & 1u, ss,
+                                                   p.dev_status);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + size_t(s) * C::kStageBytes);
-                const uint32_t d = tmem_base + buf * BN;
+                const uint32_t d = tmem_base + buf * C::kAccCols;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_e4m3(d, sw128_desc(st + kk * 32), sw128_desc(st + kTileBytes + kk * 32),
-                             idesc, kk > 0 ? 1u : 0u);
-                mma_commit(smem_u32(&ss->empty[s]));
-                mma_commit(smem_u32(&ss->tfull[buf]));
+                    mma_e4m3<PAIR>(d, sw128_desc(st + kk * 32),
+                                   sw128_desc(st + kTileBytes + kk * 32), idesc, kk > 0 ? 1u : 0u);
+                mma_commit_both<PAIR>(smem_u32(&ss->empty[s]));
+                mma_commit_both<PAIR>(smem_u32(&ss->tfull[buf]));
             }
         }
         // all MMAs issued by this thread have completed once drain fires
-        mma_commit(smem_u32(&ss->drain));
+        mma_commit<PAIR>(smem_u32(&ss->drain));
         mbar_wait(smem_u32(&ss->drain), 0, ss, nullptr);
     }
     __syncwarp();
 }
 
-// fp32 / bf16 epilogue: a warp's 32 finished row segments (64 values each)
-// are written into its parking tile in shared memory in the 128-byte swizzle
-// layout of the output tensor map (16-byte chunk c of row r at c ^ (r % 8)),
-// then one lane hands the tile to the TMA engine as bulk tensor stores.  The
-// next tile waits until the engine has read the parking tile.
+// fp32 / bf16 epilogue: a warp's 32 finished row segments are written into
+// its parking tile in shared memory in the 128-byte swizzle layout of the
+// output tensor map (16-byte chunk c of row r at c ^ (r % 8)), two 4 KB
+// boxes at a time, then one lane hands them to the TMA engine as bulk
+// tensor stores.  Before the tile is rewritten, the engine must have read it.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -487,31 +684,132 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ uint32_t bf16x2_bits(float2 f) {
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<uint32_t*>(&b2);
+}
+
+// Write this thread's NP fp32 pairs (one row, NP*2 consecutive columns
+// from `col`) of the warp's 32 rows: through the parking tile and bulk
+// tensor stores when all 32 rows are valid, else direct stores of valid rows.
+template <int NP>
+__device__ __forceinline__ void store_rows(const GemmParams& p, const uint64_t (&acc2)[NP],
+                                           char* wpark, const CUtensorMap* map_o, int lane,
+                                           int rows_here, size_t row, int y0, int col) {
+    const bool bf16_out = p.epilogue == MOE_EPI_BF16;
+    if (rows_here >= 32) {
+        if (bf16_out) {
+            // boxes of 64 bf16 (32 pairs); two per round
+            constexpr int kBoxes = NP / 32;
+#pragma unroll
+            for (int r0 = 0; r0 < kBoxes; r0 += 2) {
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+#pragma unroll
+                for (int b = r0; b < r0 + 2 && b < kBoxes; ++b) {
+                    char* box = wpark + (b - r0) * 4096;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int q0 = 32 * b + 4 * j;
+                        *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                            make_uint4(bf16x2_bits(unpack2(acc2[q0])),
+                                       bf16x2_bits(unpack2(acc2[q0 + 1])),
+                                       bf16x2_bits(unpack2(acc2[q0 + 2])),
+                                       bf16x2_bits(unpack2(acc2[q0 + 3])));
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int b = r0; b < r0 + 2 && b < kBoxes; ++b)
+                        tma_store_2d(map_o, smem_u32(wpark + (b - r0) * 4096), col + 64 * b, y0);
+                    bulk_commit();
+                }
+            }
+        } else {
+            // boxes of 32 fp32 (16 pairs); two per round
+            constexpr int kBoxes = NP / 16;
+#pragma unroll
+            for (int r0 = 0; r0 < kBoxes; r0 += 2) {
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
+#pragma unroll
+                for (int b = r0; b < r0 + 2; ++b) {
+                    char* box = wpark + (b - r0) * 4096;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float2 a = unpack2(acc2[16 * b + 2 * j]);
+                        const float2 c = unpack2(acc2[16 * b + 2 * j + 1]);
+                        *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                            make_float4(a.x, a.y, c.x, c.y);
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(map_o, smem_u32(wpark), col + 32 * r0, y0);
+                    tma_store_2d(map_o, smem_u32(wpark + 4096), col + 32 * (r0 + 1), y0);
+                    bulk_commit();
+                }
+            }
+        }
+    } else if (lane < rows_here) {
+        // the group's ragged last rows: plain stores, only the valid rows
+        if (bf16_out) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row * p.n + col);
+#pragma unroll
+            for (int j = 0; j < NP / 4; ++j)
+                dst[j] = make_uint4(bf16x2_bits(unpack2(acc2[4 * j])),
+                                    bf16x2_bits(unpack2(acc2[4 * j + 1])),
+                                    bf16x2_bits(unpack2(acc2[4 * j + 2])),
+                                    bf16x2_bits(unpack2(acc2[4 * j + 3])));
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.n + col);
+#pragma unroll
+            for (int i = 0; i < NP / 2; ++i) {
+                const float2 a = unpack2(acc2[2 * i]), c = unpack2(acc2[2 * i + 1]);
+                dst[i] = make_float4(a.x, a.y, c.x, c.y);
+            }
+        }
+    }
+}
+
 // ================================================= promotion + epilogue (warps 4-11)
-// Thread (warp w, lane l) owns token row r = 32*(w%4) + l of the tile and
-// half h = (w-4)/4 of its columns:
-//   BN = 256 (SwiGLU): gate columns [64h, 64h+64) and up columns
-//     [128+64h, 128+64h+64) (the same 64 features of W1 and W3);
-//   BN = 128: columns [64h, 64h+64) of the single weight block.
-template <int BN>
+// Thread (warp w, lane l) owns token row r = 32*(w%4) + l of its CTA's 128
+// and half h = (w-4)/4 of the partial's columns:
+//   SwiGLU: gate columns [64h, 64h+64) and up columns [128+64h, 128+64h+64)
+//     (the same 64 features of W1 and W3);
+//   fp32 / bf16, C = 256: columns [128h, 128h+128) (weight block h);
+//   fp32 / bf16, C = 128: columns [64h, 64h+64) of the single weight block.
+template <bool PAIR, bool SWIGLU>
 __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, char* park_area,
-                                         uint32_t tmem_base, const CUtensorMap* map_o) {
-    using C = Cfg<BN>;
+                                         uint32_t tmem_base, const CUtensorMap* map_o, int rank,
+                                         int unit, int units) {
+    using C = Cfg<PAIR, SWIGLU>;
+    constexpr bool kWide = C::kAccCols == 256;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     const int q = warp & 3;
     const int half = (warp - 4) >> 2;
-    const int r = q * 32 + lane;  // token row inside the tile
+    const int r = q * 32 + lane;  // token row inside the CTA's tile
     const uint32_t lane_addr = tmem_base + (uint32_t(q * 32) << 16);
-    const bool bf16_out = p.epilogue == MOE_EPI_BF16;
-    const int c0 = BN == 256 ? half * 64 : half * 64;        // first column of chunk 0
-    const int c1 = BN == 256 ? 128 + half * 64 : half * 64;  // first column of chunk 1
+    // TMEM columns of the two loads per K block and the weight block of each
+    int c0, c1, sel0, sel1;
+    if (SWIGLU) {
+        c0 = 64 * half; c1 = 128 + 64 * half; sel0 = 0; sel1 = 1;
+    } else if (kWide) {
+        c0 = 128 * half; c1 = 128 * half + 64; sel0 = half; sel1 = half;
+    } else {
+        c0 = 64 * half; c1 = 64 * half + 32; sel0 = 0; sel1 = 0;
+    }
     uint32_t tb = 0, cit = 0, parity = 0;
     bool ok = true;
     // this warp's parking tile (swizzled, 1024-byte aligned)
     char* const wpark = park_area + (warp - 4) * kParkWarpBytes;
-    for (int item = blockIdx.x; item < total_items; item += gridDim.x, parity ^= 1u) {
-        const Item w = decode_item(ss, p, item);
+    for (int item = unit; item < total_items; item += units, parity ^= 1u) {
+        const Item w = decode_item<C::kItemRows>(ss, p, item);
         uint64_t acc2[C::kPairs];  // fp32 accumulator pairs
 #pragma unroll
         for (int i = 0; i < C::kPairs; ++i) acc2[i] = 0;
@@ -519,7 +817,8 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
             const uint32_t buf = tb % C::kBufs;
             const int c = cit % kScaleSlots;
             if (lane == 0) {
-                ok = mbar_wait(smem_u32(&ss->tfull[buf]), (tb / C::kBufs) & 1u, ss, p.dev_status);
+                ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->tfull[buf]), (tb / C::kBufs) & 1u,
+                                                   ss, p.dev_status);
                 if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (cit / kScaleSlots) & 1u, ss,
                                        p.dev_status);
             }
@@ -528,111 +827,54 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
             __syncwarp();
             tc_fence_after();
             const float sa = ss->sa[c][r];
-            const float s0 = sa * ss->sb[c][0];
-            const float s1 = sa * ss->sb[c][1];
+            const float s0 = sa * ss->sb[c][sel0];
+            const float s1 = sa * ss->sb[c][sel1];
             const uint64_t s0x2 = pack2(__float_as_uint(s0), __float_as_uint(s0));
             const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
-            if (BN == 256) {
+            const uint32_t tbase = lane_addr + buf * C::kAccCols;
+            const uint32_t tempty = smem_u32(&ss->tempty[buf]);
+            if (kWide) {
                 uint32_t v[64];
-                tmem_ld64(lane_addr + buf * BN + c0, v);
+                tmem_ld64(tbase + c0, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
-                tmem_ld64(lane_addr + buf * BN + c1, v);
+                tmem_ld64(tbase + c1, v);
                 // the partial is in registers: hand the TMEM buffer back to
-                // the MMA before the last FMAs
+                // the MMA (the leader's barrier) before the last FMAs
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
+                if (lane == 0) {
+                    if (PAIR) mbar_arrive_cluster(mapa(tempty, 0));
+                    else mbar_arrive(tempty);
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     ffma2(acc2[32 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
             } else {
                 uint32_t v[32];
-                tmem_ld32(lane_addr + buf * BN + c0, v);
+                tmem_ld32(tbase + c0, v);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
-                tmem_ld32(lane_addr + buf * BN + c0 + 32, v);
+                tmem_ld32(tbase + c1, v);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
+                if (lane == 0) mbar_arrive(tempty);
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    ffma2(acc2[16 + i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
+                    ffma2(acc2[16 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
             }
         }
         // ---------------- epilogue
-        const bool row_ok = r < w.ntok;
-        const size_t row = size_t(w.row0) + r;
-        if (BN == 128) {
-            const int rows_here = w.ntok - q * 32;  // valid rows of this warp's 32
-            const int col = w.f * 128 + half * 64;
-            if (rows_here >= 32) {
-                // the engine has read the previous tile out of the parking tile
-                if (lane == 0) bulk_wait_read();
-                __syncwarp();
-                if (bf16_out) {
-                    // one 128-byte box: 64 bf16 per row
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t u[4];
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const float2 f = unpack2(acc2[4 * j + h]);
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x, f.y);
-                            u[h] = *reinterpret_cast<uint32_t*>(&b2);
-                        }
-                        *reinterpret_cast<uint4*>(wpark + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-                            make_uint4(u[0], u[1], u[2], u[3]);
-                    }
-                } else {
-                    // two 128-byte boxes: columns [0, 32) and [32, 64) of the half
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 a = unpack2(acc2[2 * i]), b = unpack2(acc2[2 * i + 1]);
-                        char* box = wpark + (i >> 3) * 4096;
-                        *reinterpret_cast<float4*>(box + lane * 128 + (((i & 7) ^ (lane & 7)) * 16)) =
-                            make_float4(a.x, a.y, b.x, b.y);
-                    }
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    const int y = w.row0 + q * 32;
-                    if (bf16_out) {
-                        tma_store_2d(map_o, smem_u32(wpark), col, y);
-                    } else {
-                        tma_store_2d(map_o, smem_u32(wpark), col, y);
-                        tma_store_2d(map_o, smem_u32(wpark + 4096), col + 32, y);
-                    }
-                    bulk_commit();
-                }
-            } else if (row_ok) {
-                // the group's ragged last rows: plain stores, only the valid rows
-                if (bf16_out) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                          row * p.n + col);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t u[4];
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const float2 f = unpack2(acc2[4 * j + h]);
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x, f.y);
-                            u[h] = *reinterpret_cast<uint32_t*>(&b2);
-                        }
-                        dst[j] = make_uint4(u[0], u[1], u[2], u[3]);
-                    }
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.n + col);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 a = unpack2(acc2[2 * i]), b = unpack2(acc2[2 * i + 1]);
-                        dst[i] = make_float4(a.x, a.y, b.x, b.y);
-                    }
-                }
-            }
+        const int my_n = cta_tokens(w, rank);
+        const int my_row0 = w.row0 + kBM * rank;
+        const bool row_ok = r < my_n;
+        const size_t row = size_t(my_row0) + r;
+        if (!SWIGLU) {
+            constexpr int kCols = C::kAccCols / 2;  // this thread's columns
+            store_rows<C::kPairs>(p, acc2, wpark, map_o, lane, my_n - q * 32, row,
+                                  my_row0 + q * 32, w.f * C::kAccCols + half * kCols);
         } else {
             // h = silu(gate) * up for this thread's 64 features, then the
             // 1x128 scale of the token's 128 features (both halves).
@@ -681,24 +923,28 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
         if (any_abort) break;
     }
     // every bulk store of this warp has completed before the CTA moves on
-    if (BN == 128 && lane == 0) bulk_wait_all();
+    if (!SWIGLU && lane == 0) bulk_wait_all();
     __syncwarp();
     tc_fence_before();
 }
 
 // ----------------------------------------------------------------- kernel
-template <int BN>
+template <bool PAIR, bool SWIGLU>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
-                        const __grid_constant__ CUtensorMap map_a,
+                        const __grid_constant__ AMaps maps_a,
                         const __grid_constant__ CUtensorMap map_o, const GemmParams p) {
-    using C = Cfg<BN>;
+    using C = Cfg<PAIR, SWIGLU>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     SharedState* ss =
         reinterpret_cast<SharedState*>(smem + size_t(C::kRingBytes) + C::kParkBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // a CTA pair works on one item at a time; a single CTA is its own unit
+    const int rank = PAIR ? int(cluster_rank()) : 0;
+    const int unit = PAIR ? int(cluster_index()) : int(blockIdx.x);
+    const int units = PAIR ? int(cluster_count()) : int(gridDim.x);
 
     // ---- prologue: barriers, TMEM, schedule
     if (threadIdx.x == 0) {
@@ -708,7 +954,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < C::kBufs; ++b) {
             mbar_init(smem_u32(&ss->tfull[b]), 1);
-            mbar_init(smem_u32(&ss->tempty[b]), kPromoters);
+            mbar_init(smem_u32(&ss->tempty[b]), kPromoters * C::kCtas);
         }
         for (int c = 0; c < kScaleSlots; ++c) {
             mbar_init(smem_u32(&ss->sfull[c]), 32);
@@ -716,14 +962,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(smem_u32(&ss->drain), 1);
         ss->abort_flag = 0;
+        ss->peer_abort = PAIR ? mapa(smem_u32(&ss->abort_flag), uint32_t(rank ^ 1)) : 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                         smem_u32(&ss->tmem_base))
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
+    if (warp == 1) tmem_alloc_all<PAIR>(smem_u32(&ss->tmem_base));
     // group offsets (validated) and an exclusive scan of work items per group
     const int G = p.n_groups;
     int bad = 0;
@@ -748,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int v = 0;
             if (g < G) {
                 const int rows = ss->goff[g + 1] - ss->goff[g];
-                v = ((rows + kBM - 1) / kBM) * p.n_ftiles;
+                v = ((rows + C::kItemRows - 1) / C::kItemRows) * p.n_ftiles;
             }
             vals[j] = v;
             sum += v;
@@ -778,34 +1020,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    // the peer's barriers are initialised before anyone signals them
+    if (PAIR) cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = ss->tmem_base;
 
     if (warp < 4) {
         set_max_regs_dec<72>();
-        if (warp == 0) producer<BN>(p, map_w, map_a, smem, ss);
-        else if (warp == 1) mma_issuer<BN>(p, smem, ss, tmem_base);
-        else if (warp == 2) scale_loader<BN>(p, ss);
+        if (warp == 0) producer<PAIR, SWIGLU>(p, &map_w, maps_a, smem, ss, rank, unit, units);
+        else if (warp == 1 && rank == 0)
+            mma_issuer<PAIR, SWIGLU>(p, smem, ss, tmem_base, unit, units);
+        else if (warp == 2) scale_loader<PAIR, SWIGLU>(p, ss, rank, unit, units);
     } else {
         set_max_regs_inc<208>();
-        promoter<BN>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base, &map_o);
+        promoter<PAIR, SWIGLU>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base,
+                               &map_o, rank, unit, units);
     }
 
     __syncthreads();
+    // neither CTA of a pair leaves (or frees TMEM) while the other may still
+    // signal its barriers or the leader's MMAs may still write its TMEM
+    if (PAIR) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem_base)
-                     : "memory");
+        tmem_free_all<PAIR>(tmem_base);
     }
 }
 
-template <int BN>
-int launch(const GemmParams& p, const CUtensorMap& mw, const CUtensorMap& ma,
-           const CUtensorMap& mo, cudaStream_t st) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem_bytes<BN>())) != cudaSuccess)
+// CTA pairs the device can hold at once for a pair kernel (cached per device).
+template <bool SWIGLU>
+int pair_units() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem_bytes<true, SWIGLU>();
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<true, SWIGLU>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem_bytes<true, SWIGLU>())) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, SWIGLU>, &cfg) !=
+                cudaSuccess || n < 1) {
+            (void)cudaGetLastError();
+            n = -1;  // pairs unavailable on this device
+        }
+        cache[dev] = std::min(n, sm_count() / 2);
+    }
+    return cache[dev];
+}
+
+template <bool PAIR, bool SWIGLU>
+int launch(const GemmParams& p, const CUtensorMap& mw, const AMaps& ma, const CUtensorMap& mo,
+           int units, cudaStream_t st) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR, SWIGLU>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem_bytes<PAIR, SWIGLU>())) != cudaSuccess)
         return MOE_ERR_CUDA;
-    grouped_gemm_kernel<BN><<<sm_count(), kThreads, smem_bytes<BN>(), st>>>(mw, ma, mo, p);
+    if (!PAIR) {
+        grouped_gemm_kernel<PAIR, SWIGLU><<<sm_count(), kThreads, smem_bytes<PAIR, SWIGLU>(), st>>>(
+            mw, ma, mo, p);
+        return check_launch();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * units, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes<PAIR, SWIGLU>();
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<PAIR, SWIGLU>, mw, ma, mo, p) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return check_launch();
 }
 
@@ -871,9 +1170,35 @@ bool device_is_sm100() {
     return major == 10;
 }
 
+// Kernel form of a call: the number of CTA pairs to launch, or 0 for single
+// CTAs.  CTA pairs halve the operand traffic per SM but double the work per
+// TMEM round trip, which pays only when most items hold 256 tokens: measured
+// on B200, pairs run the 4096-row plain GEMM 1.36x faster and a 257-expert
+// prefill W13 (about 144 rows per group) 1.5x slower.  Default: pairs for
+// fp32/bf16 output with at least 256 rows per group on average.
+// MOEFP8_GEMM_PAIR=1 / =0 in the environment forces either form (pairs only
+// where the output width is a multiple of 256).
+int gemm_pair_units(int n_groups, int max_rows, int n, bool swiglu) {
+    const char* env = getenv("MOEFP8_GEMM_PAIR");
+    const bool pair_shape = swiglu || n % 256 == 0;
+    bool want = pair_shape && !swiglu && max_rows / n_groups >= 256;
+    if (env && env[0] == '0') want = false;
+    if (env && env[0] == '1') want = pair_shape;
+    if (!want) return 0;
+    return std::max(0, swiglu ? pair_units<true>() : pair_units<false>());
+}
+
 }  // namespace moe
 
 using namespace moe;
+
+extern "C" MOE_API int moe_grouped_gemm_form(int n_groups, int max_rows, int n, int epilogue) {
+    if (n_groups < 1 || max_rows < 0 || n <= 0 || n % 128) return 0;
+    if (epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_SWIGLU_QUANT)
+        return 0;
+    if (epilogue == MOE_EPI_SWIGLU_QUANT && n % 256) return 0;
+    return gemm_pair_units(n_groups, max_rows, n, epilogue == MOE_EPI_SWIGLU_QUANT) > 0 ? 2 : 1;
+}
 
 extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_offsets,
                                             int max_rows, const uint8_t* a,
@@ -895,6 +1220,10 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     if (int64_t(n_groups) * n > INT32_MAX) return MOE_ERR_SHAPE;
     if (!device_is_sm100()) return MOE_ERR_DEVICE;
 
+    const bool swiglu = epilogue == MOE_EPI_SWIGLU_QUANT;
+    const int units = gemm_pair_units(n_groups, max_rows, n, swiglu);
+    const bool pair = units > 0;
+
     GemmParams p;
     p.group_offsets = group_offsets;
     p.n_groups = n_groups;
@@ -904,20 +1233,25 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     p.nkb = k / 128;
     p.w_scales = w_scales;
     p.n = n;
-    const bool swiglu = epilogue == MOE_EPI_SWIGLU_QUANT;
-    p.n_ftiles = swiglu ? n / 256 : n / 128;
+    p.n_ftiles = (pair || swiglu) ? n / 256 : n / 128;
     p.epilogue = epilogue;
     p.out = out;
     p.out_scales = out_scales;
     p.dev_status = dev_status;
 
-    CUtensorMap mw, ma, mo;
-    if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128) ||
-        !make_map(&ma, a, uint64_t(max_rows), uint64_t(k), 128))
-        return MOE_ERR_CUDA;
+    CUtensorMap mw, mo;
+    AMaps ma;
+    if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128)) return MOE_ERR_CUDA;
+    for (int i = 0; i < kABoxes; ++i)
+        if (!make_map(&ma.m[i], a, uint64_t(max_rows), uint64_t(k), uint32_t(128 >> i)))
+            return MOE_ERR_CUDA;
     if (swiglu) mo = mw;  // unused by the SwiGLU epilogue
     else if (!make_out_map(&mo, out, uint64_t(max_rows), uint64_t(n), epilogue == MOE_EPI_BF16))
         return MOE_ERR_CUDA;
-    return swiglu ? launch<256>(p, mw, ma, mo, as_stream(stream))
-                  : launch<128>(p, mw, ma, mo, as_stream(stream));
+    cudaStream_t st = as_stream(stream);
+    if (pair)
+        return swiglu ? launch<true, true>(p, mw, ma, mo, units, st)
+                      : launch<true, false>(p, mw, ma, mo, units, st);
+    return swiglu ? launch<false, true>(p, mw, ma, mo, 0, st)
+                  : launch<false, false>(p, mw, ma, mo, 0, st);
 }

@@ -244,12 +244,26 @@ MOE_API int moe_permute_static_ws(const MoeShape* shape, const int32_t* topk_idx
  *                          along its n/2 features: out = uint8 [max_rows, n/2],
  *                          out_scales = fp32 [n/2/128, max_rows] (kb-major)
  * Rows of A outside every group are neither read into results nor written.
+ * Kernel forms (moe_grouped_gemm_form tells which one a call uses): single
+ * CTAs, 128 tokens x 128 or 256 output columns each; or CTA pairs on two
+ * SMs (tcgen05 cta_group::2), 256 tokens x 256 columns per pair, each CTA
+ * loading one of the two 128-row weight blocks.  Pairs are the default for
+ * fp32/bf16 output with n % 256 == 0 and max_rows / n_groups >= 256; the
+ * environment variable MOEFP8_GEMM_PAIR=0 or =1 forces single CTAs or pairs
+ * (pairs only where n allows).  Both forms apply the same per-K-block
+ * promotion; results agree to fp32 accumulation order.
  * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE, MOE_ERR_ARG, MOE_ERR_ALIGN,
  * MOE_ERR_DEVICE, MOE_ERR_CUDA; MOE_DEV_TIMEOUT on dev_status. */
 MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int max_rows,
                                  const uint8_t* a, const float* a_scales, int k,
                                  const uint8_t* w, const float* w_scales, int n, int epilogue,
                                  void* out, float* out_scales, int* dev_status, void* stream);
+
+/* moe_grouped_gemm_form: CTAs per tile (1 = single CTAs, 2 = CTA pairs) that
+ * moe_grouped_gemm_fp8 uses on the current device for these arguments (same
+ * meaning as there), or 0 when they are invalid.  Host-only query; launches
+ * nothing. */
+MOE_API int moe_grouped_gemm_form(int n_groups, int max_rows, int n, int epilogue);
 
 /* ---------------------------------------------------------------- combine
  * moe_combine: y[t] = o[shared row of t] + sum_k gate[t,k] * o[row_of_pair

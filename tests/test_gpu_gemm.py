@@ -6,7 +6,13 @@ scales, FP32 accumulation promoted every 128 elements of K).
 Tolerances: with FP32 accumulation of FP8 products and per-block promotion,
 the relative error of an output is a few fp32 rounding steps (about 1e-6);
 1e-5 relative Frobenius is used for fp32 outputs.  bf16 outputs are compared
-after both sides round to bf16 (2e-3, the layer's output bound)."""
+after both sides round to bf16 (2e-3, the layer's output bound).
+
+Every test runs twice: with CTA pairs (cta_group::2, the library's default
+where the output width allows it) and with single CTAs
+(MOEFP8_GEMM_PAIR=0)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -16,6 +22,14 @@ import synthetic as S
 from gpu_util import DEV, bf16_dev, need_gpu, rel_frobenius, to_dev
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["pair", "single"])
+def cta_mode(request, monkeypatch):
+    """Select the GEMM kernel form for the test (read by the library at every
+    call)."""
+    monkeypatch.setenv("MOEFP8_GEMM_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
 
 
 def _quant_gpu(xbits):
@@ -108,7 +122,8 @@ def _check_dense(out, res, off, epilogue):
 
 @pytest.mark.parametrize("sizes,k,n", [([1], 128, 128), ([300], 512, 256), ([256], 256, 128),
                                        ([257, 0, 5, 16, 17], 384, 256),
-                                       ([40] * 9 + [600], 1024, 384)])
+                                       ([40] * 9 + [600], 1024, 384),
+                                       ([130, 1, 600, 255, 256, 17, 64, 33], 256, 512)])
 def test_grouped_fp32_output(sizes, k, n):
     import fp8_block_scaled_affinity_b200 as moe
     need_gpu()
