@@ -9,19 +9,19 @@
 //
 // Each CTA owns 128 tokens (the MMA's M side, one token per TMEM lane, so a
 // thread's token scale is one register) and, per K block, a TMEM partial of
-// 128 x C columns (C = 256, or 128 for the single-CTA fp32/bf16 form).  The
-// C columns are two 128-row weight blocks: the gate (W1) and up (W3) blocks
-// of the same 128 features for the SwiGLU epilogue, two neighbouring blocks
-// of the output otherwise.
+// 128 x C columns (C = 256; 128 for fp32/bf16 output whose width is not a
+// multiple of 256).  The 256 columns are two 128-row weight blocks: the gate
+// (W1) and up (W3) blocks of the same 128 features for the SwiGLU epilogue,
+// two neighbouring blocks of the output otherwise.
 //
 // CTA pairs (cta_group::2, the default): a cluster of two CTAs on two SMs
 // runs one M = 256, N = 256 MMA per 32-deep K step; each CTA loads its own
 // 128 tokens and ONE of the two weight blocks, so every weight byte crosses
 // L2 -> SM once per 256 tokens instead of once per 128.  The leader (rank 0)
 // issues the MMAs; both CTAs' TMA loads complete on the leader's stage
-// barrier, and the MMA commits arrive on both CTAs' barriers.  The
-// single-CTA form (cta_group::1) serves output widths that are not a
-// multiple of 256 and can be forced with MOEFP8_GEMM_PAIR=0.
+// barrier, and the MMA commits arrive on both CTAs' barriers.  Single CTAs
+// (cta_group::1) load both weight blocks themselves; gemm_pair_units picks
+// the form.
 //
 // Token boxes: the TMA box of a CTA's tokens is 128, 64, 32 or 16 rows (the
 // smallest that holds its valid rows; none when it has none), so ragged
@@ -50,7 +50,7 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kTileBytes = 128 * 128;            // one 128 x 128 FP8 tile
-constexpr int kParkWarpBytes = 2 * 4096;         // two 32-row x 128-byte output boxes
+constexpr int kBoxBytes = 4096;                  // one 32-row x 128-byte output box
 constexpr int kMaxBufs = 4;
 constexpr int kMaxStages = 6;
 constexpr int kScaleSlots = 16;
@@ -59,15 +59,21 @@ constexpr int kBM = 128;                         // tokens per CTA tile
 constexpr int kPromoters = 8;                    // promotion warps
 constexpr int kABoxes = 4;                       // token boxes of 128, 64, 32, 16 rows
 
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 struct Cfg {
-    static constexpr int kAccCols = (PAIR || SWIGLU) ? 256 : 128;  // TMEM columns per partial
+    static_assert(WIDE || !(PAIR || SWIGLU), "pairs and SwiGLU use 256-column partials");
+    static constexpr int kAccCols = WIDE ? 256 : 128;              // TMEM columns per partial
     static constexpr int kBufs = 512 / kAccCols;                   // TMEM partial buffers
     static constexpr int kWRows = PAIR ? 128 : kAccCols;           // weight rows this CTA loads
     static constexpr int kStageBytes = kTileBytes + kWRows * 128;  // tokens + weights
-    static constexpr int kStages = (PAIR && SWIGLU) ? 6 : 4;
+    // single CTAs with fp32/bf16 output and 256 columns: 48 KB stages next to
+    // the parking tiles leave room for three
+    static constexpr int kStages = (PAIR && SWIGLU) ? 6 : (!PAIR && !SWIGLU && WIDE) ? 3 : 4;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kParkBytes = SWIGLU ? 0 : kPromoters * kParkWarpBytes;
+    // output boxes parked per warp at a time (one where the operand ring is
+    // largest)
+    static constexpr int kParkBoxes = SWIGLU ? 0 : (!PAIR && WIDE) ? 1 : 2;
+    static constexpr int kParkBytes = kPromoters * kParkBoxes * kBoxBytes;
     static constexpr int kPairs = kAccCols / 4;                    // fp32 pairs per promoter thread
     static constexpr int kItemRows = PAIR ? 2 * kBM : kBM;         // tokens per work item
     static constexpr int kMmaM = PAIR ? 256 : 128;
@@ -115,13 +121,16 @@ struct SharedState {
     alignas(16) float red[2][2][kBM];         // [item parity][half][token] amax of h
 };
 
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 constexpr size_t smem_bytes() {
-    using C = Cfg<PAIR, SWIGLU>;
+    using C = Cfg<PAIR, SWIGLU, WIDE>;
     return size_t(C::kRingBytes) + C::kParkBytes + sizeof(SharedState) + 1024;
 }
-static_assert(smem_bytes<false, false>() <= 232448 && smem_bytes<false, true>() <= 232448 &&
-                  smem_bytes<true, false>() <= 232448 && smem_bytes<true, true>() <= 232448,
+static_assert(smem_bytes<false, false, false>() <= 232448 &&
+                  smem_bytes<false, false, true>() <= 232448 &&
+                  smem_bytes<false, true, true>() <= 232448 &&
+                  smem_bytes<true, false, true>() <= 232448 &&
+                  smem_bytes<true, true, true>() <= 232448,
               "dynamic shared memory above the sm_100 limit per CTA");
 
 // ------------------------------------------------------------- PTX glue
@@ -501,13 +510,13 @@ __device__ __forceinline__ uint32_t box_bytes(int n) {
 // The two 128-row weight blocks of a column tile (block-row indices inside
 // one group's [n, k] matrix): their scales go to sb[0] and sb[1], and a CTA
 // of a pair loads block b[rank].
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 __device__ __forceinline__ void weight_blocks(const GemmParams& p, const Item& w, int& b0,
                                               int& b1) {
     if (SWIGLU) {
         b0 = w.f;                // gate rows f*128 .. of W1
         b1 = p.n / 256 + w.f;    // up rows (n/2 + f*128) .. of W3
-    } else if (PAIR) {
+    } else if (WIDE) {
         b0 = 2 * w.f;
         b1 = 2 * w.f + 1;
     } else {
@@ -517,11 +526,11 @@ __device__ __forceinline__ void weight_blocks(const GemmParams& p, const Item& w
 }
 
 // ================================================= TMA producer (warp 0)
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap* map_w,
                                          const AMaps& maps_a, uint8_t* smem, SharedState* ss,
                                          int rank, int unit, int units) {
-    using C = Cfg<PAIR, SWIGLU>;
+    using C = Cfg<PAIR, SWIGLU, WIDE>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     uint32_t it = 0;
@@ -530,7 +539,7 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
     for (int item = unit; ok && item < total_items; item += units) {
         const Item w = decode_item<C::kItemRows>(ss, p, item);
         int b0, b1;
-        weight_blocks<PAIR, SWIGLU>(p, w, b0, b1);
+        weight_blocks<PAIR, SWIGLU, WIDE>(p, w, b0, b1);
         const int n0 = cta_tokens(w, 0);
         const int n1 = PAIR ? cta_tokens(w, 1) : 0;
         const int my_n = rank ? n1 : n0;
@@ -539,7 +548,7 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
         // bytes landing on the stage barrier: every CTA's tokens and weights
         const uint32_t tx = box_bytes(n0) + box_bytes(n1) + uint32_t(C::kCtas * C::kWRows * 128);
         const int wr_mine = w.g * p.n + (rank ? b1 : b0) * 128;
-        const int wr_second = w.g * p.n + b1 * 128;  // single-CTA SwiGLU: the up block
+        const int wr_second = w.g * p.n + b1 * 128;  // single CTA, 256 columns: block b1
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
             const int s = it % C::kStages;
             const uint32_t par = ((it / C::kStages) & 1u);
@@ -555,7 +564,7 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
                 if (rank == 0) mbar_arrive_expect_tx(local_full, tx);
                 if (my_n > 0) tma_load_2d<PAIR>(smem_u32(st), map_a, fb, kb * 128, a_y);
                 tma_load_2d<PAIR>(smem_u32(st + kTileBytes), map_w, fb, kb * 128, wr_mine);
-                if (!PAIR && SWIGLU)
+                if (!PAIR && WIDE)
                     tma_load_2d<PAIR>(smem_u32(st + 2 * kTileBytes), map_w, fb, kb * 128,
                                       wr_second);
                 issued_mask |= 1u << s;
@@ -577,10 +586,10 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
 // cp.async of each K block's 128 token scales (kb-major, so they are
 // contiguous) and the tile's two weight-block scales; the copies arrive on
 // sfull when they land.
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* ss, int rank,
                                              int unit, int units) {
-    using C = Cfg<PAIR, SWIGLU>;
+    using C = Cfg<PAIR, SWIGLU, WIDE>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     const int nbr = p.n / 128;  // weight block rows per group
@@ -589,7 +598,7 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
     for (int item = unit; ok && item < total_items; item += units) {
         const Item w = decode_item<C::kItemRows>(ss, p, item);
         int b0, b1;
-        weight_blocks<PAIR, SWIGLU>(p, w, b0, b1);
+        weight_blocks<PAIR, SWIGLU, WIDE>(p, w, b0, b1);
         const int my_n = cta_tokens(w, rank);
         const int my_row0 = w.row0 + kBM * rank;
         const float* sb0 = p.w_scales + (size_t(w.g) * nbr + b0) * p.nkb;
@@ -620,10 +629,10 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
 }
 
 // ================================================= MMA issuer (warp 1 of the leader)
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, SharedState* ss,
                                            uint32_t tmem_base, int unit, int units) {
-    using C = Cfg<PAIR, SWIGLU>;
+    using C = Cfg<PAIR, SWIGLU, WIDE>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
     if (lane == 0) {
@@ -661,8 +670,8 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
 
 // fp32 / bf16 epilogue: a warp's 32 finished row segments are written into
 // its parking tile in shared memory in the 128-byte swizzle layout of the
-// output tensor map (16-byte chunk c of row r at c ^ (r % 8)), two 4 KB
-// boxes at a time, then one lane hands them to the TMA engine as bulk
+// output tensor map (16-byte chunk c of row r at c ^ (r % 8)), one or two
+// 4 KB boxes at a time, then one lane hands them to the TMA engine as bulk
 // tensor stores.  Before the tile is rewritten, the engine must have read it.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
     asm volatile(
@@ -692,22 +701,22 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float2 f) {
 // Write this thread's NP fp32 pairs (one row, NP*2 consecutive columns
 // from `col`) of the warp's 32 rows: through the parking tile and bulk
 // tensor stores when all 32 rows are valid, else direct stores of valid rows.
-template <int NP>
+template <int NP, int R>
 __device__ __forceinline__ void store_rows(const GemmParams& p, const uint64_t (&acc2)[NP],
                                            char* wpark, const CUtensorMap* map_o, int lane,
                                            int rows_here, size_t row, int y0, int col) {
     const bool bf16_out = p.epilogue == MOE_EPI_BF16;
     if (rows_here >= 32) {
         if (bf16_out) {
-            // boxes of 64 bf16 (32 pairs); two per round
+            // boxes of 64 bf16 (32 pairs); R per round
             constexpr int kBoxes = NP / 32;
 #pragma unroll
-            for (int r0 = 0; r0 < kBoxes; r0 += 2) {
+            for (int r0 = 0; r0 < kBoxes; r0 += R) {
                 if (lane == 0) bulk_wait_read();
                 __syncwarp();
 #pragma unroll
-                for (int b = r0; b < r0 + 2 && b < kBoxes; ++b) {
-                    char* box = wpark + (b - r0) * 4096;
+                for (int b = r0; b < r0 + R && b < kBoxes; ++b) {
+                    char* box = wpark + (b - r0) * kBoxBytes;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int q0 = 32 * b + 4 * j;
@@ -722,21 +731,22 @@ __device__ __forceinline__ void store_rows(const GemmParams& p, const uint64_t (
                 __syncwarp();
                 if (lane == 0) {
 #pragma unroll
-                    for (int b = r0; b < r0 + 2 && b < kBoxes; ++b)
-                        tma_store_2d(map_o, smem_u32(wpark + (b - r0) * 4096), col + 64 * b, y0);
+                    for (int b = r0; b < r0 + R && b < kBoxes; ++b)
+                        tma_store_2d(map_o, smem_u32(wpark + (b - r0) * kBoxBytes), col + 64 * b,
+                                     y0);
                     bulk_commit();
                 }
             }
         } else {
-            // boxes of 32 fp32 (16 pairs); two per round
+            // boxes of 32 fp32 (16 pairs); R per round
             constexpr int kBoxes = NP / 16;
 #pragma unroll
-            for (int r0 = 0; r0 < kBoxes; r0 += 2) {
+            for (int r0 = 0; r0 < kBoxes; r0 += R) {
                 if (lane == 0) bulk_wait_read();
                 __syncwarp();
 #pragma unroll
-                for (int b = r0; b < r0 + 2; ++b) {
-                    char* box = wpark + (b - r0) * 4096;
+                for (int b = r0; b < r0 + R; ++b) {
+                    char* box = wpark + (b - r0) * kBoxBytes;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float2 a = unpack2(acc2[16 * b + 2 * j]);
@@ -748,8 +758,10 @@ __device__ __forceinline__ void store_rows(const GemmParams& p, const uint64_t (
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(map_o, smem_u32(wpark), col + 32 * r0, y0);
-                    tma_store_2d(map_o, smem_u32(wpark + 4096), col + 32 * (r0 + 1), y0);
+#pragma unroll
+                    for (int b = r0; b < r0 + R; ++b)
+                        tma_store_2d(map_o, smem_u32(wpark + (b - r0) * kBoxBytes), col + 32 * b,
+                                     y0);
                     bulk_commit();
                 }
             }
@@ -783,11 +795,11 @@ __device__ __forceinline__ void store_rows(const GemmParams& p, const uint64_t (
 //     (the same 64 features of W1 and W3);
 //   fp32 / bf16, C = 256: columns [128h, 128h+128) (weight block h);
 //   fp32 / bf16, C = 128: columns [64h, 64h+64) of the single weight block.
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, char* park_area,
                                          uint32_t tmem_base, const CUtensorMap* map_o, int rank,
                                          int unit, int units) {
-    using C = Cfg<PAIR, SWIGLU>;
+    using C = Cfg<PAIR, SWIGLU, WIDE>;
     constexpr bool kWide = C::kAccCols == 256;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
@@ -807,7 +819,7 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
     uint32_t tb = 0, cit = 0, parity = 0;
     bool ok = true;
     // this warp's parking tile (swizzled, 1024-byte aligned)
-    char* const wpark = park_area + (warp - 4) * kParkWarpBytes;
+    char* const wpark = park_area + (warp - 4) * (C::kParkBoxes * kBoxBytes);
     for (int item = unit; item < total_items; item += units, parity ^= 1u) {
         const Item w = decode_item<C::kItemRows>(ss, p, item);
         uint64_t acc2[C::kPairs];  // fp32 accumulator pairs
@@ -873,7 +885,8 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
         const size_t row = size_t(my_row0) + r;
         if (!SWIGLU) {
             constexpr int kCols = C::kAccCols / 2;  // this thread's columns
-            store_rows<C::kPairs>(p, acc2, wpark, map_o, lane, my_n - q * 32, row,
+            store_rows<C::kPairs, (C::kParkBoxes > 0 ? C::kParkBoxes : 1)>(
+                p, acc2, wpark, map_o, lane, my_n - q * 32, row,
                                   my_row0 + q * 32, w.f * C::kAccCols + half * kCols);
         } else {
             // h = silu(gate) * up for this thread's 64 features, then the
@@ -929,12 +942,12 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
 }
 
 // ----------------------------------------------------------------- kernel
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_w,
                         const __grid_constant__ AMaps maps_a,
                         const __grid_constant__ CUtensorMap map_o, const GemmParams p) {
-    using C = Cfg<PAIR, SWIGLU>;
+    using C = Cfg<PAIR, SWIGLU, WIDE>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -1027,13 +1040,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 4) {
         set_max_regs_dec<72>();
-        if (warp == 0) producer<PAIR, SWIGLU>(p, &map_w, maps_a, smem, ss, rank, unit, units);
+        if (warp == 0) producer<PAIR, SWIGLU, WIDE>(p, &map_w, maps_a, smem, ss, rank, unit, units);
         else if (warp == 1 && rank == 0)
-            mma_issuer<PAIR, SWIGLU>(p, smem, ss, tmem_base, unit, units);
-        else if (warp == 2) scale_loader<PAIR, SWIGLU>(p, ss, rank, unit, units);
+            mma_issuer<PAIR, SWIGLU, WIDE>(p, smem, ss, tmem_base, unit, units);
+        else if (warp == 2) scale_loader<PAIR, SWIGLU, WIDE>(p, ss, rank, unit, units);
     } else {
         set_max_regs_inc<208>();
-        promoter<PAIR, SWIGLU>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base,
+        promoter<PAIR, SWIGLU, WIDE>(p, ss, reinterpret_cast<char*>(smem + C::kRingBytes), tmem_base,
                                &map_o, rank, unit, units);
     }
 
@@ -1057,7 +1070,7 @@ int pair_units() {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem_bytes<true, SWIGLU>();
+        cfg.dynamicSmemBytes = smem_bytes<true, SWIGLU, true>();
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -1066,10 +1079,10 @@ int pair_units() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<true, SWIGLU>,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<true, SWIGLU, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem_bytes<true, SWIGLU>())) != cudaSuccess ||
-            cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, SWIGLU>, &cfg) !=
+                                 int(smem_bytes<true, SWIGLU, true>())) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<true, SWIGLU, true>, &cfg) !=
                 cudaSuccess || n < 1) {
             (void)cudaGetLastError();
             n = -1;  // pairs unavailable on this device
@@ -1079,22 +1092,22 @@ int pair_units() {
     return cache[dev];
 }
 
-template <bool PAIR, bool SWIGLU>
+template <bool PAIR, bool SWIGLU, bool WIDE>
 int launch(const GemmParams& p, const CUtensorMap& mw, const AMaps& ma, const CUtensorMap& mo,
            int units, cudaStream_t st) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR, SWIGLU>,
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<PAIR, SWIGLU, WIDE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem_bytes<PAIR, SWIGLU>())) != cudaSuccess)
+                             int(smem_bytes<PAIR, SWIGLU, WIDE>())) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (!PAIR) {
-        grouped_gemm_kernel<PAIR, SWIGLU><<<sm_count(), kThreads, smem_bytes<PAIR, SWIGLU>(), st>>>(
+        grouped_gemm_kernel<PAIR, SWIGLU, WIDE><<<sm_count(), kThreads, smem_bytes<PAIR, SWIGLU, WIDE>(), st>>>(
             mw, ma, mo, p);
         return check_launch();
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * units, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes<PAIR, SWIGLU>();
+    cfg.dynamicSmemBytes = smem_bytes<PAIR, SWIGLU, WIDE>();
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1103,7 +1116,7 @@ int launch(const GemmParams& p, const CUtensorMap& mw, const AMaps& ma, const CU
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<PAIR, SWIGLU>, mw, ma, mo, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<PAIR, SWIGLU, WIDE>, mw, ma, mo, p) != cudaSuccess)
         return MOE_ERR_CUDA;
     return check_launch();
 }
@@ -1171,19 +1184,20 @@ bool device_is_sm100() {
 }
 
 // Kernel form of a call: the number of CTA pairs to launch, or 0 for single
-// CTAs.  CTA pairs halve the operand traffic per SM but double the work per
-// TMEM round trip, which pays only when most items hold 256 tokens: measured
-// on B200, pairs run the 4096-row plain GEMM 1.36x faster and a 257-expert
-// prefill W13 (about 144 rows per group) 1.5x slower.  Default: pairs for
-// fp32/bf16 output with at least 256 rows per group on average.
-// MOEFP8_GEMM_PAIR=1 / =0 in the environment forces either form (pairs only
-// where the output width is a multiple of 256).
+// CTAs.  CTA pairs halve the operand traffic per SM, but on B200 that
+// traffic does not bound this kernel (the hand-off between the MMA and the
+// promotion warps does, once per K block of 128 x 256 partials in both
+// forms): measured, pairs and 256-column single CTAs run the 4096-row bf16
+// GEMM at the same 1430 TFLOP/s and the skewed W2 within 1%, while pairs
+// are 1.5x slower on the 257-expert prefill W13 (half of a pair's 256
+// tokens are padding there).  Single CTAs are therefore the default;
+// MOEFP8_GEMM_PAIR=1 in the environment selects pairs where the output
+// width is a multiple of 256 (SwiGLU always is).
 int gemm_pair_units(int n_groups, int max_rows, int n, bool swiglu) {
+    (void)n_groups;
+    (void)max_rows;
     const char* env = getenv("MOEFP8_GEMM_PAIR");
-    const bool pair_shape = swiglu || n % 256 == 0;
-    bool want = pair_shape && !swiglu && max_rows / n_groups >= 256;
-    if (env && env[0] == '0') want = false;
-    if (env && env[0] == '1') want = pair_shape;
+    const bool want = env && env[0] == '1' && (swiglu || n % 256 == 0);
     if (!want) return 0;
     return std::max(0, swiglu ? pair_units<true>() : pair_units<false>());
 }
@@ -1233,7 +1247,10 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     p.nkb = k / 128;
     p.w_scales = w_scales;
     p.n = n;
-    p.n_ftiles = (pair || swiglu) ? n / 256 : n / 128;
+    // 256 output columns per tile wherever n allows (a TMEM round trip per K
+    // block then carries twice the work); 128 otherwise
+    const bool wide = pair || swiglu || n % 256 == 0;
+    p.n_ftiles = wide ? n / 256 : n / 128;
     p.epilogue = epilogue;
     p.out = out;
     p.out_scales = out_scales;
@@ -1250,8 +1267,9 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
         return MOE_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     if (pair)
-        return swiglu ? launch<true, true>(p, mw, ma, mo, units, st)
-                      : launch<true, false>(p, mw, ma, mo, units, st);
-    return swiglu ? launch<false, true>(p, mw, ma, mo, 0, st)
-                  : launch<false, false>(p, mw, ma, mo, 0, st);
+        return swiglu ? launch<true, true, true>(p, mw, ma, mo, units, st)
+                      : launch<true, false, true>(p, mw, ma, mo, units, st);
+    if (swiglu) return launch<false, true, true>(p, mw, ma, mo, 0, st);
+    return wide ? launch<false, false, true>(p, mw, ma, mo, 0, st)
+                : launch<false, false, false>(p, mw, ma, mo, 0, st);
 }

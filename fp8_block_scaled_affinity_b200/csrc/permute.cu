@@ -190,23 +190,30 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(
     }
 }
 
-// moe_quant_permute's copy: one warp per token reads the token's bf16 row
-// once (16-byte loads, kPiece per lane in flight), quantises each 1x128 tile
-// exactly as fp8_quant_act_1x128 does (a half-warp owns one tile: amax by
-// shuffles, scale rule of quant.cu, RN products, satfinite E4M3) and writes
-// the codes and the scale K+1 times (routed rows and the shared row).
+// moe_quant_permute's copy: a work unit is one 2,048-value piece of a
+// token's bf16 row (a warp, 16-byte loads, kPiece per lane in flight), so a
+// small batch still spreads over every SM.  The warp quantises each 1x128
+// tile of the piece exactly as fp8_quant_act_1x128 does (a half-warp owns
+// one tile: amax by shuffles, scale rule of quant.cu, RN products, satfinite
+// E4M3) and writes the codes and the scale K+1 times (routed rows and the
+// shared row).
 __global__ void __launch_bounds__(256) quant_copy_rows_kernel(
     const uint4* __restrict__ x, int T, int d, int K, const int32_t* __restrict__ row_of_pair,
     int64_t rows_total, uint2* __restrict__ xq_perm, float* __restrict__ xs_perm) {
     const int lane = threadIdx.x & 31;
     const int nvec = d / 8, nkb = d / 128;  // 8 bf16 in, 8 codes out per vector
-    const int warps_total = gridDim.x * (blockDim.x / 32);
-    for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps_total) {
+    const int pieces = (nvec + 32 * kPiece - 1) / (32 * kPiece);
+    const int64_t units = int64_t(T) * pieces;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t un = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); un < units;
+         un += warps_total) {
+        const int t = int(un / pieces);
         int my_row = 0;
         if (lane < K) my_row = row_of_pair[int64_t(t) * K + lane];
         const int shared_row = T * K + t;
         const uint4* src = x + int64_t(t) * nvec;
-        for (int c0 = 0; c0 < nvec; c0 += 32 * kPiece) {
+        {
+            const int c0 = int(un - int64_t(t) * pieces) * (32 * kPiece);
             uint4 v[kPiece];
 #pragma unroll
             for (int j = 0; j < kPiece; ++j) {
@@ -428,7 +435,10 @@ extern "C" MOE_API int moe_quant_permute(const MoeShape* shape, const uint16_t* 
     rc = build_rows(shape, topk_idx, expert_counts, expert_offsets, row_of_pair,
                     static_cast<int32_t*>(ws), dev_status, st);
     if (rc != MOE_OK || T == 0) return rc;
-    quant_copy_rows_kernel<<<copy_grid(T), 256, 0, st>>>(
+    const int64_t pieces = (d / 8 + 32 * kPiece - 1) / (32 * kPiece);
+    const int64_t units = int64_t(T) * pieces;  // one warp each, 8 per block
+    const int qblocks = int(std::min<int64_t>((units + 7) / 8, int64_t(sm_count()) * 8));
+    quant_copy_rows_kernel<<<qblocks, 256, 0, st>>>(
         reinterpret_cast<const uint4*>(x), T, d, K, row_of_pair, int64_t(T) * K + T,
         reinterpret_cast<uint2*>(xq_perm), xs_perm);
     return check_launch();

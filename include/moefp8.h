@@ -245,13 +245,12 @@ MOE_API int moe_permute_static_ws(const MoeShape* shape, const int32_t* topk_idx
  *                          out_scales = fp32 [n/2/128, max_rows] (kb-major)
  * Rows of A outside every group are neither read into results nor written.
  * Kernel forms (moe_grouped_gemm_form tells which one a call uses): single
- * CTAs, 128 tokens x 128 or 256 output columns each; or CTA pairs on two
- * SMs (tcgen05 cta_group::2), 256 tokens x 256 columns per pair, each CTA
- * loading one of the two 128-row weight blocks.  Pairs are the default for
- * fp32/bf16 output with n % 256 == 0 and max_rows / n_groups >= 256; the
- * environment variable MOEFP8_GEMM_PAIR=0 or =1 forces single CTAs or pairs
- * (pairs only where n allows).  Both forms apply the same per-K-block
- * promotion; results agree to fp32 accumulation order.
+ * CTAs (the default), 128 tokens x 256 output columns each (128 when
+ * n % 256 != 0); or, when the environment variable MOEFP8_GEMM_PAIR=1 is
+ * set and n % 256 == 0, CTA pairs on two SMs (tcgen05 cta_group::2), 256
+ * tokens x 256 columns per pair, each CTA loading one of the two 128-row
+ * weight blocks.  Both forms apply the same per-K-block promotion; results
+ * agree to fp32 accumulation order.
  * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE, MOE_ERR_ARG, MOE_ERR_ALIGN,
  * MOE_ERR_DEVICE, MOE_ERR_CUDA; MOE_DEV_TIMEOUT on dev_status. */
 MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int max_rows,

@@ -43,9 +43,9 @@ def test_library_exports_every_declared_symbol(moe):
 
 
 def test_gemm_form_query(moe, monkeypatch):
-    """moe_grouped_gemm_form: invalid arguments give 0; single CTAs when
-    forced, for SwiGLU by default and for few rows per group; never a pair
-    where the output width is not a multiple of 256."""
+    """moe_grouped_gemm_form: invalid arguments give 0; single CTAs unless
+    MOEFP8_GEMM_PAIR=1; never a pair where the output width is not a
+    multiple of 256."""
     f = moe.moe_grouped_gemm_form
     assert f(0, 128, 256, moe.MOE_EPI_F32) == 0
     assert f(1, 128, 200, moe.MOE_EPI_F32) == 0
@@ -56,6 +56,7 @@ def test_gemm_form_query(moe, monkeypatch):
     monkeypatch.delenv("MOEFP8_GEMM_PAIR")
     assert f(257, 36864 + 4096, 4096, moe.MOE_EPI_SWIGLU_QUANT) == 1
     assert f(257, 1152 + 128, 7168, moe.MOE_EPI_F32) == 1
+    assert f(1, 4096, 2048, moe.MOE_EPI_BF16) == 1
     assert f(1, 4096, 384, moe.MOE_EPI_F32) == 1
     monkeypatch.setenv("MOEFP8_GEMM_PAIR", "1")
     assert f(1, 4096, 384, moe.MOE_EPI_F32) == 1
