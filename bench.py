@@ -413,7 +413,7 @@ def run_route(args, world, rank, local):
         "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * 2,
                 "d2h_bytes_per_step": idx.numel() * 4 + gate.numel() * 4},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": 7 * args.steps,
         "clocks": clk,
         "device_status": int(status.item()),
     }
@@ -829,7 +829,7 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes},
         # route 6, quant+permute 4, GEMMs 2, combine 1, bias update 1
-        "gpu_launches": 14 * args.steps,
+        "gpu_launches": 15 * args.steps,
         "clocks": clk,
         "device_status": status,
     }

@@ -28,11 +28,13 @@
 //      interval lies strictly above every rejected one.  Certified tokens get
 //      their chosen logits as fp32(u~) when [u~-B, u~+B] holds no fp32
 //      rounding boundary; others go on a list;
-//   4. route_exact_pairs_kernel: the defining FP64 sum for the chosen
-//      logits that were not settled in 3 and, when the list is short, for
-//      all N_r logits of every listed token (one sum per thread);
-//      route_logits_list_kernel does listed tokens in 64x64 FP64 tiles when
-//      the list is long;
+//   4. the defining FP64 sum for the chosen logits that were not settled
+//      in 3 and, when the list is short, for all N_r logits of every listed
+//      token: route_exact_pairs_kernel (a warp per chosen logit) settles
+//      those whose sum provably cannot round, from an exact parallel sum;
+//      route_exact_chain_kernel (a thread per sum) evaluates the rest and
+//      the listed tokens' rows in ascending k; route_logits_list_kernel
+//      does listed tokens in 64x64 FP64 tiles when the list is long;
 //   5. route_select_kernel (warp per token): exact s and s' of the chosen
 //      experts, slot order, gates and histogram for certified tokens; the
 //      full selection on the exact logits for listed ones.
@@ -639,7 +641,141 @@ __device__ __forceinline__ float exact_logit(const uint16_t* __restrict__ xr,
 // tiled kernel below.
 constexpr int kPairList = 256;
 
+// Exactness of one row pair's defining sum, decided by a warp.  Every
+// product p_k = x_k E_k is exact in FP64 and a multiple of 2^lowbit(p_k);
+// with g the smallest lowbit over the nonzero products and S = sum |p_k|,
+// every partial sum (in any order) is a multiple of 2^g of magnitude at
+// most S, hence a double when S < 2^(53+g).  Then no addition of the
+// defining ascending-k sum rounds and it equals the exact sum, which the
+// warp forms in parallel (each lane sums its k in order, then a shuffle
+// tree; every step exact).  S is accumulated rounding upward, so the test
+// is rigorous.  Returns false (no result) when the test fails or a value
+// is not finite.
+__device__ __forceinline__ bool warp_exact_logit(const uint16_t* __restrict__ xr,
+                                                 const uint16_t* __restrict__ er, int d,
+                                                 int lane, float& u) {
+    const uint4* xp = reinterpret_cast<const uint4*>(xr);
+    const uint4* ep = reinterpret_cast<const uint4*>(er);
+    double sabs = 0.0, sum = 0.0;
+    int g = INT_MAX;
+    bool finite = true;
+    for (int v = lane; v < d / 8; v += 32) {
+        const uint4 xv = __ldg(xp + v), ev = __ldg(ep + v);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const uint32_t xb = q & 1 ? xw[q >> 1] >> 16 : xw[q >> 1] & 0xFFFFu;
+            const uint32_t eb = q & 1 ? ew[q >> 1] >> 16 : ew[q >> 1] & 0xFFFFu;
+            finite = finite && ((xb >> 7) & 0xFFu) != 0xFFu && ((eb >> 7) & 0xFFu) != 0xFFu;
+            const double pk = (double)__uint_as_float(xb << 16) * (double)__uint_as_float(eb << 16);
+            sabs = __dadd_ru(sabs, fabs(pk));
+            sum = __dadd_rn(sum, pk);
+            if (pk != 0.0) {
+                // lowest set bit of the (normal, exact) double product
+                const uint64_t bits = uint64_t(__double_as_longlong(pk));
+                const int ex = int((bits >> 52) & 0x7FFu);
+                const uint64_t sig = (bits & 0xFFFFFFFFFFFFFull) | (uint64_t(1) << 52);
+                g = min(g, ex - 1075 + (__ffsll((long long)sig) - 1));
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        sabs = __dadd_ru(sabs, __shfl_xor_sync(0xffffffffu, sabs, o));
+        sum = __dadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
+        g = min(g, __shfl_xor_sync(0xffffffffu, g, o));
+    }
+    finite = __all_sync(0xffffffffu, finite);
+    if (!finite) return false;
+    if (g == INT_MAX) {  // every product is zero: the defining sum is +0
+        u = 0.0f;
+        return true;
+    }
+    if (!(sabs < ldexp(1.0, 53 + g))) return false;
+    u = __double2float_rn(sum);
+    return true;
+}
+
+// Jobs of the exact-sum kernels: the listed chosen logits (pair list) and,
+// while the list of uncertified tokens is short, every logit of those
+// tokens.  Job j -> token t, expert e and the pair index pj (-1 for a
+// listed token's logit); false (reported) when an index is out of range.
+struct ExactJobs {
+    int64_t nA, nB;
+};
+
+__device__ __forceinline__ ExactJobs exact_jobs(int T, int N, int K, const int32_t* pair_count,
+                                                const int32_t* list_count, int* dev_status,
+                                                int32_t* check, bool report) {
+    int np = *pair_count, nl = *list_count;
+    if (np > T * K || nl > T) {
+        if (report) route_bad(dev_status, check, 1, max(np, nl));
+        np = min(np, T * K);
+        nl = min(nl, T);
+    }
+    return {int64_t(np), nl <= kPairList ? int64_t(nl) * N : 0};
+}
+
+__device__ __forceinline__ bool exact_job(int64_t j, const ExactJobs& jobs, int T, int N, int K,
+                                          const int32_t* __restrict__ cand,
+                                          const int32_t* __restrict__ pair_list,
+                                          const int32_t* __restrict__ list, int& t, int& e,
+                                          int& pj) {
+    pj = -1;
+    if (j < jobs.nA) {
+        pj = pair_list[j];
+        t = pj / K;
+        e = (pj >= 0 && pj < T * K) ? cand[pj] : -1;
+    } else {
+        const int64_t jj = j - jobs.nA;
+        t = list[jj / N];
+        e = int(jj % N);
+    }
+    return t >= 0 && t < T && e >= 0 && e < N;
+}
+
+// Phase 1, one warp per pair-list job (a chosen logit of a certified token
+// whose fp32 rounding was not settled): the warp settles the job by
+// warp_exact_logit when its defining sum cannot round (nearly every row pair
+// of real data) and otherwise marks it with a NaN for phase 2.  The full
+// rows of uncertified tokens go to phase 2 directly: those tokens are
+// uncertified mostly because of values far below their row's maximum, which
+// also fail this test.
 __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d, int K,
+    const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
+    const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
+    const int32_t* __restrict__ list_count, float* __restrict__ u_exact,
+    double* __restrict__ uhat, int* dev_status, int32_t* __restrict__ check) {
+    const int lane = threadIdx.x & 31;
+    const ExactJobs jobs = exact_jobs(T, N, K, pair_count, list_count, dev_status, check,
+                                      blockIdx.x == 0 && threadIdx.x == 0);
+    const int64_t stride = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t j = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); j < jobs.nA;
+         j += stride) {
+        int t, e, pj;
+        if (!exact_job(j, jobs, T, N, K, cand, pair_list, list, t, e, pj)) {
+            if (lane == 0) route_bad(dev_status, check, 2, int(j));
+            continue;
+        }
+        // the reductions leave identical values in every lane: `fast` and u
+        // are warp-uniform
+        float u = 0.0f;
+        const bool fast = warp_exact_logit(x + int64_t(t) * d, E + int64_t(e) * d, d, lane, u);
+        if (lane == 0) {
+            if (pj >= 0) u_exact[pj] = fast ? u : __int_as_float(0x7FFFFFFF);
+            else uhat[int64_t(t) * N + e] = fast ? (double)u : __longlong_as_double(0x7FF8000000000000ll);
+        }
+    }
+}
+
+// Phase 2, one thread per job: the pair-list jobs phase 1 marked (NaN) and
+// every logit of the listed uncertified tokens get the defining sum in
+// ascending k, all in parallel (each is one dependent chain of d
+// additions).  Settled results are never NaN: phase 1 settles only finite
+// row pairs.
+__global__ void __launch_bounds__(64) route_exact_chain_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d, int K,
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
     const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
@@ -647,30 +783,16 @@ __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
     const float* __restrict__ vmin, const double* __restrict__ l2, const double* __restrict__ lb,
     float* __restrict__ u_exact, double* __restrict__ uhat, int* dev_status,
     int32_t* __restrict__ check) {
-    int np = *pair_count, nl = *list_count;
-    if (np > T * K || nl > T) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) route_bad(dev_status, check, 1, max(np, nl));
-        np = min(np, T * K);
-        nl = min(nl, T);
-    }
-    const int64_t nA = np;
-    const int64_t nB = nl <= kPairList ? int64_t(nl) * N : 0;
+    const ExactJobs jobs = exact_jobs(T, N, K, pair_count, list_count, dev_status, check, false);
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j < nA + nB; j += stride) {
-        int t, e, pj = -1;
-        if (j < nA) {
-            pj = pair_list[j];
-            t = pj / K;
-            e = (pj >= 0 && pj < T * K) ? cand[pj] : -1;
-        } else {
-            const int64_t jj = j - nA;
-            t = list[jj / N];
-            e = int(jj % N);
-        }
-        if (t < 0 || t >= T || e < 0 || e >= N) {
-            route_bad(dev_status, check, 2, int(j));
+    for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j < jobs.nA + jobs.nB;
+         j += stride) {
+        int t, e, pj;
+        if (!exact_job(j, jobs, T, N, K, cand, pair_list, list, t, e, pj)) {
+            if (j >= jobs.nA) route_bad(dev_status, check, 2, int(j));  // phase 1 saw the others
             continue;
         }
+        if (pj >= 0 && !isnan(u_exact[pj])) continue;  // settled in phase 1
         const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
                                    double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
         const float u =
@@ -1057,9 +1179,13 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
         w.pair_list, w.pair_count, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
-    // 4. the defining FP64 sums where they are needed
-    // one sum per thread (grid-stride over the jobs the lists hold)
+    // 4. the defining FP64 sums where they are needed: a warp per job where
+    // the sum provably cannot round, then a thread per remaining job
     route_exact_pairs_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
+        x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
+        w.u_exact, w.uhat, dev_status, w.check);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    route_exact_chain_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
         x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
         w.vmax, w.vmin, w.l2, w.lb, w.u_exact, w.uhat, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
