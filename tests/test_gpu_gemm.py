@@ -123,7 +123,9 @@ def _check_dense(out, res, off, epilogue):
 @pytest.mark.parametrize("sizes,k,n", [([1], 128, 128), ([300], 512, 256), ([256], 256, 128),
                                        ([257, 0, 5, 16, 17], 384, 256),
                                        ([40] * 9 + [600], 1024, 384),
-                                       ([130, 1, 600, 255, 256, 17, 64, 33], 256, 512)])
+                                       ([130, 1, 600, 255, 256, 17, 64, 33], 256, 512),
+                                       # token boxes of exactly 16, 32, 64 rows and just above
+                                       ([16, 32, 64, 65, 48, 96, 144, 160, 192], 384, 768)])
 def test_grouped_fp32_output(sizes, k, n):
     import fp8_block_scaled_affinity_b200 as moe
     need_gpu()
