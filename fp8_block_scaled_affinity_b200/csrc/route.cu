@@ -656,27 +656,40 @@ __device__ __forceinline__ bool warp_exact_logit(const uint16_t* __restrict__ xr
                                                  int lane, float& u) {
     const uint4* xp = reinterpret_cast<const uint4*>(xr);
     const uint4* ep = reinterpret_cast<const uint4*>(er);
+    constexpr int kAhead = 7;  // 16-byte vectors of each row in flight per lane
+    const int nv = d / 8;
     double sabs = 0.0, sum = 0.0;
     int g = INT_MAX;
     bool finite = true;
-    for (int v = lane; v < d / 8; v += 32) {
-        const uint4 xv = __ldg(xp + v), ev = __ldg(ep + v);
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-        const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+    for (int v0 = lane; v0 < nv; v0 += 32 * kAhead) {
+        // this lane's next kAhead vectors of both rows, loaded before use; past
+        // the row end they are zero (zero products change no sum)
+        uint4 xa[kAhead], ea[kAhead];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const uint32_t xb = q & 1 ? xw[q >> 1] >> 16 : xw[q >> 1] & 0xFFFFu;
-            const uint32_t eb = q & 1 ? ew[q >> 1] >> 16 : ew[q >> 1] & 0xFFFFu;
-            finite = finite && ((xb >> 7) & 0xFFu) != 0xFFu && ((eb >> 7) & 0xFFu) != 0xFFu;
-            const double pk = (double)__uint_as_float(xb << 16) * (double)__uint_as_float(eb << 16);
-            sabs = __dadd_ru(sabs, fabs(pk));
-            sum = __dadd_rn(sum, pk);
-            if (pk != 0.0) {
-                // lowest set bit of the (normal, exact) double product
-                const uint64_t bits = uint64_t(__double_as_longlong(pk));
-                const int ex = int((bits >> 52) & 0x7FFu);
-                const uint64_t sig = (bits & 0xFFFFFFFFFFFFFull) | (uint64_t(1) << 52);
-                g = min(g, ex - 1075 + (__ffsll((long long)sig) - 1));
+        for (int i = 0; i < kAhead; ++i) {
+            const int v = v0 + 32 * i;
+            xa[i] = v < nv ? __ldg(xp + v) : make_uint4(0u, 0u, 0u, 0u);
+            ea[i] = v < nv ? __ldg(ep + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) {
+            const uint32_t xw[4] = {xa[i].x, xa[i].y, xa[i].z, xa[i].w};
+            const uint32_t ew[4] = {ea[i].x, ea[i].y, ea[i].z, ea[i].w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t xb = q & 1 ? xw[q >> 1] >> 16 : xw[q >> 1] & 0xFFFFu;
+                const uint32_t eb = q & 1 ? ew[q >> 1] >> 16 : ew[q >> 1] & 0xFFFFu;
+                finite = finite && ((xb >> 7) & 0xFFu) != 0xFFu && ((eb >> 7) & 0xFFu) != 0xFFu;
+                const double pk = (double)__uint_as_float(xb << 16) * (double)__uint_as_float(eb << 16);
+                sabs = __dadd_ru(sabs, fabs(pk));
+                sum = __dadd_rn(sum, pk);
+                if (pk != 0.0) {
+                    // lowest set bit of the (normal, exact) double product
+                    const uint64_t bits = uint64_t(__double_as_longlong(pk));
+                    const int ex = int((bits >> 52) & 0x7FFu);
+                    const uint64_t sig = (bits & 0xFFFFFFFFFFFFFull) | (uint64_t(1) << 52);
+                    g = min(g, ex - 1075 + (__ffsll((long long)sig) - 1));
+                }
             }
         }
     }
