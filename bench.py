@@ -603,9 +603,9 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_routed": cfg.n_routed,
-                   "n_groups": cfg.n_groups, "topk_groups": cfg.topk_groups,
-                   "topk": cfg.topk, "inter": cfg.inter,
+        "config": {"workload": f"moe_layer_{cfg.name}", "T": cfg.T, "d": cfg.d,
+                   "n_routed": cfg.n_routed, "n_shared": 1, "n_groups": cfg.n_groups,
+                   "topk_groups": cfg.topk_groups, "topk": cfg.topk, "inter": cfg.inter,
                    "sample_tokens_per_step": CPU_SAMPLE_TOKENS},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count() or 1,
                          "kind": "oracle",
@@ -640,7 +640,9 @@ def run_reference_route(args, n_tok=64):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "moe_route_prefill", "T": cfg.T, "d": cfg.d,
-                   "n_routed": cfg.n_routed, "sample_tokens_per_step": n_tok},
+                   "n_routed": cfg.n_routed, "n_groups": cfg.n_groups,
+                   "topk_groups": cfg.topk_groups, "topk": cfg.topk,
+                   "sample_tokens_per_step": n_tok},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count() or 1,
                          "kind": "oracle", "sample": f"{n_tok} tokens per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
