@@ -128,10 +128,16 @@ def algorithmic_counts(cfg, counts_host):
 
 
 def gemm_source_hash() -> str:
+    """Fingerprint of the GEMM kernel's code (comments and blank lines
+    ignored), tying a committed DRAM-traffic figure to the code it was
+    measured on."""
     h = hashlib.sha256()
     for name in ("gemm.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "fp8_block_scaled_affinity_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "fp8_block_scaled_affinity_b200", "csrc", name)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,14 +14,14 @@
 // (W1) and up (W3) blocks of the same 128 features for the SwiGLU epilogue,
 // two neighbouring blocks of the output otherwise.
 //
-// CTA pairs (cta_group::2, the default): a cluster of two CTAs on two SMs
-// runs one M = 256, N = 256 MMA per 32-deep K step; each CTA loads its own
-// 128 tokens and ONE of the two weight blocks, so every weight byte crosses
-// L2 -> SM once per 256 tokens instead of once per 128.  The leader (rank 0)
-// issues the MMAs; both CTAs' TMA loads complete on the leader's stage
-// barrier, and the MMA commits arrive on both CTAs' barriers.  Single CTAs
-// (cta_group::1) load both weight blocks themselves; gemm_pair_units picks
-// the form.
+// Single CTAs (cta_group::1, the default) load both weight blocks
+// themselves.  CTA pairs (cta_group::2, MOEFP8_GEMM_PAIR=1): a cluster of
+// two CTAs on two SMs runs one M = 256, N = 256 MMA per 32-deep K step; each
+// CTA loads its own 128 tokens and ONE of the two weight blocks, so every
+// weight byte crosses L2 -> SM once per 256 tokens instead of once per 128.
+// The leader (rank 0) issues the MMAs; both CTAs' TMA loads complete on the
+// leader's stage barrier, and the MMA commits arrive on both CTAs' barriers.
+// gemm_pair_units picks the form.
 //
 // Token boxes: the TMA box of a CTA's tokens is 128, 64, 32 or 16 rows (the
 // smallest that holds its valid rows; none when it has none), so ragged
@@ -29,7 +29,8 @@
 // past the box hold stale codes; they feed only TMEM lanes whose tokens are
 // discarded.
 //
-// Roles (384 threads, one CTA per SM, persistent over work items):
+// Roles (384 threads, one CTA per SM, persistent over work items; a pair
+// shares its items):
 //   warp 0       TMA producer
 //   warp 1       TMEM owner; in the leader, the MMA issuer (one thread)
 //   warp 2       scale loader: cp.async of the K block's 128 token scales and
