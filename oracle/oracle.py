@@ -111,18 +111,47 @@ def _table():
     return _TABLE
 
 
+_POOL = None
+
+
+def _row_pieces(rows: int, step: int, fill) -> None:
+    """Run fill(r0, r1) over row ranges [r0, r1) of `step` rows (a multiple
+    of the block height) on a thread pool.  Each element is written once by
+    the same formula whatever the split: this only spreads the work over
+    the host cores."""
+    global _POOL
+    if rows <= step:
+        fill(0, rows)
+        return
+    if _POOL is None:
+        from concurrent.futures import ThreadPoolExecutor
+        _POOL = ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1)))
+    list(_POOL.map(lambda r0: fill(r0, min(rows, r0 + step)), range(0, rows, step)))
+
+
 def dequant_act(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """code value * tile scale, in FP64 (exact)."""
     rows, cols = q.shape
-    v = _table()[q].reshape(rows, cols // 128, 128)
-    return (v * s.astype(np.float64)[:, :, None]).reshape(rows, cols)
+    out = np.empty((rows, cols), dtype=np.float64)
+
+    def fill(r0, r1):
+        v = _table()[q[r0:r1]].reshape(r1 - r0, cols // 128, 128)
+        out[r0:r1] = (v * s[r0:r1].astype(np.float64)[:, :, None]).reshape(r1 - r0, cols)
+    _row_pieces(rows, 256, fill)
+    return out
 
 
 def dequant_w(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     """code value * block scale, in FP64 (exact)."""
     rows, cols = q.shape
-    v = _table()[q].reshape(rows // 128, 128, cols // 128, 128)
-    return (v * s.astype(np.float64)[:, None, :, None]).reshape(rows, cols)
+    out = np.empty((rows, cols), dtype=np.float64)
+
+    def fill(r0, r1):
+        v = _table()[q[r0:r1]].reshape((r1 - r0) // 128, 128, cols // 128, 128)
+        sb = s[r0 // 128:r1 // 128].astype(np.float64)
+        out[r0:r1] = (v * sb[:, None, :, None]).reshape(r1 - r0, cols)
+    _row_pieces(rows, 256, fill)
+    return out
 
 
 # ----------------------------------------------------------------- routing
@@ -245,8 +274,10 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
     xq, xs = quant_act_1x128(x_bf16)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     idx = r["topk_idx"][tokens]
-    o_routed = np.zeros((len(tokens), topk, d), dtype=np.float64)
-    o_shared = np.zeros((len(tokens), d), dtype=np.float64)
+    gates = r["topk_gate"][tokens].astype(np.float64)
+    # y_t = o_shared_t + sum_k g_tk o_tk in FP64, accumulated expert by
+    # expert (a token meets each expert at most once), then one bf16 rounding
+    y64 = np.zeros((len(tokens), d), dtype=np.float64)
     for e in range(n_routed + 1):
         if e == n_routed:
             sel = np.arange(len(tokens))
@@ -258,10 +289,10 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
         w = expert_weights(e)
         o = swiglu_expert(xq[tokens[sel]], xs[tokens[sel]], *w)
         if slots is None:
-            o_shared[sel] = o
+            y64[sel] += o
         else:
-            o_routed[sel, slots] = o
-    y = combine(o_shared, o_routed, r["topk_gate"][tokens])
+            y64[sel] += gates[sel, slots][:, None] * o
+    y = f64_to_bf16_bits(y64)
     r.update({"xq": xq, "xs": xs, "y": y, "tokens": tokens})
     return r
 
