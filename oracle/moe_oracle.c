@@ -161,6 +161,82 @@ void orc_quant_w_128x128(const uint16_t* w, int64_t rows, int64_t cols,
         }
 }
 
+/* ---------------------------------------- power-of-two scales (option)
+ * A numerically different option, not the pages' recipe: the scale of a
+ * tile or block is a power of two, so that block-scaled tensor-core MMAs
+ * (UE8M0 scale factors, one byte: the exponent + 127) can apply it in the
+ * MMA itself.  With amax = max |v| of the group:
+ *   e = the smallest integer with amax <= 448 * 2^e (so no code saturates),
+ *   clamped to [-127, 127]; amax = 0 gives e = 0;
+ *   code = E4M3(v * 2^-e), nearest even, saturating (the product is exact).
+ * Returns e. */
+static int pow2_exponent(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    const double a = amax;
+    int e = ilogb(a) - 9;               /* 448 * 2^e < 2^(e+9) <= a: too small */
+    while (a > ldexp(448.0, e)) ++e;    /* at most two steps */
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+static int quant_group_pow2(const float* vals, int n, uint8_t* codes_out) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(vals[i]);
+        if (a > amax) amax = a;
+    }
+    const int e = pow2_exponent(amax);
+    for (int i = 0; i < n; ++i)
+        codes_out[i] = orc_e4m3_encode((float)ldexp((double)vals[i], -e));
+    return e;
+}
+
+/* 1x128 tiles with power-of-two scales; e_out [rows, cols/128] (int32). */
+void orc_quant_act_1x128_pow2_bf16(const uint16_t* x, int64_t rows, int64_t cols,
+                                   uint8_t* q, int32_t* e_out) {
+    int64_t nt = cols / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float vals[128];
+        for (int64_t t = 0; t < nt; ++t) {
+            const uint16_t* src = x + r * cols + t * 128;
+            for (int i = 0; i < 128; ++i) vals[i] = bf16_to_f32(src[i]);
+            e_out[r * nt + t] = quant_group_pow2(vals, 128, q + r * cols + t * 128);
+        }
+    }
+}
+
+void orc_quant_act_1x128_pow2_f32(const float* x, int64_t rows, int64_t cols,
+                                  uint8_t* q, int32_t* e_out) {
+    int64_t nt = cols / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t t = 0; t < nt; ++t)
+            e_out[r * nt + t] = quant_group_pow2(x + r * cols + t * 128, 128,
+                                                 q + r * cols + t * 128);
+}
+
+/* 128x128 blocks with power-of-two scales; e_out [rows/128, cols/128]. */
+void orc_quant_w_128x128_pow2(const uint16_t* w, int64_t rows, int64_t cols,
+                              uint8_t* q, int32_t* e_out) {
+    int64_t br = rows / 128, bc = cols / 128;
+    #pragma omp parallel for schedule(static) collapse(2)
+    for (int64_t i = 0; i < br; ++i)
+        for (int64_t j = 0; j < bc; ++j) {
+            float* vals = (float*)malloc(128 * 128 * sizeof(float));
+            uint8_t* codes = (uint8_t*)malloc(128 * 128);
+            for (int r = 0; r < 128; ++r)
+                for (int c = 0; c < 128; ++c)
+                    vals[r * 128 + c] = bf16_to_f32(w[(i * 128 + r) * cols + j * 128 + c]);
+            e_out[i * bc + j] = quant_group_pow2(vals, 128 * 128, codes);
+            for (int r = 0; r < 128; ++r)
+                memcpy(q + (i * 128 + r) * cols + j * 128, codes + r * 128, 128);
+            free(vals);
+            free(codes);
+        }
+}
+
 /* ---------------------------------------------------------------- routing */
 /* Sigmoid affinity, bias-adjusted group-limited top-K, normalised gates and
  * the per-expert load histogram ("DeepSeekMoE and auxiliary-loss-free load

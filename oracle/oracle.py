@@ -20,6 +20,7 @@ __all__ = [
     "quant_w_128x128", "dequant_act", "dequant_w", "route", "update_bias",
     "permute_layout", "swiglu_expert", "f64_to_bf16_bits", "combine",
     "quantized_expert", "layer_forward", "gemm_blockscaled",
+    "quant_act_1x128_pow2", "quant_w_128x128_pow2", "pow2_scales",
 ]
 
 _LIB = None
@@ -41,6 +42,9 @@ def lib():
         L.orc_quant_act_1x128_bf16.argtypes = [P, I64, I64, P, P]
         L.orc_quant_act_1x128_f32.argtypes = [P, I64, I64, P, P]
         L.orc_quant_w_128x128.argtypes = [P, I64, I64, P, P]
+        L.orc_quant_act_1x128_pow2_bf16.argtypes = [P, I64, I64, P, P]
+        L.orc_quant_act_1x128_pow2_f32.argtypes = [P, I64, I64, P, P]
+        L.orc_quant_w_128x128_pow2.argtypes = [P, I64, I64, P, P]
         L.orc_route.restype = I
         L.orc_route.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
         L.orc_update_bias.argtypes = [I, I, I, P, ctypes.c_float, P]
@@ -99,6 +103,45 @@ def quant_w_128x128(w: np.ndarray):
     s = np.empty((rows // 128, cols // 128), dtype=np.float32)
     lib().orc_quant_w_128x128(_p(w), rows, cols, _p(q), _p(s))
     return q, s
+
+
+# ------------------------------------------- power-of-two scales (option)
+# Not the pages' recipe (their scales are arbitrary FP32 values): a
+# numerically different option whose scales are powers of two, so that
+# block-scaled tensor-core MMAs with UE8M0 scale factors can apply them.
+# Each function returns (codes, e) with e the int32 exponent of every scale
+# (scale = 2^e, UE8M0 byte = e + 127).
+
+def quant_act_1x128_pow2(x: np.ndarray):
+    """1x128 tiles, scale 2^e with e the smallest integer such that
+    amax <= 448 * 2^e; codes E4M3(v * 2^-e).  x: uint16 bf16 bits or fp32."""
+    rows, cols = x.shape
+    assert cols % 128 == 0
+    q = np.empty((rows, cols), dtype=np.uint8)
+    e = np.empty((rows, cols // 128), dtype=np.int32)
+    if x.dtype == np.uint16:
+        x = _c(x, np.uint16)
+        lib().orc_quant_act_1x128_pow2_bf16(_p(x), rows, cols, _p(q), _p(e))
+    else:
+        x = _c(x, np.float32)
+        lib().orc_quant_act_1x128_pow2_f32(_p(x), rows, cols, _p(q), _p(e))
+    return q, e
+
+
+def quant_w_128x128_pow2(w: np.ndarray):
+    """128x128 blocks of bf16 bits [rows, cols] with power-of-two scales."""
+    rows, cols = w.shape
+    assert rows % 128 == 0 and cols % 128 == 0
+    w = _c(w, np.uint16)
+    q = np.empty((rows, cols), dtype=np.uint8)
+    e = np.empty((rows // 128, cols // 128), dtype=np.int32)
+    lib().orc_quant_w_128x128_pow2(_p(w), rows, cols, _p(q), _p(e))
+    return q, e
+
+
+def pow2_scales(e: np.ndarray) -> np.ndarray:
+    """2^e as float64 (exact)."""
+    return np.ldexp(1.0, np.asarray(e, dtype=np.int32))
 
 
 _TABLE = None
