@@ -1,12 +1,16 @@
 """Benchmark of the DeepSeekMoE layer forward with FP8 block scaling on B200.
 
-Default workload: the full-size prefill layer (T=4096 tokens, d=7168, 256
-routed experts in 8 groups + 1 shared, top-4 groups, K=8, SwiGLU I=2048,
-FP8 E4M3 1x128 / 128x128 scales).  One step = the whole hot path over one
-batch: routing (+ load histogram), 1x128 quantisation of x, permutation,
-grouped GEMM W13 with SwiGLU + 1x128 quantisation of h, grouped GEMM W2,
-combine, bias update.  Expert weights are quantised once before timing (the
-offline weight quantisation is timed separately and reported).
+Default workload: the skewed large prefill (T=16384 tokens per batch,
+d=7168, 256 routed experts in 8 groups + 1 shared, top-4 groups, K=8,
+SwiGLU I=2048, FP8 E4M3 1x128 / 128x128 scales, a Zipf(1.2) prior on the
+router logits), eight successive batches cycled, each followed by the
++-gamma bias update.  One step = the whole hot path over one batch: routing
+(+ load histogram), 1x128 quantisation of x, permutation, grouped GEMM W13
+with SwiGLU + 1x128 quantisation of h, grouped GEMM W2, combine, bias
+update.  Expert weights are quantised once before timing (the offline
+weight quantisation is timed separately and reported).  Other workloads:
+--workload prefill (T=4096), decode (T=128), tiny, gemm (the block-scaled
+GEMM alone), route (the router alone), prefill_e16 (a small profiling case).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -35,7 +39,14 @@ if ROOT not in sys.path:
 METRIC = "MoE layer tokens/s and expert-GEMM FP8 TFLOPS (% of B200 FP8 dense peak)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_PER_BF16 = 2.0  # nominal dense ratio fp8 : bf16 (4.5 : 2.25 PFLOP/s)
-CPU_SAMPLE_TOKENS = 4
+# B200 datasheet figures, reported beside the measured-peak fractions
+DATASHEET = {"fp8_tflops": 4500.0, "hbm_gbs": 8000.0}
+# Oracle samples (random tokens of the batch): the CPU baseline of the GPU
+# arm (one sample, about 10-30 s of host work) and each step of the
+# reference arm (so that --steps 20 --warmup 5 ends within a few minutes)
+CPU_SAMPLE_TOKENS = {"tiny": 256, "prefill": 512, "decode": 128, "skewed": 2048,
+                     "prefill_e16": 256}
+REF_STEP_TOKENS = 64
 
 
 def load_peaks():
@@ -111,7 +122,8 @@ class ClockSampler:
 
 # --------------------------------------------------------------- workload
 def algorithmic_counts(cfg, counts_host):
-    """Algorithmic FLOPs and bytes of one layer step."""
+    """Algorithmic FLOPs and bytes of one layer step: the expert GEMMs'
+    multiply-adds, the touched experts' FP8 weights, and x in / y out."""
     d, I, K, T = cfg.d, cfg.inter, cfg.topk, cfg.T
     rows = T * K + T
     touched = int((counts_host > 0).sum()) + 1  # + shared expert
@@ -156,7 +168,7 @@ def profiled_traffic(kernel_tag: str):
     return float(t.group(1))
 
 
-def build_layer(cfg, dev):
+def build_layer(cfg, dev, scales="fp32"):
     import numpy as np
     import torch
     import fp8_block_scaled_affinity_b200 as moe
@@ -170,7 +182,8 @@ def build_layer(cfg, dev):
     shape = moe.make_shape(cfg.T, cfg.d, cfg.n_routed, cfg.n_groups, cfg.topk_groups, cfg.topk,
                            cfg.inter, cfg.gamma)
     layer = moe.MoeLayer(shape, bf16(inp["router_w"]), torch.from_numpy(inp["bias"]).to(dev),
-                         device=dev, host_io=True)
+                         device=dev, host_io="batches" if scales == "fp32" else False,
+                         scales=scales)
     small = cfg.d * cfg.inter <= 512 * 256
     wq_ms = 0.0
     st = torch.cuda.current_stream()
@@ -210,17 +223,21 @@ def stage_breakdown(layer, x, off, steps):
     pws = torch.empty((moe.moe_permute_workspace_size(sh),), dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream()
     names = ["route", "quant_permute", "gemm1_swiglu", "gemm2", "combine", "update_bias"]
+    mx = getattr(layer, "scales", "fp32") == "ue8m0"
+    if mx:  # power-of-two option: UE8M0 scale bytes, block-scaled GEMMs
+        xs_p = torch.empty((d // 128, R), dtype=torch.uint8, device=dev)
+        hs = torch.empty((I // 128, R), dtype=torch.uint8, device=dev)
+    permute = moe.moe_quant_permute_ue8m0 if mx else moe.moe_quant_permute
+    gemm = moe.moe_grouped_gemm_mxfp8 if mx else moe.moe_grouped_gemm_fp8
     calls = [
         lambda: moe.moe_route(sh, x, layer.router_w, layer.bias, off, layer.topk_idx,
                               layer.topk_gate, layer.expert_counts, rws),
-        lambda: moe.moe_quant_permute(sh, x, layer.topk_idx, layer.expert_counts, xq_p, xs_p,
-                                      layer.expert_offsets, layer.row_of_pair, pws),
-        lambda: moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, xq_p, xs_p, d,
-                                         layer.w13, layer.w13_scales, 2 * I,
-                                         _lib.MOE_EPI_SWIGLU_QUANT, hq, hs, layer.dev_status),
-        lambda: moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, hq, hs, I, layer.w2,
-                                         layer.w2_scales, d, _lib.MOE_EPI_F32, o, None,
-                                         layer.dev_status),
+        lambda: permute(sh, x, layer.topk_idx, layer.expert_counts, xq_p, xs_p,
+                        layer.expert_offsets, layer.row_of_pair, pws),
+        lambda: gemm(N + 1, layer.expert_offsets, R, xq_p, xs_p, d, layer.w13, layer.w13_scales,
+                     2 * I, _lib.MOE_EPI_SWIGLU_QUANT, hq, hs, layer.dev_status),
+        lambda: gemm(N + 1, layer.expert_offsets, R, hq, hs, I, layer.w2, layer.w2_scales, d,
+                     _lib.MOE_EPI_F32, o, None, layer.dev_status),
         lambda: moe.moe_combine(sh, o, layer.expert_offsets, layer.row_of_pair,
                                 layer.topk_gate, y),
         lambda: moe.moe_update_bias(sh, layer.expert_counts, layer.bias),
@@ -240,6 +257,9 @@ def stage_breakdown(layer, x, off, steps):
 
 
 # ------------------------------------------------------------ CPU oracle
+_ORACLE_WEIGHTS = {}  # workload -> expert -> oracle-quantised weights (reused across samples)
+
+
 def oracle_sample_time(cfg, inp, dev, n_tokens, seed=0):
     """The oracle (as it stands) on a bounded sample: n_tokens tokens through
     routing, quantisation, the experts they touch and the combine.  Expert
@@ -256,8 +276,10 @@ def oracle_sample_time(cfg, inp, dev, n_tokens, seed=0):
                      logit_offset=inp["logit_offset"])
     need = sorted(set(r["topk_idx"].ravel().tolist()) | {cfg.n_routed})
     small = cfg.d * cfg.inter <= 512 * 256
-    W = {}
+    W = _ORACLE_WEIGHTS.setdefault(cfg.name, {})
     for e in need:
+        if e in W:
+            continue
         if small:
             w = S.host_expert_weights(cfg, e)
         else:
@@ -286,7 +308,8 @@ def memory_passes(cfg, brk, alg, hbm_peak):
     out = {}
     for name, (ms, nbytes) in passes.items():
         gbs = nbytes / (ms / 1e3) / 1e9
-        out[name] = {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
+        out[name] = {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak,
+                     "frac_of_datasheet": gbs / DATASHEET["hbm_gbs"]}
     return out
 
 
@@ -314,7 +337,7 @@ def weight_quant_pass(dev, hbm_peak, rows=32768, cols=7168, reps=5):
     gbs = nbytes / (ms / 1e3) / 1e9
     del w, q, sc
     return {"ms": ms, "shape": [rows, cols], "bytes": nbytes, "gbs": gbs,
-            "frac_of_hbm": gbs / hbm_peak}
+            "frac_of_hbm": gbs / hbm_peak, "frac_of_datasheet": gbs / DATASHEET["hbm_gbs"]}
 
 
 # ------------------------------------------------------------ router alone
@@ -449,12 +472,19 @@ def run_gemm(args, world, rank, local):
             torch.bfloat16).to(dev)
 
     a, b = bf16(a_bits), bf16(b_bits)
+    mx = args.scales == "ue8m0"
+    sdt = torch.uint8 if mx else torch.float32
     aq = torch.empty((cfg.m, cfg.k), dtype=torch.uint8, device=dev)
-    as_ = torch.empty((cfg.k // 128, cfg.m), dtype=torch.float32, device=dev)
+    as_ = torch.empty((cfg.k // 128, cfg.m), dtype=sdt, device=dev)
     bq = torch.empty((cfg.n, cfg.k), dtype=torch.uint8, device=dev)
-    bs = torch.empty((cfg.n // 128, cfg.k // 128), dtype=torch.float32, device=dev)
-    moe.fp8_quant_act_1x128(a, aq, as_, scales_kb_major=True)
-    moe.fp8_quant_w_128x128(b, bq, bs)
+    bs = torch.empty((cfg.n // 128, cfg.k // 128), dtype=sdt, device=dev)
+    if mx:  # power-of-two option: UE8M0 scale bytes, block-scaled GEMM
+        moe.fp8_quant_act_1x128_ue8m0(a, aq, as_, sf_kb_major=True)
+        moe.fp8_quant_w_128x128_ue8m0(b, bq, bs)
+    else:
+        moe.fp8_quant_act_1x128(a, aq, as_, scales_kb_major=True)
+        moe.fp8_quant_w_128x128(b, bq, bs)
+    gemm_fn = moe.moe_grouped_gemm_mxfp8 if mx else moe.moe_grouped_gemm_fp8
     off = torch.tensor([0, cfg.m], dtype=torch.int32, device=dev)
     out = torch.empty((cfg.m, cfg.n), dtype=torch.bfloat16, device=dev)
     status = torch.zeros((1,), dtype=torch.int32, device=dev)
@@ -464,7 +494,7 @@ def run_gemm(args, world, rank, local):
     form = moe.moe_grouped_gemm_form(1, cfg.m, cfg.n, moe.MOE_EPI_BF16)
 
     def gemm(a_codes=aq, a_scales=as_, c=out):
-        moe.moe_grouped_gemm_fp8(1, off, cfg.m, a_codes, a_scales, cfg.k, bq, bs, cfg.n,
+        gemm_fn(1, off, cfg.m, a_codes, a_scales, cfg.k, bq, bs, cfg.n,
                                  moe.MOE_EPI_BF16, c, None, status)
 
     for _ in range(args.warmup):
@@ -514,16 +544,23 @@ def run_gemm(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8e4m3/f32", "data": "synthetic",
-        "config": {"workload": "fp8_blockscaled_gemm", "m": cfg.m, "n": cfg.n, "k": cfg.k,
+        "config": {"workload": "fp8_blockscaled_gemm", "scales": args.scales,
+                   "m": cfg.m, "n": cfg.n, "k": cfg.k,
                    "out": "bf16", "parallelism": f"replicas x{world}",
                    "l2": "256 MB buffer written between timed launches"},
         "roofline": {"bound": "tensor",
-                     "kernel": f"grouped_gemm_kernel<{int(form == 2)}, 0> "
-                               f"({'CTA pairs' if form == 2 else 'single CTAs'}; one group, bf16 out)",
+                     "kernel": ("mx_gemm_kernel<0> (block-scaled, UE8M0 scales; one group, "
+                                "bf16 out)" if mx else
+                                f"grouped_gemm_kernel<{int(form == 2)}, 0, 1> "
+                                f"({'CTA pairs' if form == 2 else 'single CTAs'}; one group, "
+                                "bf16 out)"),
                      "achieved": tflops / world, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": tflops / world / fp8_peak,
+                     "frac_of_datasheet": tflops / world / DATASHEET["fp8_tflops"],
+                     "datasheet_peak": DATASHEET["fp8_tflops"],
                      "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g} (nominal fp8:bf16)",
-                     "traffic": profiled_traffic("gemm_blockscaled_4096x7168x2048"),
+                     "traffic": profiled_traffic("gemm_ue8m0_4096x7168x2048" if mx else
+                                                 "gemm_blockscaled_4096x7168x2048"),
                      "algorithmic_flops_per_launch": flops, "launch_ms": ms / args.steps},
         "e2e": {"value": flops * args.steps * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": aq.numel() + as_.numel() * 4,
@@ -584,7 +621,7 @@ def barrier(world: int):
 
 def run_reference(args, world, rank):
     """The oracle timed on the host cores: each step is a bounded sample of
-    the workload (CPU_SAMPLE_TOKENS tokens)."""
+    the workload (REF_STEP_TOKENS random tokens)."""
     import numpy as np
     import torch
     import synthetic as S
@@ -598,12 +635,13 @@ def run_reference(args, world, rank):
     dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
     inp = S.make_layer_inputs_host(cfg, 0)
     times = []
+    n_tok = min(REF_STEP_TOKENS, cfg.T)
     for i in range(args.warmup + args.steps):
-        dt, n, cores = oracle_sample_time(cfg, inp, dev, CPU_SAMPLE_TOKENS, seed=i)
+        dt, n, cores = oracle_sample_time(cfg, inp, dev, n_tok, seed=i)
         if i >= args.warmup:
             times.append(dt)
     total = sum(times)
-    value = args.steps * CPU_SAMPLE_TOKENS / total
+    value = args.steps * n_tok / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -612,10 +650,10 @@ def run_reference(args, world, rank):
         "config": {"workload": f"moe_layer_{cfg.name}", "T": cfg.T, "d": cfg.d,
                    "n_routed": cfg.n_routed, "n_shared": 1, "n_groups": cfg.n_groups,
                    "topk_groups": cfg.topk_groups, "topk": cfg.topk, "inter": cfg.inter,
-                   "sample_tokens_per_step": CPU_SAMPLE_TOKENS},
+                   "sample_tokens_per_step": n_tok},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count() or 1,
                          "kind": "oracle",
-                         "sample": f"{CPU_SAMPLE_TOKENS} random tokens per step of the "
+                         "sample": f"{n_tok} random tokens per step of the "
                                    f"{cfg.name} batch (routing, quantisation, touched experts,"
                                    " combine)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -701,7 +739,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     cfg = S.CONFIGS[args.workload]
     peaks, peak_src = load_peaks()
-    layer, x, off, inp, wq_ms = build_layer(cfg, dev)
+    layer, x, off, inp, wq_ms = build_layer(cfg, dev, args.scales)
     st = torch.cuda.current_stream()
     y = torch.empty_like(x)
     bias0 = layer.bias.clone()
@@ -737,20 +775,38 @@ def run_ours(args, world, rank, local):
     tokens_total = cfg.T * args.steps * world
     value = tokens_total / (ms / 1e3)
 
-    # ---- end to end through the host-buffer entry point (pinned memory)
-    hosts = [b.cpu().pin_memory() for b in batches]
-    y_host = torch.empty_like(hosts[0]).pin_memory()
-    for i in range(max(1, args.warmup // 2)):
-        layer.forward_host(hosts[i % nb], y_host, update_bias=True, logit_offset=off)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for i in range(args.steps):
-        layer.forward_host(hosts[i % nb], y_host, update_bias=True, logit_offset=off)
-    e1.record(st)
-    e1.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # ---- end to end through the host-buffer entry points (pinned memory):
+    # the batches call overlaps each batch's copies with its neighbours'
+    # compute; one forward_host call per step (copies in line) is reported
+    # beside it
+    x_hosts = torch.stack([b.cpu() for b in batches]).pin_memory()  # [nb, T, d]
+    y_hosts = torch.empty_like(x_hosts).pin_memory()
+
+    def e2e_steps(pipelined):
+        done = 0
+        while done < args.steps:
+            n = min(nb, args.steps - done)  # calls start at batch 0
+            if pipelined:
+                layer.forward_host_batches(x_hosts[:n], y_hosts[:n], update_bias=True,
+                                           logit_offset=off)
+            else:
+                for j in range(n):
+                    layer.forward_host(x_hosts[j], y_hosts[j], update_bias=True,
+                                       logit_offset=off)
+            done += n
+
+    e2e = {}
+    for pipelined in ((True, False) if args.scales == "fp32" else ()):
+        layer.forward_host_batches(x_hosts[:1], y_hosts[:1], update_bias=True, logit_offset=off)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        e2e_steps(pipelined)
+        e1.record(st)
+        e1.synchronize()
+        e2e[pipelined] = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_ms = e2e.get(True)
     xbytes = cfg.T * cfg.d * 2
 
     # ---- per-batch expert load from the initial bias, batches in order
@@ -797,6 +853,12 @@ def run_ours(args, world, rank, local):
                     "algorithmic_bytes_per_launch": alg["gemm1_bytes"], "launch_ms": g1_ms}
     roofline["intensity_flop_per_byte"] = intensity
     roofline["ridge_flop_per_byte"] = ridge
+    if roofline["bound"] == "hbm":
+        roofline["frac_of_datasheet"] = achieved / DATASHEET["hbm_gbs"]
+        roofline["datasheet_peak"] = DATASHEET["hbm_gbs"]
+    else:
+        roofline["frac_of_datasheet"] = roofline["achieved"] / DATASHEET["fp8_tflops"]
+        roofline["datasheet_peak"] = DATASHEET["fp8_tflops"]
     gemm_ms = brk["gemm1_swiglu"] + brk["gemm2"]
     gemm_tflops = alg["layer_flops"] / (gemm_ms / 1e3) / 1e12
     layer_tflops = alg["layer_flops"] * args.steps * world / (ms / 1e3) / 1e12
@@ -812,9 +874,10 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8e4m3/f32",
+        "dtype": "fp8e4m3/f32" if args.scales == "fp32" else "fp8e4m3+ue8m0/f32",
         "data": "synthetic",
-        "config": {"workload": f"moe_layer_{cfg.name}", "T": cfg.T, "d": cfg.d,
+        "config": {"workload": f"moe_layer_{cfg.name}", "scales": args.scales,
+                   "T": cfg.T, "d": cfg.d,
                    "n_routed": cfg.n_routed, "n_shared": 1, "n_groups": cfg.n_groups,
                    "topk_groups": cfg.topk_groups, "topk": cfg.topk, "inter": cfg.inter,
                    "parallelism": f"replicas x{world}",
@@ -825,6 +888,7 @@ def run_ours(args, world, rank, local):
                         "ctas_per_tile": gemm_forms,
                         "frac_of_fp8_peak": gemm_tflops / fp8_peak_burst,
                         "frac_of_fp8_sustained": gemm_tflops / fp8_peak_sust,
+                        "frac_of_fp8_datasheet": gemm_tflops / DATASHEET["fp8_tflops"],
                         "gemm1_ms": brk["gemm1_swiglu"], "gemm2_ms": brk["gemm2"],
                         "flops_per_step": alg["layer_flops"]},
         "layer_tflops": layer_tflops,
@@ -834,8 +898,13 @@ def run_ours(args, world, rank, local):
         "load": {"max_over_mean": float(counts.max() / max(counts.mean(), 1e-9)),
                  "max_over_mean_per_batch": per_batch,
                  "experts_touched": alg["touched"]},
-        "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes},
+        "e2e": ({"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
+                 "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes,
+                 "api": f"moe_layer_forward_host_batches (up to {nb} batches per call, "
+                        "copies overlapped with neighbouring batches' compute)",
+                 "unpipelined_value": tokens_total / (e2e[False] / 1e3),
+                 "unpipelined_api": "moe_layer_forward_host, one call per step"}
+                if e2e else None),
         # route 6, quant+permute 4, GEMMs 2, combine 1, bias update 1
         "gpu_launches": 15 * args.steps,
         "clocks": clk,
@@ -843,7 +912,7 @@ def run_ours(args, world, rank, local):
     }
     # CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, n, cores = oracle_sample_time(cfg, inp, dev, CPU_SAMPLE_TOKENS)
+        dt, n, cores = oracle_sample_time(cfg, inp, dev, min(CPU_SAMPLE_TOKENS[cfg.name], cfg.T))
         line["cpu_baseline"] = {
             "value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{n} random tokens of the {cfg.name} batch (routing, quantisation, "
@@ -858,10 +927,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill",
+    ap.add_argument("--workload", default="skewed",
                     choices=["tiny", "prefill", "decode", "skewed", "prefill_e16", "gemm",
                              "route"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scales", choices=["fp32", "ue8m0"], default="fp32",
+                    help="fp32: the pages' recipe (default); ue8m0: the power-of-two scale "
+                         "option with block-scaled tensor-core GEMMs")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -15,11 +15,16 @@ from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QU
                    MoeError, MoeRouting, MoeShape, MoeWeights, fp8_quant_act_1x128,
                    fp8_quant_w_128x128, lib, make_routing, make_shape, make_weights,
                    moe_combine, moe_grouped_gemm_form, moe_grouped_gemm_fp8,
-                   moe_layer_forward,
-                   moe_layer_forward_host, moe_layer_host_workspace_size,
+                   moe_layer_forward, moe_layer_forward_host_batches,
+                   moe_layer_forward_host, moe_layer_host_batches_workspace_size,
+                   moe_layer_host_workspace_size,
                    moe_layer_workspace_size, moe_permute, moe_permute_workspace_size, moe_quant_permute,
                    moe_read_status, moe_route, moe_route_workspace_size, moe_update_bias,
-                   moe_version, status_string)
+                   moe_version, status_string, fp8_quant_act_1x128_ue8m0,
+                   fp8_quant_w_128x128_ue8m0, moe_grouped_gemm_mxfp8,
+                   moe_grouped_gemm_fp8_indexed, moe_plan_redundant_experts, moe_split_groups,
+                   MoeWeightsMx, make_weights_mx, moe_layer_forward_mx,
+                   moe_layer_mx_workspace_size, moe_quant_permute_ue8m0)
 
 __all__ = ["MoeLayer", "MoeShape", "MoeError", "lib", "make_shape", "moe_version"]
 
@@ -32,8 +37,16 @@ class MoeLayer:
     bias: fp32 [N_r] on the GPU (updated in place by forward(update_bias=True)).
     """
 
-    def __init__(self, shape: MoeShape, router_w, bias, device=None, host_io: bool = False):
+    def __init__(self, shape: MoeShape, router_w, bias, device=None, host_io=False,
+                 scales: str = "fp32"):
+        """scales: "fp32" (the pages' recipe: FP32 scales, per-128-K promotion)
+        or "ue8m0" (power-of-two scales, block-scaled tensor-core GEMMs)."""
         import torch
+        if scales not in ("fp32", "ue8m0"):
+            raise ValueError("scales must be 'fp32' or 'ue8m0'")
+        if scales == "ue8m0" and host_io:
+            raise ValueError("host-buffer calls use the fp32-scale layer")
+        self.scales = scales
         self.shape = shape
         dev = torch.device(device) if device is not None else router_w.device
         self.device = dev
@@ -43,9 +56,10 @@ class MoeLayer:
         self.bias = bias
         u8 = torch.uint8
         self.w13 = torch.empty((E, 2 * I, d), dtype=u8, device=dev)
-        self.w13_scales = torch.empty((E, 2 * I // 128, d // 128), dtype=torch.float32, device=dev)
+        sdt = torch.float32 if scales == "fp32" else u8  # UE8M0 bytes for "ue8m0"
+        self.w13_scales = torch.empty((E, 2 * I // 128, d // 128), dtype=sdt, device=dev)
         self.w2 = torch.empty((E, d, I), dtype=u8, device=dev)
-        self.w2_scales = torch.empty((E, d // 128, I // 128), dtype=torch.float32, device=dev)
+        self.w2_scales = torch.empty((E, d // 128, I // 128), dtype=sdt, device=dev)
         T, K = shape.T, shape.topk
         i32 = torch.int32
         self.topk_idx = torch.empty((T, K), dtype=i32, device=dev)
@@ -54,7 +68,10 @@ class MoeLayer:
         self.expert_offsets = torch.empty((N + 2,), dtype=i32, device=dev)
         self.row_of_pair = torch.empty((T, K), dtype=i32, device=dev)
         self.dev_status = torch.zeros((1,), dtype=i32, device=dev)
-        ws_bytes = (moe_layer_host_workspace_size(shape) if host_io
+        # host_io: False (device x / y), True (forward_host), "batches"
+        # (forward_host_batches as well)
+        ws_bytes = (moe_layer_host_batches_workspace_size(shape) if host_io == "batches"
+                    else moe_layer_host_workspace_size(shape) if host_io
                     else moe_layer_workspace_size(shape))
         self.ws = torch.empty((max(ws_bytes, 256),), dtype=u8, device=dev)
         self._weights = None
@@ -66,17 +83,16 @@ class MoeLayer:
         the layer's FP8 buffers with 128x128 blocks.  e = N_r is the shared
         expert."""
         I = self.shape.inter
-        fp8_quant_w_128x128(w1, self.w13[e, :I], self.w13_scales[e, :I // 128],
-                            stream=stream)
-        fp8_quant_w_128x128(w3, self.w13[e, I:], self.w13_scales[e, I // 128:],
-                            stream=stream)
-        fp8_quant_w_128x128(w2, self.w2[e], self.w2_scales[e], stream=stream)
+        quant = fp8_quant_w_128x128 if self.scales == "fp32" else fp8_quant_w_128x128_ue8m0
+        quant(w1, self.w13[e, :I], self.w13_scales[e, :I // 128], stream=stream)
+        quant(w3, self.w13[e, I:], self.w13_scales[e, I // 128:], stream=stream)
+        quant(w2, self.w2[e], self.w2_scales[e], stream=stream)
         self._weights = None
 
-    def weights(self) -> MoeWeights:
+    def weights(self):
         if self._weights is None:
-            self._weights = make_weights(self.w13, self.w13_scales, self.w2, self.w2_scales,
-                                         self.router_w)
+            mk = make_weights if self.scales == "fp32" else make_weights_mx
+            self._weights = mk(self.w13, self.w13_scales, self.w2, self.w2_scales, self.router_w)
         return self._weights
 
     def forward(self, x, y=None, update_bias: bool = False, logit_offset=None, stream=None):
@@ -84,8 +100,9 @@ class MoeLayer:
         import torch
         if y is None:
             y = torch.empty_like(x)
-        moe_layer_forward(self.shape, self.weights(), x, self.bias, logit_offset,
-                          self._routing, y, update_bias, self.ws, self.dev_status, stream)
+        fwd = moe_layer_forward if self.scales == "fp32" else moe_layer_forward_mx
+        fwd(self.shape, self.weights(), x, self.bias, logit_offset, self._routing, y,
+            update_bias, self.ws, self.dev_status, stream)
         return y
 
     def forward_host(self, x_host, y_host, update_bias: bool = False, logit_offset=None,
@@ -95,6 +112,16 @@ class MoeLayer:
         moe_layer_forward_host(self.shape, self.weights(), x_host, self.bias, logit_offset,
                                self._routing, y_host, update_bias, self.ws, self.dev_status,
                                stream)
+
+    def forward_host_batches(self, x_host, y_host, update_bias: bool = False,
+                             logit_offset=None, stream=None):
+        """Batches x_host[j] (pinned bf16 [n, T, d]) -> y_host[j], the copies
+        of neighbouring batches overlapped with the computation (the layer
+        must be built with host_io="batches").  Synchronise the stream before
+        reading y_host."""
+        moe_layer_forward_host_batches(self.shape, self.weights(), x_host, x_host.shape[0],
+                                       self.bias, logit_offset, self._routing, y_host,
+                                       update_bias, self.ws, self.dev_status, stream)
 
     def status(self, stream=None) -> int:
         """Device status word (0 = fine); synchronises the stream."""

@@ -39,6 +39,12 @@ class MoeWeights(ctypes.Structure):
                 ("router_w", ctypes.c_void_p)]
 
 
+class MoeWeightsMx(ctypes.Structure):
+    _fields_ = [("w13", ctypes.c_void_p), ("w13_sf", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("w2_sf", ctypes.c_void_p),
+                ("router_w", ctypes.c_void_p)]
+
+
 class MoeRouting(ctypes.Structure):
     _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_gate", ctypes.c_void_p),
                 ("expert_counts", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
@@ -73,6 +79,17 @@ def lib() -> ctypes.CDLL:
             "moe_quant_permute": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
             "moe_grouped_gemm_fp8": (I, [I, P, I, P, P, I, P, P, I, I, P, P, P, P]),
             "moe_grouped_gemm_form": (I, [I, I, I, I]),
+            "fp8_quant_act_1x128_ue8m0": (I, [P, I64, I64, P, P, I, P, P]),
+            "fp8_quant_w_128x128_ue8m0": (I, [P, I64, I64, P, P, P, P]),
+            "moe_grouped_gemm_mxfp8": (I, [I, P, I, P, P, I, P, P, I, I, P, P, P, P]),
+            "moe_grouped_gemm_fp8_indexed": (I, [I, P, P, I, I, P, P, I, P, P, I, I, P, P, P,
+                                                 P]),
+            "moe_plan_redundant_experts": (I, [P, I, I, P, P]),
+            "moe_quant_permute_ue8m0": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "moe_layer_mx_workspace_size": (SZ, [SP]),
+            "moe_layer_forward_mx": (I, [SP, ctypes.POINTER(MoeWeightsMx), P, P, P,
+                                         ctypes.POINTER(MoeRouting), P, I, P, SZ, P, P]),
+            "moe_split_groups": (I, [SP, P, P, P, P, I, P, P, P, P]),
             "moe_combine": (I, [SP, P, P, P, P, P, P, P]),
             "moe_update_bias": (I, [SP, P, P, P, P]),
             "moe_layer_workspace_size": (SZ, [SP]),
@@ -81,6 +98,10 @@ def lib() -> ctypes.CDLL:
             "moe_layer_host_workspace_size": (SZ, [SP]),
             "moe_layer_forward_host": (I, [SP, ctypes.POINTER(MoeWeights), P, P, P,
                                            ctypes.POINTER(MoeRouting), P, I, P, SZ, P, P]),
+            "moe_layer_host_batches_workspace_size": (SZ, [SP]),
+            "moe_layer_forward_host_batches": (I, [SP, ctypes.POINTER(MoeWeights), P, I, P, P,
+                                                   ctypes.POINTER(MoeRouting), P, I, P, SZ, P,
+                                                   P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -254,3 +275,98 @@ def moe_layer_forward_host(shape, weights: MoeWeights, x_host, bias, logit_offse
         ctypes.byref(shape), ctypes.byref(weights), _ptr(x_host), _ptr(bias),
         _ptr(logit_offset), ctypes.byref(routing), _ptr(y_host), int(bool(update_bias)),
         _ptr(ws), nbytes, _ptr(dev_status), _stream(stream)))
+
+
+def moe_layer_host_batches_workspace_size(shape: MoeShape) -> int:
+    return lib().moe_layer_host_batches_workspace_size(ctypes.byref(shape))
+
+
+def moe_layer_forward_host_batches(shape, weights: MoeWeights, x_host, n_batches, bias,
+                                   logit_offset, routing: MoeRouting, y_host, update_bias, ws,
+                                   dev_status=None, stream=None):
+    """n_batches successive batches, x_host / y_host pinned [n_batches, T, d]."""
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_layer_forward_host_batches", lib().moe_layer_forward_host_batches(
+        ctypes.byref(shape), ctypes.byref(weights), _ptr(x_host), int(n_batches), _ptr(bias),
+        _ptr(logit_offset), ctypes.byref(routing), _ptr(y_host), int(bool(update_bias)),
+        _ptr(ws), nbytes, _ptr(dev_status), _stream(stream)))
+
+
+# ------------------------------------------- power-of-two scale option
+def fp8_quant_act_1x128_ue8m0(x, q, sf, sf_kb_major=False, dev_status=None, stream=None):
+    """1x128 tiles with power-of-two scales; sf: uint8 UE8M0 bytes."""
+    rows, cols = x.shape
+    _check("fp8_quant_act_1x128_ue8m0", lib().fp8_quant_act_1x128_ue8m0(
+        _ptr(x), rows, cols, _ptr(q), _ptr(sf), int(bool(sf_kb_major)), _ptr(dev_status),
+        _stream(stream)))
+
+
+def fp8_quant_w_128x128_ue8m0(w, q, sf, dev_status=None, stream=None):
+    rows, cols = w.shape
+    _check("fp8_quant_w_128x128_ue8m0", lib().fp8_quant_w_128x128_ue8m0(
+        _ptr(w), rows, cols, _ptr(q), _ptr(sf), _ptr(dev_status), _stream(stream)))
+
+
+def moe_grouped_gemm_mxfp8(n_groups, group_offsets, max_rows, a, a_sf, k, w, w_sf, n, epilogue,
+                           out, out_sf=None, dev_status=None, stream=None):
+    _check("moe_grouped_gemm_mxfp8", lib().moe_grouped_gemm_mxfp8(
+        int(n_groups), _ptr(group_offsets), int(max_rows), _ptr(a), _ptr(a_sf), int(k), _ptr(w),
+        _ptr(w_sf), int(n), int(epilogue), _ptr(out), _ptr(out_sf), _ptr(dev_status),
+        _stream(stream)))
+
+
+# ----------------------------------------------------- redundant experts
+def moe_grouped_gemm_fp8_indexed(n_groups, group_offsets, group_weight, n_weights, max_rows, a,
+                                 a_scales, k, w, w_scales, n, epilogue, out, out_scales=None,
+                                 dev_status=None, stream=None):
+    _check("moe_grouped_gemm_fp8_indexed", lib().moe_grouped_gemm_fp8_indexed(
+        int(n_groups), _ptr(group_offsets), _ptr(group_weight), int(n_weights), int(max_rows),
+        _ptr(a), _ptr(a_scales), int(k), _ptr(w), _ptr(w_scales), int(n), int(epilogue),
+        _ptr(out), _ptr(out_scales), _ptr(dev_status), _stream(stream)))
+
+
+def moe_plan_redundant_experts(counts, n_extra):
+    """Host planner: counts (sequence of ints) -> (replicas, slot_expert) as
+    numpy int32 arrays."""
+    import numpy as np
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.int32))
+    rep = np.empty(c.size, dtype=np.int32)
+    slots = np.empty(c.size + int(n_extra), dtype=np.int32)
+    _check("moe_plan_redundant_experts", lib().moe_plan_redundant_experts(
+        c.ctypes.data, int(c.size), int(n_extra), rep.ctypes.data, slots.ctypes.data))
+    return rep, slots
+
+
+def moe_split_groups(shape, expert_offsets, replicas, slot_expert, first_slot, n_extra,
+                     slot_offsets, slot_weight, dev_status=None, stream=None):
+    _check("moe_split_groups", lib().moe_split_groups(
+        ctypes.byref(shape), _ptr(expert_offsets), _ptr(replicas), _ptr(slot_expert),
+        _ptr(first_slot), int(n_extra), _ptr(slot_offsets), _ptr(slot_weight), _ptr(dev_status),
+        _stream(stream)))
+
+
+def moe_quant_permute_ue8m0(shape, x, topk_idx, expert_counts, xq_perm, xsf_perm,
+                            expert_offsets, row_of_pair, ws, dev_status=None, stream=None):
+    """moe_quant_permute with power-of-two scales (xsf_perm: uint8 UE8M0)."""
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("moe_quant_permute_ue8m0", lib().moe_quant_permute_ue8m0(
+        ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(expert_counts), _ptr(xq_perm),
+        _ptr(xsf_perm), _ptr(expert_offsets), _ptr(row_of_pair), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_layer_mx_workspace_size(shape: MoeShape) -> int:
+    return lib().moe_layer_mx_workspace_size(ctypes.byref(shape))
+
+
+def make_weights_mx(w13, w13_sf, w2, w2_sf, router_w) -> MoeWeightsMx:
+    return MoeWeightsMx(_ptr(w13), _ptr(w13_sf), _ptr(w2), _ptr(w2_sf), _ptr(router_w))
+
+
+def moe_layer_forward_mx(shape, weights: MoeWeightsMx, x, bias, logit_offset,
+                         routing: MoeRouting, y, update_bias, ws, dev_status=None, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_layer_forward_mx", lib().moe_layer_forward_mx(
+        ctypes.byref(shape), ctypes.byref(weights), _ptr(x), _ptr(bias), _ptr(logit_offset),
+        ctypes.byref(routing), _ptr(y), int(bool(update_bias)), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))

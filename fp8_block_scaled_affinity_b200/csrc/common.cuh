@@ -33,6 +33,11 @@ int validate_shape(const MoeShape* s);
 // True when the current device is an sm_100 part.
 bool device_is_sm100();
 
+// False when p is memory the GPU cannot address (pageable host memory that
+// was never registered with CUDA); device, managed and pinned host memory
+// pass.  NULL passes (callers check required pointers separately).
+bool device_accessible(const void* p);
+
 // --------------------------------------------------------------- device
 __device__ __forceinline__ void set_status(int* st, int code) {
     if (st) atomicCAS(st, 0, code);
@@ -58,6 +63,23 @@ __device__ __forceinline__ void scale_from_amax(float amax, float& scale, float&
     }
 }
 
+// Power-of-two scale option (UE8M0 scale bytes, for the block-scaled MMA
+// form): e = the smallest integer with amax <= 448 * 2^e, clamped to
+// [-127, 127], 0 for amax = 0; the scale is 2^e (byte e + 127) and the code
+// of v is E4M3(v * 2^-e).  Every comparison is exact in FP64.
+__device__ __forceinline__ int pow2_exponent(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    const double a = (double)amax;
+    int e = int((__double_as_longlong(a) >> 52) & 0x7FF) - 1023 - 9;  // too small
+    // 448 * 2^e = 1.75 * 2^(e + 8), built from its bits
+    while (a > __longlong_as_double((int64_t(e + 8 + 1023) << 52) | (int64_t(3) << 50))) ++e;
+    return max(-127, min(127, e));
+}
+// 2^-e as fp32 for e in [-127, 127] (2^-127 is the subnormal 0x00400000)
+__device__ __forceinline__ float pow2_inverse(int e) {
+    return e < 127 ? __int_as_float((127 - e) << 23) : __int_as_float(0x00400000);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -69,6 +91,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // A wait that has not finished after this many nanoseconds is abandoned and
 // reported as MOE_DEV_TIMEOUT.  Real waits in these kernels last microseconds.
+// The limit is a kernel argument: wait_limit_ns() gives it, this default
+// unless MOEFP8_WAIT_LIMIT_NS is set in the environment.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Bounded wait limit of the next launch (host; read at every call).
+uint64_t wait_limit_ns();
+
+// Host-driven fault injection (MOEFP8_FAULT in the environment, read at
+// every call): kFaultGemmProducer makes the single-CTA grouped GEMM's TMA
+// producer withhold the loads of its first stage, so that the MMA issuer's
+// bounded wait on that stage runs out (MOE_DEV_TIMEOUT) and the kernel
+// unwinds.  Nothing faults, traps or hangs: the wait limit ends it.
+enum FaultKind { kFaultNone = 0, kFaultGemmProducer = 1 };
+int fault_injection();
 
 }  // namespace moe

@@ -63,8 +63,15 @@ constexpr int kABoxes = 4;                       // token boxes of 128, 64, 32, 
 template <bool PAIR, bool SWIGLU, bool WIDE>
 struct Cfg {
     static_assert(WIDE || !(PAIR || SWIGLU), "pairs and SwiGLU use 256-column partials");
-    static constexpr int kAccCols = WIDE ? 256 : 128;              // TMEM columns per partial
-    static constexpr int kBufs = 512 / kAccCols;                   // TMEM partial buffers
+    static constexpr int kAccCols = WIDE ? 256 : 128;              // output columns per item
+    // Single CTAs with 256-column items split each K block into two MMA
+    // chains of N = 128 (one per weight block), each into its own 128-column
+    // TMEM buffer with its own full / empty barriers: four buffers rotate,
+    // and a buffer is busy for half as long as a 256-column partial.
+    static constexpr bool kSplit = !PAIR && WIDE;
+    static constexpr int kChains = kSplit ? 2 : 1;                 // MMA chains per K block
+    static constexpr int kBufCols = kAccCols / kChains;            // TMEM columns per buffer
+    static constexpr int kBufs = 512 / kBufCols;                   // TMEM partial buffers
     static constexpr int kWRows = PAIR ? 128 : kAccCols;           // weight rows this CTA loads
     static constexpr int kStageBytes = kTileBytes + kWRows * 128;  // tokens + weights
     // single CTAs with fp32/bf16 output and 256 columns: 48 KB stages next to
@@ -96,6 +103,16 @@ struct GemmParams {
     void* out;
     float* out_scales;
     int* dev_status;
+    uint64_t wait_limit_ns;  // bound of every wait (kWaitLimitNs unless overridden)
+    int fault;               // FaultKind injected from the host (kFaultNone normally)
+    // weight matrix of each group (nullable: group g uses matrix g); lets
+    // several groups share one expert's weights (redundant experts)
+    const int32_t* group_weight;
+    int n_weights;           // weight matrices in w (== n_groups without an index)
+    // block-scaled (UE8M0) form only
+    const uint8_t* a_sf;     // [nkb, max_rows] scale bytes of the tokens' 1x128 tiles
+    const uint8_t* w_sf;     // [n_groups, n/128, nkb] scale bytes of the weight blocks
+    uint8_t* out_sf;         // SwiGLU: [n/256, max_rows] scale bytes of h
 };
 
 // Token tensor maps, one per box height (128, 64, 32, 16 rows).
@@ -111,6 +128,7 @@ struct SharedState {
     uint64_t sfull[kScaleSlots];
     uint64_t sempty[kScaleSlots];
     uint64_t drain;
+    uint64_t wait_limit;     // ns
     uint32_t tmem_base;
     int abort_flag;
     uint32_t peer_abort;     // cluster address of the peer CTA's abort_flag (0: no peer)
@@ -236,22 +254,40 @@ __device__ __forceinline__ void raise_abort(SharedState* ss) {
 }
 
 // Bounded wait: returns false (and raises the abort flags and the device
-// status) when the phase does not complete within kWaitLimitNs, or when
-// another role of the CTA (or of its peer) has already aborted.
+// status) when the phase does not complete within the launch's wait limit,
+// or when another role of the CTA (or of its peer) has already aborted.
 template <int FORM = kSuspend>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, SharedState* ss,
                                           int* dev_status) {
     if (mbar_try_wait<FORM>(bar, parity)) return true;
-    uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = ss->wait_limit;
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait<FORM>(bar, parity)) return true;
         if ((it & 15) == 0) {
             if (*reinterpret_cast<volatile int*>(&ss->abort_flag)) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit) {
                 raise_abort(ss);
                 set_status(dev_status, MOE_DEV_TIMEOUT);
                 return false;
             }
+        }
+    }
+}
+
+// Waits for work already in flight (TMA loads into this CTA's shared memory,
+// MMAs into its TMEM) before the CTA leaves: unlike mbar_wait it goes on
+// after an abort, but it still gives up after the wait limit.
+__device__ __forceinline__ bool mbar_quiesce(uint32_t bar, uint32_t parity, SharedState* ss,
+                                             int* dev_status) {
+    if (mbar_try_wait<kPoll>(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = ss->wait_limit;
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait<kPoll>(bar, parity)) return true;
+        if ((it & 15) == 0 && globaltimer_ns() - t0 > limit) {
+            set_status(dev_status, MOE_DEV_TIMEOUT);
+            return false;
         }
     }
 }
@@ -494,6 +530,18 @@ __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmPar
     return it;
 }
 
+// Weight matrix of group g (the group itself unless an index is given; an
+// out-of-range index falls back to matrix 0 and is reported).
+__device__ __forceinline__ int weight_of(const GemmParams& p, int g) {
+    if (!p.group_weight) return g;
+    const int wi = __ldg(&p.group_weight[g]);
+    if (wi < 0 || wi >= p.n_weights) {
+        set_status(p.dev_status, MOE_DEV_BAD_INPUT);
+        return 0;
+    }
+    return wi;
+}
+
 // Valid tokens of CTA `rank` in an item (0..128).
 __device__ __forceinline__ int cta_tokens(const Item& w, int rank) {
     return max(0, min(kBM, w.rows - kBM * rank));
@@ -548,8 +596,9 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
         const int a_y = w.row0 + kBM * rank;
         // bytes landing on the stage barrier: every CTA's tokens and weights
         const uint32_t tx = box_bytes(n0) + box_bytes(n1) + uint32_t(C::kCtas * C::kWRows * 128);
-        const int wr_mine = w.g * p.n + (rank ? b1 : b0) * 128;
-        const int wr_second = w.g * p.n + b1 * 128;  // single CTA, 256 columns: block b1
+        const int wg = weight_of(p, w.g);
+        const int wr_mine = wg * p.n + (rank ? b1 : b0) * 128;
+        const int wr_second = wg * p.n + b1 * 128;  // single CTA, 256 columns: block b1
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
             const int s = it % C::kStages;
             const uint32_t par = ((it / C::kStages) & 1u);
@@ -558,6 +607,9 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
                                                   p.dev_status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
+            // injected fault: the first stage is never loaded, so the MMA
+            // issuer's wait on it runs out (single CTAs only)
+            if (!PAIR && p.fault == kFaultGemmProducer && it == 0) continue;
             if (lane == 0) {
                 uint8_t* st = smem + size_t(s) * C::kStageBytes;
                 const uint32_t local_full = smem_u32(&ss->full[s]);
@@ -578,7 +630,7 @@ __device__ __forceinline__ void producer(const GemmParams& p, const CUtensorMap*
         // barriers of a pair are the leader's)
         for (int s = 0; s < C::kStages; ++s)
             if ((issued_mask >> s) & 1u)
-                mbar_wait(smem_u32(&ss->full[s]), (issued_parity >> s) & 1u, ss, nullptr);
+                mbar_quiesce(smem_u32(&ss->full[s]), (issued_parity >> s) & 1u, ss, nullptr);
     }
     __syncwarp();
 }
@@ -602,8 +654,9 @@ __device__ __forceinline__ void scale_loader(const GemmParams& p, SharedState* s
         weight_blocks<PAIR, SWIGLU, WIDE>(p, w, b0, b1);
         const int my_n = cta_tokens(w, rank);
         const int my_row0 = w.row0 + kBM * rank;
-        const float* sb0 = p.w_scales + (size_t(w.g) * nbr + b0) * p.nkb;
-        const float* sb1 = p.w_scales + (size_t(w.g) * nbr + b1) * p.nkb;
+        const int wg = weight_of(p, w.g);
+        const float* sb0 = p.w_scales + (size_t(wg) * nbr + b0) * p.nkb;
+        const float* sb1 = p.w_scales + (size_t(wg) * nbr + b1) * p.nkb;
         for (int kb = 0; kb < p.nkb; ++kb, ++cit) {
             const int c = cit % kScaleSlots;
             if (lane == 0)
@@ -639,32 +692,42 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
     if (lane == 0) {
         uint32_t it = 0, tb = 0;
         bool ok = true;
-        const uint32_t idesc = idesc_e4m3(C::kMmaM, C::kAccCols);
+        const uint32_t idesc = idesc_e4m3(C::kMmaM, C::kBufCols);
         for (int item = unit; ok && item < total_items; item += units) {
-            for (int kb = 0; kb < p.nkb; ++kb, ++it, ++tb) {
+            for (int kb = 0; ok && kb < p.nkb; ++kb, ++it) {
                 const int s = it % C::kStages;
-                const uint32_t buf = tb % C::kBufs;
-                const uint32_t tpar = (tb / C::kBufs) & 1u;
-                ok = mbar_wait<kIssuerWait<PAIR>>(smem_u32(&ss->tempty[buf]), tpar ^ 1u, ss,
-                                                   p.dev_status);
-                if (!ok) break;
-                ok = mbar_wait<kIssuerWait<PAIR>>(smem_u32(&ss->full[s]), (it / C::kStages) & 1u, ss,
-                                                   p.dev_status);
+                ok = mbar_wait<kIssuerWait<PAIR>>(smem_u32(&ss->full[s]), (it / C::kStages) & 1u,
+                                                   ss, p.dev_status);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + size_t(s) * C::kStageBytes);
-                const uint32_t d = tmem_base + buf * C::kAccCols;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_e4m3<PAIR>(d, sw128_desc(st + kk * 32),
-                                   sw128_desc(st + kTileBytes + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                mma_commit_both<PAIR>(smem_u32(&ss->empty[s]));
-                mma_commit_both<PAIR>(smem_u32(&ss->tfull[buf]));
+                for (int c = 0; c < C::kChains; ++c, ++tb) {
+                    const uint32_t buf = tb % C::kBufs;
+                    const uint32_t tpar = (tb / C::kBufs) & 1u;
+                    ok = mbar_wait<kIssuerWait<PAIR>>(smem_u32(&ss->tempty[buf]), tpar ^ 1u, ss,
+                                                       p.dev_status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + buf * C::kBufCols;
+                    // chain c multiplies the tokens by weight block c (split
+                    // form) or by the stage's whole weight tile
+                    const uint32_t b0 = st + kTileBytes + c * kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_e4m3<PAIR>(d, sw128_desc(st + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                                       kk > 0 ? 1u : 0u);
+                    // split form: the promoters free the stage once they see
+                    // the last chain complete (one commit per chain)
+                    if (!C::kSplit) mma_commit_both<PAIR>(smem_u32(&ss->empty[s]));
+                    mma_commit_both<PAIR>(smem_u32(&ss->tfull[buf]));
+                }
             }
         }
         // all MMAs issued by this thread have completed once drain fires
+        // (also after an abort: they write TMEM, which is freed at the end)
         mma_commit<PAIR>(smem_u32(&ss->drain));
-        mbar_wait(smem_u32(&ss->drain), 0, ss, nullptr);
+        mbar_quiesce(smem_u32(&ss->drain), 0, ss, nullptr);
     }
     __syncwarp();
 }
@@ -826,6 +889,69 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
         uint64_t acc2[C::kPairs];  // fp32 accumulator pairs
 #pragma unroll
         for (int i = 0; i < C::kPairs; ++i) acc2[i] = 0;
+        if (C::kSplit) {
+            // Two 128-column buffers per K block (weight blocks 0 and 1).
+            // SwiGLU: every warp reads 64 columns of each (gate and up of its
+            // 64 features); fp32 / bf16: half h reads the 128 columns of
+            // buffer h only.
+            for (int kb = 0; ok && kb < p.nkb; ++kb, tb += 2, ++cit) {
+                const int c = cit % kScaleSlots;
+                const uint32_t bufs[2] = {tb % C::kBufs, (tb + 1) % C::kBufs};
+                const uint32_t pars[2] = {(tb / C::kBufs) & 1u, ((tb + 1) / C::kBufs) & 1u};
+                const int first = SWIGLU ? 0 : half;  // buffer read first (or only)
+                if (lane == 0) {
+                    ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->tfull[bufs[first]]),
+                                                       pars[first], ss, p.dev_status);
+                    if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (cit / kScaleSlots) & 1u, ss,
+                                           p.dev_status);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                __syncwarp();
+                tc_fence_after();
+                const float sa = ss->sa[c][r];
+                const float s0 = sa * ss->sb[c][SWIGLU ? 0 : half];
+                const float s1 = sa * ss->sb[c][SWIGLU ? 1 : half];
+                const uint64_t s0x2 = pack2(__float_as_uint(s0), __float_as_uint(s0));
+                const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
+                uint32_t v[64];
+                if (SWIGLU) {
+                    tmem_ld64(lane_addr + bufs[0] * C::kBufCols + 64 * half, v);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[bufs[0]]));
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
+                    if (lane == 0)
+                        ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->tfull[bufs[1]]), pars[1],
+                                                           ss, p.dev_status);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    __syncwarp();
+                    tc_fence_after();
+                    tmem_ld64(lane_addr + bufs[1] * C::kBufCols + 64 * half, v);
+                } else {
+                    const uint32_t tbase = lane_addr + bufs[half] * C::kBufCols;
+                    tmem_ld64(tbase, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
+                    tmem_ld64(tbase + 64, v);
+                }
+                // the partial is in registers: hand the buffer back, and (one
+                // thread that saw the K block's last chain complete) the stage
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&ss->tempty[bufs[SWIGLU ? 1 : half]]));
+                    if (warp == 8) mbar_arrive(smem_u32(&ss->empty[cit % C::kStages]));
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    ffma2(acc2[32 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
+            }
+        } else
         for (int kb = 0; ok && kb < p.nkb; ++kb, ++tb, ++cit) {
             const uint32_t buf = tb % C::kBufs;
             const int c = cit % kScaleSlots;
@@ -968,13 +1094,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < C::kBufs; ++b) {
             mbar_init(smem_u32(&ss->tfull[b]), 1);
-            mbar_init(smem_u32(&ss->tempty[b]), kPromoters * C::kCtas);
+            // split fp32 / bf16 form: a buffer is read by one half of the
+            // promotion warps
+            mbar_init(smem_u32(&ss->tempty[b]),
+                      (C::kSplit && !SWIGLU ? kPromoters / 2 : kPromoters) * C::kCtas);
         }
         for (int c = 0; c < kScaleSlots; ++c) {
             mbar_init(smem_u32(&ss->sfull[c]), 32);
             mbar_init(smem_u32(&ss->sempty[c]), kPromoters);
         }
         mbar_init(smem_u32(&ss->drain), 1);
+        ss->wait_limit = p.wait_limit_ns;
         ss->abort_flag = 0;
         ss->peer_abort = PAIR ? mapa(smem_u32(&ss->abort_flag), uint32_t(rank ^ 1)) : 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1059,6 +1189,404 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_free_all<PAIR>(tmem_base);
     }
+}
+
+// ============================================== block-scaled form (UE8M0 scales)
+// A numerically different option beside the pages' recipe: with power-of-two
+// scales (UE8M0 bytes: exponent + 127) the tensor core applies the scales
+// itself (tcgen05.mma kind::mxf8f6f4.block_scale, one scale per 32 elements
+// of K; a 1x128 tile or 128x128 block repeats its scale over four of them),
+// so a K block needs no promotion and one TMEM accumulator serves the whole
+// K loop of an item.  Roles: warp 0 TMA producer (tokens + both weight
+// blocks of the 256 columns); warp 2 builds each stage's scale chunks in
+// shared memory (128 rows x 4 scales per 512 bytes: the 32-bit word of row m
+// = 32 m1 + m0 at byte 16 m0 + 4 m1, its four bytes the scales of K
+// elements 0-31, ..., 96-127); warp 1 copies them into TMEM (tcgen05.cp
+// 32x128b.warpx4) and issues the MMAs; warps 4-11 move the finished
+// accumulator out at the end of an item and run the epilogue.
+template <bool SWIGLU>
+struct MxCfg {
+    static constexpr int kStages = SWIGLU ? 4 : 3;
+    static constexpr int kStageBytes = kTileBytes + 256 * 128;  // tokens + two weight blocks
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kSfStage = 3 * 512;                    // A chunk, two B chunks
+    static constexpr int kSfBytes = kStages * kSfStage;
+    static constexpr int kParkBoxes = SWIGLU ? 0 : 1;
+    static constexpr int kParkBytes = kPromoters * kParkBoxes * kBoxBytes;
+    static constexpr int kSfCol = 256;                          // TMEM column of stage 0's scales
+    static_assert(kStages <= kMaxStages && kStages <= kScaleSlots, "ring sizes");
+};
+template <bool SWIGLU>
+constexpr size_t mx_smem_bytes() {
+    using C = MxCfg<SWIGLU>;
+    return size_t(C::kRingBytes) + C::kParkBytes + C::kSfBytes + sizeof(SharedState) + 1024;
+}
+static_assert(mx_smem_bytes<false>() <= 232448 && mx_smem_bytes<true>() <= 232448,
+              "dynamic shared memory above the sm_100 limit per CTA");
+
+// Shared-memory descriptor of a scale chunk for tcgen05.cp: K-major without
+// swizzle, 8-row x 16-byte core matrices 128 bytes apart along the rows.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+    d |= uint64_t(128 >> 4) << 16;
+    d |= uint64_t(128 >> 4) << 32;
+    d |= uint64_t(1) << 46;
+    return d;
+}
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+// kind::mxf8f6f4 block-scaled instruction descriptor: E4M3 x E4M3, UE8M0
+// scales, fp32 D, K-major; the scale byte of each operand is selected by
+// sf_id (also carried in bits 30-31 of the scale TMEM addresses).
+__device__ __forceinline__ uint32_t idesc_mx(int m, int n, uint32_t sf_id) {
+    return (sf_id << 4) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(m >> 4) << 24) |
+           (sf_id << 29);
+}
+__device__ __forceinline__ void mma_mx(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate, uint32_t sfa, uint32_t sfb) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
+}
+
+template <bool SWIGLU>
+__device__ __forceinline__ void mx_producer(const GemmParams& p, const CUtensorMap* map_w,
+                                            const AMaps& maps_a, uint8_t* smem, SharedState* ss,
+                                            int unit, int units) {
+    using C = MxCfg<SWIGLU>;
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    uint32_t it = 0, issued_mask = 0, issued_parity = 0;
+    bool ok = true;
+    for (int item = unit; ok && item < total_items; item += units) {
+        const Item w = decode_item<kBM>(ss, p, item);
+        int b0, b1;
+        weight_blocks<false, SWIGLU, true>(p, w, b0, b1);
+        const int n0 = cta_tokens(w, 0);
+        const CUtensorMap* map_a = &maps_a.m[box_index(n0)];
+        const uint32_t tx = box_bytes(n0) + uint32_t(256 * 128);
+        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+            const int s = it % C::kStages;
+            const uint32_t par = (it / C::kStages) & 1u;
+            if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
+                uint8_t* st = smem + size_t(s) * C::kStageBytes;
+                const uint32_t fb = smem_u32(&ss->full[s]);
+                mbar_arrive_expect_tx(fb, tx);
+                if (n0 > 0) tma_load_2d<false>(smem_u32(st), map_a, fb, kb * 128, w.row0);
+                tma_load_2d<false>(smem_u32(st + kTileBytes), map_w, fb, kb * 128,
+                                   w.g * p.n + b0 * 128);
+                tma_load_2d<false>(smem_u32(st + 2 * kTileBytes), map_w, fb, kb * 128,
+                                   w.g * p.n + b1 * 128);
+                issued_mask |= 1u << s;
+                issued_parity = (issued_parity & ~(1u << s)) | (par << s);
+            }
+        }
+    }
+    if (!ok && lane == 0)
+        for (int s = 0; s < C::kStages; ++s)
+            if ((issued_mask >> s) & 1u)
+                mbar_quiesce(smem_u32(&ss->full[s]), (issued_parity >> s) & 1u, ss, nullptr);
+    __syncwarp();
+}
+
+// warp 2: the stage's scale chunks (tokens, weight block 0, weight block 1)
+template <bool SWIGLU>
+__device__ __forceinline__ void mx_scale_loader(const GemmParams& p, uint8_t* sf_area,
+                                                SharedState* ss, int unit, int units) {
+    using C = MxCfg<SWIGLU>;
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    const int nbr = p.n / 128;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int item = unit; ok && item < total_items; item += units) {
+        const Item w = decode_item<kBM>(ss, p, item);
+        int b0, b1;
+        weight_blocks<false, SWIGLU, true>(p, w, b0, b1);
+        const int my_n = cta_tokens(w, 0);
+        const uint8_t* wsf0 = p.w_sf + (size_t(w.g) * nbr + b0) * p.nkb;
+        const uint8_t* wsf1 = p.w_sf + (size_t(w.g) * nbr + b1) * p.nkb;
+        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+            const int s = it % C::kStages;
+            const uint32_t par = (it / C::kStages) & 1u;
+            if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const uint8_t* asf = p.a_sf + size_t(kb) * p.max_rows + w.row0;
+            uint32_t wd[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int m = lane + 32 * j;  // row m0 = lane, m1 = j
+                const uint32_t b = m < my_n ? asf[m] : 127u;
+                wd[j] = b * 0x01010101u;
+            }
+            uint8_t* ch = sf_area + s * C::kSfStage;
+            *reinterpret_cast<uint4*>(ch + 16 * lane) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            const uint32_t w0 = uint32_t(wsf0[kb]) * 0x01010101u;
+            const uint32_t w1 = uint32_t(wsf1[kb]) * 0x01010101u;
+            *reinterpret_cast<uint4*>(ch + 512 + 16 * lane) = make_uint4(w0, w0, w0, w0);
+            *reinterpret_cast<uint4*>(ch + 1024 + 16 * lane) = make_uint4(w1, w1, w1, w1);
+            // visible to the tensor core's copy (async proxy) before the signal
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ss->sfull[s]));
+        }
+    }
+    __syncwarp();
+}
+
+// warp 1, one thread
+template <bool SWIGLU>
+__device__ __forceinline__ void mx_mma_issuer(const GemmParams& p, uint8_t* smem, uint8_t* sf_area,
+                                              SharedState* ss, uint32_t tmem_base, int unit,
+                                              int units) {
+    using C = MxCfg<SWIGLU>;
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    if (lane == 0) {
+        uint32_t it = 0, n_item = 0;
+        bool ok = true;
+        for (int item = unit; ok && item < total_items; item += units, ++n_item) {
+            // the epilogue has moved the previous item's accumulator out
+            ok = mbar_wait(smem_u32(&ss->tempty[0]), (n_item & 1u) ^ 1u, ss, p.dev_status);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+                const int s = it % C::kStages;
+                const uint32_t par = (it / C::kStages) & 1u;
+                ok = mbar_wait(smem_u32(&ss->full[s]), par, ss, p.dev_status) &&
+                     mbar_wait(smem_u32(&ss->sfull[s]), par, ss, p.dev_status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t ta = tmem_base + C::kSfCol + 12 * s, tb = ta + 4;
+                const uint32_t ch = smem_u32(sf_area + s * C::kSfStage);
+                tmem_cp_sf(ta, sf_desc(ch));
+                tmem_cp_sf(tb, sf_desc(ch + 512));
+                tmem_cp_sf(tb + 4, sf_desc(ch + 1024));
+                const uint32_t st = smem_u32(smem + size_t(s) * C::kStageBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_mx(tmem_base, sw128_desc(st + kk * 32), sw128_desc(st + kTileBytes + kk * 32),
+                           idesc_mx(128, 256, uint32_t(kk)), (kb > 0 || kk > 0) ? 1u : 0u,
+                           ta | (uint32_t(kk) << 30), tb | (uint32_t(kk) << 30));
+                mma_commit<false>(smem_u32(&ss->empty[s]));
+            }
+            if (!ok) break;
+            mma_commit<false>(smem_u32(&ss->tfull[0]));
+        }
+        mma_commit<false>(smem_u32(&ss->drain));
+        mbar_quiesce(smem_u32(&ss->drain), 0, ss, nullptr);
+    }
+    __syncwarp();
+}
+
+// warps 4-11: thread (w, l) owns token row 32 (w % 4) + l and half h = (w-4)/4
+// of the 256 columns (same mapping as the promotion form's epilogue).
+template <bool SWIGLU>
+__device__ __forceinline__ void mx_epilogue(const GemmParams& p, SharedState* ss, char* park_area,
+                                            uint32_t tmem_base, const CUtensorMap* map_o, int unit,
+                                            int units) {
+    using C = MxCfg<SWIGLU>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int r = q * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (uint32_t(q * 32) << 16);
+    const int c0 = SWIGLU ? 64 * half : 128 * half;
+    const int c1 = SWIGLU ? 128 + 64 * half : 128 * half + 64;
+    char* const wpark = park_area + (warp - 4) * (C::kParkBoxes * kBoxBytes);
+    uint32_t n_item = 0, parity = 0;
+    bool ok = true;
+    for (int item = unit; item < total_items; item += units, ++n_item, parity ^= 1u) {
+        const Item w = decode_item<kBM>(ss, p, item);
+        if (lane == 0) ok = mbar_wait(smem_u32(&ss->tfull[0]), n_item & 1u, ss, p.dev_status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        uint64_t acc2[64];
+        if (ok) {
+            __syncwarp();
+            tc_fence_after();
+            uint32_t v[64];
+            tmem_ld64(lane_addr + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc2[i] = pack2(v[2 * i], v[2 * i + 1]);
+            tmem_ld64(lane_addr + c1, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc2[32 + i] = pack2(v[2 * i], v[2 * i + 1]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[0]));  // accumulator free
+        } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc2[i] = 0;
+        }
+        const int my_n = cta_tokens(w, 0);
+        const size_t row = size_t(w.row0) + r;
+        if (!SWIGLU) {
+            store_rows<64, 1>(p, acc2, wpark, map_o, lane, my_n - q * 32, row, w.row0 + q * 32,
+                              w.f * 256 + half * 128);
+        } else {
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float2 f = unpack2(acc2[i]);
+                acc[2 * i] = f.x;
+                acc[2 * i + 1] = f.y;
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float g = acc[i];
+                const float hv = __fdividef(g, 1.0f + __expf(-g)) * acc[64 + i];
+                acc[i] = hv;
+                amax = fmaxf(amax, fabsf(hv));
+            }
+            ss->red[parity][half][r] = amax;
+            named_bar(1, kPromoters * 32);
+            amax = fmaxf(amax, ss->red[parity][half ^ 1][r]);
+            const int e = pow2_exponent(amax);
+            const float inv = pow2_inverse(e);
+            if (r < my_n) {
+                uint4* o = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + row * (p.n / 2) +
+                                                    size_t(w.f) * 128 + half * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int b = 16 * i + 4 * j;
+                        const uint32_t lo = e4m3x2(__fmul_rn(acc[b], inv), __fmul_rn(acc[b + 1], inv));
+                        const uint32_t hi = e4m3x2(__fmul_rn(acc[b + 2], inv), __fmul_rn(acc[b + 3], inv));
+                        u[j] = lo | (hi << 16);
+                    }
+                    o[i] = make_uint4(u[0], u[1], u[2], u[3]);
+                }
+                if (half == 0) p.out_sf[size_t(w.f) * p.max_rows + row] = uint8_t(e + 127);
+            }
+        }
+        const bool any_abort = named_bar_or(
+            2, kPromoters * 32, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
+        if (any_abort) break;
+    }
+    if (!SWIGLU && lane == 0) bulk_wait_all();
+    __syncwarp();
+    tc_fence_before();
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ AMaps maps_a,
+                   const __grid_constant__ CUtensorMap map_o, const GemmParams p) {
+    using C = MxCfg<SWIGLU>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    char* park = reinterpret_cast<char*>(smem + C::kRingBytes);
+    uint8_t* sf_area = smem + C::kRingBytes + C::kParkBytes;
+    SharedState* ss = reinterpret_cast<SharedState*>(sf_area + C::kSfBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int unit = int(blockIdx.x), units = int(gridDim.x);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&ss->full[s]), 1);
+            mbar_init(smem_u32(&ss->empty[s]), 1);
+            mbar_init(smem_u32(&ss->sfull[s]), 1);
+        }
+        mbar_init(smem_u32(&ss->tfull[0]), 1);
+        mbar_init(smem_u32(&ss->tempty[0]), kPromoters);
+        mbar_init(smem_u32(&ss->drain), 1);
+        ss->wait_limit = p.wait_limit_ns;
+        ss->abort_flag = 0;
+        ss->peer_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc_all<false>(smem_u32(&ss->tmem_base));
+    const int G = p.n_groups;
+    int bad = 0;
+    for (int i = threadIdx.x; i <= G; i += kThreads) {
+        const int v = p.group_offsets[i];
+        ss->goff[i] = v;
+        if (v < 0 || v > p.max_rows || (i > 0 && v < p.group_offsets[i - 1])) bad = 1;
+    }
+    if (__syncthreads_or(bad)) {
+        if (threadIdx.x == 0) set_status(p.dev_status, MOE_DEV_BAD_INPUT);
+        for (int i = threadIdx.x; i <= G; i += kThreads) ss->goff[i] = 0;
+        __syncthreads();
+    }
+    {
+        constexpr int PER = (kMaxGroups + kThreads) / kThreads;
+        int vals[PER];
+        int sum = 0;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int g = threadIdx.x * PER + j;
+            int v = 0;
+            if (g < G) {
+                const int rows = ss->goff[g + 1] - ss->goff[g];
+                v = ((rows + kBM - 1) / kBM) * p.n_ftiles;
+            }
+            vals[j] = v;
+            sum += v;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        __shared__ int wsum[kThreads / 32];
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            if (w < warp) before += wsum[w];
+            total += wsum[w];
+        }
+        int run = before + incl - sum;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int g = threadIdx.x * PER + j;
+            if (g <= G) ss->gstart[g] = run;
+            run += vals[j];
+        }
+        if (threadIdx.x == 0) ss->total_items = total;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ss->tmem_base;
+    if (warp < 4) {
+        set_max_regs_dec<72>();
+        if (warp == 0) mx_producer<SWIGLU>(p, &map_w, maps_a, smem, ss, unit, units);
+        else if (warp == 1) mx_mma_issuer<SWIGLU>(p, smem, sf_area, ss, tmem_base, unit, units);
+        else if (warp == 2) mx_scale_loader<SWIGLU>(p, sf_area, ss, unit, units);
+    } else {
+        set_max_regs_inc<208>();
+        mx_epilogue<SWIGLU>(p, ss, park, tmem_base, &map_o, unit, units);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_free_all<false>(tmem_base);
+    }
+}
+
+template <bool SWIGLU>
+int launch_mx(const GemmParams& p, const CUtensorMap& mw, const AMaps& ma, const CUtensorMap& mo,
+              cudaStream_t st) {
+    if (cudaFuncSetAttribute(mx_gemm_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(mx_smem_bytes<SWIGLU>())) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    mx_gemm_kernel<SWIGLU><<<sm_count(), kThreads, mx_smem_bytes<SWIGLU>(), st>>>(mw, ma, mo, p);
+    return check_launch();
 }
 
 // CTA pairs the device can hold at once for a pair kernel (cached per device).
@@ -1215,12 +1743,39 @@ extern "C" MOE_API int moe_grouped_gemm_form(int n_groups, int max_rows, int n, 
     return gemm_pair_units(n_groups, max_rows, n, epilogue == MOE_EPI_SWIGLU_QUANT) > 0 ? 2 : 1;
 }
 
+namespace moe {
+int grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int max_rows, const uint8_t* a,
+                     const float* a_scales, int k, const uint8_t* w, const float* w_scales, int n,
+                     int epilogue, void* out, float* out_scales, const int32_t* group_weight,
+                     int n_weights, int* dev_status, void* stream);
+}
+
 extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_offsets,
                                             int max_rows, const uint8_t* a,
                                             const float* a_scales, int k, const uint8_t* w,
                                             const float* w_scales, int n, int epilogue,
                                             void* out, float* out_scales, int* dev_status,
                                             void* stream) {
+    return grouped_gemm_fp8(n_groups, group_offsets, max_rows, a, a_scales, k, w, w_scales, n,
+                            epilogue, out, out_scales, nullptr, n_groups, dev_status, stream);
+}
+
+extern "C" MOE_API int moe_grouped_gemm_fp8_indexed(
+    int n_groups, const int32_t* group_offsets, const int32_t* group_weight, int n_weights,
+    int max_rows, const uint8_t* a, const float* a_scales, int k, const uint8_t* w,
+    const float* w_scales, int n, int epilogue, void* out, float* out_scales, int* dev_status,
+    void* stream) {
+    if (!group_weight) return MOE_ERR_NULL;
+    if (n_weights < 1) return MOE_ERR_SHAPE;
+    return grouped_gemm_fp8(n_groups, group_offsets, max_rows, a, a_scales, k, w, w_scales, n,
+                            epilogue, out, out_scales, group_weight, n_weights, dev_status, stream);
+}
+
+int moe::grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int max_rows,
+                          const uint8_t* a, const float* a_scales, int k, const uint8_t* w,
+                          const float* w_scales, int n, int epilogue, void* out,
+                          float* out_scales, const int32_t* group_weight, int n_weights,
+                          int* dev_status, void* stream) {
     if (n_groups < 1 || n_groups > kMaxGroups || max_rows < 0 || k <= 0 || k % 128 || n <= 0 ||
         n % 128)
         return MOE_ERR_SHAPE;
@@ -1232,7 +1787,7 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     if (max_rows == 0) return MOE_OK;
     if (!a || !a_scales) return MOE_ERR_NULL;
     if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MOE_ERR_ALIGN;
-    if (int64_t(n_groups) * n > INT32_MAX) return MOE_ERR_SHAPE;
+    if (int64_t(n_weights) * n > INT32_MAX) return MOE_ERR_SHAPE;
     if (!device_is_sm100()) return MOE_ERR_DEVICE;
 
     const bool swiglu = epilogue == MOE_EPI_SWIGLU_QUANT;
@@ -1256,10 +1811,14 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     p.out = out;
     p.out_scales = out_scales;
     p.dev_status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+    p.fault = fault_injection();
+    p.group_weight = group_weight;
+    p.n_weights = n_weights;
 
     CUtensorMap mw, mo;
     AMaps ma;
-    if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128)) return MOE_ERR_CUDA;
+    if (!make_map(&mw, w, uint64_t(n_weights) * n, uint64_t(k), 128)) return MOE_ERR_CUDA;
     for (int i = 0; i < kABoxes; ++i)
         if (!make_map(&ma.m[i], a, uint64_t(max_rows), uint64_t(k), uint32_t(128 >> i)))
             return MOE_ERR_CUDA;
@@ -1273,4 +1832,53 @@ extern "C" MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_o
     if (swiglu) return launch<false, true, true>(p, mw, ma, mo, 0, st);
     return wide ? launch<false, false, true>(p, mw, ma, mo, 0, st)
                 : launch<false, false, false>(p, mw, ma, mo, 0, st);
+}
+
+extern "C" MOE_API int moe_grouped_gemm_mxfp8(int n_groups, const int32_t* group_offsets,
+                                              int max_rows, const uint8_t* a, const uint8_t* a_sf,
+                                              int k, const uint8_t* w, const uint8_t* w_sf, int n,
+                                              int epilogue, void* out, uint8_t* out_sf,
+                                              int* dev_status, void* stream) {
+    if (n_groups < 1 || n_groups > kMaxGroups || max_rows < 0 || k <= 0 || k % 128 || n <= 0 ||
+        n % 256)
+        return MOE_ERR_SHAPE;
+    if (epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_SWIGLU_QUANT)
+        return MOE_ERR_ARG;
+    if (!group_offsets || !w || !w_sf || !out) return MOE_ERR_NULL;
+    if (epilogue == MOE_EPI_SWIGLU_QUANT && !out_sf) return MOE_ERR_NULL;
+    if (max_rows == 0) return MOE_OK;
+    if (!a || !a_sf) return MOE_ERR_NULL;
+    if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MOE_ERR_ALIGN;
+    if (int64_t(n_groups) * n > INT32_MAX) return MOE_ERR_SHAPE;
+    if (!device_is_sm100()) return MOE_ERR_DEVICE;
+    const bool swiglu = epilogue == MOE_EPI_SWIGLU_QUANT;
+    GemmParams p = {};
+    p.group_offsets = group_offsets;
+    p.n_groups = n_groups;
+    p.max_rows = max_rows;
+    p.k = k;
+    p.nkb = k / 128;
+    p.n = n;
+    p.n_ftiles = n / 256;
+    p.epilogue = epilogue;
+    p.out = out;
+    p.dev_status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+    p.fault = kFaultNone;
+    p.a_sf = a_sf;
+    p.w_sf = w_sf;
+    p.out_sf = out_sf;
+    p.group_weight = nullptr;
+    p.n_weights = n_groups;
+    CUtensorMap mw, mo;
+    AMaps ma;
+    if (!make_map(&mw, w, uint64_t(n_groups) * n, uint64_t(k), 128)) return MOE_ERR_CUDA;
+    for (int i = 0; i < kABoxes; ++i)
+        if (!make_map(&ma.m[i], a, uint64_t(max_rows), uint64_t(k), uint32_t(128 >> i)))
+            return MOE_ERR_CUDA;
+    if (swiglu) mo = mw;  // unused by the SwiGLU epilogue
+    else if (!make_out_map(&mo, out, uint64_t(max_rows), uint64_t(n), epilogue == MOE_EPI_BF16))
+        return MOE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    return swiglu ? launch_mx<true>(p, mw, ma, mo, st) : launch_mx<false>(p, mw, ma, mo, st);
 }

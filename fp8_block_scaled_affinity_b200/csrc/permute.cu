@@ -190,16 +190,23 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(
     }
 }
 
-// moe_quant_permute's copy: a work unit is one 2,048-value piece of a
-// token's bf16 row (a warp, 16-byte loads, kPiece per lane in flight), so a
-// small batch still spreads over every SM.  The warp quantises each 1x128
+// moe_quant_permute's copy: a work unit is one piece of 2P tiles (P = 7 or
+// 8, up to 2,048 values) of a token's bf16 row (a warp, 16-byte loads, P per
+// lane in flight), so a small batch still spreads over every SM.  The warp quantises each 1x128
 // tile of the piece exactly as fp8_quant_act_1x128 does (a half-warp owns
 // one tile: amax by shuffles, scale rule of quant.cu, RN products, satfinite
 // E4M3) and writes the codes and the scale K+1 times (routed rows and the
 // shared row).
+// P: 16-byte vectors per lane per piece (a piece is 2P tiles of 128 values);
+// the launch picks P so that the pieces tile a row exactly when it can.
+// POW2: power-of-two scales, written as UE8M0 bytes to xsf_perm instead of
+// fp32 scales to xs_perm (the block-scaled GEMM's operand layout).
+template <int P, bool POW2>
 __global__ void __launch_bounds__(256) quant_copy_rows_kernel(
     const uint4* __restrict__ x, int T, int d, int K, const int32_t* __restrict__ row_of_pair,
-    int64_t rows_total, uint2* __restrict__ xq_perm, float* __restrict__ xs_perm) {
+    int64_t rows_total, uint2* __restrict__ xq_perm, float* __restrict__ xs_perm,
+    uint8_t* __restrict__ xsf_perm) {
+    constexpr int kPiece = P;
     const int lane = threadIdx.x & 31;
     const int nvec = d / 8, nkb = d / 128;  // 8 bf16 in, 8 codes out per vector
     const int pieces = (nvec + 32 * kPiece - 1) / (32 * kPiece);
@@ -221,7 +228,7 @@ __global__ void __launch_bounds__(256) quant_copy_rows_kernel(
                 v[j] = c < nvec ? __ldcs(src + c) : make_uint4(0u, 0u, 0u, 0u);
             }
             uint2 code[kPiece];
-            float tile_scale = 1.0f;  // lane L < 16: scale of tile c0/16 + L
+            float tile_scale = 1.0f;  // lane L < 2P: scale of tile c0/16 + L
 #pragma unroll
             for (int j = 0; j < kPiece; ++j) {
                 const uint4 w = v[j];
@@ -234,7 +241,13 @@ __global__ void __launch_bounds__(256) quant_copy_rows_kernel(
                 for (int o = 8; o >= 1; o >>= 1)
                     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 float scale, inv;
-                scale_from_amax(amax, scale, inv);
+                if (POW2) {
+                    const int e = pow2_exponent(amax);
+                    inv = pow2_inverse(e);
+                    scale = __int_as_float(e + 127);  // carries the byte, not a value
+                } else {
+                    scale_from_amax(amax, scale, inv);
+                }
                 const uint32_t c0_ = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv));
                 const uint32_t c1_ = e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
                 const uint32_t c2_ = e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv));
@@ -254,7 +267,11 @@ __global__ void __launch_bounds__(256) quant_copy_rows_kernel(
                     const int c = c0 + lane + 32 * j;
                     if (c < nvec) dst[c] = code[j];
                 }
-                if (lane < 16 && tile < nkb) xs_perm[int64_t(tile) * rows_total + row] = tile_scale;
+                if (lane < 2 * kPiece && tile < nkb) {
+                    if (POW2) xsf_perm[int64_t(tile) * rows_total + row] =
+                        uint8_t(__float_as_int(tile_scale));
+                    else xs_perm[int64_t(tile) * rows_total + row] = tile_scale;
+                }
             }
         }
     }
@@ -383,6 +400,35 @@ int build_rows(const MoeShape* shape, const int32_t* topk_idx, const int32_t* ex
     return check_launch();
 }
 
+// quantise + copy pass of moe_quant_permute (xsf_perm != NULL: power-of-two
+// scales as UE8M0 bytes).  Pieces of 2P tiles: P = 7 cuts a 56-tile row
+// (d = 7168) into four full pieces; otherwise 8, the last piece of a row
+// possibly ragged.
+int launch_quant_copy(const uint16_t* x, int T, int d, int K, const int32_t* row_of_pair,
+                      uint8_t* xq_perm, float* xs_perm, uint8_t* xsf_perm, cudaStream_t st) {
+    const int nkb = d / 128;
+    const int P = (nkb % 14 == 0 && nkb % 16 != 0) ? 7 : 8;
+    const int64_t pieces = (d / 8 + 32 * P - 1) / (32 * P);
+    const int64_t units = int64_t(T) * pieces;  // one warp each, 8 per block
+    const int qblocks = int(std::min<int64_t>((units + 7) / 8, int64_t(sm_count()) * 8));
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    uint2* qv = reinterpret_cast<uint2*>(xq_perm);
+    const int64_t rows = int64_t(T) * K + T;
+    if (P == 7 && xsf_perm)
+        quant_copy_rows_kernel<7, true><<<qblocks, 256, 0, st>>>(xv, T, d, K, row_of_pair, rows,
+                                                                 qv, xs_perm, xsf_perm);
+    else if (P == 7)
+        quant_copy_rows_kernel<7, false><<<qblocks, 256, 0, st>>>(xv, T, d, K, row_of_pair, rows,
+                                                                  qv, xs_perm, xsf_perm);
+    else if (xsf_perm)
+        quant_copy_rows_kernel<8, true><<<qblocks, 256, 0, st>>>(xv, T, d, K, row_of_pair, rows,
+                                                                 qv, xs_perm, xsf_perm);
+    else
+        quant_copy_rows_kernel<8, false><<<qblocks, 256, 0, st>>>(xv, T, d, K, row_of_pair, rows,
+                                                                  qv, xs_perm, xsf_perm);
+    return check_launch();
+}
+
 int copy_grid(int T) {
     int blocks = (T + 7) / 8;
     const int cap = sm_count() * 8;
@@ -435,13 +481,29 @@ extern "C" MOE_API int moe_quant_permute(const MoeShape* shape, const uint16_t* 
     rc = build_rows(shape, topk_idx, expert_counts, expert_offsets, row_of_pair,
                     static_cast<int32_t*>(ws), dev_status, st);
     if (rc != MOE_OK || T == 0) return rc;
-    const int64_t pieces = (d / 8 + 32 * kPiece - 1) / (32 * kPiece);
-    const int64_t units = int64_t(T) * pieces;  // one warp each, 8 per block
-    const int qblocks = int(std::min<int64_t>((units + 7) / 8, int64_t(sm_count()) * 8));
-    quant_copy_rows_kernel<<<qblocks, 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(x), T, d, K, row_of_pair, int64_t(T) * K + T,
-        reinterpret_cast<uint2*>(xq_perm), xs_perm);
-    return check_launch();
+    return launch_quant_copy(x, T, d, K, row_of_pair, xq_perm, xs_perm, nullptr, st);
+}
+
+extern "C" MOE_API int moe_quant_permute_ue8m0(const MoeShape* shape, const uint16_t* x,
+                                               const int32_t* topk_idx,
+                                               const int32_t* expert_counts, uint8_t* xq_perm,
+                                               uint8_t* xsf_perm, int32_t* expert_offsets,
+                                               int32_t* row_of_pair, void* ws, size_t ws_bytes,
+                                               int* dev_status, void* stream) {
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T, d = shape->d, K = shape->topk;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_NULL;
+    if (T > 0) {
+        if (!topk_idx || !x || !xq_perm || !xsf_perm || !row_of_pair) return MOE_ERR_NULL;
+        if (!aligned16(x) || !aligned16(xq_perm)) return MOE_ERR_ALIGN;
+        if (!ws || ws_bytes < moe_permute_workspace_size(shape)) return MOE_ERR_WORKSPACE;
+    }
+    cudaStream_t st = as_stream(stream);
+    rc = build_rows(shape, topk_idx, expert_counts, expert_offsets, row_of_pair,
+                    static_cast<int32_t*>(ws), dev_status, st);
+    if (rc != MOE_OK || T == 0) return rc;
+    return launch_quant_copy(x, T, d, K, row_of_pair, xq_perm, nullptr, xsf_perm, st);
 }
 
 extern "C" MOE_API int moe_combine(const MoeShape* shape, const float* expert_out,
@@ -495,18 +557,51 @@ constexpr int64_t kStaticChunkEntries = 262144;  // int32 entries = 1 MiB
 // + 64 entries: moe_permute asks for 256 bytes of headroom on top of the counts
 __device__ __align__(256) int32_t g_permute_scratch[kStaticChunkEntries + 64];
 
-// Device address of g_permute_scratch, looked up once per device.  In host
-// code the symbol only names a host-side stand-in, never a device address.
+// Unique id of the calling thread's current CUDA context (cuCtxGetId through
+// the runtime's driver entry points), or 0 when there is none or the driver
+// cannot tell.
+unsigned long long current_context_id() {
+    typedef int (*GetCurrentFn)(void**);
+    typedef int (*GetIdFn)(void*, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(f);
+    });
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0)
+        return 0;
+    return id;
+}
+
+// Device address of g_permute_scratch in the current device's context.  In
+// host code the symbol only names a host-side stand-in, never a device
+// address.  The address is looked up once per device and context: a device
+// reset ends the context it belongs to, and the next call, seeing a new
+// context id, looks it up again.
 int32_t* static_scratch_ptr() {
     static std::mutex mu;
     static int32_t* ptrs[64] = {nullptr};
+    static unsigned long long ctx_ids[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev]) {
+    const unsigned long long id = current_context_id();
+    if (!ptrs[dev] || id == 0 || id != ctx_ids[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
         ptrs[dev] = static_cast<int32_t*>(p);
+        ctx_ids[dev] = current_context_id();  // the lookup made the context current
     }
     return ptrs[dev];
 }

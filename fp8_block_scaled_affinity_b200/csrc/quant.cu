@@ -14,9 +14,11 @@ namespace {
 // loads in flight.  Grid-strides over tiles.
 constexpr int kActUnroll = 4;
 
+// POW2: power-of-two scales written as UE8M0 bytes to sf (scales unused).
+template <bool POW2>
 __global__ void __launch_bounds__(256) quant_act_1x128_kernel(
     const uint4* __restrict__ x, int64_t rows, int64_t cols, uint2* __restrict__ q,
-    float* __restrict__ scales, int kb_major) {
+    float* __restrict__ scales, uint8_t* __restrict__ sf, int kb_major) {
     const int64_t tiles_per_row = cols >> 7;
     const int64_t n_tiles = rows * tiles_per_row;
     const int sub = threadIdx.x & 15;
@@ -48,7 +50,14 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(
             for (int o = 8; o >= 1; o >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             float scale, inv;
-            scale_from_amax(amax, scale, inv);
+            int e = 0;
+            if (POW2) {
+                e = pow2_exponent(amax);
+                inv = pow2_inverse(e);
+                scale = 0.0f;
+            } else {
+                scale_from_amax(amax, scale, inv);
+            }
             uint32_t c0 = e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv));
             uint32_t c1 = e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv));
             uint32_t c2 = e4m3x2(__fmul_rn(v[4], inv), __fmul_rn(v[5], inv));
@@ -56,8 +65,9 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(
             if (r[u] < 0) continue;
             q[vec[u]] = make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
             if (sub == 0) {
-                if (kb_major) scales[t[u] * rows + r[u]] = scale;
-                else scales[r[u] * tiles_per_row + t[u]] = scale;
+                const int64_t at = kb_major ? t[u] * rows + r[u] : r[u] * tiles_per_row + t[u];
+                if (POW2) sf[at] = uint8_t(e + 127);
+                else scales[at] = scale;
             }
         }
     }
@@ -69,9 +79,10 @@ __global__ void __launch_bounds__(256) quant_act_1x128_kernel(
 // block is reduced and stored, so every thread keeps its loads in flight.
 constexpr int kWThreads = 512;
 
+template <bool POW2>
 __global__ void __launch_bounds__(kWThreads) quant_w_128x128_kernel(
     const uint4* __restrict__ w, int64_t rows, int64_t cols, uint4* __restrict__ q,
-    float* __restrict__ scales) {
+    float* __restrict__ scales, uint8_t* __restrict__ sf) {
     constexpr int kWarps = kWThreads / 32;
     __shared__ float warp_max[2][kWarps];
     const int64_t bc = cols >> 7;
@@ -118,7 +129,14 @@ __global__ void __launch_bounds__(kWThreads) quant_w_128x128_kernel(
 #pragma unroll
         for (int i = 1; i < kWarps; ++i) amax = fmaxf(amax, wm[i]);
         float scale, inv;
-        scale_from_amax(amax, scale, inv);
+        int e = 0;
+        if (POW2) {
+            e = pow2_exponent(amax);
+            inv = pow2_inverse(e);
+            scale = 0.0f;
+        } else {
+            scale_from_amax(amax, scale, inv);
+        }
         const int64_t bi = b / bc, bj = b - bi * bc;
         const int64_t qbase = ((bi * 128 + row) * cols + bj * 128 + quarter * 32) / 16;
 #pragma unroll
@@ -136,7 +154,10 @@ __global__ void __launch_bounds__(kWThreads) quant_w_128x128_kernel(
             }
             __stcs(q + qbase + i, make_uint4(o[0], o[1], o[2], o[3]));
         }
-        if (threadIdx.x == 0) scales[b] = scale;
+        if (threadIdx.x == 0) {
+            if (POW2) sf[b] = uint8_t(e + 127);
+            else scales[b] = scale;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[i] = nv[i];
     }
@@ -146,6 +167,44 @@ __global__ void __launch_bounds__(kWThreads) quant_w_128x128_kernel(
 }  // namespace moe
 
 using namespace moe;
+
+namespace moe {
+namespace {
+
+int launch_act(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+               uint8_t* sf, int kb_major, void* stream) {
+    const int64_t threads = rows * (cols / 128) * 16;
+    int64_t blocks = (threads + 256 * kActUnroll - 1) / (256 * kActUnroll);
+    const int64_t cap = int64_t(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (sf)
+        quant_act_1x128_kernel<true><<<unsigned(blocks), 256, 0, as_stream(stream)>>>(
+            reinterpret_cast<const uint4*>(x), rows, cols, reinterpret_cast<uint2*>(q), scales, sf,
+            kb_major);
+    else
+        quant_act_1x128_kernel<false><<<unsigned(blocks), 256, 0, as_stream(stream)>>>(
+            reinterpret_cast<const uint4*>(x), rows, cols, reinterpret_cast<uint2*>(q), scales, sf,
+            kb_major);
+    return check_launch();
+}
+
+int launch_w(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+             uint8_t* sf, void* stream) {
+    const int64_t n_blocks = (rows / 128) * (cols / 128);
+    int64_t grid = n_blocks;
+    const int64_t cap = int64_t(sm_count()) * 4;  // 4 CTAs of 512 threads per SM
+    if (grid > cap) grid = cap;
+    if (sf)
+        quant_w_128x128_kernel<true><<<unsigned(grid), kWThreads, 0, as_stream(stream)>>>(
+            reinterpret_cast<const uint4*>(w), rows, cols, reinterpret_cast<uint4*>(q), scales, sf);
+    else
+        quant_w_128x128_kernel<false><<<unsigned(grid), kWThreads, 0, as_stream(stream)>>>(
+            reinterpret_cast<const uint4*>(w), rows, cols, reinterpret_cast<uint4*>(q), scales, sf);
+    return check_launch();
+}
+
+}  // namespace
+}  // namespace moe
 
 extern "C" MOE_API int fp8_quant_act_1x128(const uint16_t* x, int64_t rows, int64_t cols,
                                            uint8_t* q, float* scales, int scales_kb_major,
@@ -157,14 +216,7 @@ extern "C" MOE_API int fp8_quant_act_1x128(const uint16_t* x, int64_t rows, int6
     if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
         return MOE_ERR_ALIGN;
     if (scales_kb_major != 0 && scales_kb_major != 1) return MOE_ERR_ARG;
-    const int64_t threads = rows * (cols / 128) * 16;
-    int64_t blocks = (threads + 256 * kActUnroll - 1) / (256 * kActUnroll);
-    const int64_t cap = int64_t(sm_count()) * 8;
-    if (blocks > cap) blocks = cap;
-    quant_act_1x128_kernel<<<unsigned(blocks), 256, 0, as_stream(stream)>>>(
-        reinterpret_cast<const uint4*>(x), rows, cols, reinterpret_cast<uint2*>(q), scales,
-        scales_kb_major);
-    return check_launch();
+    return launch_act(x, rows, cols, q, scales, nullptr, scales_kb_major, stream);
 }
 
 extern "C" MOE_API int fp8_quant_w_128x128(const uint16_t* w, int64_t rows, int64_t cols,
@@ -176,11 +228,28 @@ extern "C" MOE_API int fp8_quant_w_128x128(const uint16_t* w, int64_t rows, int6
     if (!w || !q || !scales) return MOE_ERR_NULL;
     if (!aligned16(w) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3))
         return MOE_ERR_ALIGN;
-    const int64_t n_blocks = (rows / 128) * (cols / 128);
-    int64_t grid = n_blocks;
-    const int64_t cap = int64_t(sm_count()) * 4;  // 4 CTAs of 512 threads per SM
-    if (grid > cap) grid = cap;
-    quant_w_128x128_kernel<<<unsigned(grid), kWThreads, 0, as_stream(stream)>>>(
-        reinterpret_cast<const uint4*>(w), rows, cols, reinterpret_cast<uint4*>(q), scales);
-    return check_launch();
+    return launch_w(w, rows, cols, q, scales, nullptr, stream);
+}
+
+extern "C" MOE_API int fp8_quant_act_1x128_ue8m0(const uint16_t* x, int64_t rows, int64_t cols,
+                                                 uint8_t* q, uint8_t* sf, int sf_kb_major,
+                                                 int* dev_status, void* stream) {
+    (void)dev_status;
+    if (rows < 0 || cols < 0 || cols % 128) return MOE_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!x || !q || !sf) return MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q)) return MOE_ERR_ALIGN;
+    if (sf_kb_major != 0 && sf_kb_major != 1) return MOE_ERR_ARG;
+    return launch_act(x, rows, cols, q, nullptr, sf, sf_kb_major, stream);
+}
+
+extern "C" MOE_API int fp8_quant_w_128x128_ue8m0(const uint16_t* w, int64_t rows, int64_t cols,
+                                                 uint8_t* q, uint8_t* sf, int* dev_status,
+                                                 void* stream) {
+    (void)dev_status;
+    if (rows < 0 || cols < 0 || rows % 128 || cols % 128) return MOE_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!w || !q || !sf) return MOE_ERR_NULL;
+    if (!aligned16(w) || !aligned16(q)) return MOE_ERR_ALIGN;
+    return launch_w(w, rows, cols, q, nullptr, sf, stream);
 }

@@ -224,7 +224,8 @@ constexpr size_t kImmaSmem = size_t(kIStages) * kIStageBytes + 1024 + sizeof(Imm
 
 __global__ void __launch_bounds__(128, 1) route_imma_kernel(
     const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_e, int T,
-    int N, int nchunks, int chunks_per_split, int32_t* __restrict__ acc, int* dev_status) {
+    int N, int nchunks, int chunks_per_split, int32_t* __restrict__ acc, int* dev_status,
+    uint64_t wait_ns) {
     extern __shared__ __align__(1024) uint8_t imma_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(imma_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(128, 1) route_imma_kernel(
             const int st = issued % kIStages;
             if (issued >= kIStages &&
                 !tc::mbar_wait(tc::smem_u32(&ss->empty[st]), ((issued / kIStages) - 1) & 1,
-                               &ss->abort, dev_status))
+                               &ss->abort, dev_status, wait_ns))
                 break;
             const uint32_t bar = tc::smem_u32(&ss->full[st]);
             tc::mbar_arrive_expect_tx(bar, kIStageBytes);
@@ -273,16 +274,17 @@ __global__ void __launch_bounds__(128, 1) route_imma_kernel(
                                 c * kIK, r * N + e0);
         }
         // the copies of the last stages have landed before the CTA moves on
+        // (also after an abort: they write this CTA's shared memory)
         for (int i = max(0, issued - kIStages); i < issued; ++i)
-            tc::mbar_wait(tc::smem_u32(&ss->full[i % kIStages]), (i / kIStages) & 1, &ss->abort,
-                          dev_status);
+            tc::mbar_quiesce(tc::smem_u32(&ss->full[i % kIStages]), (i / kIStages) & 1,
+                             dev_status, wait_ns);
     } else if (warp == 1 && lane == 0) {
         // MMA issuer
         const uint32_t idesc = tc::idesc_s8(kIM, kIN);
         for (int c = c0, i = 0; c < c1; ++c, ++i) {
             const int st = i % kIStages;
             if (!tc::mbar_wait(tc::smem_u32(&ss->full[st]), (i / kIStages) & 1, &ss->abort,
-                               dev_status))
+                               dev_status, wait_ns))
                 break;
             tc::fence_after();
             const uint32_t a0 = tc::smem_u32(smem + size_t(st) * kIStageBytes);
@@ -304,8 +306,10 @@ __global__ void __launch_bounds__(128, 1) route_imma_kernel(
         tc::commit(tc::smem_u32(&ss->done));  // after every MMA issued above
     }
     __syncwarp();
-    // levels out: warp w holds TMEM lanes (tokens) 32w .. 32w+31
-    bool ok = tc::mbar_wait(tc::smem_u32(&ss->done), 0, &ss->abort, dev_status) &&
+    // levels out: warp w holds TMEM lanes (tokens) 32w .. 32w+31.  Every MMA
+    // issued has completed once `done` fires, abort or not (TMEM is freed
+    // below).
+    bool ok = tc::mbar_quiesce(tc::smem_u32(&ss->done), 0, dev_status, wait_ns) &&
               !*reinterpret_cast<volatile int*>(&ss->abort);
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
     tc::fence_after();
@@ -1143,6 +1147,13 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
     if (!x || !topk_idx || !topk_gate) return MOE_ERR_NULL;
     if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_ALIGN;
     if (!ws || ws_bytes < moe_route_workspace_size(shape)) return MOE_ERR_WORKSPACE;
+    // every buffer the kernels touch must be addressable by the GPU (a
+    // pageable host array here would fault the kernels)
+    for (const void* ptr : {(const void*)x, (const void*)router_w, (const void*)bias,
+                            (const void*)logit_offset, (const void*)topk_idx,
+                            (const void*)topk_gate, (const void*)expert_counts, (const void*)ws,
+                            (const void*)dev_status})
+        if (!device_accessible(ptr)) return MOE_ERR_ARG;
     const RouteWs w = route_carve(shape, ws);
     const int sms = sm_count();
     if (!device_is_sm100()) return MOE_ERR_DEVICE;
@@ -1175,7 +1186,7 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
         return MOE_ERR_CUDA;
     dim3 gi((T + kIM - 1) / kIM, (N + kIN - 1) / kIN, splits);
     route_imma_kernel<<<gi, 128, kImmaSmem, st>>>(mx, me, T, N, nchunks, per_split, w.acc,
-                                                  dev_status);
+                                                  dev_status, wait_limit_ns());
     if ((rc = check_launch()) != MOE_OK) return rc;
 
     // 3. certify the choice of every token; gamma_d of FP64 bounds the

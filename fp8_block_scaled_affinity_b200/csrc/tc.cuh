@@ -41,20 +41,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with `parity`; gives up (raising *abort and the
-// device status) after kWaitLimitNs, or when *abort is already raised.
+// device status) after limit_ns, or when *abort is already raised.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* abort,
-                                          int* dev_status) {
+                                          int* dev_status, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15) == 0) {
             if (*reinterpret_cast<volatile int*>(abort)) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 atomicExch(abort, 1);
                 set_status(dev_status, MOE_DEV_TIMEOUT);
                 return false;
             }
+        }
+    }
+}
+
+// Waits for work already in flight (TMA copies, MMAs) before a CTA frees
+// what that work writes: like mbar_wait but it does not stop when the CTA
+// has aborted; it still gives up after limit_ns.
+__device__ __forceinline__ bool mbar_quiesce(uint32_t bar, uint32_t parity, int* dev_status,
+                                             uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15) == 0 && globaltimer_ns() - t0 > limit_ns) {
+            set_status(dev_status, MOE_DEV_TIMEOUT);
+            return false;
         }
     }
 }

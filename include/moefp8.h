@@ -40,6 +40,17 @@
  *     the supported range.
  *   - Thread safety: the library keeps no state between calls; concurrent
  *     calls on different buffers are independent.
+ *   - Bounded waits: every wait of a kernel on an mbarrier (TMA loads, MMA
+ *     completion, hand-overs between warps) gives up after a limit, 2 s by
+ *     default, sets MOE_DEV_TIMEOUT and lets the kernel unwind (work already
+ *     in flight is waited for, TMEM is freed); the context stays usable.
+ *     The environment variable MOEFP8_WAIT_LIMIT_NS (read at every call)
+ *     sets another limit in nanoseconds (at least 1000).
+ *   - Fault injection for tests of that path: MOEFP8_FAULT=gemm_producer
+ *     (read at every call) makes the single-CTA grouped GEMM's TMA producer
+ *     withhold the loads of its first stage, so that the MMA issuer's wait
+ *     on that stage runs out.  Nothing faults or hangs; the call's results
+ *     are garbage and dev_status reads MOE_DEV_TIMEOUT.  Unset in normal use.
  */
 #ifndef MOEFP8_H
 #define MOEFP8_H
@@ -125,7 +136,8 @@ MOE_API int moe_read_status(const int* dev_status, int* host_status, void* strea
  *   slot order.
  * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE (d % 128, T < 0, N_r range),
  * MOE_ERR_ROUTE, MOE_ERR_ALIGN (x, router_w not 16-byte aligned),
- * MOE_ERR_WORKSPACE, MOE_ERR_DEVICE (not sm_100), MOE_ERR_CUDA;
+ * MOE_ERR_WORKSPACE, MOE_ERR_ARG (a pointer the GPU cannot address, e.g.
+ * pageable host memory), MOE_ERR_DEVICE (not sm_100), MOE_ERR_CUDA;
  * MOE_DEV_TIMEOUT or MOE_DEV_BAD_INPUT on dev_status (may be NULL).
  * The logits are computed exactly on the tensor cores from int8 digit
  * planes of x and E wherever a rigorous bound settles the result, and with
@@ -208,8 +220,10 @@ MOE_API int moe_quant_permute(const MoeShape* shape, const uint16_t* x, const in
  *   ceil(T / 64) * N_r <= 262144 (e.g. T <= 65536 with N_r = 256); larger
  *   shapes return MOE_ERR_STATIC_LIMIT without doing anything.
  *   The first call on a device looks the array's device address up (once
- *   per device, with that device current), so make that first call before
- *   any stream capture.
+ *   per device and CUDA context, with that device current), so make that
+ *   first call before any stream capture.  After cudaDeviceReset the next
+ *   call sees a new context and looks the address up again (so make it
+ *   outside a capture too).
  *   All calls share the one array: two calls whose work overlaps on the GPU
  *   (different streams, or different host threads, on one device) race and
  *   give wrong results.  Each call overwrites every scratch entry it reads,
@@ -257,6 +271,105 @@ MOE_API int moe_grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int
                                  const uint8_t* a, const float* a_scales, int k,
                                  const uint8_t* w, const float* w_scales, int n, int epilogue,
                                  void* out, float* out_scales, int* dev_status, void* stream);
+
+/* ------------------------------------------- power-of-two scale option
+ * A numerically different option beside the pages' recipe (whose scales
+ * are arbitrary FP32 values): every 1x128 tile / 128x128 block gets the
+ * scale 2^e with e the smallest integer such that amax <= 448 * 2^e
+ * (clamped to [-127, 127]; amax = 0 gives e = 0), stored as one UE8M0 byte
+ * e + 127, and codes E4M3(v * 2^-e) (nearest even, saturating; the product
+ * is exact).  The pages wish for hardware support of tile / block scaling
+ * (section "FP8 mixed precision training", discussion): B200's block-scaled
+ * MMA (tcgen05.mma kind::mxf8f6f4.block_scale) applies such scales inside
+ * the tensor core, so the GEMM needs no per-K-block promotion.
+ *
+ * fp8_quant_act_1x128_ue8m0: as fp8_quant_act_1x128 with power-of-two
+ *   scales; sf uint8 [rows, cols/128] (sf_kb_major = 0) or [cols/128, rows]
+ *   (sf_kb_major = 1, the layout moe_grouped_gemm_mxfp8 reads).
+ * fp8_quant_w_128x128_ue8m0: as fp8_quant_w_128x128; sf uint8
+ *   [rows/128, cols/128].
+ * Bit-exact contract: codes and scale bytes as the rule above. */
+MOE_API int fp8_quant_act_1x128_ue8m0(const uint16_t* x, int64_t rows, int64_t cols,
+                                      uint8_t* q, uint8_t* sf, int sf_kb_major,
+                                      int* dev_status, void* stream);
+MOE_API int fp8_quant_w_128x128_ue8m0(const uint16_t* w, int64_t rows, int64_t cols,
+                                      uint8_t* q, uint8_t* sf, int* dev_status, void* stream);
+
+/* moe_grouped_gemm_mxfp8: moe_grouped_gemm_fp8 for operands quantised with
+ * power-of-two scales: the scales are applied by the tensor core (one UE8M0
+ * byte per 32 elements of K, each 1x128 tile's byte repeated over its four
+ * 32-element pieces) and the whole K range accumulates in one FP32 TMEM
+ * accumulator per 128 x 256 output tile.
+ *   a_sf       uint8 [k/128, max_rows] (kb-major)
+ *   w_sf       uint8 [n_groups, n/128, k/128]
+ *   n          a multiple of 256
+ *   epilogue   MOE_EPI_F32, MOE_EPI_BF16, or MOE_EPI_SWIGLU_QUANT (h =
+ *              silu(gate) * up quantised 1x128 with power-of-two scales:
+ *              out uint8 [max_rows, n/2], out_sf uint8 [n/2/128, max_rows])
+ * Other arguments, layouts and errors as moe_grouped_gemm_fp8. */
+MOE_API int moe_grouped_gemm_mxfp8(int n_groups, const int32_t* group_offsets, int max_rows,
+                                   const uint8_t* a, const uint8_t* a_sf, int k,
+                                   const uint8_t* w, const uint8_t* w_sf, int n, int epilogue,
+                                   void* out, uint8_t* out_sf, int* dev_status, void* stream);
+
+/* moe_grouped_gemm_fp8_indexed: moe_grouped_gemm_fp8 where group g uses
+ * weight matrix group_weight[g] (device int32 [n_groups], each in
+ * [0, n_weights)) of w [n_weights, n, k] and w_scales [n_weights, n/128,
+ * k/128], so that several groups can share one expert's weights (redundant
+ * experts).  An index out of range is reported (MOE_DEV_BAD_INPUT) and
+ * matrix 0 is used.  Other arguments as moe_grouped_gemm_fp8. */
+MOE_API int moe_grouped_gemm_fp8_indexed(int n_groups, const int32_t* group_offsets,
+                                         const int32_t* group_weight, int n_weights,
+                                         int max_rows, const uint8_t* a, const float* a_scales,
+                                         int k, const uint8_t* w, const float* w_scales, int n,
+                                         int epilogue, void* out, float* out_scales,
+                                         int* dev_status, void* stream);
+
+/* moe_quant_permute_ue8m0: moe_quant_permute with power-of-two scales:
+ * xsf_perm uint8 [d/128, T*K + T] (kb-major UE8M0 bytes) replaces xs_perm.
+ * Bit-exact contract: equal to fp8_quant_act_1x128_ue8m0 followed by the
+ * permutation of moe_permute. */
+MOE_API int moe_quant_permute_ue8m0(const MoeShape* shape, const uint16_t* x,
+                                    const int32_t* topk_idx, const int32_t* expert_counts,
+                                    uint8_t* xq_perm, uint8_t* xsf_perm,
+                                    int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
+                                    size_t ws_bytes, int* dev_status, void* stream);
+
+/* ------------------------------------------------------ redundant experts
+ * The most loaded experts get extra copies so that their rows can be split
+ * over several groups (618zxw.cn news article on DeepSeek-V3, redundant
+ * experts for inference load balance).  On one GPU the copies share the
+ * expert's weights (moe_grouped_gemm_fp8_indexed); every output row is
+ * computed exactly as without copies.
+ *
+ * moe_plan_redundant_experts (HOST memory, synchronous): distributes
+ * n_extra extra slots over n_experts experts with loads counts[e] (e.g. the
+ * expert_counts of a batch): each extra slot goes to the expert with the
+ * largest rows per copy ceil(counts[e] / replicas[e]) (ties to the lower
+ * expert), which minimises the largest rows per copy.
+ *   replicas    int32 [n_experts] out: copies per expert (>= 1)
+ *   slot_expert int32 [n_experts + n_extra] out: the expert of each slot,
+ *               experts ascending, an expert's copies adjacent
+ * Errors: MOE_ERR_NULL, MOE_ERR_SHAPE (n_experts + n_extra + 1 > 1040),
+ * MOE_ERR_ARG (a negative count).
+ *
+ * moe_split_groups (device): the group table of the copies.  Expert e's rows
+ * [off[e], off[e+1]) of the permutation are cut into replicas[e] consecutive
+ * pieces whose sizes differ by at most one (the first ones longer).
+ *   expert_offsets  int32 [N_r + 2] from moe_permute / moe_quant_permute
+ *   replicas, slot_expert   as planned above (device copies)
+ *   first_slot      int32 [N_r] first slot of each expert (device)
+ *   slot_offsets    int32 [N_r + n_extra + 2] out: group s owns rows
+ *                   [slot_offsets[s], slot_offsets[s+1]); the last group is
+ *                   the shared expert's rows
+ *   slot_weight     int32 [N_r + n_extra + 1] out: weight matrix of each
+ *                   group (slot_expert, then N_r for the shared expert) */
+MOE_API int moe_plan_redundant_experts(const int32_t* counts, int n_experts, int n_extra,
+                                       int32_t* replicas, int32_t* slot_expert);
+MOE_API int moe_split_groups(const MoeShape* shape, const int32_t* expert_offsets,
+                             const int32_t* replicas, const int32_t* slot_expert,
+                             const int32_t* first_slot, int n_extra, int32_t* slot_offsets,
+                             int32_t* slot_weight, int* dev_status, void* stream);
 
 /* moe_grouped_gemm_form: CTAs per tile (1 = single CTAs, 2 = CTA pairs) that
  * moe_grouped_gemm_fp8 uses on the current device for these arguments (same
@@ -333,6 +446,52 @@ MOE_API int moe_layer_forward_host(const MoeShape* shape, const MoeWeights* weig
                                    const float* logit_offset, MoeRouting* routing,
                                    uint16_t* y_host, int update_bias, void* ws,
                                    size_t ws_bytes, int* dev_status, void* stream);
+
+/* The whole layer with the power-of-two scale option: weights quantised
+ * with fp8_quant_w_128x128_ue8m0, x and h with power-of-two 1x128 scales,
+ * both expert GEMMs block-scaled (moe_grouped_gemm_mxfp8).  Routing,
+ * permutation, combine and bias update as moe_layer_forward.  d and I must
+ * be multiples of 256.
+ *   w13_sf uint8 [N_r+1, 2I/128, d/128], w2_sf uint8 [N_r+1, d/128, I/128]
+ *   ws, ws_bytes scratch of moe_layer_mx_workspace_size(shape) */
+typedef struct {
+    const uint8_t* w13;
+    const uint8_t* w13_sf;
+    const uint8_t* w2;
+    const uint8_t* w2_sf;
+    const uint16_t* router_w;
+} MoeWeightsMx;
+MOE_API size_t moe_layer_mx_workspace_size(const MoeShape* shape);
+MOE_API int moe_layer_forward_mx(const MoeShape* shape, const MoeWeightsMx* weights,
+                                 const uint16_t* x, float* bias, const float* logit_offset,
+                                 MoeRouting* routing, uint16_t* y, int update_bias, void* ws,
+                                 size_t ws_bytes, int* dev_status, void* stream);
+
+/* moe_layer_forward_host_batches: n_batches successive batches of the layer
+ * with x and y in HOST memory (pinned), the transfers overlapped with the
+ * computation: while batch j runs on `stream`, x of batch j+1 is copied in
+ * on one internal copy stream and y of batch j-1 out on another (two device
+ * buffers of x and of y alternate in the workspace).  Every output token
+ * needs the outputs of every expert, so inside one batch the copies cannot
+ * overlap the work; across batches they can.
+ *   x_host       bf16 [n_batches, T, d] (pinned for the copies to be
+ *                asynchronous);  y_host bf16 [n_batches, T, d] out
+ *   bias         updated after each batch when update_bias != 0: batch j
+ *                routes with the bias batch j-1 left, exactly as n_batches
+ *                calls of moe_layer_forward_host would
+ *   routing      holds the last batch's routing when the call completes
+ *   ws, ws_bytes scratch of moe_layer_host_batches_workspace_size(shape)
+ * Work already queued on `stream` is finished before the first copy starts;
+ * `stream` completes after the last copy out: synchronise it before reading
+ * y_host.  The two copy streams and the events are created and released by
+ * the call.  Errors: those of moe_layer_forward, MOE_ERR_ARG (n_batches <
+ * 0).  n_batches = 0 does nothing. */
+MOE_API size_t moe_layer_host_batches_workspace_size(const MoeShape* shape);
+MOE_API int moe_layer_forward_host_batches(const MoeShape* shape, const MoeWeights* weights,
+                                           const uint16_t* x_host, int n_batches, float* bias,
+                                           const float* logit_offset, MoeRouting* routing,
+                                           uint16_t* y_host, int update_bias, void* ws,
+                                           size_t ws_bytes, int* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -21,6 +21,7 @@ __all__ = [
     "permute_layout", "swiglu_expert", "f64_to_bf16_bits", "combine",
     "quantized_expert", "layer_forward", "gemm_blockscaled",
     "quant_act_1x128_pow2", "quant_w_128x128_pow2", "pow2_scales",
+    "redundant_plan", "split_groups", "quantized_expert_pow2", "quant_act_1x128_pow2_values",
 ]
 
 _LIB = None
@@ -144,6 +145,43 @@ def pow2_scales(e: np.ndarray) -> np.ndarray:
     return np.ldexp(1.0, np.asarray(e, dtype=np.int32))
 
 
+# ------------------------------------------------------ redundant experts
+# The pages name redundant experts for inference load balance (the 618zxw.cn
+# news article) without an algorithm.  Reading: copies are given so as to
+# minimise the largest number of rows one copy serves, max_e ceil(c_e/r_e),
+# each extra copy to the expert whose copies currently serve the most rows
+# (ties to the lower expert); an expert's rows (in token order) are cut into
+# r_e consecutive pieces whose sizes differ by at most one, longer first.
+
+def redundant_plan(counts, n_extra: int):
+    """-> replicas [N] (copies per expert), slot_expert [N + n_extra]."""
+    c = [int(v) for v in counts]
+    rep = [1] * len(c)
+    for _ in range(int(n_extra)):
+        loads = [-(-c[e] // rep[e]) for e in range(len(c))]  # ceil
+        best = max(range(len(c)), key=lambda e: (loads[e], -e))
+        rep[best] += 1
+    slots = [e for e in range(len(c)) for _ in range(rep[e])]
+    return np.array(rep, np.int32), np.array(slots, np.int32)
+
+
+def split_groups(expert_offsets, replicas):
+    """Group table of the copies: (slot_offsets [S + 2], slot_weight [S + 1])
+    for S = sum(replicas) slots; the last group is the shared expert's."""
+    off = [int(v) for v in expert_offsets]
+    N = len(replicas)
+    starts, weights = [], []
+    for e in range(N):
+        c, r = off[e + 1] - off[e], int(replicas[e])
+        q, extra = divmod(c, r)
+        for j in range(r):
+            starts.append(off[e] + j * q + min(j, extra))
+            weights.append(e)
+    starts += [off[N], off[N + 1]]
+    weights.append(N)
+    return np.array(starts, np.int32), np.array(weights, np.int32)
+
+
 _TABLE = None
 
 
@@ -248,8 +286,24 @@ def quantized_expert(w1_bf16, w3_bf16, w2_bf16):
     return quant_w_128x128(w1_bf16), quant_w_128x128(w3_bf16), quant_w_128x128(w2_bf16)
 
 
+def quantized_expert_pow2(w1_bf16, w3_bf16, w2_bf16):
+    """Oracle quantisation of one expert with power-of-two 128x128 scales;
+    the scales are returned as float32 values 2^e (exact)."""
+    out = []
+    for w in (w1_bf16, w3_bf16, w2_bf16):
+        q, e = quant_w_128x128_pow2(w)
+        out.append((q, pow2_scales(e).astype(np.float32)))
+    return tuple(out)
+
+
+def quant_act_1x128_pow2_values(x: np.ndarray):
+    """quant_act_1x128_pow2 with the scales as float32 values 2^e."""
+    q, e = quant_act_1x128_pow2(x)
+    return q, pow2_scales(e).astype(np.float32)
+
+
 def swiglu_expert(xq: np.ndarray, xs: np.ndarray, w1, w3, w2,
-                  return_h: bool = False):
+                  return_h: bool = False, h_quant=None):
     """One expert on FP8 rows (xq, xs = 1x128 codes and scales).
 
     w1, w3, w2 = (codes, scales) pairs, [I,d], [I,d], [d,I].
@@ -264,7 +318,7 @@ def swiglu_expert(xq: np.ndarray, xs: np.ndarray, w1, w3, w2,
     c = X @ W3.T
     h = (a / (1.0 + np.exp(-a))) * c
     h32 = h.astype(np.float32)
-    hq, hs = quant_act_1x128(h32)
+    hq, hs = (h_quant or quant_act_1x128)(h32)
     o = dequant_act(hq, hs) @ dequant_w(*w2).T
     if return_h:
         return o, h32, hq, hs
@@ -305,7 +359,7 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
                   n_groups: int, topk_groups: int, topk: int,
                   expert_weights: Callable[[int], tuple],
                   logit_offset: Optional[np.ndarray] = None,
-                  tokens: Optional[np.ndarray] = None) -> dict:
+                  tokens: Optional[np.ndarray] = None, scales: str = "fp32") -> dict:
     """Whole layer for all tokens (routing) and the chosen ``tokens`` (output).
 
     expert_weights(e) returns ((w1q,w1s),(w3q,w3s),(w2q,w2s)) for expert e;
@@ -314,7 +368,10 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
     T, d = x_bf16.shape
     n_routed = router_w_bf16.shape[0]
     r = route(x_bf16, router_w_bf16, bias, n_groups, topk_groups, topk, logit_offset)
-    xq, xs = quant_act_1x128(x_bf16)
+    # scales = "pow2": the power-of-two option for x and h (the expert
+    # weights come quantised that way from expert_weights)
+    act_quant = quant_act_1x128 if scales == "fp32" else quant_act_1x128_pow2_values
+    xq, xs = act_quant(x_bf16)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     idx = r["topk_idx"][tokens]
     gates = r["topk_gate"][tokens].astype(np.float64)
@@ -330,7 +387,7 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
             if sel.size == 0:
                 continue
         w = expert_weights(e)
-        o = swiglu_expert(xq[tokens[sel]], xs[tokens[sel]], *w)
+        o = swiglu_expert(xq[tokens[sel]], xs[tokens[sel]], *w, h_quant=act_quant)
         if slots is None:
             y64[sel] += o
         else:

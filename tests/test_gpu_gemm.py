@@ -8,9 +8,9 @@ the relative error of an output is a few fp32 rounding steps (about 1e-6);
 1e-5 relative Frobenius is used for fp32 outputs.  bf16 outputs are compared
 after both sides round to bf16 (2e-3, the layer's output bound).
 
-Every test runs twice: with CTA pairs (cta_group::2, the library's default
-where the output width allows it) and with single CTAs
-(MOEFP8_GEMM_PAIR=0)."""
+Every test runs twice: with single CTAs (the library's default) and with
+CTA pairs (cta_group::2, selected with MOEFP8_GEMM_PAIR=1 where the output
+width allows it)."""
 import os
 
 import numpy as np
@@ -50,7 +50,7 @@ def _quant_w_gpu(wbits):
     return q, s
 
 
-def run_grouped(sizes, k, n, epilogue, seed, pad_rows=0, outliers=False):
+def run_grouped(sizes, k, n, epilogue, seed, pad_rows=0, outliers=False, inputs=None):
     """Random A rows split into groups of `sizes`, one weight matrix per group.
     Returns (gpu_out, oracle_results_per_group, offsets, extras)."""
     import fp8_block_scaled_affinity_b200 as moe
@@ -63,6 +63,8 @@ def run_grouped(sizes, k, n, epilogue, seed, pad_rows=0, outliers=False):
         va *= np.where(rng.random((R, k)) < 0.001, 100.0, 1.0).astype(np.float32)
     a = S.f32_to_bf16_bits(va)
     w = S.host_normal_bf16(rng, (G * n, k), 0.05)
+    if inputs is not None:
+        inputs.update(a=a, w=w)
     aq, as_ = _quant_gpu(a)
     wq, ws = _quant_w_gpu(w)
     if epilogue == moe.MOE_EPI_SWIGLU_QUANT:
@@ -201,3 +203,75 @@ def test_gemm_rejects_bad_arguments():
         with pytest.raises(moe.MoeError) as e:
             moe.moe_grouped_gemm_fp8(*args)
         assert e.value.status == code
+
+
+# ----------------------------------------------------------------------
+# Many work items per CTA, compared element by element.
+#
+# The GEMM is persistent: one CTA (or CTA pair) per SM walks a strided list
+# of (group, column tile, token tile) items, handing TMEM partial buffers,
+# stage barriers and (SwiGLU) the alternating amax exchange over from item
+# to item.  With 64 groups of 130-300 rows there are well over 2 x 148
+# items, so every CTA runs several of them.
+
+def _rank(codes):
+    """Order-preserving integer of an E4M3 code (both zeros -> 0)."""
+    c = codes.astype(np.int32)
+    mag = c & 0x7F
+    return np.where(c & 0x80, -mag, mag)
+
+
+def _many_items_sizes(seed):
+    return np.random.default_rng(seed).integers(130, 301, size=64).tolist()
+
+
+@pytest.mark.parametrize("epilogue_name,n,k", [("f32", 2048, 512), ("swiglu", 4096, 512),
+                                                ("f32", 768, 1024)])
+def test_many_items_per_cta_element_wise(epilogue_name, n, k):
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    epi = moe.MOE_EPI_F32 if epilogue_name == "f32" else moe.MOE_EPI_SWIGLU_QUANT
+    sizes = _many_items_sizes(seed=n + k)
+    ctas = 2 if moe.moe_grouped_gemm_form(len(sizes), sum(sizes), n, epi) == 2 else 1
+    tile_rows = 128 * ctas
+    tile_cols = 256 if (epi == moe.MOE_EPI_SWIGLU_QUANT or n % 256 == 0) else 128
+    items = sum((s + tile_rows - 1) // tile_rows for s in sizes) * (n // tile_cols)
+    assert items > 2 * (148 // ctas)  # several items per CTA (pair)
+    inp = {}
+    out, out_s, res, off = run_grouped(sizes, k, n, epi, seed=n * 7 + k, pad_rows=5, inputs=inp)
+    nkb = k // 128
+    if epi == moe.MOE_EPI_F32:
+        got = out.cpu().numpy().astype(np.float64)
+        # every element: FP32 accumulation of 128 exact products per K block
+        # (at most 127 roundings) and one promotion FMA per block, each
+        # rounding at most one fp32 ulp (2^-23 relative, whatever the
+        # rounding mode), so |got - exact| <= 2^-23 (128 + nkb + 2)
+        # sum_k |a_k b_k| s_a s_b
+        a, w = inp["a"], inp["w"]
+        qa, sa = oracle.quant_act_1x128(a)
+        for g, ref in enumerate(res):
+            r0, r1 = off[g], off[g + 1]
+            wq, ws = oracle.quant_w_128x128(w[g * n:(g + 1) * n])
+            absum = np.abs(oracle.dequant_act(qa[r0:r1], sa[r0:r1])) @ \
+                np.abs(oracle.dequant_w(wq, ws)).T
+            bound = 2.0 ** -23 * (128 + nkb + 2) * absum
+            err = np.abs(got[r0:r1] - ref)
+            bad = err > bound
+            assert not bad.any(), (g, int(bad.sum()), float(err.max()))
+        assert np.all(np.isnan(got[off[-1]:]))
+    else:
+        q = out.cpu().numpy()
+        s = out_s.cpu().numpy().T
+        for g, ref in enumerate(res):
+            r0, r1 = off[g], off[g + 1]
+            h32, hq_ref, hs_ref = ref
+            # scales: the same amax up to fp32 accumulation order
+            assert np.allclose(s[r0:r1], hs_ref, rtol=1e-5, atol=0), g
+            # codes: every one equal or one E4M3 step away (h at a rounding
+            # boundary), and almost all equal
+            step = np.abs(_rank(q[r0:r1]) - _rank(hq_ref))
+            assert step.max() <= 1, (g, int(step.max()))
+            assert (step == 0).mean() > 0.999, g
+        # rows outside every group are not written
+        assert np.all(q[off[-1]:] == 0xEE)
+        assert np.all(s[off[-1]:] == -1.0)

@@ -7,6 +7,9 @@ dispatch / MLP / combine stages of "DualPipe").
 Bit-exact: expert indices, gates, counts, offsets, row_of_pair, bias.
 Output y (bf16): relative Frobenius error <= 2e-3 against the oracle's FP64
 result rounded once to bf16 (the bound the layer is built to)."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -19,6 +22,10 @@ from gpu_util import (DEV, OracleExperts, bf16_dev, expert_bf16, host_bits, need
 pytestmark = pytest.mark.gpu
 
 Y_TOL = 2e-3
+# Per token: both sides round y once to bf16, so a token's error is a few
+# one-step bf16 differences where the fp32 and FP64 sums straddle a rounding
+# boundary (and rare one-step h code differences); a wrong row gives ~1.
+Y_TOKEN_TOL = 1e-2
 
 
 def build_layer(cfg, T=None, host_io=False):
@@ -104,6 +111,28 @@ def test_host_buffer_entry_point_matches_device_entry_point():
     assert torch.equal(y_dev.cpu().view(torch.int16), y_host.view(torch.int16))
 
 
+def y_errors(name, got, ref_bits):
+    """Relative Frobenius error of y over the compared tokens and the worst
+    per-token relative error; asserted against the layer bound (Frobenius)
+    and a per-token bound that a single wrong token would break.  The
+    figures are appended to the file named by MOEFP8_PARITY_REPORT, if set."""
+    ref = S.bf16_bits_to_f32(ref_bits).astype(np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    fro = rel_frobenius(got, ref)
+    tok = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    rec = {"case": name, "tokens": int(got.shape[0]), "rel_frobenius": fro,
+           "worst_token_rel": float(tok.max()), "median_token_rel": float(np.median(tok)),
+           "bf16_equal_frac": float(np.mean(got == ref))}
+    print(json.dumps(rec))
+    path = os.environ.get("MOEFP8_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+    assert fro <= Y_TOL, rec
+    assert tok.max() <= Y_TOKEN_TOL, rec
+    return rec
+
+
 def _full(cfg_name, n_sample, seed):
     need_gpu()
     cfg = S.CONFIGS[cfg_name]
@@ -113,40 +142,90 @@ def _full(cfg_name, n_sample, seed):
                       else to_dev(inp["logit_offset"]))
     torch.cuda.synchronize()
     assert layer.status() == 0
-    sample = np.sort(np.random.default_rng(seed).choice(cfg.T, n_sample, replace=False))
+    sample = (np.arange(cfg.T) if n_sample >= cfg.T else
+              np.sort(np.random.default_rng(seed).choice(cfg.T, n_sample, replace=False)))
     ref = check_layer(cfg, layer, inp, x, inp["bias"], sample, OracleExperts(cfg),
                       offset=inp["logit_offset"])
     got = _y_host(y)[sample]
-    err = rel_frobenius(got, S.bf16_bits_to_f32(ref["y"]))
-    assert err <= Y_TOL, err
+    y_errors(f"{cfg_name}: {len(sample)} of {cfg.T} tokens", got, ref["y"])
     return layer, got
 
 
-def test_decode_layer_full_size():
-    _full("decode", 12, 3)
+def test_decode_layer_full_size_all_tokens():
+    _full("decode", 128, 3)
 
 
 def test_prefill_layer_full_size():
-    _full("prefill", 6, 2)
+    _full("prefill", 512, 2)
 
 
-def test_skewed_layer_two_batches():
-    """Skewed prefill: batch 0 routes with the initial bias and updates it;
-    batch 1 routes with the updated bias.  Routing and bias bit-exact each
-    batch, y on sampled tokens of batch 1."""
+def test_skewed_layer_eight_batches():
+    """Skewed prefill, the eight batches in sequence: batch j routes with the
+    bias left by batch j-1.  Routing, offsets, rows and the bias are bit-exact
+    after every batch; y is compared on every token of batch 0 and on 1,024
+    sampled tokens of batch 1."""
     need_gpu()
     cfg = S.CONFIGS["skewed"]
     layer, inp = build_layer(cfg)
     off = to_dev(inp["logit_offset"])
     b_ref = inp["bias"].copy()
     experts = OracleExperts(cfg)
-    for j in range(2):
+    for j in range(cfg.batches):
         x = S.make_layer_inputs_host(cfg, j)["x"]
         y = layer.forward(bf16_dev(x), update_bias=True, logit_offset=off)
         torch.cuda.synchronize()
-        sample = np.array([0, 4097, cfg.T - 1]) if j == 1 else np.array([5])
-        ref = check_layer(cfg, layer, inp, x, b_ref, sample, experts, offset=inp["logit_offset"])
-        b_ref = oracle.update_bias(ref["counts"], b_ref, cfg.T, cfg.topk, cfg.gamma)
+        assert layer.status() == 0
+        if j == 0:
+            sample = np.arange(cfg.T)
+        elif j == 1:
+            sample = np.sort(np.random.default_rng(41).choice(cfg.T, 1024, replace=False))
+        else:
+            sample = np.zeros(0, dtype=np.int64)
+        if len(sample):
+            ref = check_layer(cfg, layer, inp, x, b_ref, sample, experts,
+                              offset=inp["logit_offset"])
+            y_errors(f"skewed batch {j}: {len(sample)} of {cfg.T} tokens", _y_host(y)[sample],
+                     ref["y"])
+            counts = ref["counts"]
+        else:
+            r = oracle.route(x, inp["router_w"], b_ref, cfg.n_groups, cfg.topk_groups, cfg.topk,
+                             logit_offset=inp["logit_offset"])
+            assert np.array_equal(layer.topk_idx.cpu().numpy(), r["topk_idx"])
+            assert np.array_equal(layer.topk_gate.cpu().numpy().view(np.uint32),
+                                  r["topk_gate"].view(np.uint32))
+            assert np.array_equal(layer.expert_counts.cpu().numpy(), r["counts"])
+            counts = r["counts"]
+        b_ref = oracle.update_bias(counts, b_ref, cfg.T, cfg.topk, cfg.gamma)
         assert np.array_equal(layer.bias.cpu().numpy().view(np.uint32), b_ref.view(np.uint32))
-        got = _y_host(y)[sample]
-        assert rel_frobenius(got, S.bf16_bits_to_f32(ref["y"])) <= Y_TOL
+
+
+def test_host_batches_entry_point_matches_single_batch_calls():
+    """moe_layer_forward_host_batches (copies of neighbouring batches
+    overlapped with compute) gives, bit for bit, the outputs and the bias
+    trajectory of one moe_layer_forward_host call per batch."""
+    need_gpu()
+    cfg = S.CONFIGS["tiny"]
+    n = 5
+    layer_a, inp = build_layer(cfg, host_io=True)
+    layer_b, _ = build_layer(cfg, host_io="batches")
+    xs = np.stack([S.make_layer_inputs_host(cfg, j)["x"] for j in range(n)])
+    x_host = torch.from_numpy(xs.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_a = torch.empty_like(x_host).pin_memory()
+    y_b = torch.empty_like(x_host).pin_memory()
+    for j in range(n):
+        layer_a.forward_host(x_host[j], y_a[j], update_bias=True)
+    layer_b.forward_host_batches(x_host, y_b, update_bias=True)
+    torch.cuda.synchronize()
+    assert layer_a.status() == 0 and layer_b.status() == 0
+    assert torch.equal(y_a.view(torch.int16), y_b.view(torch.int16))
+    assert torch.equal(layer_a.bias.view(torch.int32), layer_b.bias.view(torch.int32))
+    # and the last batch against the oracle
+    experts = OracleExperts(cfg)
+    b = inp["bias"].copy()
+    for j in range(n):
+        r = oracle.route(xs[j], inp["router_w"], b, cfg.n_groups, cfg.topk_groups, cfg.topk)
+        if j < n - 1:
+            b = oracle.update_bias(r["counts"], b, cfg.T, cfg.topk, cfg.gamma)
+    ref = oracle.layer_forward(xs[n - 1], inp["router_w"], b, cfg.n_groups, cfg.topk_groups,
+                               cfg.topk, experts)
+    y_errors("tiny, last of 5 pipelined host batches", _y_host(y_b[n - 1]), ref["y"])

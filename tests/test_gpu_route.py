@@ -207,3 +207,89 @@ def test_empty_batch_zeroes_counts():
     bad = moe.make_shape(4, 128, 10, 3, 1, 2, 128)  # N_r % G != 0
     with pytest.raises(moe.MoeError):
         gpu_route(bad, inp["x"][:4, :128], inp["router_w"][:10, :128], inp["bias"][:10])
+
+
+# ----------------------------------------------------------------------
+# Near ties: biased scores a few fp32 ulps apart without being equal.
+#
+# The router certifies each token's choice from intervals around scores
+# computed from exact integer logits; an interval that is too narrow would
+# certify a wrong choice exactly when two candidates are one or two ulps
+# apart.  Here every router row is the same base row except in its own
+# "perturbation slot", an element whose value is tiny (2^-e for a spread of
+# e), so all N_r logits of a token agree except in their last few bits:
+# every group boundary and every K-th / (K+1)-th boundary is a near tie.
+
+def _near_tie_router(N, d, rng):
+    base = S.bf16_bits_to_f32(S.host_normal_bf16(rng, (d,), 0.02)).astype(np.float32)
+    slots = np.arange(N) * (d // N)  # one slot per expert, spread over k
+    base[slots] = 0.0
+    E = np.tile(base, (N, 1))
+    # slot value 2^-e with e from 14 to 24: the logit differences x_k 2^-e
+    # then span a few ulps of |u| ~ 1
+    e = 14 + (np.arange(N) * 7) % 11
+    E[np.arange(N), slots] = np.ldexp(1.0, -e).astype(np.float32)
+    return S.f32_to_bf16_bits(E)
+
+
+@pytest.mark.parametrize("N,G,M,K,d", [(16, 4, 2, 4, 512), (64, 8, 4, 8, 1024),
+                                       (256, 8, 4, 8, 7168)])
+def test_near_tied_scores_bit_exact(N, G, M, K, d):
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    rng = np.random.default_rng(N + d)
+    T = 1024
+    E = _near_tie_router(N, d, rng)
+    x = S.host_normal_bf16(rng, (T, d), 1.0)
+    bias = np.zeros(N, np.float32)  # equal biases keep the scores' last bits in play
+    shape = moe.make_shape(T, d, N, G, M, K, 256, 0.001)
+    idx, gate, counts = gpu_route(shape, x, E, bias)
+    ref = oracle.route(x, E, bias, G, M, K, want_scores=True)
+    assert np.array_equal(idx, ref["topk_idx"])
+    assert np.array_equal(gate.view(np.uint32), ref["topk_gate"].view(np.uint32))
+    assert np.array_equal(counts, ref["counts"])
+    # the case is adversarial: count tokens whose K-th and (K+1)-th best
+    # biased scores (over all experts) are 1 or 2 fp32 ulps apart
+    s = np.sort(ref["scores"].astype(np.float32) + bias, axis=1)[:, ::-1]
+    gap = s[:, K - 1].view(np.int32).astype(np.int64) - s[:, K].view(np.int32).astype(np.int64)
+    assert np.sum((gap >= 1) & (gap <= 2)) >= T // 20
+
+
+def test_near_tied_scores_with_offsets_and_biases():
+    """The same near-tied router with a logit offset and biases that differ
+    by single ulps."""
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    N, G, M, K, d, T = 64, 8, 4, 8, 1024, 1024
+    rng = np.random.default_rng(5)
+    E = _near_tie_router(N, d, rng)
+    x = S.host_normal_bf16(rng, (T, d), 1.0)
+    b0 = np.float32(0.0125)
+    bias = (np.full(N, b0).view(np.int32) + (np.arange(N) % 3)).view(np.float32)
+    offset = (np.full(N, np.float32(-1.5)).view(np.int32) + (np.arange(N) % 2)).view(np.float32)
+    shape = moe.make_shape(T, d, N, G, M, K, 256, 0.001)
+    idx, gate, counts = gpu_route(shape, x, E, bias, offset)
+    ref = oracle.route(x, E, bias, G, M, K, logit_offset=offset)
+    assert np.array_equal(idx, ref["topk_idx"])
+    assert np.array_equal(gate.view(np.uint32), ref["topk_gate"].view(np.uint32))
+    assert np.array_equal(counts, ref["counts"])
+
+
+def test_pageable_host_pointer_is_rejected_not_dereferenced():
+    """A pageable host array passed where device memory is expected (here the
+    logit offset) returns MOE_ERR_ARG before any kernel is launched."""
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    cfg = S.CONFIGS["tiny"]
+    inp = S.make_layer_inputs_host(cfg, 0)
+    shape = shape_of(cfg, 64)
+    idx = torch.empty((64, cfg.topk), dtype=torch.int32, device=DEV)
+    gate = torch.empty((64, cfg.topk), dtype=torch.float32, device=DEV)
+    counts = torch.empty((cfg.n_routed,), dtype=torch.int32, device=DEV)
+    ws = torch.empty((moe.moe_route_workspace_size(shape),), dtype=torch.uint8, device=DEV)
+    host_offset = torch.zeros(cfg.n_routed, dtype=torch.float32)  # pageable host memory
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_route(shape, bf16_dev(inp["x"][:64]), bf16_dev(inp["router_w"]),
+                      to_dev(inp["bias"]), host_offset, idx, gate, counts, ws)
+    assert e.value.status == -7
+    torch.cuda.synchronize()

@@ -157,3 +157,38 @@ def test_layer_forward_tiny_consistency():
     assert np.array_equal(out["y"][t], oracle.f64_to_bf16_bits(acc))
     y = S.bf16_bits_to_f32(out["y"])
     assert np.isfinite(y).all() and np.abs(y).max() > 0
+
+
+def test_layer_forward_pow2_option_recomposes():
+    """The power-of-two scale option of the whole-layer oracle: a token's y is
+    the shared expert plus the gate-weighted selected experts, with x, the
+    weights and h quantised by the power-of-two rule (pinned in
+    test_oracle_pow2.py) and the routing of the pages' recipe unchanged."""
+    cfg = S.CONFIGS["tiny"]
+    inp = S.make_layer_inputs_host(cfg)
+    W = {e: oracle.quantized_expert_pow2(*S.host_expert_weights(cfg, e))
+         for e in range(cfg.n_routed + 1)}
+    out = oracle.layer_forward(inp["x"], inp["router_w"], inp["bias"], cfg.n_groups,
+                               cfg.topk_groups, cfg.topk, W.__getitem__, scales="pow2")
+    ref = oracle.route(inp["x"], inp["router_w"], inp["bias"], cfg.n_groups, cfg.topk_groups,
+                       cfg.topk)
+    assert np.array_equal(out["topk_idx"], ref["topk_idx"])
+    qx, ex = oracle.quant_act_1x128_pow2(inp["x"])
+    assert np.array_equal(out["xq"], qx)
+    assert np.array_equal(out["xs"], np.ldexp(1.0, ex).astype(np.float32))
+    t = 29
+    xq, xs = out["xq"][t:t + 1], out["xs"][t:t + 1]
+    hq = oracle.quant_act_1x128_pow2_values
+    acc = oracle.swiglu_expert(xq, xs, *W[cfg.n_routed], h_quant=hq)[0].copy()
+    for k, e in enumerate(out["topk_idx"][t]):
+        acc += float(out["topk_gate"][t, k]) * oracle.swiglu_expert(xq, xs, *W[int(e)],
+                                                                      h_quant=hq)[0]
+    assert np.array_equal(out["y"][t], oracle.f64_to_bf16_bits(acc))
+    # a different rounding of the same layer: close to the FP32-scale result
+    W32 = {e: oracle.quantized_expert(*S.host_expert_weights(cfg, e))
+           for e in range(cfg.n_routed + 1)}
+    y32 = oracle.layer_forward(inp["x"], inp["router_w"], inp["bias"], cfg.n_groups,
+                               cfg.topk_groups, cfg.topk, W32.__getitem__)["y"]
+    a, b = S.bf16_bits_to_f32(out["y"]), S.bf16_bits_to_f32(y32)
+    rel = np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert 0 < rel < 0.1
