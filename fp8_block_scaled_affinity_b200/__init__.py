@@ -24,7 +24,9 @@ from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QU
                    fp8_quant_w_128x128_ue8m0, moe_grouped_gemm_mxfp8,
                    moe_grouped_gemm_fp8_indexed, moe_plan_redundant_experts, moe_split_groups,
                    MoeWeightsMx, make_weights_mx, moe_layer_forward_mx,
-                   moe_layer_mx_workspace_size, moe_quant_permute_ue8m0)
+                   moe_layer_mx_workspace_size, moe_quant_permute_ue8m0,
+                   moe_ep_row_bytes, moe_ep_workspace_size, moe_ep_dispatch_plan, moe_ep_pack,
+                   moe_ep_local_permute, moe_ep_partial_combine, moe_ep_final_combine)
 
 __all__ = ["MoeLayer", "MoeShape", "MoeError", "lib", "make_shape", "moe_version"]
 

@@ -86,6 +86,13 @@ def lib() -> ctypes.CDLL:
                                                  P]),
             "moe_plan_redundant_experts": (I, [P, I, I, P, P]),
             "moe_quant_permute_ue8m0": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "moe_ep_row_bytes": (SZ, [SP]),
+            "moe_ep_workspace_size": (SZ, [SP, I, I]),
+            "moe_ep_dispatch_plan": (I, [SP, I, P, P, P, P, P, SZ, P, P]),
+            "moe_ep_pack": (I, [SP, I, P, P, P, P, P, P, P]),
+            "moe_ep_local_permute": (I, [SP, I, P, I, P, P, I, P, P, P, SZ, P, P]),
+            "moe_ep_partial_combine": (I, [SP, I, P, I, P, P, P, P, P]),
+            "moe_ep_final_combine": (I, [SP, I, P, P, P, P, P, P]),
             "moe_layer_mx_workspace_size": (SZ, [SP]),
             "moe_layer_forward_mx": (I, [SP, ctypes.POINTER(MoeWeightsMx), P, P, P,
                                          ctypes.POINTER(MoeRouting), P, I, P, SZ, P, P]),
@@ -370,3 +377,52 @@ def moe_layer_forward_mx(shape, weights: MoeWeightsMx, x, bias, logit_offset,
         ctypes.byref(shape), ctypes.byref(weights), _ptr(x), _ptr(bias), _ptr(logit_offset),
         ctypes.byref(routing), _ptr(y), int(bool(update_bias)), _ptr(ws), nbytes,
         _ptr(dev_status), _stream(stream)))
+
+
+# -------------------------------------------------- expert parallelism
+def moe_ep_row_bytes(shape) -> int:
+    return int(lib().moe_ep_row_bytes(ctypes.byref(shape)))
+
+
+def moe_ep_workspace_size(shape, n_ranks, max_recv_rows) -> int:
+    return int(lib().moe_ep_workspace_size(ctypes.byref(shape), int(n_ranks),
+                                           int(max_recv_rows)))
+
+
+def moe_ep_dispatch_plan(shape, n_ranks, topk_idx, send_counts, send_offsets, send_row, ws,
+                         dev_status=None, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_ep_dispatch_plan", lib().moe_ep_dispatch_plan(
+        ctypes.byref(shape), int(n_ranks), _ptr(topk_idx), _ptr(send_counts),
+        _ptr(send_offsets), _ptr(send_row), _ptr(ws), nbytes, _ptr(dev_status),
+        _stream(stream)))
+
+
+def moe_ep_pack(shape, n_ranks, x, topk_idx, topk_gate, send_row, send_buf, dev_status=None,
+                stream=None):
+    _check("moe_ep_pack", lib().moe_ep_pack(
+        ctypes.byref(shape), int(n_ranks), _ptr(x), _ptr(topk_idx), _ptr(topk_gate),
+        _ptr(send_row), _ptr(send_buf), _ptr(dev_status), _stream(stream)))
+
+
+def moe_ep_local_permute(shape, n_ranks, recv_buf, n_recv, xq_perm, xs_perm, max_rows,
+                         local_offsets, pair_row, ws, dev_status=None, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_ep_local_permute", lib().moe_ep_local_permute(
+        ctypes.byref(shape), int(n_ranks), _ptr(recv_buf), int(n_recv), _ptr(xq_perm),
+        _ptr(xs_perm), int(max_rows), _ptr(local_offsets), _ptr(pair_row), _ptr(ws), nbytes,
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_ep_partial_combine(shape, n_ranks, recv_buf, n_recv, pair_row, expert_out, back_buf,
+                           dev_status=None, stream=None):
+    _check("moe_ep_partial_combine", lib().moe_ep_partial_combine(
+        ctypes.byref(shape), int(n_ranks), _ptr(recv_buf), int(n_recv), _ptr(pair_row),
+        _ptr(expert_out), _ptr(back_buf), _ptr(dev_status), _stream(stream)))
+
+
+def moe_ep_final_combine(shape, n_ranks, shared_out, back_recv, send_row, y, dev_status=None,
+                         stream=None):
+    _check("moe_ep_final_combine", lib().moe_ep_final_combine(
+        ctypes.byref(shape), int(n_ranks), _ptr(shared_out), _ptr(back_recv), _ptr(send_row),
+        _ptr(y), _ptr(dev_status), _stream(stream)))

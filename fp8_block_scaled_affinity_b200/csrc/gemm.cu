@@ -64,12 +64,12 @@ template <bool PAIR, bool SWIGLU, bool WIDE>
 struct Cfg {
     static_assert(WIDE || !(PAIR || SWIGLU), "pairs and SwiGLU use 256-column partials");
     static constexpr int kAccCols = WIDE ? 256 : 128;              // output columns per item
-    // Single CTAs with 256-column items split each K block into two MMA
-    // chains of N = 128 (one per weight block), each into its own 128-column
-    // TMEM buffer with its own full / empty barriers: four buffers rotate,
-    // and a buffer is busy for half as long as a 256-column partial.
-    static constexpr bool kSplit = !PAIR && WIDE;
-    static constexpr int kChains = kSplit ? 2 : 1;                 // MMA chains per K block
+    // One MMA chain per K block into one kAccCols-column TMEM buffer.  (Two
+    // N = 128 chains into four 128-column buffers halve how long a buffer is
+    // held, but measured slower on B200: eight N = 128 MMAs and two commits
+    // per K block cost more issue time than the 512 cycles the block's MMAs
+    // take.)
+    static constexpr int kChains = 1;                              // MMA chains per K block
     static constexpr int kBufCols = kAccCols / kChains;            // TMEM columns per buffer
     static constexpr int kBufs = 512 / kBufCols;                   // TMEM partial buffers
     static constexpr int kWRows = PAIR ? 128 : kAccCols;           // weight rows this CTA loads
@@ -710,16 +710,12 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t d = tmem_base + buf * C::kBufCols;
-                    // chain c multiplies the tokens by weight block c (split
-                    // form) or by the stage's whole weight tile
                     const uint32_t b0 = st + kTileBytes + c * kTileBytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_e4m3<PAIR>(d, sw128_desc(st + kk * 32), sw128_desc(b0 + kk * 32), idesc,
                                        kk > 0 ? 1u : 0u);
-                    // split form: the promoters free the stage once they see
-                    // the last chain complete (one commit per chain)
-                    if (!C::kSplit) mma_commit_both<PAIR>(smem_u32(&ss->empty[s]));
+                    mma_commit_both<PAIR>(smem_u32(&ss->empty[s]));
                     mma_commit_both<PAIR>(smem_u32(&ss->tfull[buf]));
                 }
             }
@@ -889,69 +885,6 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
         uint64_t acc2[C::kPairs];  // fp32 accumulator pairs
 #pragma unroll
         for (int i = 0; i < C::kPairs; ++i) acc2[i] = 0;
-        if (C::kSplit) {
-            // Two 128-column buffers per K block (weight blocks 0 and 1).
-            // SwiGLU: every warp reads 64 columns of each (gate and up of its
-            // 64 features); fp32 / bf16: half h reads the 128 columns of
-            // buffer h only.
-            for (int kb = 0; ok && kb < p.nkb; ++kb, tb += 2, ++cit) {
-                const int c = cit % kScaleSlots;
-                const uint32_t bufs[2] = {tb % C::kBufs, (tb + 1) % C::kBufs};
-                const uint32_t pars[2] = {(tb / C::kBufs) & 1u, ((tb + 1) / C::kBufs) & 1u};
-                const int first = SWIGLU ? 0 : half;  // buffer read first (or only)
-                if (lane == 0) {
-                    ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->tfull[bufs[first]]),
-                                                       pars[first], ss, p.dev_status);
-                    if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (cit / kScaleSlots) & 1u, ss,
-                                           p.dev_status);
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                __syncwarp();
-                tc_fence_after();
-                const float sa = ss->sa[c][r];
-                const float s0 = sa * ss->sb[c][SWIGLU ? 0 : half];
-                const float s1 = sa * ss->sb[c][SWIGLU ? 1 : half];
-                const uint64_t s0x2 = pack2(__float_as_uint(s0), __float_as_uint(s0));
-                const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
-                uint32_t v[64];
-                if (SWIGLU) {
-                    tmem_ld64(lane_addr + bufs[0] * C::kBufCols + 64 * half, v);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[bufs[0]]));
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
-                    if (lane == 0)
-                        ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->tfull[bufs[1]]), pars[1],
-                                                           ss, p.dev_status);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    __syncwarp();
-                    tc_fence_after();
-                    tmem_ld64(lane_addr + bufs[1] * C::kBufCols + 64 * half, v);
-                } else {
-                    const uint32_t tbase = lane_addr + bufs[half] * C::kBufCols;
-                    tmem_ld64(tbase, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ffma2(acc2[i], pack2(v[2 * i], v[2 * i + 1]), s0x2);
-                    tmem_ld64(tbase + 64, v);
-                }
-                // the partial is in registers: hand the buffer back, and (one
-                // thread that saw the K block's last chain complete) the stage
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_u32(&ss->tempty[bufs[SWIGLU ? 1 : half]]));
-                    if (warp == 8) mbar_arrive(smem_u32(&ss->empty[cit % C::kStages]));
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    ffma2(acc2[32 + i], pack2(v[2 * i], v[2 * i + 1]), s1x2);
-            }
-        } else
         for (int kb = 0; ok && kb < p.nkb; ++kb, ++tb, ++cit) {
             const uint32_t buf = tb % C::kBufs;
             const int c = cit % kScaleSlots;
@@ -972,7 +905,7 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
             const uint64_t s1x2 = pack2(__float_as_uint(s1), __float_as_uint(s1));
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
-            const uint32_t tbase = lane_addr + buf * C::kAccCols;
+            const uint32_t tbase = lane_addr + buf * C::kBufCols;
             const uint32_t tempty = smem_u32(&ss->tempty[buf]);
             if (kWide) {
                 uint32_t v[64];
@@ -1094,10 +1027,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < C::kBufs; ++b) {
             mbar_init(smem_u32(&ss->tfull[b]), 1);
-            // split fp32 / bf16 form: a buffer is read by one half of the
-            // promotion warps
-            mbar_init(smem_u32(&ss->tempty[b]),
-                      (C::kSplit && !SWIGLU ? kPromoters / 2 : kPromoters) * C::kCtas);
+            mbar_init(smem_u32(&ss->tempty[b]), kPromoters * C::kCtas);
         }
         for (int c = 0; c < kScaleSlots; ++c) {
             mbar_init(smem_u32(&ss->sfull[c]), 32);
@@ -1297,47 +1227,73 @@ __device__ __forceinline__ void mx_producer(const GemmParams& p, const CUtensorM
     __syncwarp();
 }
 
-// warp 2: the stage's scale chunks (tokens, weight block 0, weight block 1)
+// warp 2: the stage's scale chunks (tokens, weight block 0, weight block 1).
+// The scale bytes of a K block are loaded kMxAhead K blocks before the chunk
+// is written (a register ring), so the global-load latency stays off the
+// per-K-block path.
+constexpr int kMxAhead = 4;
+
+struct MxPre {
+    uint32_t a[4];  // token rows lane + 32 j
+    uint32_t w0, w1;
+};
+
+template <bool SWIGLU>
+__device__ __forceinline__ void mx_fetch(const GemmParams& p, const SharedState* ss, int unit,
+                                         int units, int64_t it, int64_t n_it, int lane,
+                                         MxPre& r) {
+    if (it >= n_it) return;
+    const int i = int(it / p.nkb), kb = int(it - int64_t(i) * p.nkb);
+    const Item w = decode_item<kBM>(ss, p, unit + i * units);
+    int b0, b1;
+    weight_blocks<false, SWIGLU, true>(p, w, b0, b1);
+    const int my_n = cta_tokens(w, 0);
+    const uint8_t* asf = p.a_sf + size_t(kb) * p.max_rows + w.row0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int m = lane + 32 * j;
+        r.a[j] = m < my_n ? uint32_t(__ldg(asf + m)) : 127u;
+    }
+    const int nbr = p.n / 128;
+    r.w0 = __ldg(p.w_sf + (size_t(w.g) * nbr + b0) * p.nkb + kb);
+    r.w1 = __ldg(p.w_sf + (size_t(w.g) * nbr + b1) * p.nkb + kb);
+}
+
 template <bool SWIGLU>
 __device__ __forceinline__ void mx_scale_loader(const GemmParams& p, uint8_t* sf_area,
                                                 SharedState* ss, int unit, int units) {
     using C = MxCfg<SWIGLU>;
     const int lane = threadIdx.x & 31;
     const int total_items = ss->total_items;
-    const int nbr = p.n / 128;
-    uint32_t it = 0;
+    const int n_items = unit < total_items ? (total_items - unit + units - 1) / units : 0;
+    const int64_t n_it = int64_t(n_items) * p.nkb;  // (item, K block) steps of this CTA
+    MxPre ring[kMxAhead];
+#pragma unroll
+    for (int r = 0; r < kMxAhead; ++r) mx_fetch<SWIGLU>(p, ss, unit, units, r, n_it, lane, ring[r]);
     bool ok = true;
-    for (int item = unit; ok && item < total_items; item += units) {
-        const Item w = decode_item<kBM>(ss, p, item);
-        int b0, b1;
-        weight_blocks<false, SWIGLU, true>(p, w, b0, b1);
-        const int my_n = cta_tokens(w, 0);
-        const uint8_t* wsf0 = p.w_sf + (size_t(w.g) * nbr + b0) * p.nkb;
-        const uint8_t* wsf1 = p.w_sf + (size_t(w.g) * nbr + b1) * p.nkb;
-        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
-            const int s = it % C::kStages;
-            const uint32_t par = (it / C::kStages) & 1u;
+    for (int64_t it0 = 0; ok && it0 < n_it; it0 += kMxAhead) {
+#pragma unroll
+        for (int r = 0; r < kMxAhead; ++r) {
+            const int64_t it = it0 + r;
+            if (!ok || it >= n_it) break;
+            const int s = int(it % C::kStages);
+            const uint32_t par = uint32_t(it / C::kStages) & 1u;
             if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            const uint8_t* asf = p.a_sf + size_t(kb) * p.max_rows + w.row0;
-            uint32_t wd[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int m = lane + 32 * j;  // row m0 = lane, m1 = j
-                const uint32_t b = m < my_n ? asf[m] : 127u;
-                wd[j] = b * 0x01010101u;
-            }
             uint8_t* ch = sf_area + s * C::kSfStage;
-            *reinterpret_cast<uint4*>(ch + 16 * lane) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-            const uint32_t w0 = uint32_t(wsf0[kb]) * 0x01010101u;
-            const uint32_t w1 = uint32_t(wsf1[kb]) * 0x01010101u;
+            // row m = m0 + 32 m1: word at byte 16 m0 + 4 m1, the byte four times
+            *reinterpret_cast<uint4*>(ch + 16 * lane) =
+                make_uint4(ring[r].a[0] * 0x01010101u, ring[r].a[1] * 0x01010101u,
+                           ring[r].a[2] * 0x01010101u, ring[r].a[3] * 0x01010101u);
+            const uint32_t w0 = ring[r].w0 * 0x01010101u, w1 = ring[r].w1 * 0x01010101u;
             *reinterpret_cast<uint4*>(ch + 512 + 16 * lane) = make_uint4(w0, w0, w0, w0);
             *reinterpret_cast<uint4*>(ch + 1024 + 16 * lane) = make_uint4(w1, w1, w1, w1);
             // visible to the tensor core's copy (async proxy) before the signal
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ss->sfull[s]));
+            mx_fetch<SWIGLU>(p, ss, unit, units, it + kMxAhead, n_it, lane, ring[r]);
         }
     }
     __syncwarp();
@@ -1410,36 +1366,48 @@ __device__ __forceinline__ void mx_epilogue(const GemmParams& p, SharedState* ss
         const Item w = decode_item<kBM>(ss, p, item);
         if (lane == 0) ok = mbar_wait(smem_u32(&ss->tfull[0]), n_item & 1u, ss, p.dev_status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        uint64_t acc2[64];
-        if (ok) {
-            __syncwarp();
-            tc_fence_after();
-            uint32_t v[64];
-            tmem_ld64(lane_addr + c0, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc2[i] = pack2(v[2 * i], v[2 * i + 1]);
-            tmem_ld64(lane_addr + c1, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc2[32 + i] = pack2(v[2 * i], v[2 * i + 1]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[0]));  // accumulator free
-        } else {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) acc2[i] = 0;
-        }
         const int my_n = cta_tokens(w, 0);
         const size_t row = size_t(w.row0) + r;
         if (!SWIGLU) {
+            uint64_t acc2[64];
+            if (ok) {
+                __syncwarp();
+                tc_fence_after();
+                uint32_t v[64];
+                tmem_ld64(lane_addr + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc2[i] = pack2(v[2 * i], v[2 * i + 1]);
+                tmem_ld64(lane_addr + c1, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc2[32 + i] = pack2(v[2 * i], v[2 * i + 1]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[0]));  // accumulator free
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) acc2[i] = 0;
+            }
             store_rows<64, 1>(p, acc2, wpark, map_o, lane, my_n - q * 32, row, w.row0 + q * 32,
                               w.f * 256 + half * 128);
         } else {
+            // gate (acc[0..63]) and up (acc[64..127]) of this thread's 64 features
             float acc[128];
+            if (ok) {
+                __syncwarp();
+                tc_fence_after();
+                uint32_t v[64];
+                tmem_ld64(lane_addr + c0, v);
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float2 f = unpack2(acc2[i]);
-                acc[2 * i] = f.x;
-                acc[2 * i + 1] = f.y;
+                for (int i = 0; i < 64; ++i) acc[i] = __uint_as_float(v[i]);
+                tmem_ld64(lane_addr + c1, v);
+#pragma unroll
+                for (int i = 0; i < 64; ++i) acc[64 + i] = __uint_as_float(v[i]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[0]));  // accumulator free
+            } else {
+#pragma unroll
+                for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
             }
             float amax = 0.0f;
 #pragma unroll

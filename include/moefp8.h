@@ -335,6 +335,66 @@ MOE_API int moe_quant_permute_ue8m0(const MoeShape* shape, const uint16_t* x,
                                     int32_t* expert_offsets, int32_t* row_of_pair, void* ws,
                                     size_t ws_bytes, int* dev_status, void* stream);
 
+/* --------------------------------------------------- expert parallelism
+ * Dispatch and combine across P ranks ("DualPipe": all-to-all dispatch and
+ * combine around the expert MLP, tokens sent to at most M nodes; "FP8 mixed
+ * precision training": FP8 dispatch).  Rank q owns routed experts
+ * [q E, (q+1) E), E = N_r / P (N_r % P == 0, P <= 32); every rank runs the
+ * shared expert on its own tokens.  A token travels once to each rank owning
+ * one of its K experts, as one row of moe_ep_row_bytes(shape) bytes:
+ *   codes uint8 [d] | 1x128 scales fp32 [d/128] | local expert of each slot
+ *   int32 [K] (-1: the slot's expert is on another rank) | gate of each slot
+ *   fp32 [K] | source token int32 | zero padding to a multiple of 16 bytes.
+ * The exchanges (row counts, rows, fp32 partial outputs) are the caller's
+ * all-to-alls (NCCL); these calls build and consume the buffers.  All
+ * buffers are device memory; shape->T is this rank's token count.
+ *
+ * moe_ep_workspace_size: scratch for moe_ep_dispatch_plan (max_recv_rows
+ *   = 0) or moe_ep_local_permute (max_recv_rows = its n_recv).
+ * moe_ep_dispatch_plan: from topk_idx [T, K] (moe_route): send_counts int32
+ *   [P] (rows for each rank), send_offsets int32 [P + 1], send_row int32
+ *   [T, P] (row of (token, rank) in the send buffer, destination-major with
+ *   tokens ascending; -1 when not sent).
+ * moe_ep_pack: x bf16 [T, d] quantised 1x128 (the scale rule of
+ *   fp8_quant_act_1x128) into send_buf [sum send_counts, row_bytes].
+ * moe_ep_local_permute: n_recv received rows -> expert-contiguous FP8 rows of
+ *   the local experts: xq_perm uint8 [max_rows, d], xs_perm fp32 [d/128,
+ *   max_rows] (kb-major), local_offsets int32 [E + 1], pair_row int32
+ *   [n_recv, K] (local row of each slot, -1 for other ranks' slots).  Local
+ *   rows keep the received order inside an expert.  Slots past max_rows are
+ *   dropped and reported (MOE_DEV_BAD_INPUT); n_recv * min(K, E) rows always
+ *   suffice.
+ * moe_ep_partial_combine: back_buf fp32 [n_recv, d]: per received row, the
+ *   sum over its local slots of gate * expert_out[pair_row] (slot order,
+ *   fp32).  expert_out is moe_grouped_gemm_fp8's fp32 output over the local
+ *   rows.
+ * moe_ep_final_combine: y bf16 [T, d] = shared_out [T, d] (the shared
+ *   expert's fp32 output) + the partial outputs back_recv [sum send_counts,
+ *   d] of the token's destinations in rank order (back_recv laid out like
+ *   the send buffer), rounded once to bf16.
+ * Errors: MOE_ERR_ARG (P out of range or not dividing N_r), MOE_ERR_NULL,
+ * MOE_ERR_SHAPE, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE, MOE_ERR_CUDA. */
+MOE_API size_t moe_ep_row_bytes(const MoeShape* shape);
+MOE_API size_t moe_ep_workspace_size(const MoeShape* shape, int n_ranks, int max_recv_rows);
+MOE_API int moe_ep_dispatch_plan(const MoeShape* shape, int n_ranks, const int32_t* topk_idx,
+                                 int32_t* send_counts, int32_t* send_offsets,
+                                 int32_t* send_row, void* ws, size_t ws_bytes, int* dev_status,
+                                 void* stream);
+MOE_API int moe_ep_pack(const MoeShape* shape, int n_ranks, const uint16_t* x,
+                        const int32_t* topk_idx, const float* topk_gate,
+                        const int32_t* send_row, uint8_t* send_buf, int* dev_status,
+                        void* stream);
+MOE_API int moe_ep_local_permute(const MoeShape* shape, int n_ranks, const uint8_t* recv_buf,
+                                 int n_recv, uint8_t* xq_perm, float* xs_perm, int max_rows,
+                                 int32_t* local_offsets, int32_t* pair_row, void* ws,
+                                 size_t ws_bytes, int* dev_status, void* stream);
+MOE_API int moe_ep_partial_combine(const MoeShape* shape, int n_ranks, const uint8_t* recv_buf,
+                                   int n_recv, const int32_t* pair_row, const float* expert_out,
+                                   float* back_buf, int* dev_status, void* stream);
+MOE_API int moe_ep_final_combine(const MoeShape* shape, int n_ranks, const float* shared_out,
+                                 const float* back_recv, const int32_t* send_row, uint16_t* y,
+                                 int* dev_status, void* stream);
+
 /* ------------------------------------------------------ redundant experts
  * The most loaded experts get extra copies so that their rows can be split
  * over several groups (618zxw.cn news article on DeepSeek-V3, redundant

@@ -24,8 +24,12 @@ pytestmark = pytest.mark.gpu
 Y_TOL = 2e-3
 # Per token: both sides round y once to bf16, so a token's error is a few
 # one-step bf16 differences where the fp32 and FP64 sums straddle a rounding
-# boundary (and rare one-step h code differences); a wrong row gives ~1.
-Y_TOKEN_TOL = 1e-2
+# boundary, plus the rare h codes that land one E4M3 step apart (h is
+# re-quantised from FP32 on the GPU and from FP64 in the oracle; one step is
+# 6-12% of that h value, and on a token with a small output it moves y by
+# up to about a percent: the worst token of the 16384 skewed-batch tokens is
+# at 1.07e-2).  A wrong row gives an error of order 1.
+Y_TOKEN_TOL = 5e-2
 
 
 def build_layer(cfg, T=None, host_io=False):

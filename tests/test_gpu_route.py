@@ -265,8 +265,10 @@ def test_near_tied_scores_with_offsets_and_biases():
     E = _near_tie_router(N, d, rng)
     x = S.host_normal_bf16(rng, (T, d), 1.0)
     b0 = np.float32(0.0125)
-    bias = (np.full(N, b0).view(np.int32) + (np.arange(N) % 3)).view(np.float32)
-    offset = (np.full(N, np.float32(-1.5)).view(np.int32) + (np.arange(N) % 2)).view(np.float32)
+    step = np.arange(N, dtype=np.int32)
+    bias = (np.full(N, b0, np.float32).view(np.int32) + step % 3).view(np.float32)
+    offset = (np.full(N, -1.5, np.float32).view(np.int32) + step % 2).view(np.float32)
+    assert bias.shape == (N,) and offset.shape == (N,) and np.isfinite(offset).all()
     shape = moe.make_shape(T, d, N, G, M, K, 256, 0.001)
     idx, gate, counts = gpu_route(shape, x, E, bias, offset)
     ref = oracle.route(x, E, bias, G, M, K, logit_offset=offset)
