@@ -22,6 +22,7 @@ __all__ = [
     "quantized_expert", "layer_forward", "gemm_blockscaled",
     "quant_act_1x128_pow2", "quant_w_128x128_pow2", "pow2_scales",
     "redundant_plan", "split_groups", "quantized_expert_pow2", "quant_act_1x128_pow2_values",
+    "gate_backward", "router_backward", "expert_backward", "layer_backward", "swiglu_backward",
 ]
 
 _LIB = None
@@ -400,3 +401,127 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
 def gemm_blockscaled(aq, a_s, bq, b_s):
     """C = dq(A) dq(B)^T in FP64; A [m,k] 1x128-scaled, B [n,k] 128x128-scaled."""
     return dequant_act(aq, a_s) @ dequant_w(bq, b_s).T
+
+
+# ---------------------------------------------------------------- backward
+# The gradient of the layer with respect to x and the router weights for an
+# upstream gradient dy ("DeepSeek-V3 Technical Report" notes page, section
+# "FP8 mixed precision training": the Fprop, Dgrad and Wgrad GEMMs run in
+# FP8, gating stays in high precision; section "DeepSeekMoE and
+# auxiliary-loss-free load balancing": gates are the normalised unbiased
+# affinities of the selected experts, the bias only selects).  Readings:
+#   - the selection is piecewise constant: no gradient flows through the
+#     top-K choice or the bias;
+#   - gates g_k = s_k / S with S the sum of the chosen s: dL/ds_j =
+#     (dg_j - sum_k g_k dg_k) / S for chosen j; dL/du_j = dL/ds_j s_j (1-s_j);
+#   - the expert MLP's Dgrad GEMMs take FP8 operands quantised like the
+#     forward's: do = g dy (fp32 product) per routed row (dy for the shared
+#     row) in 1x128 tiles along d, and [da | dc] in 1x128 tiles along 2I;
+#     the weights keep their 128x128 blocks, transposed (exact);
+#   - SwiGLU derivative: silu'(a) = sigma(a) (1 + a (1 - sigma(a))).
+
+def gate_backward(dy_bf16: np.ndarray, o_routed: np.ndarray, scores: np.ndarray):
+    """dg [T,K] = <dy_t, o_tk>, du [T,K] = dL/du of the chosen logits.
+    o_routed: FP64 [T,K,d] routed expert outputs; scores: fp32 [T,K] the
+    chosen experts' unbiased s."""
+    dy = _bf16_to_f64(dy_bf16)
+    dg = np.einsum("td,tkd->tk", dy, o_routed)
+    s = scores.astype(np.float64)
+    S = s.sum(axis=1, keepdims=True)
+    g = s / S
+    ds = (dg - (g * dg).sum(axis=1, keepdims=True)) / S
+    du = ds * s * (1.0 - s)
+    return dg, du
+
+
+def router_backward(du: np.ndarray, topk_idx: np.ndarray, x_bf16: np.ndarray,
+                    router_w_bf16: np.ndarray):
+    """dx_router [T,d] = sum_k du_tk E_{e_k};  dE [N_r,d] = sum du_tk x_t."""
+    x = _bf16_to_f64(x_bf16)
+    E = _bf16_to_f64(router_w_bf16)
+    dx = np.einsum("tk,tkd->td", du, E[topk_idx])
+    dE = np.zeros_like(E)
+    np.add.at(dE, topk_idx.ravel(), (du[:, :, None] * x[:, None, :]).reshape(-1, x.shape[1]))
+    return dx, dE
+
+
+def swiglu_backward(dh, a, c):
+    """h = silu(a) c:  da = dh c silu'(a) with silu'(a) = sigma(a) (1 + a (1 -
+    sigma(a))), dc = dh silu(a); FP64."""
+    a = np.asarray(a, np.float64)
+    sig = 1.0 / (1.0 + np.exp(-a))
+    da = np.asarray(dh, np.float64) * np.asarray(c, np.float64) * sig * (1.0 + a * (1.0 - sig))
+    dc = np.asarray(dh, np.float64) * a * sig
+    return da, dc
+
+
+def expert_backward(do_rows_f32: np.ndarray, xq: np.ndarray, xs: np.ndarray, w1, w3, w2,
+                    quant: bool = True):
+    """Dgrad through one expert for its rows: do (fp32 [rows, d], the
+    gate-scaled dy) quantised 1x128 -> dh = dq(do) W2 (FP64); a, c
+    recomputed from the forward's FP8 x; da = dh c silu'(a), dc = dh silu(a)
+    rounded to fp32 and quantised 1x128 along [da | dc]; dx = dq([da|dc])
+    [W1; W3] (FP64).  Returns dx [rows, d] FP64.
+    quant=False (for checks against derivatives): no quantisation of do and
+    [da | dc], and xq is taken as the FP64 input itself (xs ignored)."""
+    W1, W3, W2 = dequant_w(*w1), dequant_w(*w3), dequant_w(*w2)
+    if quant:
+        dq_, ds_ = quant_act_1x128(np.ascontiguousarray(do_rows_f32, np.float32))
+        dh = dequant_act(dq_, ds_) @ W2
+        X = dequant_act(xq, xs)
+    else:
+        dh = np.asarray(do_rows_f32, np.float64) @ W2
+        X = np.asarray(xq, np.float64)
+    a, c = X @ W1.T, X @ W3.T
+    dac = np.concatenate(swiglu_backward(dh, a, c), axis=1)
+    if quant:
+        qq, qs = quant_act_1x128(dac.astype(np.float32))
+        dac = dequant_act(qq, qs)
+    return dac @ np.concatenate([W1, W3], axis=0)
+
+
+def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def layer_backward(dy_bf16, x_bf16, router_w_bf16, bias, n_groups, topk_groups, topk,
+                   expert_weights, logit_offset=None, quant=True):
+    """dx [T,d] (FP64) and dE [N_r,d] (FP64) of the whole layer for dy.
+    quant=False (for checks against derivatives): the experts take x itself
+    and nothing is quantised (the routing is the same)."""
+    T, d = x_bf16.shape
+    n_routed = router_w_bf16.shape[0]
+    r = route(x_bf16, router_w_bf16, bias, n_groups, topk_groups, topk, logit_offset,
+              want_scores=True)
+    idx = r["topk_idx"]
+    scores = np.take_along_axis(r["scores"], idx, axis=1)
+    xq, xs = quant_act_1x128(x_bf16)
+    dy32 = _bf16_to_f64(dy_bf16).astype(np.float32)
+    gates = r["topk_gate"]
+    o_routed = np.zeros((T, topk, d))
+    dx = np.zeros((T, d))
+    for e in range(n_routed + 1):
+        if e == n_routed:
+            sel, slots = np.arange(T), None
+            do = dy32
+        else:
+            sel, slots = np.nonzero(idx == e)
+            if sel.size == 0:
+                continue
+            do = (gates[sel, slots].astype(np.float32)[:, None] * dy32[sel]).astype(np.float32)
+        w = expert_weights(e)
+        if quant:
+            if slots is not None:
+                o_routed[sel, slots] = swiglu_expert(xq[sel], xs[sel], *w)
+            dx[sel] += expert_backward(do, xq[sel], xs[sel], *w)
+        else:
+            X = _bf16_to_f64(x_bf16[sel])
+            if slots is not None:
+                W1, W3, W2 = (dequant_w(*m) for m in w)
+                a, c = X @ W1.T, X @ W3.T
+                o_routed[sel, slots] = (a / (1.0 + np.exp(-a)) * c) @ W2.T
+            dx[sel] += expert_backward(do, X, None, *w, quant=False)
+    dg, du = gate_backward(dy_bf16, o_routed, scores)
+    dxr, dE = router_backward(du, idx, x_bf16, router_w_bf16)
+    return {"dx": dx + dxr, "dE": dE, "dg": dg, "du": du, "topk_idx": idx, "scores": scores}
