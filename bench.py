@@ -921,6 +921,129 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_backward(args, world, rank, local):
+    """The layer's backward pass (dx and the router gradient for an upstream
+    gradient dy) on the workload's batch: forward_train once, then timed
+    backward calls with dy resident in HBM; beside it end to end with dy
+    copied in from pinned host memory and dx copied out every step."""
+    import numpy as np
+    import torch
+    import synthetic as S
+
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.CONFIGS[args.workload]
+    peaks, peak_src = load_peaks()
+    layer, x, off, inp, _ = build_layer(cfg, dev)
+    st = torch.cuda.current_stream()
+    layer.forward_train(x, logit_offset=off)
+    T, d, I, K = cfg.T, cfg.d, cfg.inter, cfg.topk
+    dy_host = torch.from_numpy(S.host_normal_bf16(np.random.default_rng(cfg.seed + 100),
+                                                  (T, d), 1.0).view(np.int16)).view(
+        torch.bfloat16).pin_memory()
+    dy = dy_host.to(dev)
+    for _ in range(args.warmup):
+        layer.backward(dy)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(args.steps):
+        layer.backward(dy)
+    ev1.record(st)
+    ev1.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    status = layer.status()
+    tokens_total = T * args.steps * world
+
+    # end to end: dy in from pinned host memory, dx out, every step
+    dx_host = torch.empty((T, d), dtype=torch.float32).pin_memory()
+    dy_dev = torch.empty_like(dy)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        dy_dev.copy_(dy_host, non_blocking=True)
+        dx, _dE = layer.backward(dy_dev)
+        dx_host.copy_(dx, non_blocking=True)
+    e1.record(st)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    # per-stage times (events between the stages, same launches)
+    tot = {}
+    for it in range(args.steps + 2):
+        marks = []
+        layer.backward(dy, marks=marks)
+        marks[-1][1].synchronize()
+        if it >= 2:
+            for (_, a), (n, b) in zip(marks[:-1], marks[1:]):
+                tot[n] = tot.get(n, 0.0) + a.elapsed_time(b)
+    brk = {n: v / args.steps for n, v in tot.items()}
+    R = T * K + T
+    flops = {"gemm_dh": 2.0 * R * d * I, "gemm_ac_recompute": 2.0 * R * d * 2 * I,
+             "gemm_dx": 2.0 * R * 2 * I * d}
+    top = max(flops, key=lambda n: brk[n])
+    fp8_peak = float(peaks["bf16_tflops"]) * FP8_PER_BF16
+    ach = flops[top] / (brk[top] / 1e3) / 1e12
+    gemm_ms = sum(brk[n] for n in flops)
+    hbm_peak = float(peaks["hbm_gbs"])
+    mem_bytes = {
+        "combine_backward_quant": T * d * 2 + R * d + R * (d // 128) * 4,
+        "swiglu_backward_quant": R * I * 4 + R * 2 * I * 4 + R * 2 * I + R * (2 * I // 128) * 4,
+        "gate_backward": T * K * d * 4 + T * d * 2,
+        "dx_combine": R * d * 4 + T * d * 4 + T * d * 4,
+    }
+    line = {
+        "metric": "backward_tokens_per_s",
+        "value": tokens_total / (ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3/f32",
+        "data": "synthetic",
+        "config": {"workload": f"moe_layer_backward_{cfg.name}", "T": T, "d": d,
+                   "n_routed": cfg.n_routed, "topk": K, "inter": I,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (FP8 weights and their transposes, "
+                         "fp32 row buffers of several GB)"},
+        "roofline": {"bound": "tensor", "kernel": f"grouped_gemm ({top})", "achieved": ach,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": ach / fp8_peak,
+                     "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g}",
+                     "traffic": None, "algorithmic_flops_per_launch": flops[top],
+                     "launch_ms": brk[top],
+                     "frac_of_datasheet": ach / DATASHEET["fp8_tflops"]},
+        "dgrad_gemms": {"tflops": sum(flops.values()) / (gemm_ms / 1e3) / 1e12,
+                        "frac_of_fp8_peak": sum(flops.values()) / (gemm_ms / 1e3) / 1e12
+                        / fp8_peak, "ms": gemm_ms},
+        "memory_passes": {n: {"ms": brk[n], "gbs": b / (brk[n] / 1e3) / 1e9,
+                              "frac_of_hbm": b / (brk[n] / 1e3) / 1e9 / hbm_peak}
+                          for n, b in mem_bytes.items()},
+        "breakdown_ms": brk,
+        "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4,
+                "api": "MoeLayer.backward with dy copied in and dx copied out each step"},
+        # combine quant 1, GEMMs 3, SwiGLU quant 1, gate 1, router 3, dx 1
+        "gpu_launches": 10 * args.steps,
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -934,6 +1057,8 @@ def main(argv=None):
     ap.add_argument("--scales", choices=["fp32", "ue8m0"], default="fp32",
                     help="fp32: the pages' recipe (default); ue8m0: the power-of-two scale "
                          "option with block-scaled tensor-core GEMMs")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
+                    help="backward: time the layer's backward pass (dx, router gradient)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -945,6 +1070,8 @@ def main(argv=None):
             run_gemm(args, world, rank, local)
         elif args.workload == "route":
             run_route(args, world, rank, local)
+        elif args.which == "backward":
+            run_backward(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -26,7 +26,10 @@ from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QU
                    MoeWeightsMx, make_weights_mx, moe_layer_forward_mx,
                    moe_layer_mx_workspace_size, moe_quant_permute_ue8m0,
                    moe_ep_row_bytes, moe_ep_workspace_size, moe_ep_dispatch_plan, moe_ep_pack,
-                   moe_ep_local_permute, moe_ep_partial_combine, moe_ep_final_combine)
+                   moe_ep_local_permute, moe_ep_partial_combine, moe_ep_final_combine,
+                   moe_route_scores, fp8_transpose_w_128x128, moe_combine_backward_quant,
+                   moe_swiglu_backward_quant, moe_gate_backward, moe_router_backward,
+                   moe_dx_combine)
 
 __all__ = ["MoeLayer", "MoeShape", "MoeError", "lib", "make_shape", "moe_version"]
 
@@ -77,6 +80,8 @@ class MoeLayer:
                     else moe_layer_workspace_size(shape))
         self.ws = torch.empty((max(ws_bytes, 256),), dtype=u8, device=dev)
         self._weights = None
+        self._transposed = None
+        self._train = None
         self._routing = make_routing(self.topk_idx, self.topk_gate, self.expert_counts,
                                      self.expert_offsets, self.row_of_pair)
 
@@ -90,6 +95,7 @@ class MoeLayer:
         quant(w3, self.w13[e, I:], self.w13_scales[e, I // 128:], stream=stream)
         quant(w2, self.w2[e], self.w2_scales[e], stream=stream)
         self._weights = None
+        self._transposed = None
 
     def weights(self):
         if self._weights is None:
@@ -124,6 +130,149 @@ class MoeLayer:
         moe_layer_forward_host_batches(self.shape, self.weights(), x_host, x_host.shape[0],
                                        self.bias, logit_offset, self._routing, y_host,
                                        update_bias, self.ws, self.dev_status, stream)
+
+    # ------------------------------------------------------------ training
+    def _train_buffers(self):
+        import torch
+        if self._train is None:
+            sh, dev = self.shape, self.device
+            T, d, I, K = sh.T, sh.d, sh.inter, sh.topk
+            R = T * K + T
+            u8, f32, i32 = torch.uint8, torch.float32, torch.int32
+            self._train = {
+                "score": torch.empty((T, K), dtype=f32, device=dev),
+                "route_ws": torch.empty((max(moe_route_workspace_size(sh), 256),), dtype=u8,
+                                        device=dev),
+                "perm_ws": torch.empty((max(moe_permute_workspace_size(sh), 256),), dtype=u8,
+                                       device=dev),
+                "xq": torch.empty((R, d), dtype=u8, device=dev),
+                "xs": torch.empty((d // 128, R), dtype=f32, device=dev),
+                "hq": torch.empty((R, I), dtype=u8, device=dev),
+                "hs": torch.empty((I // 128, R), dtype=f32, device=dev),
+                "o": torch.empty((R, d), dtype=f32, device=dev),
+                "x": None,
+            }
+        return self._train
+
+    def forward_train(self, x, y=None, update_bias: bool = False, logit_offset=None,
+                      stream=None):
+        """The forward pass (fp32-scale recipe) through the stage entry points,
+        keeping what backward() needs: the chosen affinities, the permuted FP8
+        rows and the expert outputs.  y equals forward()'s bit for bit; x
+        must stay unchanged until backward() has run."""
+        import torch
+        if self.scales != "fp32":
+            raise ValueError("the backward pass uses the fp32-scale layer")
+        sh, b = self.shape, self._train_buffers()
+        N, d, I, K, T = sh.n_routed, sh.d, sh.inter, sh.topk, sh.T
+        R = T * K + T
+        if y is None:
+            y = torch.empty_like(x)
+        st = self.dev_status
+        moe_route_scores(sh, x, self.router_w, self.bias, logit_offset, self.topk_idx,
+                         self.topk_gate, b["score"], self.expert_counts, b["route_ws"], st,
+                         stream)
+        moe_quant_permute(sh, x, self.topk_idx, self.expert_counts, b["xq"], b["xs"],
+                          self.expert_offsets, self.row_of_pair, b["perm_ws"], st, stream)
+        moe_grouped_gemm_fp8(N + 1, self.expert_offsets, R, b["xq"], b["xs"], d, self.w13,
+                             self.w13_scales, 2 * I, MOE_EPI_SWIGLU_QUANT, b["hq"], b["hs"], st,
+                             stream)
+        moe_grouped_gemm_fp8(N + 1, self.expert_offsets, R, b["hq"], b["hs"], I, self.w2,
+                             self.w2_scales, d, MOE_EPI_F32, b["o"], None, st, stream)
+        moe_combine(sh, b["o"], self.expert_offsets, self.row_of_pair, self.topk_gate, y, st,
+                    stream)
+        if update_bias:
+            moe_update_bias(sh, self.expert_counts, self.bias, st, stream)
+        b["x"] = x
+        return y
+
+    def _transposed_weights(self, stream=None):
+        """W2 and W13 with rows and columns swapped (the Dgrad GEMMs' B
+        operands): the same FP8 codes and 128x128 scales, moved."""
+        import torch
+        if self._transposed is None:
+            sh, dev = self.shape, self.device
+            E, d, I = sh.n_routed + 1, sh.d, sh.inter
+            u8, f32 = torch.uint8, torch.float32
+            w2t = torch.empty((E, I, d), dtype=u8, device=dev)
+            w2t_s = torch.empty((E, I // 128, d // 128), dtype=f32, device=dev)
+            w13t = torch.empty((E, d, 2 * I), dtype=u8, device=dev)
+            w13t_s = torch.empty((E, d // 128, 2 * I // 128), dtype=f32, device=dev)
+            fp8_transpose_w_128x128(self.w2, self.w2_scales, w2t, w2t_s, self.dev_status, stream)
+            fp8_transpose_w_128x128(self.w13, self.w13_scales, w13t, w13t_s, self.dev_status,
+                                    stream)
+            self._transposed = (w2t, w2t_s, w13t, w13t_s)
+        return self._transposed
+
+    def backward(self, dy, stream=None, marks=None):
+        """Gradients of the last forward_train() for the upstream gradient dy
+        (bf16 [T, d]): returns (dx fp32 [T, d], d_router_w fp32 [N_r, d]).
+
+        Dgrad through the experts with FP8 operands (the gate-scaled output
+        gradient and [da | dc] quantised in 1x128 tiles, the weights' own
+        128x128 blocks transposed), a and c recomputed from the forward's FP8
+        rows; the gate and router gradients in high precision.  The top-K
+        choice and the bias carry no gradient.
+
+        marks: a list, or None; given a list, a timing CUDA event recorded on
+        the stream after each stage is appended as (stage name, event), with
+        ("start", event) first."""
+        import torch
+        b = self._train
+        if b is None or b["x"] is None:
+            raise RuntimeError("backward() needs a forward_train() first")
+        sh, dev, st = self.shape, self.device, self.dev_status
+        N, d, I, K, T = sh.n_routed, sh.d, sh.inter, sh.topk, sh.T
+        R = T * K + T
+        u8, f32, i32 = torch.uint8, torch.float32, torch.int32
+        w2t, w2t_s, w13t, w13t_s = self._transposed_weights(stream)
+        cuda_stream = (torch.cuda.current_stream(dev) if stream is None else
+                       torch.cuda.ExternalStream(stream) if isinstance(stream, int) else stream)
+
+        def mark(name):
+            if marks is not None:
+                ev = torch.cuda.Event(enable_timing=True)
+                ev.record(cuda_stream)
+                marks.append((name, ev))
+        mark("start")
+        off = self.expert_offsets
+        do_q = torch.empty((R, d), dtype=u8, device=dev)
+        do_s = torch.empty((d // 128, R), dtype=f32, device=dev)
+        moe_combine_backward_quant(sh, dy, self.row_of_pair, self.topk_gate, do_q, do_s, st,
+                                   stream)
+        mark("combine_backward_quant")
+        dh = torch.empty((R, I), dtype=f32, device=dev)
+        moe_grouped_gemm_fp8(N + 1, off, R, do_q, do_s, d, w2t, w2t_s, I, MOE_EPI_F32, dh, None,
+                             st, stream)
+        mark("gemm_dh")
+        ac = torch.empty((R, 2 * I), dtype=f32, device=dev)
+        moe_grouped_gemm_fp8(N + 1, off, R, b["xq"], b["xs"], d, self.w13, self.w13_scales,
+                             2 * I, MOE_EPI_F32, ac, None, st, stream)
+        mark("gemm_ac_recompute")
+        gq = torch.empty((R, 2 * I), dtype=u8, device=dev)
+        gs = torch.empty((2 * I // 128, R), dtype=f32, device=dev)
+        moe_swiglu_backward_quant(dh, ac, R, I, R, gq, gs, st, stream)
+        mark("swiglu_backward_quant")
+        del dh, ac
+        dx_rows = torch.empty((R, d), dtype=f32, device=dev)
+        moe_grouped_gemm_fp8(N + 1, off, R, gq, gs, 2 * I, w13t, w13t_s, d, MOE_EPI_F32,
+                             dx_rows, None, st, stream)
+        mark("gemm_dx")
+        dgate = torch.empty((T, K), dtype=f32, device=dev)
+        du = torch.empty((T, K), dtype=f32, device=dev)
+        moe_gate_backward(sh, dy, b["o"], self.row_of_pair, b["score"], dgate, du, st, stream)
+        mark("gate_backward")
+        dx_router = torch.empty((T, d), dtype=f32, device=dev)
+        d_router_w = torch.empty((N, d), dtype=f32, device=dev)
+        pair_scratch = torch.empty((max(T * K, 1),), dtype=i32, device=dev)
+        moe_router_backward(sh, b["x"], self.router_w, du, self.topk_idx, off, self.row_of_pair,
+                            pair_scratch, dx_router, d_router_w, st, stream)
+        mark("router_backward")
+        dx = torch.empty((T, d), dtype=f32, device=dev)
+        moe_dx_combine(sh, dx_rows, dx_router, self.row_of_pair, dx, st, stream)
+        mark("dx_combine")
+        self.last_dgate, self.last_du = dgate, du
+        return dx, d_router_w
 
     def status(self, stream=None) -> int:
         """Device status word (0 = fine); synchronises the stream."""

@@ -71,6 +71,13 @@ def lib() -> ctypes.CDLL:
             "moe_read_status": (I, [P, P, P]),
             "moe_route_workspace_size": (SZ, [SP]),
             "moe_route": (I, [SP, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "moe_route_scores": (I, [SP, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "fp8_transpose_w_128x128": (I, [P, P, I64, I64, I64, P, P, P, P]),
+            "moe_combine_backward_quant": (I, [SP, P, P, P, P, P, P, P]),
+            "moe_swiglu_backward_quant": (I, [P, P, I64, I, I64, P, P, P, P]),
+            "moe_gate_backward": (I, [SP, P, P, P, P, P, P, P, P]),
+            "moe_router_backward": (I, [SP, P, P, P, P, P, P, P, P, P, P, P]),
+            "moe_dx_combine": (I, [SP, P, P, P, P, P, P]),
             "fp8_quant_act_1x128": (I, [P, I64, I64, P, P, I, P, P]),
             "fp8_quant_w_128x128": (I, [P, I64, I64, P, P, P, P]),
             "moe_permute_workspace_size": (SZ, [SP]),
@@ -171,6 +178,16 @@ def moe_route(shape, x, router_w, bias, logit_offset, topk_idx, topk_gate, exper
         ctypes.byref(shape), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(logit_offset),
         _ptr(topk_idx), _ptr(topk_gate), _ptr(expert_counts), _ptr(ws), nbytes,
         _ptr(dev_status), _stream(stream)))
+
+
+def moe_route_scores(shape, x, router_w, bias, logit_offset, topk_idx, topk_gate, topk_score,
+                     expert_counts, ws, dev_status=None, stream=None) -> None:
+    """moe_route that also returns the chosen unbiased affinities (topk_score)."""
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("moe_route_scores", lib().moe_route_scores(
+        ctypes.byref(shape), _ptr(x), _ptr(router_w), _ptr(bias), _ptr(logit_offset),
+        _ptr(topk_idx), _ptr(topk_gate), _ptr(topk_score), _ptr(expert_counts), _ptr(ws),
+        nbytes, _ptr(dev_status), _stream(stream)))
 
 
 def fp8_quant_act_1x128(x, q, scales, scales_kb_major=False, dev_status=None, stream=None):
@@ -426,3 +443,49 @@ def moe_ep_final_combine(shape, n_ranks, shared_out, back_recv, send_row, y, dev
     _check("moe_ep_final_combine", lib().moe_ep_final_combine(
         ctypes.byref(shape), int(n_ranks), _ptr(shared_out), _ptr(back_recv), _ptr(send_row),
         _ptr(y), _ptr(dev_status), _stream(stream)))
+
+
+# ------------------------------------------------------------- backward
+def fp8_transpose_w_128x128(q, scales, qt, scales_t, dev_status=None, stream=None):
+    """q uint8 [mats, rows, cols] (or [rows, cols]), scales fp32
+    [mats, rows/128, cols/128] -> the transposed codes and scales."""
+    rows, cols = q.shape[-2], q.shape[-1]
+    mats = q.numel() // max(rows * cols, 1) if rows * cols else 0
+    _check("fp8_transpose_w_128x128", lib().fp8_transpose_w_128x128(
+        _ptr(q), _ptr(scales), int(mats), int(rows), int(cols), _ptr(qt), _ptr(scales_t),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_combine_backward_quant(shape, dy, row_of_pair, topk_gate, do_q, do_scales,
+                               dev_status=None, stream=None):
+    _check("moe_combine_backward_quant", lib().moe_combine_backward_quant(
+        ctypes.byref(shape), _ptr(dy), _ptr(row_of_pair), _ptr(topk_gate), _ptr(do_q),
+        _ptr(do_scales), _ptr(dev_status), _stream(stream)))
+
+
+def moe_swiglu_backward_quant(dh, ac, rows, inter, rows_total, q, q_scales, dev_status=None,
+                              stream=None):
+    _check("moe_swiglu_backward_quant", lib().moe_swiglu_backward_quant(
+        _ptr(dh), _ptr(ac), int(rows), int(inter), int(rows_total), _ptr(q), _ptr(q_scales),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_gate_backward(shape, dy, expert_out, row_of_pair, topk_score, dgate, du,
+                      dev_status=None, stream=None):
+    _check("moe_gate_backward", lib().moe_gate_backward(
+        ctypes.byref(shape), _ptr(dy), _ptr(expert_out), _ptr(row_of_pair), _ptr(topk_score),
+        _ptr(dgate), _ptr(du), _ptr(dev_status), _stream(stream)))
+
+
+def moe_router_backward(shape, x, router_w, du, topk_idx, expert_offsets, row_of_pair,
+                        pair_scratch, dx_router, d_router_w, dev_status=None, stream=None):
+    _check("moe_router_backward", lib().moe_router_backward(
+        ctypes.byref(shape), _ptr(x), _ptr(router_w), _ptr(du), _ptr(topk_idx),
+        _ptr(expert_offsets), _ptr(row_of_pair), _ptr(pair_scratch), _ptr(dx_router),
+        _ptr(d_router_w), _ptr(dev_status), _stream(stream)))
+
+
+def moe_dx_combine(shape, dx_rows, dx_router, row_of_pair, dx, dev_status=None, stream=None):
+    _check("moe_dx_combine", lib().moe_dx_combine(
+        ctypes.byref(shape), _ptr(dx_rows), _ptr(dx_router), _ptr(row_of_pair), _ptr(dx),
+        _ptr(dev_status), _stream(stream)))

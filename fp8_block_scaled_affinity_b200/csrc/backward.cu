@@ -1,0 +1,490 @@
+// Backward pass of the MoE layer with respect to x and the router weights
+// ("DeepSeek-V3 Technical Report" notes page, section "FP8 mixed precision
+// training": the Dgrad GEMMs take FP8 operands with fine-grained scales,
+// gating stays in high precision; section "DeepSeekMoE and
+// auxiliary-loss-free load balancing": gates are the normalised unbiased
+// affinities of the chosen experts, the bias only selects, so no gradient
+// flows through the choice or the bias).
+//
+// For an upstream gradient dy of y:
+//   1. moe_combine_backward_quant: do = g_k dy (fp32 product) for each
+//      routed row, dy for the shared row, quantised in 1x128 tiles along d
+//      (the forward's activation rule) into the permuted row order;
+//   2. dh = do W2 (grouped FP8 GEMM on the transposed W2, k = d);
+//   3. a, c recomputed (grouped GEMM on W13 with fp32 output, k = d);
+//   4. moe_swiglu_backward_quant: da = dh c silu'(a), dc = dh silu(a),
+//      [da | dc] quantised in 1x128 tiles along 2I;
+//   5. dx rows = [da | dc] [W1; W3] (grouped FP8 GEMM on the transposed W13,
+//      k = 2I);
+//   6. moe_gate_backward: dg_k = <dy, o_k>, dL/ds_j = (dg_j - sum_k g_k dg_k)
+//      / S over the chosen experts, dL/du_j = dL/ds_j s_j (1 - s_j) (FP64);
+//   7. moe_router_backward: dx_router[t] = sum_k du_tk E[e_k] and
+//      dE[e] = sum over the expert's tokens of du x (fp32, fixed order);
+//   8. moe_dx_combine: dx[t] = shared row + routed rows + dx_router[t].
+// fp8_transpose_w_128x128 gives the transposed weights: a 128x128 block's
+// codes move and its scale stays, so the transposed matrix holds the same
+// values (the transposed-GEMM need the pages raise in their discussion).
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+int warp_blocks(int64_t units) {
+    const int64_t cap = int64_t(sm_count()) * 8;
+    return int(std::max<int64_t>(1, std::min<int64_t>((units + 7) / 8, cap)));
+}
+
+// ------------------------------------------- 1. do rows, quantised 1x128
+// A warp per (token, piece of 2P tiles): dy read once in bf16; for every
+// destination row the values g * dy (fp32) are quantised with the forward's
+// rule (a half-warp per 1x128 tile) and written to that row.
+template <int PC>
+__global__ void __launch_bounds__(256) combine_backward_quant_kernel(
+    const uint4* __restrict__ dy, int T, int d, int K, const int32_t* __restrict__ row_of_pair,
+    const float* __restrict__ gate, int64_t rows_total, uint2* __restrict__ dq,
+    float* __restrict__ ds) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = d / 8, nkb = d / 128;
+    const int pieces = (nvec + 32 * PC - 1) / (32 * PC);
+    const int64_t units = int64_t(T) * pieces;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t un = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); un < units;
+         un += warps_total) {
+        const int t = int(un / pieces);
+        const int c0 = int(un - int64_t(t) * pieces) * (32 * PC);
+        int my_row = 0;
+        float my_g = 1.0f;
+        if (lane < K) {
+            my_row = row_of_pair[int64_t(t) * K + lane];
+            my_g = gate[int64_t(t) * K + lane];
+        }
+        uint4 v[PC];
+#pragma unroll
+        for (int j = 0; j < PC; ++j) {
+            const int c = c0 + lane + 32 * j;
+            v[j] = c < nvec ? __ldg(dy + int64_t(t) * nvec + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const int tile = c0 / 16 + lane;
+        for (int k = 0; k <= K; ++k) {
+            const int row = k < K ? __shfl_sync(0xffffffffu, my_row, k) : T * K + t;
+            const float g = k < K ? __shfl_sync(0xffffffffu, my_g, k) : 1.0f;
+            if (row < 0) continue;
+            float tile_scale = 1.0f;
+#pragma unroll
+            for (int j = 0; j < PC; ++j) {
+                const uint4 w = v[j];
+                float f[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                              bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    f[i] = __fmul_rn(g, f[i]);
+                    amax = fmaxf(amax, fabsf(f[i]));
+                }
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                float scale, inv;
+                scale_from_amax(amax, scale, inv);
+                const uint32_t a0 = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv));
+                const uint32_t a1 = e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
+                const uint32_t a2 = e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv));
+                const uint32_t a3 = e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv));
+                const int c = c0 + lane + 32 * j;
+                if (c < nvec) dq[int64_t(row) * nvec + c] = make_uint2(a0 | (a1 << 16), a2 | (a3 << 16));
+                const float sj = __shfl_sync(0xffffffffu, scale, (lane & 1) * 16);
+                if ((lane >> 1) == j) tile_scale = sj;
+            }
+            if (lane < 2 * PC && tile < nkb) ds[int64_t(tile) * rows_total + row] = tile_scale;
+        }
+    }
+}
+
+// ------------------------------------------- 4. SwiGLU backward, quantised
+// A warp per (row, piece of 2P tiles of the 2I-wide row [da | dc]).
+template <int PC>
+__global__ void __launch_bounds__(256) swiglu_backward_quant_kernel(
+    const float* __restrict__ dh, const float* __restrict__ ac, int64_t rows, int I,
+    int64_t rows_total, uint2* __restrict__ q, float* __restrict__ qs) {
+    const int lane = threadIdx.x & 31;
+    const int n2 = 2 * I;
+    const int nvec = n2 / 8, nkb = n2 / 128;
+    const int pieces = (nvec + 32 * PC - 1) / (32 * PC);
+    const int64_t units = rows * pieces;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t un = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); un < units;
+         un += warps_total) {
+        const int64_t r = un / pieces;
+        const int c0 = int(un - r * pieces) * (32 * PC);
+        const float* dhr = dh + r * I;
+        const float* ar = ac + r * n2;
+        float tile_scale = 1.0f;
+#pragma unroll
+        for (int j = 0; j < PC; ++j) {
+            const int c = c0 + lane + 32 * j;  // vector of 8 values of [da | dc]
+            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (c < nvec) {
+                const int col = 8 * c;
+                const bool is_da = col < I;
+                const int feat = is_da ? col : col - I;
+                const float4 h0 = *reinterpret_cast<const float4*>(dhr + feat);
+                const float4 h1 = *reinterpret_cast<const float4*>(dhr + feat + 4);
+                const float4 a0 = *reinterpret_cast<const float4*>(ar + feat);
+                const float4 a1 = *reinterpret_cast<const float4*>(ar + feat + 4);
+                const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                float cv[8];
+                if (is_da) {
+                    const float4 u0 = *reinterpret_cast<const float4*>(ar + I + feat);
+                    const float4 u1 = *reinterpret_cast<const float4*>(ar + I + feat + 4);
+                    cv[0] = u0.x; cv[1] = u0.y; cv[2] = u0.z; cv[3] = u0.w;
+                    cv[4] = u1.x; cv[5] = u1.y; cv[6] = u1.z; cv[7] = u1.w;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float a = av[i];
+                    const float sg = 1.0f / (1.0f + expf(-a));
+                    f[i] = is_da ? hv[i] * cv[i] * sg * (1.0f + a * (1.0f - sg)) : hv[i] * a * sg;
+                }
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            float scale, inv;
+            scale_from_amax(amax, scale, inv);
+            const uint32_t b0 = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv));
+            const uint32_t b1 = e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
+            const uint32_t b2 = e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv));
+            const uint32_t b3 = e4m3x2(__fmul_rn(f[6], inv), __fmul_rn(f[7], inv));
+            if (c < nvec) q[r * nvec + c] = make_uint2(b0 | (b1 << 16), b2 | (b3 << 16));
+            const float sj = __shfl_sync(0xffffffffu, scale, (lane & 1) * 16);
+            if ((lane >> 1) == j) tile_scale = sj;
+        }
+        const int tile = c0 / 16 + lane;
+        if (lane < 2 * PC && tile < nkb) qs[int64_t(tile) * rows_total + r] = tile_scale;
+    }
+}
+
+// ------------------------------------------- 6. gate gradients (FP64)
+// A warp per token: dg_k = <dy, o_k> summed in FP64 (lane-strided, then a
+// shuffle tree); the chosen scores' gradients in FP64.
+__global__ void __launch_bounds__(256) gate_backward_kernel(
+    const uint16_t* __restrict__ dy, const float* __restrict__ o, int T, int d, int K,
+    const int32_t* __restrict__ row_of_pair, const float* __restrict__ score,
+    float* __restrict__ dgate, float* __restrict__ du) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    double my_dg = 0.0;
+    for (int k = 0; k < K; ++k) {
+        const int row = row_of_pair[int64_t(t) * K + k];
+        double acc = 0.0;
+        if (row >= 0)
+            for (int c = lane; c < d; c += 32)
+                acc += double(__uint_as_float(uint32_t(dy[int64_t(t) * d + c]) << 16)) *
+                       double(o[int64_t(row) * d + c]);
+#pragma unroll
+        for (int s = 16; s >= 1; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+        if (lane == k) my_dg = acc;
+    }
+    const double s = lane < K ? double(score[int64_t(t) * K + lane]) : 0.0;
+    double S = s, gdg = 0.0;
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o2);
+    double term = lane < K ? (s / S) * my_dg : 0.0;
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o2);
+    gdg = term;
+    if (lane < K) {
+        const double ds = (my_dg - gdg) / S;
+        dgate[int64_t(t) * K + lane] = float(my_dg);
+        du[int64_t(t) * K + lane] = float(ds * s * (1.0 - s));
+    }
+}
+
+// ------------------------------------------- 7. router gradients
+// dx_router: a warp per (token, 64-float4 slice), the K chosen router rows
+// weighted by du in slot order.
+__global__ void __launch_bounds__(256) router_dx_kernel(
+    const uint16_t* __restrict__ E, const float* __restrict__ du,
+    const int32_t* __restrict__ topk_idx, int T, int d, int K, int n_routed,
+    float* __restrict__ dx, int* dev_status) {
+    const int lane = threadIdx.x & 31;
+    const int chunks = (d + 255) / 256;  // 256 values (8 per lane) per unit
+    const int64_t units = int64_t(T) * chunks;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t u = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); u < units;
+         u += warps_total) {
+        const int64_t t = u / chunks;
+        const int c = int(u - t * chunks) * 256 + lane * 8;
+        if (c >= d) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < K; ++k) {
+            const int e = topk_idx[t * K + k];
+            if (e < 0 || e >= n_routed) {
+                set_status(dev_status, MOE_DEV_BAD_INPUT);
+                continue;
+            }
+            const float g = du[t * K + k];
+            const uint4 w = *reinterpret_cast<const uint4*>(E + int64_t(e) * d + c);
+            const float ev[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                 bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(g, ev[i], acc[i]);
+        }
+        float4* out = reinterpret_cast<float4*>(dx + t * d + c);
+        out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
+// pair_of_row[row] = t*K + k for each routed row (the permutation's inverse)
+__global__ void pair_of_row_kernel(const int32_t* __restrict__ row_of_pair, int64_t pairs,
+                                   int64_t routed_rows, int32_t* __restrict__ pair_of_row) {
+    const int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (p >= pairs) return;
+    const int r = row_of_pair[p];
+    if (r >= 0 && r < routed_rows) pair_of_row[r] = int32_t(p);
+}
+
+// dE: a warp per (expert, 256-value slice), the expert's rows in permutation
+// order (tokens ascending), du times the token's x, fp32.
+__global__ void __launch_bounds__(256) router_dE_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ du,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ pair_of_row, int d, int K,
+    int n_routed, float* __restrict__ dE) {
+    const int lane = threadIdx.x & 31;
+    const int chunks = (d + 255) / 256;
+    const int64_t units = int64_t(n_routed) * chunks;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t u = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); u < units;
+         u += warps_total) {
+        const int e = int(u / chunks);
+        const int c = int(u - int64_t(e) * chunks) * 256 + lane * 8;
+        if (c >= d) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int r = offsets[e]; r < offsets[e + 1]; ++r) {
+            const int p = pair_of_row[r];
+            const int t = p / K;
+            const float g = du[p];
+            const uint4 w = *reinterpret_cast<const uint4*>(x + int64_t(t) * d + c);
+            const float xv[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                 bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(g, xv[i], acc[i]);
+        }
+        float4* out = reinterpret_cast<float4*>(dE + int64_t(e) * d + c);
+        out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
+// ------------------------------------------- 8. dx
+__global__ void __launch_bounds__(256) dx_combine_kernel(
+    const float4* __restrict__ dx_rows, const float4* __restrict__ dx_router, int T, int d,
+    int K, const int32_t* __restrict__ row_of_pair, float4* __restrict__ dx) {
+    const int lane = threadIdx.x & 31;
+    const int nv = d / 4;
+    const int chunks = (nv + 63) / 64;
+    const int64_t units = int64_t(T) * chunks;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t u = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); u < units;
+         u += warps_total) {
+        const int64_t t = u / chunks;
+        int my_row = -1;
+        if (lane < K) my_row = row_of_pair[t * K + lane];
+        for (int j = 0; j < 2; ++j) {
+            const int c = int(u - t * chunks) * 64 + lane + 32 * j;
+            if (c >= nv) continue;
+            float4 a = dx_rows[(int64_t(T) * K + t) * nv + c];  // the shared expert's row
+            for (int k = 0; k < K; ++k) {
+                const int row = __shfl_sync(0xffffffffu, my_row, k);
+                if (row < 0) continue;
+                const float4 v = dx_rows[int64_t(row) * nv + c];
+                a.x = __fadd_rn(a.x, v.x);
+                a.y = __fadd_rn(a.y, v.y);
+                a.z = __fadd_rn(a.z, v.z);
+                a.w = __fadd_rn(a.w, v.w);
+            }
+            if (dx_router) {
+                const float4 v = dx_router[t * nv + c];
+                a.x = __fadd_rn(a.x, v.x);
+                a.y = __fadd_rn(a.y, v.y);
+                a.z = __fadd_rn(a.z, v.z);
+                a.w = __fadd_rn(a.w, v.w);
+            }
+            dx[t * nv + c] = a;
+        }
+    }
+}
+
+// ------------------------------------------- transposed weights
+// A CTA per 128x128 block: codes through shared memory, transposed; the
+// block's scale moves to the transposed position.
+__global__ void __launch_bounds__(256) transpose_w_kernel(
+    const uint8_t* __restrict__ q, const float* __restrict__ s, int64_t mats, int rows,
+    int cols, uint8_t* __restrict__ qt, float* __restrict__ st) {
+    __shared__ uint8_t tile[128][129];
+    const int rb = rows / 128, cb = cols / 128;
+    const int64_t blocks = mats * rb * cb;
+    for (int64_t b = blockIdx.x; b < blocks; b += gridDim.x) {
+        const int64_t m = b / (int64_t(rb) * cb);
+        const int i = int((b / cb) % rb), j = int(b % cb);
+        const uint8_t* src = q + (m * rows + int64_t(i) * 128) * cols + int64_t(j) * 128;
+        for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x)
+            tile[e / 128][e % 128] = src[int64_t(e / 128) * cols + (e % 128)];
+        __syncthreads();
+        uint8_t* dst = qt + (m * cols + int64_t(j) * 128) * rows + int64_t(i) * 128;
+        for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x)
+            dst[int64_t(e / 128) * rows + (e % 128)] = tile[e % 128][e / 128];
+        if (threadIdx.x == 0) st[(m * cb + j) * rb + i] = s[(m * rb + i) * cb + j];
+        __syncthreads();
+    }
+}
+
+int pieces_per(int n, int& PC) {
+    const int nkb = n / 128;
+    PC = (nkb % 14 == 0 && nkb % 16 != 0) ? 7 : 8;
+    return (n / 8 + 32 * PC - 1) / (32 * PC);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" MOE_API int fp8_transpose_w_128x128(const uint8_t* q, const float* scales,
+                                               int64_t mats, int64_t rows, int64_t cols,
+                                               uint8_t* qt, float* scales_t, int* dev_status,
+                                               void* stream) {
+    (void)dev_status;
+    if (mats < 0 || rows < 0 || cols < 0 || rows % 128 || cols % 128 || rows > INT32_MAX ||
+        cols > INT32_MAX)
+        return MOE_ERR_SHAPE;
+    if (mats == 0 || rows == 0 || cols == 0) return MOE_OK;
+    if (!q || !scales || !qt || !scales_t) return MOE_ERR_NULL;
+    const int64_t blocks = mats * (rows / 128) * (cols / 128);
+    const int grid = int(std::min<int64_t>(blocks, int64_t(sm_count()) * 8));
+    transpose_w_kernel<<<grid, 256, 0, as_stream(stream)>>>(q, scales, mats, int(rows), int(cols),
+                                                            qt, scales_t);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_combine_backward_quant(const MoeShape* shape, const uint16_t* dy,
+                                                  const int32_t* row_of_pair,
+                                                  const float* topk_gate, uint8_t* do_q,
+                                                  float* do_scales, int* dev_status,
+                                                  void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T, d = shape->d, K = shape->topk;
+    if (T == 0) return MOE_OK;
+    if (!dy || !row_of_pair || !topk_gate || !do_q || !do_scales) return MOE_ERR_NULL;
+    if (!aligned16(dy) || !aligned16(do_q)) return MOE_ERR_ALIGN;
+    int PC;
+    const int pieces = pieces_per(d, PC);
+    const int grid = warp_blocks(int64_t(T) * pieces);
+    const int64_t R = int64_t(T) * K + T;
+    if (PC == 7)
+        combine_backward_quant_kernel<7><<<grid, 256, 0, as_stream(stream)>>>(
+            reinterpret_cast<const uint4*>(dy), T, d, K, row_of_pair, topk_gate, R,
+            reinterpret_cast<uint2*>(do_q), do_scales);
+    else
+        combine_backward_quant_kernel<8><<<grid, 256, 0, as_stream(stream)>>>(
+            reinterpret_cast<const uint4*>(dy), T, d, K, row_of_pair, topk_gate, R,
+            reinterpret_cast<uint2*>(do_q), do_scales);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_swiglu_backward_quant(const float* dh, const float* ac, int64_t rows,
+                                                 int inter, int64_t rows_total, uint8_t* q,
+                                                 float* q_scales, int* dev_status,
+                                                 void* stream) {
+    (void)dev_status;
+    if (rows < 0 || inter <= 0 || inter % 128 || rows_total < rows) return MOE_ERR_SHAPE;
+    if (rows == 0) return MOE_OK;
+    if (!dh || !ac || !q || !q_scales) return MOE_ERR_NULL;
+    if (!aligned16(dh) || !aligned16(ac) || !aligned16(q)) return MOE_ERR_ALIGN;
+    int PC;
+    const int pieces = pieces_per(2 * inter, PC);
+    const int grid = warp_blocks(rows * pieces);
+    if (PC == 7)
+        swiglu_backward_quant_kernel<7><<<grid, 256, 0, as_stream(stream)>>>(
+            dh, ac, rows, inter, rows_total, reinterpret_cast<uint2*>(q), q_scales);
+    else
+        swiglu_backward_quant_kernel<8><<<grid, 256, 0, as_stream(stream)>>>(
+            dh, ac, rows, inter, rows_total, reinterpret_cast<uint2*>(q), q_scales);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_gate_backward(const MoeShape* shape, const uint16_t* dy,
+                                         const float* expert_out, const int32_t* row_of_pair,
+                                         const float* topk_score, float* dgate, float* du,
+                                         int* dev_status, void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T;
+    if (T == 0) return MOE_OK;
+    if (!dy || !expert_out || !row_of_pair || !topk_score || !dgate || !du) return MOE_ERR_NULL;
+    gate_backward_kernel<<<(T + 7) / 8, 256, 0, as_stream(stream)>>>(
+        dy, expert_out, T, shape->d, shape->topk, row_of_pair, topk_score, dgate, du);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t* x,
+                                           const uint16_t* router_w, const float* du,
+                                           const int32_t* topk_idx,
+                                           const int32_t* expert_offsets,
+                                           const int32_t* row_of_pair, int32_t* pair_scratch,
+                                           float* dx_router, float* d_router_w,
+                                           int* dev_status, void* stream) {
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T, d = shape->d, K = shape->topk, N = shape->n_routed;
+    if (!d_router_w) return MOE_ERR_NULL;
+    cudaStream_t st = as_stream(stream);
+    if (T == 0)
+        return cudaMemsetAsync(d_router_w, 0, sizeof(float) * N * d, st) == cudaSuccess
+                   ? MOE_OK : MOE_ERR_CUDA;
+    if (!x || !router_w || !du || !topk_idx || !expert_offsets || !row_of_pair ||
+        !pair_scratch || !dx_router)
+        return MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(dx_router) || !aligned16(d_router_w))
+        return MOE_ERR_ALIGN;
+    const int chunks = (d + 255) / 256;
+    router_dx_kernel<<<warp_blocks(int64_t(T) * chunks), 256, 0, st>>>(
+        router_w, du, topk_idx, T, d, K, N, dx_router, dev_status);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    const int64_t pairs = int64_t(T) * K;
+    pair_of_row_kernel<<<int((pairs + 255) / 256), 256, 0, st>>>(row_of_pair, pairs, pairs,
+                                                                  pair_scratch);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    router_dE_kernel<<<warp_blocks(int64_t(N) * chunks), 256, 0, st>>>(
+        x, du, expert_offsets, pair_scratch, d, K, N, d_router_w);
+    return check_launch();
+}
+
+extern "C" MOE_API int moe_dx_combine(const MoeShape* shape, const float* dx_rows,
+                                      const float* dx_router, const int32_t* row_of_pair,
+                                      float* dx, int* dev_status, void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    const int T = shape->T;
+    if (T == 0) return MOE_OK;
+    if (!dx_rows || !row_of_pair || !dx) return MOE_ERR_NULL;
+    if (!aligned16(dx_rows) || !aligned16(dx) || (dx_router && !aligned16(dx_router)))
+        return MOE_ERR_ALIGN;
+    const int chunks = (shape->d / 4 + 63) / 64;
+    dx_combine_kernel<<<warp_blocks(int64_t(T) * chunks), 256, 0, as_stream(stream)>>>(
+        reinterpret_cast<const float4*>(dx_rows), reinterpret_cast<const float4*>(dx_router), T,
+        shape->d, shape->topk, row_of_pair, reinterpret_cast<float4*>(dx));
+    return check_launch();
+}

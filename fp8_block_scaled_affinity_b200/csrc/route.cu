@@ -936,7 +936,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(
     const int32_t* __restrict__ cand, const float* __restrict__ u_exact, int T, int n_routed,
     int n_groups, int topk_groups, int topk, const float* __restrict__ bias,
     const float* __restrict__ logit_offset, int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_gate, int32_t* __restrict__ counts, int* dev_status,
+    float* __restrict__ topk_gate, float* __restrict__ topk_score,
+    int32_t* __restrict__ counts, int* dev_status,
     int32_t* __restrict__ check) {
     extern __shared__ __align__(16) float sel_smem[];
     int* hist = reinterpret_cast<int*>(sel_smem);
@@ -1042,6 +1043,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) route_select_kernel(
         if (lane < topk) {
             topk_idx[int64_t(t) * topk + lane] = my_idx;
             topk_gate[int64_t(t) * topk + lane] = __double2float_rn((double)sv / S);
+            if (topk_score) topk_score[int64_t(t) * topk + lane] = sv;
             atomicAdd(&hist[my_idx], 1);
         }
     }
@@ -1131,11 +1133,12 @@ extern "C" MOE_API size_t moe_route_workspace_size(const MoeShape* shape) {
     return route_carve(shape, nullptr).bytes;
 }
 
-extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
-                                 const uint16_t* router_w, const float* bias,
-                                 const float* logit_offset, int32_t* topk_idx, float* topk_gate,
-                                 int32_t* expert_counts, void* ws, size_t ws_bytes,
-                                 int* dev_status, void* stream) {
+extern "C" MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x,
+                                        const uint16_t* router_w, const float* bias,
+                                        const float* logit_offset, int32_t* topk_idx,
+                                        float* topk_gate, float* topk_score,
+                                        int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                        int* dev_status, void* stream) {
     int rc = validate_shape(shape);
     if (rc != MOE_OK) return rc;
     if (!router_w || !bias || !expert_counts) return MOE_ERR_NULL;
@@ -1151,8 +1154,8 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
     // pageable host array here would fault the kernels)
     for (const void* ptr : {(const void*)x, (const void*)router_w, (const void*)bias,
                             (const void*)logit_offset, (const void*)topk_idx,
-                            (const void*)topk_gate, (const void*)expert_counts, (const void*)ws,
-                            (const void*)dev_status})
+                            (const void*)topk_gate, (const void*)topk_score,
+                            (const void*)expert_counts, (const void*)ws, (const void*)dev_status})
         if (!device_accessible(ptr)) return MOE_ERR_ARG;
     const RouteWs w = route_carve(shape, ws);
     const int sms = sm_count();
@@ -1226,6 +1229,15 @@ extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
         return MOE_ERR_CUDA;
     route_select_kernel<<<(T + kSelWarps - 1) / kSelWarps, kSelWarps * 32, smem, st>>>(
         w.uhat, w.cert, w.cand, w.u_exact, T, N, shape->n_groups, shape->topk_groups, K, bias,
-        logit_offset, topk_idx, topk_gate, expert_counts, dev_status, w.check);
+        logit_offset, topk_idx, topk_gate, topk_score, expert_counts, dev_status, w.check);
     return check_launch();
+}
+
+extern "C" MOE_API int moe_route(const MoeShape* shape, const uint16_t* x,
+                                 const uint16_t* router_w, const float* bias,
+                                 const float* logit_offset, int32_t* topk_idx, float* topk_gate,
+                                 int32_t* expert_counts, void* ws, size_t ws_bytes,
+                                 int* dev_status, void* stream) {
+    return moe_route_scores(shape, x, router_w, bias, logit_offset, topk_idx, topk_gate, nullptr,
+                            expert_counts, ws, ws_bytes, dev_status, stream);
 }

@@ -148,6 +148,14 @@ MOE_API int moe_route(const MoeShape* shape, const uint16_t* x, const uint16_t* 
                       float* topk_gate, int32_t* expert_counts, void* ws, size_t ws_bytes,
                       int* dev_status, void* stream);
 
+/* moe_route_scores: moe_route that also writes topk_score fp32 [T, K]: the
+ * unbiased affinity s of each chosen expert, in slot order (the values the
+ * gates are normalised from; the backward pass needs them). */
+MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x, const uint16_t* router_w,
+                             const float* bias, const float* logit_offset, int32_t* topk_idx,
+                             float* topk_gate, float* topk_score, int32_t* expert_counts,
+                             void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
 /* ----------------------------------------------------------- quantisation
  * fp8_quant_act_1x128: online 1x128 tile quantisation of activations
  * ("FP8 mixed precision training", fine-grained quantisation).
@@ -552,6 +560,100 @@ MOE_API int moe_layer_forward_host_batches(const MoeShape* shape, const MoeWeigh
                                            const float* logit_offset, MoeRouting* routing,
                                            uint16_t* y_host, int update_bias, void* ws,
                                            size_t ws_bytes, int* dev_status, void* stream);
+
+/* ====================================================================
+ * Backward pass (dx and the router's gradient) of the layer, fp32-scale
+ * recipe ("DeepSeek-V3 Technical Report" notes page, section "FP8 mixed
+ * precision training": the Dgrad GEMMs take FP8 operands with 1x128 tiles
+ * for activation gradients and 128x128 blocks for weights, accumulation in
+ * FP32 with per-128-K promotion; section "DeepSeekMoE and
+ * auxiliary-loss-free load balancing": the gates are the chosen unbiased
+ * affinities normalised, the bias and the top-K choice carry no gradient).
+ * The steps for an upstream gradient dy (bf16 [T, d]), with the rows of the
+ * forward's permutation (R = T*K + T, the shared expert's row of token t is
+ * T*K + t):
+ *   moe_combine_backward_quant -> do rows, FP8 1x128 (d)
+ *   moe_grouped_gemm_fp8 (do, W2 transposed, n = I, F32)     -> dh
+ *   moe_grouped_gemm_fp8 (forward FP8 x rows, W13, n = 2I, F32) -> [a | c]
+ *   moe_swiglu_backward_quant -> [da | dc] FP8 1x128 (2I)
+ *   moe_grouped_gemm_fp8 ([da|dc], W13 transposed, n = d, F32) -> dx rows
+ *   moe_gate_backward, moe_router_backward, moe_dx_combine -> dx, dE.
+ * Gradients of the expert weights (Wgrad) are not part of the library.
+ * ==================================================================== */
+
+/* fp8_transpose_w_128x128: for mats matrices of FP8 codes [rows, cols] with
+ * fp32 scales [rows/128, cols/128] (the 128x128 block quantiser's output),
+ * write the transposed codes [cols, rows] and scales [cols/128, rows/128].
+ * A block keeps its scale, so the transposed matrix holds the same values
+ * exactly (no requantisation).  Bit-exact.  rows, cols multiples of 128.
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_CUDA. */
+MOE_API int fp8_transpose_w_128x128(const uint8_t* q, const float* scales, int64_t mats,
+                                    int64_t rows, int64_t cols, uint8_t* qt, float* scales_t,
+                                    int* dev_status, void* stream);
+
+/* moe_combine_backward_quant: the gradient of each expert row's output,
+ * do = fp32(gate[t,k] * dy[t]) for the row of (t, k) and do = dy[t] for the
+ * shared row of t, quantised like the forward's activations (1x128 tiles
+ * along d, scale = amax/448 in fp32, code = E4M3(v * (448/amax))).
+ *   dy           bf16 [T, d] device, 16-byte aligned
+ *   row_of_pair  int32 [T, K] (the forward's; entries < 0 are skipped)
+ *   topk_gate    fp32 [T, K] (the forward's gates)
+ *   do_q         uint8 [R, d] out;  do_scales fp32 [d/128, R] out (k-block
+ *                major, the grouped GEMM's A-scale layout)
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_CUDA. */
+MOE_API int moe_combine_backward_quant(const MoeShape* shape, const uint16_t* dy,
+                                       const int32_t* row_of_pair, const float* topk_gate,
+                                       uint8_t* do_q, float* do_scales, int* dev_status,
+                                       void* stream);
+
+/* moe_swiglu_backward_quant: for rows of dh (fp32 [rows, I]) and the
+ * pre-activations [a | c] (fp32 [rows, 2I]), da = dh c silu'(a) with
+ * silu'(a) = sigma(a)(1 + a(1 - sigma(a))) and dc = dh silu(a), in fp32, the
+ * row [da | dc] quantised in 1x128 tiles along 2I into q (uint8 [rows, 2I])
+ * and q_scales (fp32 [2I/128, rows_total], k-block major).  inter % 128 ==
+ * 0; dh, ac, q 16-byte aligned.  Errors: MOE_ERR_SHAPE, MOE_ERR_NULL,
+ * MOE_ERR_ALIGN, MOE_ERR_CUDA. */
+MOE_API int moe_swiglu_backward_quant(const float* dh, const float* ac, int64_t rows, int inter,
+                                      int64_t rows_total, uint8_t* q, float* q_scales,
+                                      int* dev_status, void* stream);
+
+/* moe_gate_backward: dgate[t,k] = <dy[t], o[row of (t,k)]> (FP64 sum, stored
+ * fp32) and du[t,k], the gradient of the chosen expert's logit:
+ * ds_k = (dgate_k - sum_j g_j dgate_j) / S with S = sum of the chosen s,
+ * du_k = ds_k s_k (1 - s_k) (FP64, stored fp32).
+ *   dy bf16 [T, d]; expert_out fp32 [R, d] (the forward's expert outputs,
+ *   ungated); row_of_pair int32 [T, K]; topk_score fp32 [T, K] (from
+ *   moe_route_scores); dgate, du fp32 [T, K] out.
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_CUDA. */
+MOE_API int moe_gate_backward(const MoeShape* shape, const uint16_t* dy, const float* expert_out,
+                              const int32_t* row_of_pair, const float* topk_score, float* dgate,
+                              float* du, int* dev_status, void* stream);
+
+/* moe_router_backward: the router's two gradients from du (fp32 [T, K]):
+ *   dx_router[t] = sum_k du[t,k] E[topk_idx[t,k]]     (fp32 [T, d] out,
+ *                  fp32 fused multiply-adds in slot order)
+ *   d_router_w[e] = sum over the tokens choosing e, ascending, of du x[t]
+ *                  (fp32 [N_r, d] out; every row written, zero for an
+ *                  unchosen expert)
+ *   x bf16 [T, d]; router_w bf16 [N_r, d]; topk_idx int32 [T, K];
+ *   expert_offsets int32 [N_r + 2] and row_of_pair int32 [T, K] (the
+ *   forward's permutation); pair_scratch int32 [T*K] scratch.
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_CUDA;
+ * MOE_DEV_BAD_INPUT on dev_status for an expert index out of range. */
+MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t* x,
+                                const uint16_t* router_w, const float* du,
+                                const int32_t* topk_idx, const int32_t* expert_offsets,
+                                const int32_t* row_of_pair, int32_t* pair_scratch,
+                                float* dx_router, float* d_router_w, int* dev_status,
+                                void* stream);
+
+/* moe_dx_combine: dx[t] = dx_rows[shared row of t] + sum_k dx_rows[row of
+ * (t,k)] (slot order) + dx_router[t] (NULL: none), fp32 [T, d] out.
+ *   dx_rows fp32 [R, d] (the expert rows' input gradients).
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_CUDA. */
+MOE_API int moe_dx_combine(const MoeShape* shape, const float* dx_rows, const float* dx_router,
+                           const int32_t* row_of_pair, float* dx, int* dev_status,
+                           void* stream);
 
 #ifdef __cplusplus
 }
