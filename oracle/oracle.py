@@ -23,6 +23,7 @@ __all__ = [
     "quant_act_1x128_pow2", "quant_w_128x128_pow2", "pow2_scales",
     "redundant_plan", "split_groups", "quantized_expert_pow2", "quant_act_1x128_pow2_values",
     "gate_backward", "router_backward", "expert_backward", "layer_backward", "swiglu_backward",
+    "quant_act_128x1",
 ]
 
 _LIB = None
@@ -455,15 +456,35 @@ def swiglu_backward(dh, a, c):
     return da, dc
 
 
+def quant_act_128x1(x: np.ndarray):
+    """128x1 tiles along the rows: a [rows, cols] matrix (one expert's rows)
+    is cut into blocks of 128 rows from its first row, and every column of a
+    block takes its own scale (the 1x128 rule applied to the transpose, the
+    rows padded with zeros to a multiple of 128).  x: uint16 bf16 bits or
+    float32.  Returns (codes uint8 [cols, rows_pad], scales float32
+    [cols, rows_pad/128]): the transposed operand of a weight-gradient GEMM."""
+    rows, cols = x.shape
+    pad = -(-rows // 128) * 128
+    t = np.zeros((cols, pad), dtype=x.dtype)
+    t[:, :rows] = x.T
+    return quant_act_1x128(t)
+
+
 def expert_backward(do_rows_f32: np.ndarray, xq: np.ndarray, xs: np.ndarray, w1, w3, w2,
-                    quant: bool = True):
+                    quant: bool = True, x_rows=None):
     """Dgrad through one expert for its rows: do (fp32 [rows, d], the
     gate-scaled dy) quantised 1x128 -> dh = dq(do) W2 (FP64); a, c
     recomputed from the forward's FP8 x; da = dh c silu'(a), dc = dh silu(a)
     rounded to fp32 and quantised 1x128 along [da | dc]; dx = dq([da|dc])
     [W1; W3] (FP64).  Returns dx [rows, d] FP64.
     quant=False (for checks against derivatives): no quantisation of do and
-    [da | dc], and xq is taken as the FP64 input itself (xs ignored)."""
+    [da | dc], and xq is taken as the FP64 input itself (xs ignored).
+
+    With x_rows (the rows' layer input: bf16 bits, or FP64 when quant=False)
+    also the weight gradients, contracting over the rows: returns (dx,
+    dW13 [2I, d] = [da | dc]^T x, dW2 [d, I] = do^T h) with h = silu(a) c.
+    Each operand is quantised in 128x1 tiles along the rows from its fp32
+    value (do; h and [da | dc] rounded to fp32; x from bf16)."""
     W1, W3, W2 = dequant_w(*w1), dequant_w(*w3), dequant_w(*w2)
     if quant:
         dq_, ds_ = quant_act_1x128(np.ascontiguousarray(do_rows_f32, np.float32))
@@ -473,11 +494,30 @@ def expert_backward(do_rows_f32: np.ndarray, xq: np.ndarray, xs: np.ndarray, w1,
         dh = np.asarray(do_rows_f32, np.float64) @ W2
         X = np.asarray(xq, np.float64)
     a, c = X @ W1.T, X @ W3.T
-    dac = np.concatenate(swiglu_backward(dh, a, c), axis=1)
+    dac_exact = np.concatenate(swiglu_backward(dh, a, c), axis=1)
     if quant:
-        qq, qs = quant_act_1x128(dac.astype(np.float32))
+        qq, qs = quant_act_1x128(dac_exact.astype(np.float32))
         dac = dequant_act(qq, qs)
-    return dac @ np.concatenate([W1, W3], axis=0)
+    else:
+        dac = dac_exact
+    dx = dac @ np.concatenate([W1, W3], axis=0)
+    if x_rows is None:
+        return dx
+    h = a / (1.0 + np.exp(-a)) * c
+    if quant:
+        rows = X.shape[0]
+
+        def t128(m):  # dequantised transposed 128x1 operand, [cols, rows]
+            q_, s_ = quant_act_128x1(m)
+            return dequant_act(q_, s_)[:, :rows]
+        dW2 = t128(np.ascontiguousarray(do_rows_f32, np.float32)) @ \
+            t128(h.astype(np.float32)).T
+        dW13 = t128(dac_exact.astype(np.float32)) @ \
+            t128(np.ascontiguousarray(x_rows, np.uint16)).T
+    else:
+        dW2 = np.asarray(do_rows_f32, np.float64).T @ h
+        dW13 = dac_exact.T @ np.asarray(x_rows, np.float64)
+    return dx, dW13, dW2
 
 
 def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -486,10 +526,13 @@ def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 def layer_backward(dy_bf16, x_bf16, router_w_bf16, bias, n_groups, topk_groups, topk,
-                   expert_weights, logit_offset=None, quant=True):
+                   expert_weights, logit_offset=None, quant=True, wgrad_experts=()):
     """dx [T,d] (FP64) and dE [N_r,d] (FP64) of the whole layer for dy.
     quant=False (for checks against derivatives): the experts take x itself
-    and nothing is quantised (the routing is the same)."""
+    and nothing is quantised (the routing is the same).
+    wgrad_experts: experts (N_r = the shared one) whose weight gradients to
+    return as "dW" {e: (dW13 [2I, d], dW2 [d, I])} (zeros for an expert no
+    token chose)."""
     T, d = x_bf16.shape
     n_routed = router_w_bf16.shape[0]
     r = route(x_bf16, router_w_bf16, bias, n_groups, topk_groups, topk, logit_offset,
@@ -501,6 +544,7 @@ def layer_backward(dy_bf16, x_bf16, router_w_bf16, bias, n_groups, topk_groups, 
     gates = r["topk_gate"]
     o_routed = np.zeros((T, topk, d))
     dx = np.zeros((T, d))
+    dW = {}
     for e in range(n_routed + 1):
         if e == n_routed:
             sel, slots = np.arange(T), None
@@ -511,17 +555,29 @@ def layer_backward(dy_bf16, x_bf16, router_w_bf16, bias, n_groups, topk_groups, 
                 continue
             do = (gates[sel, slots].astype(np.float32)[:, None] * dy32[sel]).astype(np.float32)
         w = expert_weights(e)
+        want_w = e in wgrad_experts
         if quant:
             if slots is not None:
                 o_routed[sel, slots] = swiglu_expert(xq[sel], xs[sel], *w)
-            dx[sel] += expert_backward(do, xq[sel], xs[sel], *w)
+            res = expert_backward(do, xq[sel], xs[sel], *w,
+                                  x_rows=x_bf16[sel] if want_w else None)
         else:
             X = _bf16_to_f64(x_bf16[sel])
             if slots is not None:
                 W1, W3, W2 = (dequant_w(*m) for m in w)
                 a, c = X @ W1.T, X @ W3.T
                 o_routed[sel, slots] = (a / (1.0 + np.exp(-a)) * c) @ W2.T
-            dx[sel] += expert_backward(do, X, None, *w, quant=False)
+            res = expert_backward(do, X, None, *w, quant=False, x_rows=X if want_w else None)
+        if want_w:
+            dx[sel] += res[0]
+            dW[e] = (res[1], res[2])
+        else:
+            dx[sel] += res
+    for e in wgrad_experts:
+        if e not in dW:
+            I2, dd = expert_weights(e)[0][0].shape
+            dW[e] = (np.zeros((2 * I2, dd)), np.zeros((dd, I2)))
     dg, du = gate_backward(dy_bf16, o_routed, scores)
     dxr, dE = router_backward(du, idx, x_bf16, router_w_bf16)
-    return {"dx": dx + dxr, "dE": dE, "dg": dg, "du": du, "topk_idx": idx, "scores": scores}
+    return {"dx": dx + dxr, "dE": dE, "dg": dg, "du": du, "topk_idx": idx, "scores": scores,
+            "dW": dW}

@@ -140,3 +140,79 @@ def test_layer_backward_matches_finite_differences():
     scale_x, scale_E = np.abs(num_dx).max(), np.abs(num_dE).max()
     assert np.abs(got["dx"] - num_dx).max() <= 1e-5 * scale_x
     assert np.abs(got["dE"] - num_dE).max() <= 1e-5 * scale_E
+
+
+def test_quant_act_128x1_blocks_follow_the_rows():
+    """Blocks of 128 rows from the first row, one scale per column and
+    block, stored transposed; the ragged last block is padded with zero
+    codes.  Every (block, column) gets a distinct amax, so a transposed or
+    shifted index moves a scale to the wrong place."""
+    rows, cols = 300, 5
+    rng = np.random.default_rng(5)
+    x = rng.uniform(-1.0, 1.0, (rows, cols)).astype(np.float32)
+    amax = np.zeros((3, cols), np.float32)
+    for b in range(3):
+        for j in range(cols):
+            a = np.float32(2.0 + 3 * b + 0.25 * j)
+            r = 128 * b + (7 * j + 3 * b) % min(128, rows - 128 * b)
+            x[r, j] = -a if (b + j) % 2 else a
+            amax[b, j] = a
+    q, s = oracle.quant_act_128x1(x)
+    assert q.shape == (cols, 384) and s.shape == (cols, 3)
+    assert np.allclose(s.T * 448.0, amax, rtol=1e-6)
+    assert np.all(q[:, rows:] == 0)
+    deq = oracle.dequant_act(q, s)[:, :rows].T
+    assert np.all(np.abs(deq - x) <= 2.0**-4 * np.abs(x) + 2.0**-9 * np.repeat(s.T, 128, 0)[:rows])
+
+
+def test_layer_weight_gradients_match_finite_differences():
+    """dW1, dW3, dW2 of every expert (shared one included) from the
+    unquantised chain against central differences of the FP64 forward in a
+    sample of weight entries; an expert no token chose has zero gradients."""
+    rng = np.random.default_rng(6)
+    T, d, N, G, M, K, I = 3, 128, 4, 2, 2, 2, 128
+    x = S.f32_to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    E = S.f32_to_bf16_bits((rng.standard_normal((N, d)) * 0.1).astype(np.float32))
+    bias = np.array([0.0, 0.0, 0.0, -5.0], np.float32)  # expert 3 is never chosen
+    dy = S.f32_to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    ws = [oracle.quantized_expert(*(S.host_normal_bf16(rng, sh, 0.1)
+                                    for sh in ((I, d), (I, d), (d, I))))
+          for _ in range(N + 1)]
+    got = oracle.layer_backward(dy, x, E, bias, G, M, K, lambda e: ws[e], quant=False,
+                                wgrad_experts=tuple(range(N + 1)))
+    idx = got["topk_idx"]
+    assert not np.any(idx == 3)
+    W = [[oracle.dequant_w(*m) for m in w] for w in ws]
+    xv = S.bf16_bits_to_f32(x).astype(np.float64)
+    Ev = S.bf16_bits_to_f32(E).astype(np.float64)
+    dyv = S.bf16_bits_to_f32(dy).astype(np.float64)
+    s = 1.0 / (1.0 + np.exp(-(xv @ Ev.T)))
+    sk = np.take_along_axis(s, idx, axis=1)
+    g = sk / sk.sum(axis=1, keepdims=True)
+
+    def loss(Wl):
+        def expert(e, X):
+            W1, W3, W2 = Wl[e]
+            a, c = X @ W1.T, X @ W3.T
+            return (a / (1.0 + np.exp(-a)) * c) @ W2.T
+        y = expert(N, xv)
+        for t in range(T):
+            for k in range(K):
+                y[t] += g[t, k] * expert(idx[t, k], xv[t:t + 1])[0]
+        return float(np.sum(dyv * y))
+    h = 1e-5
+    for e in range(N + 1):
+        dW13, dW2 = got["dW"][e]
+        grads = (dW13[:I], dW13[I:], dW2)
+        for m in range(3):
+            for _ in range(12):
+                i, j = rng.integers(0, W[e][m].shape[0]), rng.integers(0, W[e][m].shape[1])
+                Wp = [[w.copy() for w in we] for we in W]
+                Wm = [[w.copy() for w in we] for we in W]
+                Wp[e][m][i, j] += h
+                Wm[e][m][i, j] -= h
+                num = (loss(Wp) - loss(Wm)) / (2 * h)
+                scale = max(np.abs(grads[m]).max(), 1e-12)
+                assert abs(grads[m][i, j] - num) <= 1e-6 * scale + 1e-9, (e, m, i, j)
+        if e == 3:
+            assert not np.any(dW13) and not np.any(dW2)
