@@ -23,7 +23,7 @@ __all__ = [
     "quant_act_1x128_pow2", "quant_w_128x128_pow2", "pow2_scales",
     "redundant_plan", "split_groups", "quantized_expert_pow2", "quant_act_1x128_pow2_values",
     "gate_backward", "router_backward", "expert_backward", "layer_backward", "swiglu_backward",
-    "quant_act_128x1",
+    "quant_act_128x1", "gemm_wgrad",
 ]
 
 _LIB = None
@@ -402,6 +402,21 @@ def layer_forward(x_bf16: np.ndarray, router_w_bf16: np.ndarray, bias: np.ndarra
 def gemm_blockscaled(aq, a_s, bq, b_s):
     """C = dq(A) dq(B)^T in FP64; A [m,k] 1x128-scaled, B [n,k] 128x128-scaled."""
     return dequant_act(aq, a_s) @ dequant_w(bq, b_s).T
+
+
+def gemm_wgrad(a_t, a_scales, b_t, b_scales, kb_offsets):
+    """Weight-gradient GEMM with K groups: out[g] = dq(A)[:, K_g] dq(B)[:, K_g]^T
+    in FP64, K_g the 128-column blocks [kb_offsets[g], kb_offsets[g+1]).
+    a_t [m, nkb*128] codes with scales [nkb, m] (one per row and K block),
+    b_t [n, nkb*128] likewise.  Returns [G, m, n]."""
+    A = dequant_act(a_t, np.ascontiguousarray(a_scales.T))
+    B = dequant_act(b_t, np.ascontiguousarray(b_scales.T))
+    G = len(kb_offsets) - 1
+    out = np.zeros((G, A.shape[0], B.shape[0]))
+    for g in range(G):
+        k0, k1 = 128 * int(kb_offsets[g]), 128 * int(kb_offsets[g + 1])
+        out[g] = A[:, k0:k1] @ B[:, k0:k1].T
+    return out
 
 
 # ---------------------------------------------------------------- backward

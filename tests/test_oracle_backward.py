@@ -216,3 +216,29 @@ def test_layer_weight_gradients_match_finite_differences():
                 assert abs(grads[m][i, j] - num) <= 1e-6 * scale + 1e-9, (e, m, i, j)
         if e == 3:
             assert not np.any(dW13) and not np.any(dW2)
+
+
+def test_gemm_wgrad_brute_force():
+    """The K-grouped GEMM against a loop over groups, rows, columns and K
+    with each product scaled by its row's and column's block scales; an
+    empty group is zero."""
+    rng = np.random.default_rng(7)
+    m, n, nkb = 3, 2, 4
+    table = oracle.e4m3_decode_table()
+    finite = np.nonzero(np.isfinite(table))[0].astype(np.uint8)
+    a = rng.choice(finite, (m, 128 * nkb))
+    b = rng.choice(finite, (n, 128 * nkb))
+    sa = rng.uniform(0.5, 2.0, (nkb, m)).astype(np.float32)
+    sb = rng.uniform(0.5, 2.0, (nkb, n)).astype(np.float32)
+    kb_off = np.array([0, 1, 1, 4], np.int32)
+    got = oracle.gemm_wgrad(a, sa, b, sb, kb_off)
+    for g in range(3):
+        for i in range(m):
+            for j in range(n):
+                ref = 0.0
+                for k in range(128 * kb_off[g], 128 * kb_off[g + 1]):
+                    kb = k // 128
+                    ref += float(table[a[i, k]]) * float(sa[kb, i]) * float(table[b[j, k]]) * \
+                        float(sb[kb, j])
+                assert abs(got[g, i, j] - ref) <= 1e-9 * max(1.0, abs(ref))
+    assert not np.any(got[1])
