@@ -29,7 +29,9 @@ from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QU
                    moe_ep_local_permute, moe_ep_partial_combine, moe_ep_final_combine,
                    moe_route_scores, fp8_transpose_w_128x128, moe_combine_backward_quant,
                    moe_swiglu_backward_quant, moe_gate_backward, moe_router_backward,
-                   moe_dx_combine)
+                   moe_dx_combine, moe_wgrad_max_blocks, moe_wgrad_layout, moe_wgrad_quant_x,
+                   moe_wgrad_quant_do, moe_wgrad_quant_h, moe_wgrad_quant_dac,
+                   moe_grouped_gemm_wgrad)
 
 __all__ = ["MoeLayer", "MoeShape", "MoeError", "lib", "make_shape", "moe_version"]
 
@@ -204,15 +206,21 @@ class MoeLayer:
             self._transposed = (w2t, w2t_s, w13t, w13t_s)
         return self._transposed
 
-    def backward(self, dy, stream=None, marks=None):
+    def backward(self, dy, stream=None, marks=None, wgrad: bool = False):
         """Gradients of the last forward_train() for the upstream gradient dy
-        (bf16 [T, d]): returns (dx fp32 [T, d], d_router_w fp32 [N_r, d]).
+        (bf16 [T, d]): returns (dx fp32 [T, d], d_router_w fp32 [N_r, d]), and
+        with wgrad=True also the expert weights' gradients dW13 (fp32
+        [N_r + 1, 2I, d], W1 rows then W3 rows) and dW2 (fp32 [N_r + 1, d, I]),
+        the shared expert last.
 
         Dgrad through the experts with FP8 operands (the gate-scaled output
         gradient and [da | dc] quantised in 1x128 tiles, the weights' own
         128x128 blocks transposed), a and c recomputed from the forward's FP8
         rows; the gate and router gradients in high precision.  The top-K
-        choice and the bias carry no gradient.
+        choice and the bias carry no gradient.  The weight gradients are FP8
+        GEMMs over each expert's rows with both operands quantised in 128x1
+        tiles along the rows (x from the layer input, do = gate dy, h and
+        [da | dc] from the recomputed fp32 a, c).
 
         marks: a list, or None; given a list, a timing CUDA event recorded on
         the stream after each stage is appended as (stage name, event), with
@@ -253,7 +261,6 @@ class MoeLayer:
         gs = torch.empty((2 * I // 128, R), dtype=f32, device=dev)
         moe_swiglu_backward_quant(dh, ac, R, I, R, gq, gs, st, stream)
         mark("swiglu_backward_quant")
-        del dh, ac
         dx_rows = torch.empty((R, d), dtype=f32, device=dev)
         moe_grouped_gemm_fp8(N + 1, off, R, gq, gs, 2 * I, w13t, w13t_s, d, MOE_EPI_F32,
                              dx_rows, None, st, stream)
@@ -272,7 +279,37 @@ class MoeLayer:
         moe_dx_combine(sh, dx_rows, dx_router, self.row_of_pair, dx, st, stream)
         mark("dx_combine")
         self.last_dgate, self.last_du = dgate, du
-        return dx, d_router_w
+        if not wgrad:
+            return dx, d_router_w
+        # ---- weight gradients (pair_scratch holds the permutation's inverse)
+        G = N + 1
+        nb = moe_wgrad_max_blocks(R, G)
+        kb_off = torch.empty((G + 1,), dtype=i32, device=dev)
+        blocks = torch.empty((nb, 2), dtype=i32, device=dev)
+        moe_wgrad_layout(G, off, kb_off, blocks, st, stream)
+        KP = nb * 128
+        xt = torch.empty((d, KP), dtype=u8, device=dev)
+        xts = torch.empty((nb, d), dtype=f32, device=dev)
+        moe_wgrad_quant_x(sh, b["x"], pair_scratch, blocks, xt, xts, st, stream)
+        dact = torch.empty((2 * I, KP), dtype=u8, device=dev)
+        dacts = torch.empty((nb, 2 * I), dtype=f32, device=dev)
+        moe_wgrad_quant_dac(dh, ac, I, blocks, dact, dacts, st, stream)
+        mark("wgrad_quant_x_dac")
+        dW13 = torch.empty((G, 2 * I, d), dtype=f32, device=dev)
+        moe_grouped_gemm_wgrad(G, kb_off, nb, dact, dacts, 2 * I, xt, xts, d, dW13, st, stream)
+        mark("gemm_dw13")
+        del xt, xts, dact, dacts
+        dot = torch.empty((d, KP), dtype=u8, device=dev)
+        dots = torch.empty((nb, d), dtype=f32, device=dev)
+        moe_wgrad_quant_do(sh, dy, self.topk_gate, pair_scratch, blocks, dot, dots, st, stream)
+        ht = torch.empty((I, KP), dtype=u8, device=dev)
+        hts = torch.empty((nb, I), dtype=f32, device=dev)
+        moe_wgrad_quant_h(ac, I, blocks, ht, hts, st, stream)
+        mark("wgrad_quant_do_h")
+        dW2 = torch.empty((G, d, I), dtype=f32, device=dev)
+        moe_grouped_gemm_wgrad(G, kb_off, nb, dot, dots, d, ht, hts, I, dW2, st, stream)
+        mark("gemm_dw2")
+        return dx, d_router_w, dW13, dW2
 
     def status(self, stream=None) -> int:
         """Device status word (0 = fine); synchronises the stream."""

@@ -78,6 +78,13 @@ def lib() -> ctypes.CDLL:
             "moe_gate_backward": (I, [SP, P, P, P, P, P, P, P, P]),
             "moe_router_backward": (I, [SP, P, P, P, P, P, P, P, P, P, P, P]),
             "moe_dx_combine": (I, [SP, P, P, P, P, P, P]),
+            "moe_wgrad_max_blocks": (I, [I64, I]),
+            "moe_wgrad_layout": (I, [I, P, I, P, P, P, P]),
+            "moe_wgrad_quant_x": (I, [SP, P, P, P, I, P, P, P, P]),
+            "moe_wgrad_quant_do": (I, [SP, P, P, P, P, I, P, P, P, P]),
+            "moe_wgrad_quant_h": (I, [P, I, P, I, P, P, P, P]),
+            "moe_wgrad_quant_dac": (I, [P, P, I, P, I, P, P, P, P]),
+            "moe_grouped_gemm_wgrad": (I, [I, P, I, P, P, I, P, P, I, P, P, P]),
             "fp8_quant_act_1x128": (I, [P, I64, I64, P, P, I, P, P]),
             "fp8_quant_w_128x128": (I, [P, I64, I64, P, P, P, P]),
             "moe_permute_workspace_size": (SZ, [SP]),
@@ -489,3 +496,48 @@ def moe_dx_combine(shape, dx_rows, dx_router, row_of_pair, dx, dev_status=None, 
     _check("moe_dx_combine", lib().moe_dx_combine(
         ctypes.byref(shape), _ptr(dx_rows), _ptr(dx_router), _ptr(row_of_pair), _ptr(dx),
         _ptr(dev_status), _stream(stream)))
+
+
+# ------------------------------------------------------- weight gradients
+def moe_wgrad_max_blocks(rows, n_groups) -> int:
+    return int(lib().moe_wgrad_max_blocks(int(rows), int(n_groups)))
+
+
+def moe_wgrad_layout(n_groups, row_offsets, kb_offsets, blocks, dev_status=None, stream=None):
+    """blocks: int32 [max_blocks, 2]."""
+    _check("moe_wgrad_layout", lib().moe_wgrad_layout(
+        int(n_groups), _ptr(row_offsets), int(blocks.shape[0]), _ptr(kb_offsets), _ptr(blocks),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_wgrad_quant_x(shape, x, pair_of_row, blocks, xt, xt_scales, dev_status=None,
+                      stream=None):
+    _check("moe_wgrad_quant_x", lib().moe_wgrad_quant_x(
+        ctypes.byref(shape), _ptr(x), _ptr(pair_of_row), _ptr(blocks), int(blocks.shape[0]),
+        _ptr(xt), _ptr(xt_scales), _ptr(dev_status), _stream(stream)))
+
+
+def moe_wgrad_quant_do(shape, dy, topk_gate, pair_of_row, blocks, dot, dot_scales,
+                       dev_status=None, stream=None):
+    _check("moe_wgrad_quant_do", lib().moe_wgrad_quant_do(
+        ctypes.byref(shape), _ptr(dy), _ptr(topk_gate), _ptr(pair_of_row), _ptr(blocks),
+        int(blocks.shape[0]), _ptr(dot), _ptr(dot_scales), _ptr(dev_status), _stream(stream)))
+
+
+def moe_wgrad_quant_h(ac, inter, blocks, ht, ht_scales, dev_status=None, stream=None):
+    _check("moe_wgrad_quant_h", lib().moe_wgrad_quant_h(
+        _ptr(ac), int(inter), _ptr(blocks), int(blocks.shape[0]), _ptr(ht), _ptr(ht_scales),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moe_wgrad_quant_dac(dh, ac, inter, blocks, dact, dact_scales, dev_status=None, stream=None):
+    _check("moe_wgrad_quant_dac", lib().moe_wgrad_quant_dac(
+        _ptr(dh), _ptr(ac), int(inter), _ptr(blocks), int(blocks.shape[0]), _ptr(dact),
+        _ptr(dact_scales), _ptr(dev_status), _stream(stream)))
+
+
+def moe_grouped_gemm_wgrad(n_groups, kb_offsets, nkb_total, a_t, a_scales, m, b_t, b_scales, n,
+                           out, dev_status=None, stream=None):
+    _check("moe_grouped_gemm_wgrad", lib().moe_grouped_gemm_wgrad(
+        int(n_groups), _ptr(kb_offsets), int(nkb_total), _ptr(a_t), _ptr(a_scales), int(m),
+        _ptr(b_t), _ptr(b_scales), int(n), _ptr(out), _ptr(dev_status), _stream(stream)))

@@ -347,6 +347,170 @@ __global__ void __launch_bounds__(256) transpose_w_kernel(
     }
 }
 
+
+// ------------------------------------------- weight gradients: 128x1 operands
+// K blocks of the weight-gradient GEMMs: each expert's rows (in the
+// permutation's order) cut into blocks of 128 from its first row.
+// kb_offsets[g] = first block of group g; blocks[b] = (first row, rows).
+__global__ void __launch_bounds__(1024) wgrad_layout_kernel(
+    const int32_t* __restrict__ row_offsets, int G, int max_blocks, int32_t* __restrict__ kb_offsets,
+    int2* __restrict__ blocks, int* dev_status) {
+    __shared__ int sums[1024];
+    __shared__ int total_s;
+    // blocks per group, exclusive scan (G <= 1040: a thread may hold two groups)
+    const int t = threadIdx.x;
+    int nb[2] = {0, 0};
+    for (int j = 0; j < 2; ++j) {
+        const int g = 2 * t + j;
+        if (g < G) {
+            const int rows = row_offsets[g + 1] - row_offsets[g];
+            nb[j] = rows > 0 ? (rows + 127) / 128 : 0;
+        }
+    }
+    sums[t] = nb[0] + nb[1];
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        const int v = t >= o ? sums[t - o] : 0;
+        __syncthreads();
+        sums[t] += v;
+        __syncthreads();
+    }
+    int run = sums[t] - nb[0] - nb[1];
+    if (t == 1023) total_s = sums[t];
+    for (int j = 0; j < 2; ++j) {
+        const int g = 2 * t + j;
+        if (g < G) kb_offsets[g] = min(run, max_blocks);
+        run += nb[j];
+    }
+    __syncthreads();
+    const int total = total_s;
+    if (t == 0) {
+        kb_offsets[G] = min(total, max_blocks);
+        if (total > max_blocks) set_status(dev_status, MOE_DEV_BAD_INPUT);
+    }
+    // the block table
+    for (int g = 0; g < G; ++g) {
+        const int r0 = row_offsets[g], rows = row_offsets[g + 1] - r0;
+        const int b0 = kb_offsets[g];
+        for (int j = t; j * 128 < rows; j += blockDim.x) {
+            const int b = b0 + j;
+            if (b < max_blocks) blocks[b] = make_int2(r0 + 128 * j, min(128, rows - 128 * j));
+        }
+    }
+    for (int b = total + t; b < max_blocks; b += blockDim.x) blocks[b] = make_int2(0, 0);
+}
+
+enum WgSource { kWgX = 0, kWgDo = 1, kWgH = 2, kWgDac = 3 };
+
+struct WgSrc {
+    const uint16_t* x;          // x or dy, bf16 [T, d]
+    const float* gate;          // [T, K]
+    const int32_t* pair_of_row; // [T * K]
+    const float* dh;            // [rows, I]
+    const float* ac;            // [rows, 2I]
+    int T, K, I;
+};
+
+// token of a permutation row and the gate its gradient carries
+__device__ __forceinline__ int wg_token(const WgSrc& s, int r, float& g) {
+    const int TK = s.T * s.K;
+    if (r >= TK) {
+        g = 1.0f;
+        return r - TK;
+    }
+    const int p = s.pair_of_row[r];
+    g = s.gate ? s.gate[p] : 1.0f;
+    return p / s.K;
+}
+
+__device__ __forceinline__ float wg_sigmoid(float a) { return 1.0f / (1.0f + expf(-a)); }
+
+// A CTA per (128-row block, 64 output features): the block's values in
+// shared memory, one amax per feature over the block's rows, codes written
+// transposed (the block's 128 codes of a feature contiguous).
+template <int SRC>
+__global__ void __launch_bounds__(256) wgrad_quant_kernel(
+    WgSrc src, const int2* __restrict__ blocks, int n_blocks, int F, int64_t kpitch,
+    uint8_t* __restrict__ qt, float* __restrict__ st) {
+    __shared__ __align__(16) float tile[128][68];
+    __shared__ float red[4][64];
+    const int fchunks = F / 64;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int64_t u = blockIdx.x; u < int64_t(n_blocks) * fchunks; u += gridDim.x) {
+        const int b = int(u / fchunks);
+        const int f0 = int(u - int64_t(b) * fchunks) * 64;
+        const int2 blk = blocks[b];
+        if (blk.y <= 0) continue;  // past the last expert's rows: never read
+        // ---- load: warp w, rows w, w + 8, ...; lane: features f0 + 2 lane, +1
+        for (int rr = warp; rr < 128; rr += 8) {
+            float v0 = 0.0f, v1 = 0.0f;
+            if (rr < blk.y) {
+                const int r = blk.x + rr;
+                const int f = f0 + 2 * lane;
+                if (SRC == kWgX || SRC == kWgDo) {
+                    float g;
+                    const int t = wg_token(src, r, g);
+                    const uint32_t w2 =
+                        *reinterpret_cast<const uint32_t*>(src.x + int64_t(t) * F + f);
+                    v0 = bf16_lo(w2);
+                    v1 = bf16_hi(w2);
+                    if (SRC == kWgDo) {
+                        v0 = __fmul_rn(g, v0);
+                        v1 = __fmul_rn(g, v1);
+                    }
+                } else if (SRC == kWgH) {
+                    const float* ar = src.ac + int64_t(r) * 2 * src.I;
+                    const float2 a = *reinterpret_cast<const float2*>(ar + f);
+                    const float2 c = *reinterpret_cast<const float2*>(ar + src.I + f);
+                    v0 = a.x / (1.0f + expf(-a.x)) * c.x;
+                    v1 = a.y / (1.0f + expf(-a.y)) * c.y;
+                } else {  // [da | dc]
+                    const float* ar = src.ac + int64_t(r) * 2 * src.I;
+                    const bool is_da = f < src.I;
+                    const int j = is_da ? f : f - src.I;
+                    const float2 h = *reinterpret_cast<const float2*>(src.dh + int64_t(r) * src.I + j);
+                    const float2 a = *reinterpret_cast<const float2*>(ar + j);
+                    const float sg0 = wg_sigmoid(a.x), sg1 = wg_sigmoid(a.y);
+                    if (is_da) {
+                        const float2 c = *reinterpret_cast<const float2*>(ar + src.I + j);
+                        v0 = h.x * c.x * sg0 * (1.0f + a.x * (1.0f - sg0));
+                        v1 = h.y * c.y * sg1 * (1.0f + a.y * (1.0f - sg1));
+                    } else {
+                        v0 = h.x * a.x * sg0;
+                        v1 = h.y * a.y * sg1;
+                    }
+                }
+            }
+            *reinterpret_cast<float2*>(&tile[rr][2 * lane]) = make_float2(v0, v1);
+        }
+        __syncthreads();
+        // ---- amax per feature, then codes: thread (feature f, quarter q)
+        const int f = threadIdx.x & 63, qr = threadIdx.x >> 6;
+        float amax = 0.0f;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(tile[32 * qr + i][f]));
+        red[qr][f] = amax;
+        __syncthreads();
+        amax = fmaxf(fmaxf(red[0][f], red[1][f]), fmaxf(red[2][f], red[3][f]));
+        float scale, inv;
+        scale_from_amax(amax, scale, inv);
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float* c = &tile[32 * qr + 4 * i][f];
+            const uint32_t lo = e4m3x2(__fmul_rn(c[0], inv), __fmul_rn(c[68], inv));
+            const uint32_t hi = e4m3x2(__fmul_rn(c[2 * 68], inv), __fmul_rn(c[3 * 68], inv));
+            w[i] = lo | (hi << 16);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(qt + int64_t(f0 + f) * kpitch + int64_t(b) * 128 +
+                                              32 * qr);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (qr == 0) st[int64_t(b) * F + f0 + f] = scale;
+        __syncthreads();
+    }
+}
+
 int pieces_per(int n, int& PC) {
     const int nkb = n / 128;
     PC = (nkb % 14 == 0 && nkb % 16 != 0) ? 7 : 8;
@@ -487,4 +651,82 @@ extern "C" MOE_API int moe_dx_combine(const MoeShape* shape, const float* dx_row
         reinterpret_cast<const float4*>(dx_rows), reinterpret_cast<const float4*>(dx_router), T,
         shape->d, shape->topk, row_of_pair, reinterpret_cast<float4*>(dx));
     return check_launch();
+}
+
+extern "C" MOE_API int moe_wgrad_max_blocks(int64_t rows, int n_groups) {
+    if (rows < 0 || n_groups < 1) return -1;
+    const int64_t b = (rows + 127) / 128 + n_groups;
+    return b > INT32_MAX / 128 ? -1 : int(b);
+}
+
+extern "C" MOE_API int moe_wgrad_layout(int n_groups, const int32_t* row_offsets,
+                                        int max_blocks, int32_t* kb_offsets, int32_t* blocks,
+                                        int* dev_status, void* stream) {
+    if (n_groups < 1 || n_groups > 2048 || max_blocks < 1) return MOE_ERR_SHAPE;
+    if (!row_offsets || !kb_offsets || !blocks) return MOE_ERR_NULL;
+    wgrad_layout_kernel<<<1, 1024, 0, as_stream(stream)>>>(row_offsets, n_groups, max_blocks,
+                                                           kb_offsets,
+                                                           reinterpret_cast<int2*>(blocks),
+                                                           dev_status);
+    return check_launch();
+}
+
+namespace {
+template <int SRC>
+int launch_wgrad_quant(const WgSrc& src, const int32_t* blocks, int n_blocks, int F,
+                       uint8_t* qt, float* st, void* stream) {
+    if (n_blocks < 0 || F <= 0 || F % 64) return MOE_ERR_SHAPE;
+    if (n_blocks == 0) return MOE_OK;
+    if (!blocks || !qt || !st) return MOE_ERR_NULL;
+    if (!aligned16(qt)) return MOE_ERR_ALIGN;
+    const int64_t units = int64_t(n_blocks) * (F / 64);
+    const int grid = int(std::min<int64_t>(units, int64_t(sm_count()) * 8));
+    wgrad_quant_kernel<SRC><<<grid, 256, 0, as_stream(stream)>>>(
+        src, reinterpret_cast<const int2*>(blocks), n_blocks, F, int64_t(n_blocks) * 128, qt, st);
+    return check_launch();
+}
+}  // namespace
+
+extern "C" MOE_API int moe_wgrad_quant_x(const MoeShape* shape, const uint16_t* x,
+                                         const int32_t* pair_of_row, const int32_t* blocks,
+                                         int n_blocks, uint8_t* xt, float* xt_scales,
+                                         int* dev_status, void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    if (shape->T > 0 && (!x || !pair_of_row)) return MOE_ERR_NULL;
+    WgSrc s{x, nullptr, pair_of_row, nullptr, nullptr, shape->T, shape->topk, shape->inter};
+    return launch_wgrad_quant<kWgX>(s, blocks, n_blocks, shape->d, xt, xt_scales, stream);
+}
+
+extern "C" MOE_API int moe_wgrad_quant_do(const MoeShape* shape, const uint16_t* dy,
+                                          const float* topk_gate, const int32_t* pair_of_row,
+                                          const int32_t* blocks, int n_blocks, uint8_t* dot,
+                                          float* dot_scales, int* dev_status, void* stream) {
+    (void)dev_status;
+    int rc = validate_shape(shape);
+    if (rc != MOE_OK) return rc;
+    if (shape->T > 0 && (!dy || !topk_gate || !pair_of_row)) return MOE_ERR_NULL;
+    WgSrc s{dy, topk_gate, pair_of_row, nullptr, nullptr, shape->T, shape->topk, shape->inter};
+    return launch_wgrad_quant<kWgDo>(s, blocks, n_blocks, shape->d, dot, dot_scales, stream);
+}
+
+extern "C" MOE_API int moe_wgrad_quant_h(const float* ac, int inter, const int32_t* blocks,
+                                         int n_blocks, uint8_t* ht, float* ht_scales,
+                                         int* dev_status, void* stream) {
+    (void)dev_status;
+    if (inter <= 0 || inter % 128) return MOE_ERR_SHAPE;
+    if (n_blocks > 0 && !ac) return MOE_ERR_NULL;
+    WgSrc s{nullptr, nullptr, nullptr, nullptr, ac, 0, 1, inter};
+    return launch_wgrad_quant<kWgH>(s, blocks, n_blocks, inter, ht, ht_scales, stream);
+}
+
+extern "C" MOE_API int moe_wgrad_quant_dac(const float* dh, const float* ac, int inter,
+                                           const int32_t* blocks, int n_blocks, uint8_t* dact,
+                                           float* dact_scales, int* dev_status, void* stream) {
+    (void)dev_status;
+    if (inter <= 0 || inter % 128) return MOE_ERR_SHAPE;
+    if (n_blocks > 0 && (!dh || !ac)) return MOE_ERR_NULL;
+    WgSrc s{nullptr, nullptr, nullptr, dh, ac, 0, 1, inter};
+    return launch_wgrad_quant<kWgDac>(s, blocks, n_blocks, 2 * inter, dact, dact_scales, stream);
 }

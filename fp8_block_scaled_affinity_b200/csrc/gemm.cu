@@ -1618,6 +1618,328 @@ int launch(const GemmParams& p, const CUtensorMap& mw, const AMaps& ma, const CU
     return check_launch();
 }
 
+// ============================================== weight-gradient form (K-grouped)
+// out[g] (fp32 [M, N]) = sum over the K blocks of group g of the products of
+// A rows and B rows, with a scale per (row, K block) on BOTH operands: the
+// weight gradients, whose contraction runs over one expert's token rows and
+// whose two operands are activations quantised in 128x1 tiles along the
+// tokens ("DeepSeek-V3 Technical Report" notes page, section "FP8 mixed
+// precision training": all three linear GEMMs take FP8 inputs; the
+// transposed activations need tiles along the other dimension).  A and B are
+// stored transposed, K (the tokens, each group's rows padded to a multiple of
+// 128) contiguous, so the tensor core sees ordinary K-major tiles; a group is
+// a range of K blocks, not of rows.  The promotion is the forward's with the
+// combined scale sa[row of A] * sb[row of B] per element (one more multiply
+// per pair of values).  Every item covers 128 rows of A and 256 of B; an
+// item whose group has no K blocks stores zeros (an expert no token chose).
+struct WgCfg {
+    static constexpr int kStages = 3;
+    static constexpr int kStageBytes = kTileBytes + 256 * 128;  // A tile + two B boxes
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kParkBytes = kPromoters * kBoxBytes;
+    static constexpr int kSbBytes = kScaleSlots * 256 * 4;      // B scales of a K block
+    static constexpr int kBufs = 2;                             // 256-column TMEM partials
+};
+constexpr size_t wg_smem_bytes() {
+    return size_t(WgCfg::kRingBytes) + WgCfg::kParkBytes + WgCfg::kSbBytes +
+           sizeof(SharedState) + 1024;
+}
+static_assert(wg_smem_bytes() <= 232448, "dynamic shared memory above the sm_100 limit per CTA");
+
+struct WgParams {
+    const int32_t* kb_offsets;  // [n_groups + 1] K-block ranges of the groups
+    int n_groups;
+    int m, n;                   // rows of A and of B (output [n_groups, m, n])
+    int nkb_total;              // K blocks of A and B
+    int m_tiles, n_tiles;       // m / 128, n / 256
+    const float* a_scales;      // [nkb_total, m]
+    const float* b_scales;      // [nkb_total, n]
+    int* dev_status;
+    uint64_t wait_limit_ns;
+    GemmParams out;             // epilogue fields (fp32 output, row pitch n)
+};
+
+struct WgItem {
+    int g, mt, f, kb0, kb1;
+};
+__device__ __forceinline__ WgItem wg_item(const SharedState* ss, const WgParams& p, int item) {
+    const int per = p.m_tiles * p.n_tiles;
+    WgItem w;
+    w.g = item / per;
+    const int local = item - w.g * per;
+    w.f = local / p.m_tiles;  // m tiles fastest: neighbouring CTAs share B
+    w.mt = local - w.f * p.m_tiles;
+    w.kb0 = ss->goff[w.g];
+    w.kb1 = ss->goff[w.g + 1];
+    return w;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ void wg_producer(const WgParams& p, const CUtensorMap* map_a,
+                                            const CUtensorMap* map_b, uint8_t* smem,
+                                            SharedState* ss, int unit, int units) {
+    using C = WgCfg;
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    uint32_t it = 0, issued_mask = 0, issued_parity = 0;
+    bool ok = true;
+    for (int item = unit; ok && item < total_items; item += units) {
+        const WgItem w = wg_item(ss, p, item);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+            const int s = it % C::kStages;
+            const uint32_t par = (it / C::kStages) & 1u;
+            if (lane == 0) ok = mbar_wait(smem_u32(&ss->empty[s]), par ^ 1u, ss, p.dev_status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
+                uint8_t* st = smem + size_t(s) * C::kStageBytes;
+                const uint32_t fb = smem_u32(&ss->full[s]);
+                mbar_arrive_expect_tx(fb, uint32_t(C::kStageBytes));
+                tma_load_2d<false>(smem_u32(st), map_a, fb, kb * 128, w.mt * 128);
+                tma_load_2d<false>(smem_u32(st + kTileBytes), map_b, fb, kb * 128, w.f * 256);
+                tma_load_2d<false>(smem_u32(st + 2 * kTileBytes), map_b, fb, kb * 128,
+                                   w.f * 256 + 128);
+                issued_mask |= 1u << s;
+                issued_parity = (issued_parity & ~(1u << s)) | (par << s);
+            }
+        }
+    }
+    if (!ok && lane == 0)
+        for (int s = 0; s < C::kStages; ++s)
+            if ((issued_mask >> s) & 1u)
+                mbar_quiesce(smem_u32(&ss->full[s]), (issued_parity >> s) & 1u, ss, nullptr);
+    __syncwarp();
+}
+
+// warp 2: per K block, the 128 A scales into sa[slot] and the 256 B scales
+// into the slot's row of sb_area (16-byte asynchronous copies).
+__device__ __forceinline__ void wg_scale_loader(const WgParams& p, float* sb_area,
+                                                SharedState* ss, int unit, int units) {
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    uint32_t cit = 0;
+    bool ok = true;
+    for (int item = unit; ok && item < total_items; item += units) {
+        const WgItem w = wg_item(ss, p, item);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++cit) {
+            const int c = cit % kScaleSlots;
+            if (lane == 0)
+                ok = mbar_wait(smem_u32(&ss->sempty[c]), ((cit / kScaleSlots) & 1u) ^ 1u, ss,
+                               p.dev_status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const float* sa = p.a_scales + size_t(kb) * p.m + w.mt * 128;
+            const float* sb = p.b_scales + size_t(kb) * p.n + w.f * 256;
+            cp_async16(&ss->sa[c][4 * lane], sa + 4 * lane);
+            cp_async16(sb_area + c * 256 + 4 * lane, sb + 4 * lane);
+            cp_async16(sb_area + c * 256 + 128 + 4 * lane, sb + 128 + 4 * lane);
+            cp_async_arrive(smem_u32(&ss->sfull[c]));
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncwarp();
+}
+
+__device__ __forceinline__ void wg_mma_issuer(const WgParams& p, uint8_t* smem, SharedState* ss,
+                                              uint32_t tmem_base, int unit, int units) {
+    using C = WgCfg;
+    const int lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        const uint32_t idesc = idesc_e4m3(128, 256);
+        for (int item = unit; ok && item < total_items; item += units) {
+            const WgItem w = wg_item(ss, p, item);
+            for (int kb = w.kb0; ok && kb < w.kb1; ++kb, ++it) {
+                const int s = it % C::kStages;
+                const uint32_t buf = it % C::kBufs;
+                ok = mbar_wait(smem_u32(&ss->full[s]), (it / C::kStages) & 1u, ss, p.dev_status) &&
+                     mbar_wait(smem_u32(&ss->tempty[buf]), ((it / C::kBufs) & 1u) ^ 1u, ss,
+                               p.dev_status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = smem_u32(smem + size_t(s) * C::kStageBytes);
+                const uint32_t d = tmem_base + buf * 256;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_e4m3<false>(d, sw128_desc(st + kk * 32),
+                                    sw128_desc(st + kTileBytes + kk * 32), idesc, kk > 0 ? 1u : 0u);
+                mma_commit<false>(smem_u32(&ss->empty[s]));
+                mma_commit<false>(smem_u32(&ss->tfull[buf]));
+            }
+        }
+        mma_commit<false>(smem_u32(&ss->drain));
+        mbar_quiesce(smem_u32(&ss->drain), 0, ss, nullptr);
+    }
+    __syncwarp();
+}
+
+// A shared-memory load the compiler keeps in program order (plain loads of
+// the B scales were all hoisted to the top of the K block, and the
+// registers they took spilled the accumulators).
+__device__ __forceinline__ uint64_t ld_shared_volatile(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.volatile.shared.b64 %0, [%1];" : "=l"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
+// acc2[o + i] += v pair i * (sa * sb pair o + i) for 16 pairs, eight pairs
+// of B scales at a time.
+__device__ __forceinline__ void wg_fold(uint64_t (&acc2)[64], const uint32_t (&v)[32],
+                                        uint64_t sa2, const uint64_t* sb2, int o) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        uint64_t s[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i] = fmul2(sa2, ld_shared_volatile(sb2 + o + 8 * j + i));
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            ffma2(acc2[o + 8 * j + i], pack2(v[2 * (8 * j + i)], v[2 * (8 * j + i) + 1]), s[i]);
+    }
+}
+
+// warps 4-11: thread (w, l) owns A row 32 (w % 4) + l of the item and the
+// 128 B rows [128 h, 128 h + 128) of its 256, h = (w - 4) / 4.
+__device__ __forceinline__ void wg_promoter(const WgParams& p, SharedState* ss,
+                                            const float* sb_area, char* park_area,
+                                            uint32_t tmem_base, const CUtensorMap* map_o,
+                                            int unit, int units) {
+    using C = WgCfg;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total_items = ss->total_items;
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int r = q * 32 + lane;
+    const uint32_t lane_addr = tmem_base + (uint32_t(q * 32) << 16);
+    const int c0 = 128 * half;
+    uint32_t it = 0;
+    bool ok = true;
+    char* const wpark = park_area + (warp - 4) * kBoxBytes;
+    for (int item = unit; item < total_items; item += units) {
+        const WgItem w = wg_item(ss, p, item);
+        uint64_t acc2[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc2[i] = 0;
+        for (int kb = w.kb0; ok && kb < w.kb1; ++kb, ++it) {
+            const uint32_t buf = it % C::kBufs;
+            const int c = it % kScaleSlots;
+            if (lane == 0) {
+                ok = mbar_wait(smem_u32(&ss->tfull[buf]), (it / C::kBufs) & 1u, ss, p.dev_status);
+                if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (it / kScaleSlots) & 1u, ss,
+                                       p.dev_status);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            __syncwarp();
+            tc_fence_after();
+            const float sa = ss->sa[c][r];
+            const uint64_t sa2 = pack2(__float_as_uint(sa), __float_as_uint(sa));
+            const uint64_t* sb2 = reinterpret_cast<const uint64_t*>(sb_area + c * 256 + c0);
+            const uint32_t tbase = lane_addr + buf * 256;
+            // 32 columns per TMEM load (the per-column scales need the
+            // registers a 64-column load would take)
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                tmem_ld32(tbase + c0 + 32 * j, v);
+                wg_fold(acc2, v, sa2, sb2, 16 * j);
+            }
+            tmem_ld32(tbase + c0 + 96, v);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ss->tempty[buf]));
+            wg_fold(acc2, v, sa2, sb2, 48);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
+        }
+        store_rows<64, 1>(p.out, acc2, wpark, map_o, lane, 32, 0,
+                          w.g * p.m + w.mt * 128 + q * 32, w.f * 256 + c0);
+        const bool any_abort = named_bar_or(
+            2, kPromoters * 32, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
+        if (any_abort) break;
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+    tc_fence_before();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                      const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_o, const WgParams p) {
+    using C = WgCfg;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    char* park = reinterpret_cast<char*>(smem + C::kRingBytes);
+    float* sb_area = reinterpret_cast<float*>(smem + C::kRingBytes + C::kParkBytes);
+    SharedState* ss = reinterpret_cast<SharedState*>(smem + size_t(C::kRingBytes) + C::kParkBytes +
+                                                     C::kSbBytes);
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&ss->full[s]), 1);
+            mbar_init(smem_u32(&ss->empty[s]), 1);
+        }
+        for (int b = 0; b < C::kBufs; ++b) {
+            mbar_init(smem_u32(&ss->tfull[b]), 1);
+            mbar_init(smem_u32(&ss->tempty[b]), kPromoters);
+        }
+        for (int c = 0; c < kScaleSlots; ++c) {
+            mbar_init(smem_u32(&ss->sfull[c]), 32);
+            mbar_init(smem_u32(&ss->sempty[c]), kPromoters);
+        }
+        mbar_init(smem_u32(&ss->drain), 1);
+        ss->wait_limit = p.wait_limit_ns;
+        ss->abort_flag = 0;
+        ss->peer_abort = 0u;
+        ss->total_items = p.n_groups * p.m_tiles * p.n_tiles;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc_all<false>(smem_u32(&ss->tmem_base));
+    // K-block ranges (validated: non-decreasing, inside [0, nkb_total])
+    const int G = p.n_groups;
+    int bad = 0;
+    for (int i = threadIdx.x; i <= G; i += kThreads) {
+        const int v = p.kb_offsets[i];
+        ss->goff[i] = v;
+        if (v < 0 || v > p.nkb_total || (i > 0 && v < p.kb_offsets[i - 1])) bad = 1;
+    }
+    if (__syncthreads_or(bad)) {
+        if (threadIdx.x == 0) set_status(p.dev_status, MOE_DEV_BAD_INPUT);
+        for (int i = threadIdx.x; i <= G; i += kThreads) ss->goff[i] = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ss->tmem_base;
+    const int unit = int(blockIdx.x), units = int(gridDim.x);
+    if (warp < 4) {
+        set_max_regs_dec<72>();
+        if (warp == 0) wg_producer(p, &map_a, &map_b, smem, ss, unit, units);
+        else if (warp == 1) wg_mma_issuer(p, smem, ss, tmem_base, unit, units);
+        else if (warp == 2) wg_scale_loader(p, sb_area, ss, unit, units);
+    } else {
+        set_max_regs_inc<208>();
+        wg_promoter(p, ss, sb_area, park, tmem_base, &map_o, unit, units);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_free_all<false>(tmem_base);
+    }
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ host
@@ -1849,4 +2171,58 @@ extern "C" MOE_API int moe_grouped_gemm_mxfp8(int n_groups, const int32_t* group
         return MOE_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     return swiglu ? launch_mx<true>(p, mw, ma, mo, st) : launch_mx<false>(p, mw, ma, mo, st);
+}
+
+extern "C" MOE_API int moe_grouped_gemm_wgrad(int n_groups, const int32_t* kb_offsets,
+                                              int nkb_total, const uint8_t* a_t,
+                                              const float* a_scales, int m, const uint8_t* b_t,
+                                              const float* b_scales, int n, float* out,
+                                              int* dev_status, void* stream) {
+    if (n_groups < 1 || n_groups > kMaxGroups || nkb_total < 0 || m <= 0 || m % 128 || n <= 0 ||
+        n % 256)
+        return MOE_ERR_SHAPE;
+    if (int64_t(n_groups) * m > INT32_MAX || int64_t(nkb_total) * 128 > INT32_MAX)
+        return MOE_ERR_SHAPE;
+    if (!kb_offsets || !out) return MOE_ERR_NULL;
+    const bool empty_k = nkb_total == 0;
+    if (!empty_k && (!a_t || !a_scales || !b_t || !b_scales)) return MOE_ERR_NULL;
+    if (!aligned16(out) || (!empty_k && (!aligned16(a_t) || !aligned16(b_t) ||
+                                         !aligned16(a_scales) || !aligned16(b_scales))))
+        return MOE_ERR_ALIGN;
+    if (!device_is_sm100()) return MOE_ERR_DEVICE;
+    cudaStream_t st = as_stream(stream);
+    if (empty_k) {
+        // no token rows at all: every gradient is zero
+        return cudaMemsetAsync(out, 0, sizeof(float) * size_t(n_groups) * m * n, st) ==
+                       cudaSuccess
+                   ? MOE_OK
+                   : MOE_ERR_CUDA;
+    }
+    WgParams p;
+    p.kb_offsets = kb_offsets;
+    p.n_groups = n_groups;
+    p.m = m;
+    p.n = n;
+    p.nkb_total = nkb_total;
+    p.m_tiles = m / 128;
+    p.n_tiles = n / 256;
+    p.a_scales = a_scales;
+    p.b_scales = b_scales;
+    p.dev_status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+    p.out = GemmParams{};
+    p.out.epilogue = MOE_EPI_F32;
+    p.out.out = out;
+    p.out.n = n;
+    p.out.dev_status = dev_status;
+    CUtensorMap ma, mb, mo;
+    const uint64_t kcols = uint64_t(nkb_total) * 128;
+    if (!make_map(&ma, a_t, uint64_t(m), kcols, 128) || !make_map(&mb, b_t, uint64_t(n), kcols, 128) ||
+        !make_out_map(&mo, out, uint64_t(n_groups) * m, uint64_t(n), false))
+        return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(wgrad_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(wg_smem_bytes())) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    wgrad_gemm_kernel<<<sm_count(), kThreads, wg_smem_bytes(), st>>>(ma, mb, mo, p);
+    return check_launch();
 }

@@ -578,7 +578,7 @@ MOE_API int moe_layer_forward_host_batches(const MoeShape* shape, const MoeWeigh
  *   moe_swiglu_backward_quant -> [da | dc] FP8 1x128 (2I)
  *   moe_grouped_gemm_fp8 ([da|dc], W13 transposed, n = d, F32) -> dx rows
  *   moe_gate_backward, moe_router_backward, moe_dx_combine -> dx, dE.
- * Gradients of the expert weights (Wgrad) are not part of the library.
+ * The expert weights' gradients (Wgrad) follow below.
  * ==================================================================== */
 
 /* fp8_transpose_w_128x128: for mats matrices of FP8 codes [rows, cols] with
@@ -637,7 +637,8 @@ MOE_API int moe_gate_backward(const MoeShape* shape, const uint16_t* dy, const f
  *                  unchosen expert)
  *   x bf16 [T, d]; router_w bf16 [N_r, d]; topk_idx int32 [T, K];
  *   expert_offsets int32 [N_r + 2] and row_of_pair int32 [T, K] (the
- *   forward's permutation); pair_scratch int32 [T*K] scratch.
+ *   forward's permutation); pair_scratch int32 [T*K] out: the
+ *   permutation's inverse over the routed rows (pair t*K + k of each row).
  * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_CUDA;
  * MOE_DEV_BAD_INPUT on dev_status for an expert index out of range. */
 MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t* x,
@@ -654,6 +655,78 @@ MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t* x,
 MOE_API int moe_dx_combine(const MoeShape* shape, const float* dx_rows, const float* dx_router,
                            const int32_t* row_of_pair, float* dx, int* dev_status,
                            void* stream);
+
+/* -------------------------------------------------- weight gradients
+ * dW13_e [2I, d] = sum over expert e's rows of [da | dc]^T x and
+ * dW2_e [d, I] = sum of do^T h (h = silu(a) c), as FP8 GEMMs whose operands
+ * are quantised in 128x1 tiles along the rows ("DeepSeek-V3 Technical
+ * Report" notes page, section "FP8 mixed precision training": Wgrad in FP8;
+ * the pages' request for transposed-operand support).  Each expert's rows,
+ * in the forward's permutation order, are cut into K blocks of 128 from its
+ * first row; an operand is stored transposed, [features, n_blocks * 128]
+ * uint8 codes (a block's 128 codes of a feature contiguous, rows past the
+ * expert's end zero) with fp32 scales [n_blocks, features], one per feature
+ * and block (amax/448 rule of the 1x128 quantiser).  The value sources:
+ * x from the layer input (bf16), do = fp32(gate dy), h and [da | dc] from
+ * the recomputed fp32 a and c and dh. */
+
+/* Blocks an operand array must hold for `rows` permutation rows in
+ * n_groups groups: ceil(rows/128) + n_groups (-1 for invalid arguments). */
+MOE_API int moe_wgrad_max_blocks(int64_t rows, int n_groups);
+
+/* moe_wgrad_layout: from row_offsets (int32 [n_groups + 1], the forward's
+ * expert_offsets with the shared expert as the last group) the K-block
+ * offsets kb_offsets (int32 [n_groups + 1] out) and the block table blocks
+ * (int32 [max_blocks, 2] out: first row, rows; (0, 0) past the last block).
+ * One CTA.  More blocks than max_blocks: MOE_DEV_BAD_INPUT on dev_status.
+ * Errors: MOE_ERR_SHAPE (n_groups outside [1, 2048], max_blocks < 1),
+ * MOE_ERR_NULL, MOE_ERR_CUDA. */
+MOE_API int moe_wgrad_layout(int n_groups, const int32_t* row_offsets, int max_blocks,
+                             int32_t* kb_offsets, int32_t* blocks, int* dev_status, void* stream);
+
+/* The 128x1 quantisers (blocks / n_blocks: the layout's table and its
+ * length, which is also the K extent of the output arrays):
+ *   moe_wgrad_quant_x:   x bf16 [T, d] -> xt [d, n_blocks*128], scales
+ *                        [n_blocks, d]; row r takes the token of its pair
+ *                        (pair_of_row, the permutation's inverse over the
+ *                        T*K routed rows, as moe_router_backward leaves it in
+ *                        pair_scratch), shared row T*K + t token t;
+ *   moe_wgrad_quant_do:  the same with fp32(topk_gate[pair] * dy) (dy on the
+ *                        shared rows) -> dot [d, ...];
+ *   moe_wgrad_quant_h:   ac fp32 [rows, 2I] -> ht [I, ...] of
+ *                        h = a / (1 + e^-a) * c;
+ *   moe_wgrad_quant_dac: dh fp32 [rows, I], ac -> dact [2I, ...] of
+ *                        [da | dc] as moe_swiglu_backward_quant forms them.
+ * Output codes 16-byte aligned.  Errors: MOE_ERR_SHAPE, MOE_ERR_NULL,
+ * MOE_ERR_ALIGN, MOE_ERR_CUDA. */
+MOE_API int moe_wgrad_quant_x(const MoeShape* shape, const uint16_t* x,
+                              const int32_t* pair_of_row, const int32_t* blocks, int n_blocks,
+                              uint8_t* xt, float* xt_scales, int* dev_status, void* stream);
+MOE_API int moe_wgrad_quant_do(const MoeShape* shape, const uint16_t* dy, const float* topk_gate,
+                               const int32_t* pair_of_row, const int32_t* blocks, int n_blocks,
+                               uint8_t* dot, float* dot_scales, int* dev_status, void* stream);
+MOE_API int moe_wgrad_quant_h(const float* ac, int inter, const int32_t* blocks, int n_blocks,
+                              uint8_t* ht, float* ht_scales, int* dev_status, void* stream);
+MOE_API int moe_wgrad_quant_dac(const float* dh, const float* ac, int inter,
+                                const int32_t* blocks, int n_blocks, uint8_t* dact,
+                                float* dact_scales, int* dev_status, void* stream);
+
+/* moe_grouped_gemm_wgrad: out[g] (fp32 [m, n], groups back to back) =
+ * sum over the K blocks kb in [kb_offsets[g], kb_offsets[g+1]) of
+ * a_scales[kb, i] b_scales[kb, j] sum_{k in kb} A[i, k] B[j, k], the
+ * products exact on the tensor cores, each K block promoted into an FP32
+ * accumulator with its two scales; a group with no K blocks gets zeros.
+ *   a_t uint8 [m, nkb_total*128] (E4M3), a_scales fp32 [nkb_total, m];
+ *   b_t uint8 [n, nkb_total*128], b_scales fp32 [nkb_total, n];
+ *   kb_offsets int32 [n_groups + 1], non-decreasing, within [0, nkb_total]
+ *   (else MOE_DEV_BAD_INPUT on dev_status and nothing is computed).
+ * m % 128 == 0, n % 256 == 0, pointers 16-byte aligned.  Errors:
+ * MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_DEVICE, MOE_ERR_CUDA;
+ * MOE_DEV_TIMEOUT as the forward GEMM. */
+MOE_API int moe_grouped_gemm_wgrad(int n_groups, const int32_t* kb_offsets, int nkb_total,
+                                   const uint8_t* a_t, const float* a_scales, int m,
+                                   const uint8_t* b_t, const float* b_scales, int n, float* out,
+                                   int* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -266,3 +266,228 @@ def test_layer_backward_full_expert_shapes_16_experts():
 
 def test_layer_backward_decode_full_size():
     _layer_case("decode", S.CONFIGS["decode"])
+
+
+# ------------------------------------------------------ weight gradients
+def _inverse(rop, R):
+    """pair_of_row of the routed rows from row_of_pair (host)."""
+    inv = np.zeros((rop.size,), np.int32)
+    inv[rop.ravel()] = np.arange(rop.size, dtype=np.int32)
+    return inv
+
+
+def _layout_ref(off, max_blocks):
+    G = len(off) - 1
+    kb = np.zeros(G + 1, np.int32)
+    blocks = np.zeros((max_blocks, 2), np.int32)
+    for g in range(G):
+        rows = int(off[g + 1] - off[g])
+        nb = -(-rows // 128)
+        kb[g + 1] = kb[g] + nb
+        for j in range(nb):
+            blocks[kb[g] + j] = (off[g] + 128 * j, min(128, rows - 128 * j))
+    return kb, blocks
+
+
+def test_wgrad_layout_bit_exact():
+    need_gpu()
+    moe = _moe()
+    sizes = [0, 1, 127, 128, 129, 0, 300, 5, 0]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    nb = moe.moe_wgrad_max_blocks(off[-1], len(sizes))
+    kb = torch.empty((len(sizes) + 1,), dtype=torch.int32, device=DEV)
+    blocks = torch.full((nb, 2), 9, dtype=torch.int32, device=DEV)
+    moe.moe_wgrad_layout(len(sizes), to_dev(off), kb, blocks)
+    torch.cuda.synchronize()
+    kb_ref, blocks_ref = _layout_ref(off, nb)
+    assert np.array_equal(kb.cpu().numpy(), kb_ref)
+    assert np.array_equal(blocks.cpu().numpy(), blocks_ref)
+
+
+def _wgrad_setup(T, d, N, K, seed):
+    rng = np.random.default_rng(seed)
+    idx, counts, off, rop = _routing(rng, T, N, K, n_choosable=N - 1)
+    R = T * K + T
+    moe = _moe()
+    nb = moe.moe_wgrad_max_blocks(R, N + 1)
+    kb = torch.empty((N + 2,), dtype=torch.int32, device=DEV)
+    blocks = torch.empty((nb, 2), dtype=torch.int32, device=DEV)
+    moe.moe_wgrad_layout(N + 1, to_dev(off), kb, blocks)
+    torch.cuda.synchronize()
+    return rng, idx, off, rop, R, nb, kb, blocks
+
+
+def _expert_rows(off, e):
+    return np.arange(off[e], off[e + 1])
+
+
+@pytest.mark.parametrize("source", ["x", "do"])
+def test_wgrad_quant_x_and_do_bit_exact(source):
+    """The transposed 128x1 operands of x and of do = fp32(gate dy) equal the
+    oracle's 128x1 quantisation of each expert's rows (in permutation order),
+    codes and scales; an unchosen expert has no blocks."""
+    need_gpu()
+    moe = _moe()
+    T, d, N, G, M, K = 150, 256, 8, 2, 2, 2
+    rng, idx, off, rop, R, nb, kb, blocks = _wgrad_setup(T, d, N, K, 80)
+    x = S.host_normal_bf16(rng, (T, d), 1.0)
+    gate = rng.random((T, K)).astype(np.float32)
+    inv = _inverse(rop, R)
+    sh = moe.make_shape(T, d, N, G, M, K, 128)
+    q = torch.zeros((d, nb * 128), dtype=torch.uint8, device=DEV)
+    s = torch.zeros((nb, d), dtype=torch.float32, device=DEV)
+    if source == "x":
+        moe.moe_wgrad_quant_x(sh, bf16_dev(x), to_dev(inv), blocks, q, s)
+    else:
+        moe.moe_wgrad_quant_do(sh, bf16_dev(x), to_dev(gate), to_dev(inv), blocks, q, s)
+    torch.cuda.synchronize()
+    q, s, kbh = q.cpu().numpy(), s.cpu().numpy(), kb.cpu().numpy()
+    x32 = S.bf16_bits_to_f32(x)
+    for e in range(N + 1):
+        rows = _expert_rows(off, e)
+        if rows.size == 0:
+            assert kbh[e] == kbh[e + 1]
+            continue
+        toks = np.where(rows >= T * K, rows - T * K, inv[np.minimum(rows, T * K - 1)] // K)
+        if source == "x":
+            vals = x[toks]
+        else:
+            g = np.where(rows >= T * K, np.float32(1.0),
+                         gate.ravel()[inv[np.minimum(rows, T * K - 1)]]).astype(np.float32)
+            vals = (g[:, None] * x32[toks]).astype(np.float32)
+        q_ref, s_ref = oracle.quant_act_128x1(np.ascontiguousarray(vals))
+        k0, k1 = int(kbh[e]), int(kbh[e + 1])
+        assert np.array_equal(q[:, 128 * k0:128 * k1], q_ref), e
+        assert np.array_equal(s[k0:k1].T.view(U32), s_ref.view(U32)), e
+
+
+@pytest.mark.parametrize("source", ["h", "dac"])
+def test_wgrad_quant_h_and_dac(source):
+    """h = silu(a) c and [da | dc] from fp32 inputs: codes equal the oracle's
+    quantisation of the FP64 values (rounded to fp32) except at rare E4M3
+    rounding boundaries; dequantised within one step of the exact value."""
+    need_gpu()
+    moe = _moe()
+    T, d, N, K, I = 150, 256, 8, 2, 256
+    rng, idx, off, rop, R, nb, kb, blocks = _wgrad_setup(T, d, N, K, 81)
+    ac = (rng.standard_normal((R, 2 * I)) * 2.0).astype(np.float32)
+    dh = rng.standard_normal((R, I)).astype(np.float32)
+    F = I if source == "h" else 2 * I
+    q = torch.zeros((F, nb * 128), dtype=torch.uint8, device=DEV)
+    s = torch.zeros((nb, F), dtype=torch.float32, device=DEV)
+    if source == "h":
+        moe.moe_wgrad_quant_h(to_dev(ac), I, blocks, q, s)
+    else:
+        moe.moe_wgrad_quant_dac(to_dev(dh), to_dev(ac), I, blocks, q, s)
+    torch.cuda.synchronize()
+    q, s, kbh = q.cpu().numpy(), s.cpu().numpy(), kb.cpu().numpy()
+    a64, c64 = ac[:, :I].astype(np.float64), ac[:, I:].astype(np.float64)
+    if source == "h":
+        exact = a64 / (1.0 + np.exp(-a64)) * c64
+    else:
+        exact = np.concatenate(oracle.swiglu_backward(dh, a64, c64), axis=1)
+    same, total = 0, 0
+    for e in range(N + 1):
+        rows = _expert_rows(off, e)
+        if rows.size == 0:
+            continue
+        k0, k1 = int(kbh[e]), int(kbh[e + 1])
+        q_ref, s_ref = oracle.quant_act_128x1(exact[rows].astype(np.float32))
+        qe, se = q[:, 128 * k0:128 * k1], s[k0:k1].T.copy()
+        assert np.all(np.abs(se - s_ref) <= 16 * 2.0**-24 * np.abs(s_ref)), e
+        same += int(np.sum(qe == q_ref))
+        total += qe.size
+        deq = oracle.dequant_act(qe, se)[:, :rows.size].T
+        step = np.repeat(se.T, 128, axis=0)[:rows.size]
+        ex = exact[rows]
+        assert np.all(np.abs(deq - ex) <= 2.0**-3 * np.abs(ex) + 2.0**-9 * step), e
+    _report({"case": f"wgrad quant {source}", "codes_equal_frac": same / total})
+    assert same / total >= 0.999
+
+
+@pytest.mark.parametrize("m,n,kbs", [(256, 512, [0, 3, 3, 5, 9]), (128, 256, [0, 1]),
+                                     (384, 768, [0, 0, 2, 2, 20])])
+def test_grouped_gemm_wgrad(m, n, kbs):
+    """K-grouped GEMM with per-row scales on both operands against the
+    oracle, within the FP32 accumulation bound; empty groups give zeros."""
+    need_gpu()
+    moe = _moe()
+    rng = np.random.default_rng(90 + m)
+    nkb = kbs[-1] + 1  # one trailing block no group uses
+    table = oracle.e4m3_decode_table()
+    finite = np.nonzero(np.isfinite(table))[0].astype(np.uint8)
+    a = rng.choice(finite, (m, 128 * nkb)).astype(np.uint8)
+    b = rng.choice(finite, (n, 128 * nkb)).astype(np.uint8)
+    sa = (2.0 ** rng.uniform(-12, -6, (nkb, m))).astype(np.float32)
+    sb = (2.0 ** rng.uniform(-12, -6, (nkb, n))).astype(np.float32)
+    kb_off = np.array(kbs, np.int32)
+    G = len(kbs) - 1
+    out = torch.full((G, m, n), 3.0, dtype=torch.float32, device=DEV)
+    st = torch.zeros((1,), dtype=torch.int32, device=DEV)
+    moe.moe_grouped_gemm_wgrad(G, to_dev(kb_off), nkb, to_dev(a), to_dev(sa), m, to_dev(b),
+                               to_dev(sb), n, out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = oracle.gemm_wgrad(a, sa, b, sb, kb_off)
+    # the same sums over |products|: codes with the sign bit cleared
+    mag = oracle.gemm_wgrad((a & 0x7F).astype(np.uint8), sa, (b & 0x7F).astype(np.uint8), sb,
+                            kb_off)
+    got = out.cpu().numpy()
+    nk = np.diff(kb_off)[:, None, None]
+    assert np.all(np.abs(got - ref) <= 2.0**-23 * (128 + nk + 2) * mag)
+    for g in range(G):
+        if kb_off[g] == kb_off[g + 1]:
+            assert np.all(got[g] == 0.0)
+
+
+DW_TOL = 2e-3
+
+
+def _wgrad_case(name, cfg, T=None, experts=None, seed=71):
+    need_gpu()
+    moe = _moe()
+    inp = S.make_layer_inputs_host(cfg, 0)
+    T = cfg.T if T is None else T
+    layer = moe.MoeLayer(shape_of(cfg, T), bf16_dev(inp["router_w"]), to_dev(inp["bias"]),
+                         device=DEV)
+    for e in range(cfg.n_routed + 1):
+        layer.set_expert(e, *expert_bf16(cfg, e))
+    x = inp["x"][:T]
+    off = inp["logit_offset"]
+    layer.forward_train(bf16_dev(x), logit_offset=None if off is None else to_dev(off))
+    dy = S.host_normal_bf16(np.random.default_rng(seed), (T, cfg.d), 1.0)
+    dx, dE, dW13, dW2 = layer.backward(bf16_dev(dy), wgrad=True)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    counts = layer.expert_counts.cpu().numpy()
+    if experts is None:
+        experts = list(range(cfg.n_routed + 1))
+    ref = oracle.layer_backward(dy, x, inp["router_w"], inp["bias"], cfg.n_groups,
+                                cfg.topk_groups, cfg.topk, OracleExperts(cfg), logit_offset=off,
+                                wgrad_experts=tuple(experts))
+    worst = 0.0
+    for e in experts:
+        r13, r2 = ref["dW"][e]
+        g13, g2 = dW13[e].cpu().numpy(), dW2[e].cpu().numpy()
+        if e < cfg.n_routed and counts[e] == 0:
+            assert not np.any(g13) and not np.any(g2), e
+            continue
+        err = max(rel_frobenius(g13, r13), rel_frobenius(g2, r2))
+        worst = max(worst, err)
+        assert err <= DW_TOL, (e, err)
+    _report({"case": f"wgrad {name}: {T} tokens, {len(experts)} experts",
+             "worst_dW_rel_frobenius": worst})
+
+
+def test_layer_wgrad_tiny_all_experts():
+    _wgrad_case("tiny", S.CONFIGS["tiny"])
+
+
+def test_layer_wgrad_tiny_ragged():
+    _wgrad_case("tiny", S.CONFIGS["tiny"], T=13)
+
+
+def test_layer_wgrad_full_expert_shapes():
+    """d = 7168, I = 2048, 16 routed experts: the shared expert and three
+    routed ones (the oracle's FP64 weight gradients are 0.35 GB each)."""
+    _wgrad_case("prefill_e16", S.CONFIGS["prefill_e16"], experts=[16, 0, 5, 11])
