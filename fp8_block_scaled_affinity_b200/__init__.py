@@ -29,6 +29,7 @@ from ._lib import (MOE_DEV_TIMEOUT, MOE_EPI_BF16, MOE_EPI_F32, MOE_EPI_SWIGLU_QU
                    moe_ep_local_permute, moe_ep_partial_combine, moe_ep_final_combine,
                    moe_route_scores, fp8_transpose_w_128x128, moe_combine_backward_quant,
                    moe_swiglu_backward_quant, moe_gate_backward, moe_router_backward,
+                   moe_router_backward_workspace_size,
                    moe_dx_combine, moe_wgrad_max_blocks, moe_wgrad_layout, moe_wgrad_quant_x,
                    moe_wgrad_quant_do, moe_wgrad_quant_h, moe_wgrad_quant_dac,
                    moe_grouped_gemm_wgrad)
@@ -272,8 +273,10 @@ class MoeLayer:
         dx_router = torch.empty((T, d), dtype=f32, device=dev)
         d_router_w = torch.empty((N, d), dtype=f32, device=dev)
         pair_scratch = torch.empty((max(T * K, 1),), dtype=i32, device=dev)
+        rbw = torch.empty((max(moe_router_backward_workspace_size(sh), 256),), dtype=u8,
+                          device=dev)
         moe_router_backward(sh, b["x"], self.router_w, du, self.topk_idx, off, self.row_of_pair,
-                            pair_scratch, dx_router, d_router_w, st, stream)
+                            pair_scratch, dx_router, d_router_w, rbw, st, stream)
         mark("router_backward")
         dx = torch.empty((T, d), dtype=f32, device=dev)
         moe_dx_combine(sh, dx_rows, dx_router, self.row_of_pair, dx, st, stream)

@@ -76,7 +76,8 @@ def lib() -> ctypes.CDLL:
             "moe_combine_backward_quant": (I, [SP, P, P, P, P, P, P, P]),
             "moe_swiglu_backward_quant": (I, [P, P, I64, I, I64, P, P, P, P]),
             "moe_gate_backward": (I, [SP, P, P, P, P, P, P, P, P]),
-            "moe_router_backward": (I, [SP, P, P, P, P, P, P, P, P, P, P, P]),
+            "moe_router_backward_workspace_size": (SZ, [SP]),
+            "moe_router_backward": (I, [SP, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
             "moe_dx_combine": (I, [SP, P, P, P, P, P, P]),
             "moe_wgrad_max_blocks": (I, [I64, I]),
             "moe_wgrad_layout": (I, [I, P, I, P, P, P, P]),
@@ -484,12 +485,17 @@ def moe_gate_backward(shape, dy, expert_out, row_of_pair, topk_score, dgate, du,
         _ptr(dgate), _ptr(du), _ptr(dev_status), _stream(stream)))
 
 
+def moe_router_backward_workspace_size(shape) -> int:
+    return int(lib().moe_router_backward_workspace_size(ctypes.byref(shape)))
+
+
 def moe_router_backward(shape, x, router_w, du, topk_idx, expert_offsets, row_of_pair,
-                        pair_scratch, dx_router, d_router_w, dev_status=None, stream=None):
+                        pair_scratch, dx_router, d_router_w, ws, dev_status=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check("moe_router_backward", lib().moe_router_backward(
         ctypes.byref(shape), _ptr(x), _ptr(router_w), _ptr(du), _ptr(topk_idx),
         _ptr(expert_offsets), _ptr(row_of_pair), _ptr(pair_scratch), _ptr(dx_router),
-        _ptr(d_router_w), _ptr(dev_status), _stream(stream)))
+        _ptr(d_router_w), _ptr(ws), nbytes, _ptr(dev_status), _stream(stream)))
 
 
 def moe_dx_combine(shape, dx_rows, dx_router, row_of_pair, dx, dev_status=None, stream=None):

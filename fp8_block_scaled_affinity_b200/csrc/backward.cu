@@ -171,8 +171,12 @@ __global__ void __launch_bounds__(256) swiglu_backward_quant_kernel(
 }
 
 // ------------------------------------------- 6. gate gradients (FP64)
-// A warp per token: dg_k = <dy, o_k> summed in FP64 (lane-strided, then a
-// shuffle tree); the chosen scores' gradients in FP64.
+// A warp per token: dg_k = <dy, o_k> summed in FP64.  A lane takes four
+// consecutive values per step (one 8-byte load of dy, one 16-byte load of
+// each of the KM rows, all in flight together) and keeps KM FP64 partial
+// sums; one shuffle tree per slot at the end.  Then the chosen scores'
+// gradients in FP64.
+template <int KM>
 __global__ void __launch_bounds__(256) gate_backward_kernel(
     const uint16_t* __restrict__ dy, const float* __restrict__ o, int T, int d, int K,
     const int32_t* __restrict__ row_of_pair, const float* __restrict__ score,
@@ -180,28 +184,44 @@ __global__ void __launch_bounds__(256) gate_backward_kernel(
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (t >= T) return;
-    double my_dg = 0.0;
-    for (int k = 0; k < K; ++k) {
-        const int row = row_of_pair[int64_t(t) * K + k];
-        double acc = 0.0;
-        if (row >= 0)
-            for (int c = lane; c < d; c += 32)
-                acc += double(__uint_as_float(uint32_t(dy[int64_t(t) * d + c]) << 16)) *
-                       double(o[int64_t(row) * d + c]);
+    const float4* rows[KM];
+    double acc[KM];
 #pragma unroll
-        for (int s = 16; s >= 1; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-        if (lane == k) my_dg = acc;
+    for (int k = 0; k < KM; ++k) {
+        const int row = k < K ? row_of_pair[int64_t(t) * K + k] : -1;
+        rows[k] = row >= 0 ? reinterpret_cast<const float4*>(o + int64_t(row) * d) : nullptr;
+        acc[k] = 0.0;
+    }
+    const uint2* dyr = reinterpret_cast<const uint2*>(dy + int64_t(t) * d);
+    for (int c = lane; c < d / 4; c += 32) {
+        const uint2 w = __ldg(dyr + c);
+        const double y0 = bf16_lo(w.x), y1 = bf16_hi(w.x), y2 = bf16_lo(w.y), y3 = bf16_hi(w.y);
+        float4 v[KM];
+#pragma unroll
+        for (int k = 0; k < KM; ++k)
+            v[k] = rows[k] ? __ldg(rows[k] + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < KM; ++k)
+            acc[k] += y0 * double(v[k].x) + y1 * double(v[k].y) + y2 * double(v[k].z) +
+                      y3 * double(v[k].w);
+    }
+    double my_dg = 0.0;
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+        double a = acc[k];
+#pragma unroll
+        for (int s2 = 16; s2 >= 1; s2 >>= 1) a += __shfl_xor_sync(0xffffffffu, a, s2);
+        if (lane == k) my_dg = a;
     }
     const double s = lane < K ? double(score[int64_t(t) * K + lane]) : 0.0;
-    double S = s, gdg = 0.0;
+    double S = s;
 #pragma unroll
     for (int o2 = 16; o2 >= 1; o2 >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o2);
     double term = lane < K ? (s / S) * my_dg : 0.0;
 #pragma unroll
     for (int o2 = 16; o2 >= 1; o2 >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o2);
-    gdg = term;
     if (lane < K) {
-        const double ds = (my_dg - gdg) / S;
+        const double ds = (my_dg - term) / S;
         dgate[int64_t(t) * K + lane] = float(my_dg);
         du[int64_t(t) * K + lane] = float(ds * s * (1.0 - s));
     }
@@ -252,23 +272,28 @@ __global__ void pair_of_row_kernel(const int32_t* __restrict__ row_of_pair, int6
     if (r >= 0 && r < routed_rows) pair_of_row[r] = int32_t(p);
 }
 
-// dE: a warp per (expert, 256-value slice), the expert's rows in permutation
-// order (tokens ascending), du times the token's x, fp32.
-__global__ void __launch_bounds__(256) router_dE_kernel(
+// dE in two phases over the experts' 128-row blocks (the layout of the
+// weight-gradient operands): a warp per (block, 256-value slice) sums its
+// rows in order into a partial row, then a warp per (expert, slice) adds its
+// blocks' partials in order.  Every expert's rows are summed in the same
+// fixed order whatever the launch shape (deterministic); the hot expert of a
+// skewed batch is spread over as many warps as it has blocks.
+__global__ void __launch_bounds__(256) router_dE_partial_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ du,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ pair_of_row, int d, int K,
-    int n_routed, float* __restrict__ dE) {
+    const int2* __restrict__ blocks, int n_blocks, const int32_t* __restrict__ pair_of_row, int d,
+    int K, float* __restrict__ partial) {
     const int lane = threadIdx.x & 31;
     const int chunks = (d + 255) / 256;
-    const int64_t units = int64_t(n_routed) * chunks;
+    const int64_t units = int64_t(n_blocks) * chunks;
     const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
     for (int64_t u = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); u < units;
          u += warps_total) {
-        const int e = int(u / chunks);
-        const int c = int(u - int64_t(e) * chunks) * 256 + lane * 8;
-        if (c >= d) continue;
+        const int b = int(u / chunks);
+        const int c = int(u - int64_t(b) * chunks) * 256 + lane * 8;
+        const int2 blk = blocks[b];
+        if (blk.y <= 0 || c >= d) continue;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int r = offsets[e]; r < offsets[e + 1]; ++r) {
+        for (int r = blk.x; r < blk.x + blk.y; ++r) {
             const int p = pair_of_row[r];
             const int t = p / K;
             const float g = du[p];
@@ -278,9 +303,33 @@ __global__ void __launch_bounds__(256) router_dE_kernel(
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(g, xv[i], acc[i]);
         }
-        float4* out = reinterpret_cast<float4*>(dE + int64_t(e) * d + c);
+        float4* out = reinterpret_cast<float4*>(partial + int64_t(b) * d + c);
         out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
+__global__ void __launch_bounds__(256) router_dE_reduce_kernel(
+    const float* __restrict__ partial, const int32_t* __restrict__ kb_offsets, int n_routed,
+    int d, float* __restrict__ dE) {
+    const int lane = threadIdx.x & 31;
+    const int chunks = (d + 127) / 128;
+    const int64_t units = int64_t(n_routed) * chunks;
+    const int64_t warps_total = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t u = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); u < units;
+         u += warps_total) {
+        const int e = int(u / chunks);
+        const int c = int(u - int64_t(e) * chunks) * 128 + lane * 4;
+        if (c >= d) continue;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int b = kb_offsets[e]; b < kb_offsets[e + 1]; ++b) {
+            const float4 v = *reinterpret_cast<const float4*>(partial + int64_t(b) * d + c);
+            a.x = __fadd_rn(a.x, v.x);
+            a.y = __fadd_rn(a.y, v.y);
+            a.z = __fadd_rn(a.z, v.z);
+            a.w = __fadd_rn(a.w, v.w);
+        }
+        *reinterpret_cast<float4*>(dE + int64_t(e) * d + c) = a;
     }
 }
 
@@ -511,6 +560,24 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
     }
 }
 
+// Workspace of moe_router_backward: the routed experts' 128-row blocks and
+// one fp32 partial row of dE per block.
+struct RouterBwdWs {
+    int n_blocks;
+    size_t kb_off, blocks, partial, total;
+};
+RouterBwdWs router_bwd_ws(const MoeShape& s) {
+    RouterBwdWs w;
+    const int64_t pairs = int64_t(s.T) * s.topk;
+    w.n_blocks = int((pairs + 127) / 128 + s.n_routed);
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    w.kb_off = 0;
+    w.blocks = up(sizeof(int32_t) * (s.n_routed + 1));
+    w.partial = w.blocks + up(sizeof(int32_t) * 2 * size_t(w.n_blocks));
+    w.total = w.partial + up(sizeof(float) * size_t(w.n_blocks) * s.d);
+    return w;
+}
+
 int pieces_per(int n, int& PC) {
     const int nkb = n / 128;
     PC = (nkb % 14 == 0 && nkb % 16 != 0) ? 7 : 8;
@@ -597,8 +664,21 @@ extern "C" MOE_API int moe_gate_backward(const MoeShape* shape, const uint16_t* 
     const int T = shape->T;
     if (T == 0) return MOE_OK;
     if (!dy || !expert_out || !row_of_pair || !topk_score || !dgate || !du) return MOE_ERR_NULL;
-    gate_backward_kernel<<<(T + 7) / 8, 256, 0, as_stream(stream)>>>(
-        dy, expert_out, T, shape->d, shape->topk, row_of_pair, topk_score, dgate, du);
+    const int K = shape->topk, grid = (T + 7) / 8;
+    cudaStream_t st = as_stream(stream);
+    if (!aligned16(expert_out) || (reinterpret_cast<uintptr_t>(dy) & 7)) return MOE_ERR_ALIGN;
+    if (K <= 4)
+        gate_backward_kernel<4><<<grid, 256, 0, st>>>(dy, expert_out, T, shape->d, K, row_of_pair,
+                                                      topk_score, dgate, du);
+    else if (K <= 8)
+        gate_backward_kernel<8><<<grid, 256, 0, st>>>(dy, expert_out, T, shape->d, K, row_of_pair,
+                                                      topk_score, dgate, du);
+    else if (K <= 16)
+        gate_backward_kernel<16><<<grid, 256, 0, st>>>(dy, expert_out, T, shape->d, K,
+                                                       row_of_pair, topk_score, dgate, du);
+    else
+        gate_backward_kernel<32><<<grid, 256, 0, st>>>(dy, expert_out, T, shape->d, K,
+                                                       row_of_pair, topk_score, dgate, du);
     return check_launch();
 }
 
@@ -607,8 +687,8 @@ extern "C" MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t
                                            const int32_t* topk_idx,
                                            const int32_t* expert_offsets,
                                            const int32_t* row_of_pair, int32_t* pair_scratch,
-                                           float* dx_router, float* d_router_w,
-                                           int* dev_status, void* stream) {
+                                           float* dx_router, float* d_router_w, void* ws,
+                                           size_t ws_bytes, int* dev_status, void* stream) {
     int rc = validate_shape(shape);
     if (rc != MOE_OK) return rc;
     const int T = shape->T, d = shape->d, K = shape->topk, N = shape->n_routed;
@@ -618,10 +698,16 @@ extern "C" MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t
         return cudaMemsetAsync(d_router_w, 0, sizeof(float) * N * d, st) == cudaSuccess
                    ? MOE_OK : MOE_ERR_CUDA;
     if (!x || !router_w || !du || !topk_idx || !expert_offsets || !row_of_pair ||
-        !pair_scratch || !dx_router)
+        !pair_scratch || !dx_router || !ws)
         return MOE_ERR_NULL;
     if (!aligned16(x) || !aligned16(router_w) || !aligned16(dx_router) || !aligned16(d_router_w))
         return MOE_ERR_ALIGN;
+    const RouterBwdWs W = router_bwd_ws(*shape);
+    if (ws_bytes < W.total) return MOE_ERR_WORKSPACE;
+    char* base = static_cast<char*>(ws);
+    int32_t* kb_off = reinterpret_cast<int32_t*>(base + W.kb_off);
+    int2* blocks = reinterpret_cast<int2*>(base + W.blocks);
+    float* partial = reinterpret_cast<float*>(base + W.partial);
     const int chunks = (d + 255) / 256;
     router_dx_kernel<<<warp_blocks(int64_t(T) * chunks), 256, 0, st>>>(
         router_w, du, topk_idx, T, d, K, N, dx_router, dev_status);
@@ -630,9 +716,20 @@ extern "C" MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t
     pair_of_row_kernel<<<int((pairs + 255) / 256), 256, 0, st>>>(row_of_pair, pairs, pairs,
                                                                   pair_scratch);
     if ((rc = check_launch()) != MOE_OK) return rc;
-    router_dE_kernel<<<warp_blocks(int64_t(N) * chunks), 256, 0, st>>>(
-        x, du, expert_offsets, pair_scratch, d, K, N, d_router_w);
+    wgrad_layout_kernel<<<1, 1024, 0, st>>>(expert_offsets, N, W.n_blocks, kb_off, blocks,
+                                            dev_status);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    router_dE_partial_kernel<<<warp_blocks(int64_t(W.n_blocks) * chunks), 256, 0, st>>>(
+        x, du, blocks, W.n_blocks, pair_scratch, d, K, partial);
+    if ((rc = check_launch()) != MOE_OK) return rc;
+    router_dE_reduce_kernel<<<warp_blocks(int64_t(N) * ((d + 127) / 128)), 256, 0, st>>>(
+        partial, kb_off, N, d, d_router_w);
     return check_launch();
+}
+
+extern "C" MOE_API size_t moe_router_backward_workspace_size(const MoeShape* shape) {
+    if (validate_shape(shape) != MOE_OK) return 0;
+    return router_bwd_ws(*shape).total;
 }
 
 extern "C" MOE_API int moe_dx_combine(const MoeShape* shape, const float* dx_rows,

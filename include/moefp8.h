@@ -632,21 +632,26 @@ MOE_API int moe_gate_backward(const MoeShape* shape, const uint16_t* dy, const f
 /* moe_router_backward: the router's two gradients from du (fp32 [T, K]):
  *   dx_router[t] = sum_k du[t,k] E[topk_idx[t,k]]     (fp32 [T, d] out,
  *                  fp32 fused multiply-adds in slot order)
- *   d_router_w[e] = sum over the tokens choosing e, ascending, of du x[t]
- *                  (fp32 [N_r, d] out; every row written, zero for an
- *                  unchosen expert)
+ *   d_router_w[e] = sum over the tokens choosing e of du x[t] (fp32 [N_r, d]
+ *                  out; every row written, zero for an unchosen expert),
+ *                  summed in a fixed order: the expert's rows (tokens
+ *                  ascending) in blocks of 128, each block's rows in order
+ *                  into a partial sum, the partials then added in order
  *   x bf16 [T, d]; router_w bf16 [N_r, d]; topk_idx int32 [T, K];
  *   expert_offsets int32 [N_r + 2] and row_of_pair int32 [T, K] (the
  *   forward's permutation); pair_scratch int32 [T*K] out: the
- *   permutation's inverse over the routed rows (pair t*K + k of each row).
- * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_CUDA;
- * MOE_DEV_BAD_INPUT on dev_status for an expert index out of range. */
+ *   permutation's inverse over the routed rows (pair t*K + k of each row);
+ *   ws, ws_bytes scratch of moe_router_backward_workspace_size(shape).
+ * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_WORKSPACE,
+ * MOE_ERR_CUDA; MOE_DEV_BAD_INPUT on dev_status for an expert index out of
+ * range. */
+MOE_API size_t moe_router_backward_workspace_size(const MoeShape* shape);
 MOE_API int moe_router_backward(const MoeShape* shape, const uint16_t* x,
                                 const uint16_t* router_w, const float* du,
                                 const int32_t* topk_idx, const int32_t* expert_offsets,
                                 const int32_t* row_of_pair, int32_t* pair_scratch,
-                                float* dx_router, float* d_router_w, int* dev_status,
-                                void* stream);
+                                float* dx_router, float* d_router_w, void* ws, size_t ws_bytes,
+                                int* dev_status, void* stream);
 
 /* moe_dx_combine: dx[t] = dx_rows[shared row of t] + sum_k dx_rows[row of
  * (t,k)] (slot order) + dx_router[t] (NULL: none), fp32 [T, d] out.
