@@ -841,15 +841,15 @@ def run_ours(args, world, rank, local):
     if intensity < ridge:
         roofline = {"bound": "hbm", "kernel": label, "achieved": achieved, "peak": hbm_peak,
                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": peak_src,
-                    "traffic": profiled_traffic("gemm_swiglu_prefill") if cfg.name == "prefill"
-                    else None,
+                    "traffic": profiled_traffic(f"gemm_swiglu_{cfg.name}"),
                     "algorithmic_bytes_per_launch": alg["gemm1_bytes"], "launch_ms": g1_ms}
     else:
         g1_tflops = alg["flops_gemm1"] / (g1_ms / 1e3) / 1e12
         roofline = {"bound": "tensor", "kernel": label, "achieved": g1_tflops,
                     "peak": fp8_peak_burst, "unit": "TFLOP/s", "frac": g1_tflops / fp8_peak_burst,
                     "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g} (fp8:bf16 nominal)",
-                    "traffic": None, "algorithmic_flops_per_launch": alg["flops_gemm1"],
+                    "traffic": profiled_traffic(f"gemm_swiglu_{cfg.name}"),
+                    "algorithmic_flops_per_launch": alg["flops_gemm1"],
                     "algorithmic_bytes_per_launch": alg["gemm1_bytes"], "launch_ms": g1_ms}
     roofline["intensity_flop_per_byte"] = intensity
     roofline["ridge_flop_per_byte"] = ridge
@@ -922,8 +922,9 @@ def run_ours(args, world, rank, local):
 
 
 def run_backward(args, world, rank, local):
-    """The layer's backward pass (dx and the router gradient for an upstream
-    gradient dy) on the workload's batch: forward_train once, then timed
+    """The layer's backward pass (dx, the router gradient and, unless
+    --no-wgrad, the expert weight gradients for an upstream gradient dy) on
+    the workload's batch: forward_train once, then timed
     backward calls with dy resident in HBM; beside it end to end with dy
     copied in from pinned host memory and dx copied out every step."""
     import numpy as np
@@ -942,8 +943,9 @@ def run_backward(args, world, rank, local):
                                                   (T, d), 1.0).view(np.int16)).view(
         torch.bfloat16).pin_memory()
     dy = dy_host.to(dev)
+    wg = not args.no_wgrad
     for _ in range(args.warmup):
-        layer.backward(dy)
+        layer.backward(dy, wgrad=wg)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -953,7 +955,7 @@ def run_backward(args, world, rank, local):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(st)
     for _ in range(args.steps):
-        layer.backward(dy)
+        layer.backward(dy, wgrad=wg)
     ev1.record(st)
     ev1.synchronize()
     clk = clocks.stop()
@@ -971,7 +973,7 @@ def run_backward(args, world, rank, local):
     e0.record(st)
     for _ in range(args.steps):
         dy_dev.copy_(dy_host, non_blocking=True)
-        dx, _dE = layer.backward(dy_dev)
+        dx = layer.backward(dy_dev, wgrad=wg)[0]
         dx_host.copy_(dx, non_blocking=True)
     e1.record(st)
     e1.synchronize()
@@ -981,20 +983,40 @@ def run_backward(args, world, rank, local):
     tot = {}
     for it in range(args.steps + 2):
         marks = []
-        layer.backward(dy, marks=marks)
+        layer.backward(dy, marks=marks, wgrad=wg)
         marks[-1][1].synchronize()
         if it >= 2:
             for (_, a), (n, b) in zip(marks[:-1], marks[1:]):
                 tot[n] = tot.get(n, 0.0) + a.elapsed_time(b)
     brk = {n: v / args.steps for n, v in tot.items()}
     R = T * K + T
+    G = cfg.n_routed + 1
     flops = {"gemm_dh": 2.0 * R * d * I, "gemm_ac_recompute": 2.0 * R * d * 2 * I,
              "gemm_dx": 2.0 * R * 2 * I * d}
+    # weight gradients: fp32 outputs for every expert (zeros for unchosen ones)
+    out_bytes = {}
+    if wg:
+        flops.update({"gemm_dw13": 2.0 * R * 2 * I * d, "gemm_dw2": 2.0 * R * d * I})
+        out_bytes = {"gemm_dw13": 4.0 * G * 2 * I * d, "gemm_dw2": 4.0 * G * d * I}
     top = max(flops, key=lambda n: brk[n])
     fp8_peak = float(peaks["bf16_tflops"]) * FP8_PER_BF16
+    hbm_peak = float(peaks["hbm_gbs"])
     ach = flops[top] / (brk[top] / 1e3) / 1e12
     gemm_ms = sum(brk[n] for n in flops)
-    hbm_peak = float(peaks["hbm_gbs"])
+    if top in out_bytes and out_bytes[top] / (hbm_peak * 1e9) > flops[top] / (fp8_peak * 1e12):
+        # the gradient write bounds this launch, not the tensor cores
+        gbs = out_bytes[top] / (brk[top] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": f"wgrad_gemm_kernel ({top})", "achieved": gbs,
+                "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                "peak_source": peak_src, "traffic": None,
+                "algorithmic_bytes_per_launch": out_bytes[top], "launch_ms": brk[top],
+                "tflops": ach, "frac_of_datasheet": gbs / DATASHEET["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "kernel": f"grouped GEMM ({top})", "achieved": ach,
+                "peak": fp8_peak, "unit": "TFLOP/s", "frac": ach / fp8_peak,
+                "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g}",
+                "traffic": None, "algorithmic_flops_per_launch": flops[top],
+                "launch_ms": brk[top], "frac_of_datasheet": ach / DATASHEET["fp8_tflops"]}
     mem_bytes = {
         "combine_backward_quant": T * d * 2 + R * d + R * (d // 128) * 4,
         "swiglu_backward_quant": R * I * 4 + R * 2 * I * 4 + R * 2 * I + R * (2 * I // 128) * 4,
@@ -1014,20 +1036,16 @@ def run_backward(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "fp8e4m3/f32",
         "data": "synthetic",
-        "config": {"workload": f"moe_layer_backward_{cfg.name}", "T": T, "d": d,
+        "config": {"workload": f"moe_layer_backward_{cfg.name}", "wgrad": wg, "T": T, "d": d,
                    "n_routed": cfg.n_routed, "topk": K, "inter": I,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (FP8 weights and their transposes, "
                          "fp32 row buffers of several GB)"},
-        "roofline": {"bound": "tensor", "kernel": f"grouped_gemm ({top})", "achieved": ach,
-                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": ach / fp8_peak,
-                     "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g}",
-                     "traffic": None, "algorithmic_flops_per_launch": flops[top],
-                     "launch_ms": brk[top],
-                     "frac_of_datasheet": ach / DATASHEET["fp8_tflops"]},
-        "dgrad_gemms": {"tflops": sum(flops.values()) / (gemm_ms / 1e3) / 1e12,
-                        "frac_of_fp8_peak": sum(flops.values()) / (gemm_ms / 1e3) / 1e12
-                        / fp8_peak, "ms": gemm_ms},
+        "roofline": roof,
+        "backward_gemms": {n: {"ms": brk[n], "tflops": f / (brk[n] / 1e3) / 1e12,
+                               "frac_of_fp8_peak": f / (brk[n] / 1e3) / 1e12 / fp8_peak}
+                           for n, f in flops.items()},
+        "gemm_tflops": sum(flops.values()) / (gemm_ms / 1e3) / 1e12,
         "memory_passes": {n: {"ms": brk[n], "gbs": b / (brk[n] / 1e3) / 1e9,
                               "frac_of_hbm": b / (brk[n] / 1e3) / 1e9 / hbm_peak}
                           for n, b in mem_bytes.items()},
@@ -1035,8 +1053,9 @@ def run_backward(args, world, rank, local):
         "e2e": {"value": tokens_total / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4,
                 "api": "MoeLayer.backward with dy copied in and dx copied out each step"},
-        # combine quant 1, GEMMs 3, SwiGLU quant 1, gate 1, router 3, dx 1
-        "gpu_launches": 10 * args.steps,
+        # combine quant 1, GEMMs 3, SwiGLU quant 1, gate 1, router 3, dx 1;
+        # weight gradients: layout 1, quantisers 4, GEMMs 2
+        "gpu_launches": (17 if wg else 10) * args.steps,
         "clocks": clk,
         "device_status": status,
     }
@@ -1058,7 +1077,10 @@ def main(argv=None):
                     help="fp32: the pages' recipe (default); ue8m0: the power-of-two scale "
                          "option with block-scaled tensor-core GEMMs")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
-                    help="backward: time the layer's backward pass (dx, router gradient)")
+                    help="backward: time the layer's backward pass (dx, router and expert "
+                         "weight gradients)")
+    ap.add_argument("--no-wgrad", action="store_true",
+                    help="backward without the expert weight gradients")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
