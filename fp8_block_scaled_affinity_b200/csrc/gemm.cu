@@ -522,9 +522,13 @@ __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmPar
     it.g = lo;
     const int local = item - ss->gstart[lo];
     const int rows = ss->goff[lo + 1] - ss->goff[lo];
-    const int mtiles = (rows + ITEM_ROWS - 1) / ITEM_ROWS;
-    it.f = local / mtiles;
-    const int mt = local - it.f * mtiles;
+    // column tiles fastest: the CTAs running at the same time share a few
+    // token tiles and walk all of the expert's weight tiles, so a large group
+    // (the hot experts of a skewed batch, 128 token tiles) reads its token
+    // rows from HBM once while its weights (29 MB at most) stay in L2; with
+    // token tiles fastest the token rows were read once per column tile
+    const int mt = local / p.n_ftiles;
+    it.f = local - mt * p.n_ftiles;
     it.row0 = ss->goff[lo] + mt * ITEM_ROWS;
     it.rows = rows - mt * ITEM_ROWS;
     return it;
@@ -1838,8 +1842,19 @@ __device__ __forceinline__ void wg_promoter(const WgParams& p, SharedState* ss,
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ss->sempty[c]));  // scales read
         }
-        store_rows<64, 1>(p.out, acc2, wpark, map_o, lane, 32, 0,
-                          w.g * p.m + w.mt * 128 + q * 32, w.f * 256 + c0);
+        if (w.kb0 < w.kb1) {
+            store_rows<64, 1>(p.out, acc2, wpark, map_o, lane, 32, 0,
+                              w.g * p.m + w.mt * 128 + q * 32, w.f * 256 + c0);
+        } else {
+            // no K blocks (an expert no token chose): zeros, one 512-byte row
+            // segment per store instruction, no staging
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out.out) +
+                                                    size_t(w.g * p.m + w.mt * 128 + q * 32) * p.n +
+                                                    w.f * 256 + c0) + lane;
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i)
+                dst[size_t(i) * (p.n / 4)] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         const bool any_abort = named_bar_or(
             2, kPromoters * 32, !ok || *reinterpret_cast<volatile int*>(&ss->abort_flag));
         if (any_abort) break;
