@@ -490,47 +490,85 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
         const int f0 = int(u - int64_t(b) * fchunks) * 64;
         const int2 blk = blocks[b];
         if (blk.y <= 0) continue;  // past the last expert's rows: never read
-        // ---- load: warp w, rows w, w + 8, ...; lane: features f0 + 2 lane, +1
-        for (int rr = warp; rr < 128; rr += 8) {
-            float v0 = 0.0f, v1 = 0.0f;
-            if (rr < blk.y) {
-                const int r = blk.x + rr;
-                const int f = f0 + 2 * lane;
-                if (SRC == kWgX || SRC == kWgDo) {
-                    float g;
-                    const int t = wg_token(src, r, g);
-                    const uint32_t w2 =
-                        *reinterpret_cast<const uint32_t*>(src.x + int64_t(t) * F + f);
-                    v0 = bf16_lo(w2);
-                    v1 = bf16_hi(w2);
+        // ---- load: warp w, rows w, w + 8, ...; lane: features f0 + 2 lane, +1.
+        // Eight rows at a time: their token indices first, then all their
+        // loads, then the arithmetic (a warp keeps eight loads in flight).
+        const int fl = f0 + 2 * lane;
+        for (int i0 = 0; i0 < 16; i0 += 8) {
+            float v0[8], v1[8];
+            if (SRC == kWgX || SRC == kWgDo) {
+                int tok[8];
+                float g[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = warp + 8 * (i0 + i);
+                    g[i] = 0.0f;
+                    tok[i] = rr < blk.y ? wg_token(src, blk.x + rr, g[i]) : -1;
+                }
+                uint32_t w2[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    w2[i] = tok[i] >= 0
+                                ? __ldg(reinterpret_cast<const uint32_t*>(src.x + int64_t(tok[i]) * F + fl))
+                                : 0u;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    v0[i] = bf16_lo(w2[i]);
+                    v1[i] = bf16_hi(w2[i]);
                     if (SRC == kWgDo) {
-                        v0 = __fmul_rn(g, v0);
-                        v1 = __fmul_rn(g, v1);
+                        v0[i] = __fmul_rn(g[i], v0[i]);
+                        v1[i] = __fmul_rn(g[i], v1[i]);
                     }
-                } else if (SRC == kWgH) {
-                    const float* ar = src.ac + int64_t(r) * 2 * src.I;
-                    const float2 a = *reinterpret_cast<const float2*>(ar + f);
-                    const float2 c = *reinterpret_cast<const float2*>(ar + src.I + f);
-                    v0 = a.x / (1.0f + expf(-a.x)) * c.x;
-                    v1 = a.y / (1.0f + expf(-a.y)) * c.y;
-                } else {  // [da | dc]
-                    const float* ar = src.ac + int64_t(r) * 2 * src.I;
-                    const bool is_da = f < src.I;
-                    const int j = is_da ? f : f - src.I;
-                    const float2 h = *reinterpret_cast<const float2*>(src.dh + int64_t(r) * src.I + j);
-                    const float2 a = *reinterpret_cast<const float2*>(ar + j);
-                    const float sg0 = wg_sigmoid(a.x), sg1 = wg_sigmoid(a.y);
+                }
+            } else if (SRC == kWgH) {
+                float2 a[8], c[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = warp + 8 * (i0 + i);
+                    a[i] = c[i] = make_float2(0.f, 0.f);
+                    if (rr < blk.y) {
+                        const float* ar = src.ac + int64_t(blk.x + rr) * 2 * src.I;
+                        a[i] = __ldg(reinterpret_cast<const float2*>(ar + fl));
+                        c[i] = __ldg(reinterpret_cast<const float2*>(ar + src.I + fl));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    v0[i] = a[i].x / (1.0f + expf(-a[i].x)) * c[i].x;
+                    v1[i] = a[i].y / (1.0f + expf(-a[i].y)) * c[i].y;
+                }
+            } else {  // [da | dc]
+                const bool is_da = fl < src.I;
+                const int j = is_da ? fl : fl - src.I;
+                float2 h[8], a[8], c[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = warp + 8 * (i0 + i);
+                    h[i] = a[i] = c[i] = make_float2(0.f, 0.f);
+                    if (rr < blk.y) {
+                        const int64_t r = blk.x + rr;
+                        const float* ar = src.ac + r * 2 * src.I;
+                        h[i] = __ldg(reinterpret_cast<const float2*>(src.dh + r * src.I + j));
+                        a[i] = __ldg(reinterpret_cast<const float2*>(ar + j));
+                        if (is_da) c[i] = __ldg(reinterpret_cast<const float2*>(ar + src.I + j));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float sg0 = wg_sigmoid(a[i].x), sg1 = wg_sigmoid(a[i].y);
                     if (is_da) {
-                        const float2 c = *reinterpret_cast<const float2*>(ar + src.I + j);
-                        v0 = h.x * c.x * sg0 * (1.0f + a.x * (1.0f - sg0));
-                        v1 = h.y * c.y * sg1 * (1.0f + a.y * (1.0f - sg1));
+                        v0[i] = h[i].x * c[i].x * sg0 * (1.0f + a[i].x * (1.0f - sg0));
+                        v1[i] = h[i].y * c[i].y * sg1 * (1.0f + a[i].y * (1.0f - sg1));
                     } else {
-                        v0 = h.x * a.x * sg0;
-                        v1 = h.y * a.y * sg1;
+                        v0[i] = h[i].x * a[i].x * sg0;
+                        v1[i] = h[i].y * a[i].y * sg1;
                     }
                 }
             }
-            *reinterpret_cast<float2*>(&tile[rr][2 * lane]) = make_float2(v0, v1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<float2*>(&tile[warp + 8 * (i0 + i)][2 * lane]) =
+                    make_float2(v0[i], v1[i]);
         }
         __syncthreads();
         // ---- amax per feature, then codes: thread (feature f, quarter q)

@@ -1764,13 +1764,11 @@ __device__ __forceinline__ void wg_mma_issuer(const WgParams& p, uint8_t* smem, 
     __syncwarp();
 }
 
-// A shared-memory load the compiler keeps in program order (plain loads of
-// the B scales were all hoisted to the top of the K block, and the
-// registers they took spilled the accumulators).
-__device__ __forceinline__ uint64_t ld_shared_volatile(const uint64_t* p) {
-    uint64_t v;
-    asm volatile("ld.volatile.shared.b64 %0, [%1];" : "=l"(v) : "r"(smem_u32(p)));
-    return v;
+// Two B-scale pairs from shared memory in one 16-byte load that the compiler
+// keeps in program order (plain loads were all hoisted to the top of the K
+// block, and the registers they took spilled the accumulators).
+__device__ __forceinline__ void ld_shared_volatile2(const uint64_t* p, uint64_t& a, uint64_t& b) {
+    asm volatile("ld.volatile.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(smem_u32(p)));
 }
 
 // acc2[o + i] += v pair i * (sa * sb pair o + i) for 16 pairs, eight pairs
@@ -1781,7 +1779,12 @@ __device__ __forceinline__ void wg_fold(uint64_t (&acc2)[64], const uint32_t (&v
     for (int j = 0; j < 2; ++j) {
         uint64_t s[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s[i] = fmul2(sa2, ld_shared_volatile(sb2 + o + 8 * j + i));
+        for (int i = 0; i < 8; i += 2) {
+            uint64_t b0, b1;
+            ld_shared_volatile2(sb2 + o + 8 * j + i, b0, b1);
+            s[i] = fmul2(sa2, b0);
+            s[i + 1] = fmul2(sa2, b1);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             ffma2(acc2[o + 8 * j + i], pack2(v[2 * (8 * j + i)], v[2 * (8 * j + i) + 1]), s[i]);
