@@ -451,6 +451,93 @@ def run_route(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_permute(args, world, rank, local):
+    """The 1x128 activation quantisation fused with the permutation copy
+    (moe_quant_permute) alone, on the prefill batch (T=4096, d=7168, K=8):
+    x read once in bf16, codes and kb-major scales written to the K + 1
+    destination rows.  Routing runs once beforehand, untimed; a 256 MB buffer
+    is written between timed launches (x is smaller than L2)."""
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    import synthetic as S
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.CONFIGS["prefill"]
+    inp = S.make_layer_inputs_host(cfg, 0)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    x, rw = bf16(inp["x"]), bf16(inp["router_w"])
+    bias = torch.from_numpy(inp["bias"]).to(dev)
+    T, d, K, N = cfg.T, cfg.d, cfg.topk, cfg.n_routed
+    R = T * K + T
+    shape = moe.make_shape(T, d, N, cfg.n_groups, cfg.topk_groups, K, cfg.inter, cfg.gamma)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty((N,), dtype=torch.int32, device=dev)
+    rws = torch.empty((moe.moe_route_workspace_size(shape),), dtype=torch.uint8, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    moe.moe_route(shape, x, rw, bias, None, idx, gate, counts, rws, status)
+    xq = torch.empty((R, d), dtype=torch.uint8, device=dev)
+    xs = torch.empty((d // 128, R), dtype=torch.float32, device=dev)
+    off = torch.empty((N + 2,), dtype=torch.int32, device=dev)
+    rop = torch.empty((T, K), dtype=torch.int32, device=dev)
+    pws = torch.empty((moe.moe_permute_workspace_size(shape),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_quant_permute(shape, x, idx, counts, xq, xs, off, rop, pws, status)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(st)
+        step()
+        e1.record(st)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs), world)
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    nbytes = T * d * 2 + R * (d + 4 * (d // 128))  # x in; codes + scales out
+    gbs = nbytes * args.steps / (ms / 1e3) / 1e9
+    tok = T * args.steps * world
+    line = {
+        "metric": METRIC, "value": tok / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->fp8e4m3", "data": "synthetic",
+        "config": {"workload": "moe_quant_permute_prefill", "T": T, "d": d, "n_routed": N,
+                   "topk": K, "parallelism": f"replicas x{world}",
+                   "l2": "256 MB buffer written between timed launches"},
+        "roofline": {"bound": "hbm", "kernel": "quant_copy_rows_kernel (+ permutation ranks)",
+                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "frac_of_datasheet": gbs / DATASHEET["hbm_gbs"]},
+        "e2e": None,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+        "device_status": int(status.item()),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------- GEMM-alone workload
 def run_gemm(args, world, rank, local):
     """The FP8 block-scaled GEMM alone: A [4096, 7168] (1x128 scales) times B
@@ -1075,7 +1162,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="skewed",
                     choices=["tiny", "prefill", "decode", "skewed", "prefill_e16", "gemm",
-                             "route"])
+                             "route", "permute"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scales", choices=["fp32", "ue8m0"], default="fp32",
                     help="fp32: the pages' recipe (default); ue8m0: the power-of-two scale "
@@ -1096,6 +1183,8 @@ def main(argv=None):
             run_gemm(args, world, rank, local)
         elif args.workload == "route":
             run_route(args, world, rank, local)
+        elif args.workload == "permute":
+            run_permute(args, world, rank, local)
         elif args.which == "backward":
             run_backward(args, world, rank, local)
         else:

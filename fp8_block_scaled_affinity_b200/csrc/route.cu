@@ -600,17 +600,19 @@ __device__ __forceinline__ float exact_logit_unordered(const uint16_t* __restric
 __device__ __forceinline__ float exact_logit(const uint16_t* __restrict__ xr,
                                              const uint16_t* __restrict__ er, int d,
                                              bool fp32_products) {
-    // 16-byte vectors (8 k) of both rows stream through an 8-deep register
-    // ring: slot i is consumed, then refilled with the vector 8 further on.
+    // 16-byte vectors (8 k) of both rows stream through a 16-deep register
+    // ring: slot i is consumed, then refilled with the vector 16 further on
+    // (the few threads of this kernel are bound by load latency, so each
+    // keeps 32 loads in flight).
     // The products of the next vector are formed and widened before the
     // FP64 adds of the current one, so the conversions overlap the add
     // chain.  Each product of two bf16 values is exact in FP64 (and in fp32
     // under fp32_products), so adding it equals the FP64 fma of the
     // definition.
-    constexpr int kRing = 8;
+    constexpr int kRing = 16;
     const uint4* xp = reinterpret_cast<const uint4*>(xr);
     const uint4* ep = reinterpret_cast<const uint4*>(er);
-    const int nv = d / 8;  // a multiple of 16
+    const int nv = d / 8;  // a multiple of 16 = kRing
     uint4 xv[kRing], ev[kRing];
 #pragma unroll
     for (int i = 0; i < kRing; ++i) {
