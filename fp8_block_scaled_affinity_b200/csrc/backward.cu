@@ -373,24 +373,46 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(
 }
 
 // ------------------------------------------- transposed weights
-// A CTA per 128x128 block: codes through shared memory, transposed; the
-// block's scale moves to the transposed position.
+// A CTA per 128x128 block: the block's rows read with 16-byte loads into
+// shared memory (rows padded to 144 bytes), then each thread gathers 16
+// consecutive source rows of one column into one 16-byte store of the
+// transposed row.  The block's scale moves to the transposed position.
+constexpr int kTPitch = 144;  // bytes per staged row (16-byte aligned, spreads banks)
 __global__ void __launch_bounds__(256) transpose_w_kernel(
     const uint8_t* __restrict__ q, const float* __restrict__ s, int64_t mats, int rows,
     int cols, uint8_t* __restrict__ qt, float* __restrict__ st) {
-    __shared__ uint8_t tile[128][129];
+    __shared__ __align__(16) uint8_t tile[128 * kTPitch];
     const int rb = rows / 128, cb = cols / 128;
     const int64_t blocks = mats * rb * cb;
     for (int64_t b = blockIdx.x; b < blocks; b += gridDim.x) {
         const int64_t m = b / (int64_t(rb) * cb);
         const int i = int((b / cb) % rb), j = int(b % cb);
         const uint8_t* src = q + (m * rows + int64_t(i) * 128) * cols + int64_t(j) * 128;
-        for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x)
-            tile[e / 128][e % 128] = src[int64_t(e / 128) * cols + (e % 128)];
+        // 128 rows x 8 vectors of 16 bytes: four per thread
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = threadIdx.x + 256 * u;
+            const int r = e >> 3, v = e & 7;
+            *reinterpret_cast<uint4*>(tile + r * kTPitch + 16 * v) =
+                __ldg(reinterpret_cast<const uint4*>(src + int64_t(r) * cols) + v);
+        }
         __syncthreads();
         uint8_t* dst = qt + (m * cols + int64_t(j) * 128) * rows + int64_t(i) * 128;
-        for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x)
-            dst[int64_t(e / 128) * rows + (e % 128)] = tile[e % 128][e / 128];
+        // output row c (source column c) = 8 vectors of 16 source rows each
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = threadIdx.x + 256 * u;
+            const int c = e & 127, v = e >> 7;  // consecutive threads: consecutive columns
+            uint32_t w[4];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const uint8_t* col = tile + (16 * v + 4 * q4) * kTPitch + c;
+                w[q4] = uint32_t(col[0]) | (uint32_t(col[kTPitch]) << 8) |
+                        (uint32_t(col[2 * kTPitch]) << 16) | (uint32_t(col[3 * kTPitch]) << 24);
+            }
+            *reinterpret_cast<uint4*>(dst + int64_t(c) * rows + 16 * v) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
         if (threadIdx.x == 0) st[(m * cb + j) * rb + i] = s[(m * rb + i) * cb + j];
         __syncthreads();
     }
@@ -637,6 +659,7 @@ extern "C" MOE_API int fp8_transpose_w_128x128(const uint8_t* q, const float* sc
         return MOE_ERR_SHAPE;
     if (mats == 0 || rows == 0 || cols == 0) return MOE_OK;
     if (!q || !scales || !qt || !scales_t) return MOE_ERR_NULL;
+    if (!aligned16(q) || !aligned16(qt)) return MOE_ERR_ALIGN;
     const int64_t blocks = mats * (rows / 128) * (cols / 128);
     const int grid = int(std::min<int64_t>(blocks, int64_t(sm_count()) * 8));
     transpose_w_kernel<<<grid, 256, 0, as_stream(stream)>>>(q, scales, mats, int(rows), int(cols),

@@ -59,6 +59,7 @@ constexpr int kMaxGroups = 1040;
 constexpr int kBM = 128;                         // tokens per CTA tile
 constexpr int kPromoters = 8;                    // promotion warps
 constexpr int kABoxes = 4;                       // token boxes of 128, 64, 32, 16 rows
+constexpr int kTokenTilesFirst = 16;             // groups up to this many token tiles: token tiles fastest
 
 template <bool PAIR, bool SWIGLU, bool WIDE>
 struct Cfg {
@@ -70,6 +71,7 @@ struct Cfg {
     // per K block cost more issue time than the 512 cycles the block's MMAs
     // take.)
     static constexpr int kChains = 1;                              // MMA chains per K block
+    static_assert(kChains == 1, "the promotion waits on the stage barrier of its K block");
     static constexpr int kBufCols = kAccCols / kChains;            // TMEM columns per buffer
     static constexpr int kBufs = 512 / kBufCols;                   // TMEM partial buffers
     static constexpr int kWRows = PAIR ? 128 : kAccCols;           // weight rows this CTA loads
@@ -522,13 +524,22 @@ __device__ __forceinline__ Item decode_item(const SharedState* ss, const GemmPar
     it.g = lo;
     const int local = item - ss->gstart[lo];
     const int rows = ss->goff[lo + 1] - ss->goff[lo];
-    // column tiles fastest: the CTAs running at the same time share a few
-    // token tiles and walk all of the expert's weight tiles, so a large group
-    // (the hot experts of a skewed batch, 128 token tiles) reads its token
-    // rows from HBM once while its weights (29 MB at most) stay in L2; with
-    // token tiles fastest the token rows were read once per column tile
-    const int mt = local / p.n_ftiles;
-    it.f = local - mt * p.n_ftiles;
+    const int mtiles = (rows + ITEM_ROWS - 1) / ITEM_ROWS;
+    // Order inside a group.  Small groups (a few token tiles, the common
+    // case): token tiles fastest, so the tiles that read one weight tile run
+    // side by side and the weight tile crosses HBM once.  Large groups (the
+    // hot experts of a skewed batch, up to 128 token tiles): column tiles
+    // fastest, so the CTAs running together share a few token tiles and walk
+    // the expert's weight tiles (29 MB at most, kept in L2), and the token
+    // rows cross HBM once instead of once per column tile.
+    int mt;
+    if (mtiles <= kTokenTilesFirst) {
+        it.f = local / mtiles;
+        mt = local - it.f * mtiles;
+    } else {
+        mt = local / p.n_ftiles;
+        it.f = local - mt * p.n_ftiles;
+    }
     it.row0 = ss->goff[lo] + mt * ITEM_ROWS;
     it.rows = rows - mt * ITEM_ROWS;
     return it;
@@ -719,8 +730,10 @@ __device__ __forceinline__ void mma_issuer(const GemmParams& p, uint8_t* smem, S
                     for (int kk = 0; kk < 4; ++kk)
                         mma_e4m3<PAIR>(d, sw128_desc(st + kk * 32), sw128_desc(b0 + kk * 32), idesc,
                                        kk > 0 ? 1u : 0u);
+                    // one commit per K block: its completion frees the
+                    // stage for the producer AND hands the partial to the
+                    // promotion warps (who wait on the same barrier)
                     mma_commit_both<PAIR>(smem_u32(&ss->empty[s]));
-                    mma_commit_both<PAIR>(smem_u32(&ss->tfull[buf]));
                 }
             }
         }
@@ -893,8 +906,12 @@ __device__ __forceinline__ void promoter(const GemmParams& p, SharedState* ss, c
             const uint32_t buf = tb % C::kBufs;
             const int c = cit % kScaleSlots;
             if (lane == 0) {
-                ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->tfull[buf]), (tb / C::kBufs) & 1u,
-                                                   ss, p.dev_status);
+                // the K block's MMAs have completed: the stage barrier the
+                // producer refills on (the stage cannot complete again before
+                // this wait: its next K block needs this warp's release of
+                // the TMEM buffer one block later)
+                ok = mbar_wait<kRemoteWait<PAIR>>(smem_u32(&ss->empty[tb % C::kStages]),
+                                                   (tb / C::kStages) & 1u, ss, p.dev_status);
                 if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (cit / kScaleSlots) & 1u, ss,
                                        p.dev_status);
             }
@@ -1754,8 +1771,7 @@ __device__ __forceinline__ void wg_mma_issuer(const WgParams& p, uint8_t* smem, 
                 for (int kk = 0; kk < 4; ++kk)
                     mma_e4m3<false>(d, sw128_desc(st + kk * 32),
                                     sw128_desc(st + kTileBytes + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                mma_commit<false>(smem_u32(&ss->empty[s]));
-                mma_commit<false>(smem_u32(&ss->tfull[buf]));
+                mma_commit<false>(smem_u32(&ss->empty[s]));  // stage free, partial ready
             }
         }
         mma_commit<false>(smem_u32(&ss->drain));
@@ -1817,7 +1833,8 @@ __device__ __forceinline__ void wg_promoter(const WgParams& p, SharedState* ss,
             const uint32_t buf = it % C::kBufs;
             const int c = it % kScaleSlots;
             if (lane == 0) {
-                ok = mbar_wait(smem_u32(&ss->tfull[buf]), (it / C::kBufs) & 1u, ss, p.dev_status);
+                ok = mbar_wait(smem_u32(&ss->empty[it % C::kStages]), (it / C::kStages) & 1u, ss,
+                               p.dev_status);
                 if (ok) ok = mbar_wait(smem_u32(&ss->sfull[c]), (it / kScaleSlots) & 1u, ss,
                                        p.dev_status);
             }

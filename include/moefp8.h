@@ -585,8 +585,9 @@ MOE_API int moe_layer_forward_host_batches(const MoeShape* shape, const MoeWeigh
  * fp32 scales [rows/128, cols/128] (the 128x128 block quantiser's output),
  * write the transposed codes [cols, rows] and scales [cols/128, rows/128].
  * A block keeps its scale, so the transposed matrix holds the same values
- * exactly (no requantisation).  Bit-exact.  rows, cols multiples of 128.
- * Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_CUDA. */
+ * exactly (no requantisation).  Bit-exact.  rows, cols multiples of 128; q
+ * and qt 16-byte aligned.  Errors: MOE_ERR_SHAPE, MOE_ERR_NULL, MOE_ERR_ALIGN,
+ * MOE_ERR_CUDA. */
 MOE_API int fp8_transpose_w_128x128(const uint8_t* q, const float* scales, int64_t mats,
                                     int64_t rows, int64_t cols, uint8_t* qt, float* scales_t,
                                     int* dev_status, void* stream);
