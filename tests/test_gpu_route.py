@@ -295,3 +295,34 @@ def test_pageable_host_pointer_is_rejected_not_dereferenced():
                       to_dev(inp["bias"]), host_offset, idx, gate, counts, ws)
     assert e.value.status == -7
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("cfg_name,T,with_offset", [("tiny", 256, False), ("skewed", 2048, True)])
+def test_route_scores_are_the_chosen_unbiased_affinities(cfg_name, T, with_offset):
+    """moe_route_scores writes, besides moe_route's outputs (bit-identical),
+    the unbiased affinity s of each chosen expert in slot order, equal to
+    the oracle's s at those experts bit for bit (the values the gates are
+    normalised from and the backward pass differentiates)."""
+    need_gpu()
+    import fp8_block_scaled_affinity_b200 as moe
+    cfg = S.CONFIGS[cfg_name]
+    inp = S.make_layer_inputs_host(cfg, 0)
+    x = inp["x"][:T]
+    off = inp["logit_offset"] if with_offset else None
+    shape = shape_of(cfg, T)
+    K, N = cfg.topk, cfg.n_routed
+    idx = torch.empty((T, K), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, K), dtype=torch.float32, device=DEV)
+    score = torch.empty((T, K), dtype=torch.float32, device=DEV)
+    counts = torch.empty((N,), dtype=torch.int32, device=DEV)
+    ws = torch.empty((moe.moe_route_workspace_size(shape),), dtype=torch.uint8, device=DEV)
+    moe.moe_route_scores(shape, bf16_dev(x), bf16_dev(inp["router_w"]), to_dev(inp["bias"]),
+                         None if off is None else to_dev(off), idx, gate, score, counts, ws)
+    torch.cuda.synchronize()
+    ref = oracle.route(x, inp["router_w"], inp["bias"], cfg.n_groups, cfg.topk_groups, K,
+                       logit_offset=off, want_scores=True)
+    assert np.array_equal(idx.cpu().numpy(), ref["topk_idx"])
+    assert np.array_equal(gate.cpu().numpy().view(np.uint32), ref["topk_gate"].view(np.uint32))
+    assert np.array_equal(counts.cpu().numpy(), ref["counts"])
+    s_ref = np.take_along_axis(ref["scores"], ref["topk_idx"], axis=1)
+    assert np.array_equal(score.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
