@@ -538,6 +538,227 @@ def run_permute(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_ep(args, world, rank, local):
+    """Expert-parallel layer stages, P = 8 ranks emulated on one GPU: each
+    rank owns 32 of the prefill layer's 256 routed experts (plus the shared
+    one) and routes its own 2,048 tokens (16,384 in all); every rank's
+    stages run through the library and each all-to-all is a device copy
+    that hands rank p's rows for rank q to rank q.  All ranks' stages run
+    one after another on one stream, so the value is the serialised
+    throughput of the EP kernels, not a multi-GPU figure; the per-stage
+    times and the EP kernels' GB/s are the point."""
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    from fp8_block_scaled_affinity_b200.ep import EpMoeLayer
+    import synthetic as S
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.CONFIGS["prefill"]
+    P, T = 8, 2048
+    inp = S.make_layer_inputs_host(cfg, 0)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    shape = moe.make_shape(T, cfg.d, cfg.n_routed, cfg.n_groups, cfg.topk_groups, cfg.topk,
+                           cfg.inter, cfg.gamma)
+    rw, bias = bf16(inp["router_w"]), torch.from_numpy(inp["bias"]).to(dev)
+    layers = [EpMoeLayer(shape, q, P, rw, bias.clone(), device=dev) for q in range(P)]
+    for e in range(cfg.n_routed + 1):
+        w = S.device_expert_weights(cfg, e, dev)
+        for l in layers:
+            l.set_expert(e, *w)
+    xs = [bf16(S.make_layer_inputs_host(cfg, 1 + q)["x"][:T]) for q in range(P)]
+    d = cfg.d
+
+    def step(marks=None):
+        sends = [l.route_and_pack(x, marks=marks) for l, x in zip(layers, xs)]
+        offs = [np.concatenate([[0], np.cumsum(c)]) for _, c in sends]
+        recv, src = [], []
+        for q in range(P):  # the dispatch all-to-all as device copies
+            recv.append(torch.cat([sends[p][0][offs[p][q]:offs[p][q + 1]] for p in range(P)]))
+            src.append(np.concatenate([[0], np.cumsum([sends[p][1][q] for p in range(P)])]))
+        backs = [layers[q].experts(recv[q], int(src[q][-1]), marks=marks) for q in range(P)]
+        ys = []
+        for p in range(P):  # the combine all-to-all as device copies
+            back = torch.cat([backs[q][src[q][p]:src[q][p + 1]] for q in range(P)])
+            ys.append(layers[p].shared_and_combine(xs[p], back, marks=marks))
+        return sends, recv
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        sends, recv = step()
+    e1.record(st)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    # per-stage times, all ranks summed (events between the library calls)
+    tot = {}
+    for it in range(args.steps):
+        marks = []
+        step(marks)
+        torch.cuda.synchronize()
+        prev = None
+        for name, ev in marks:
+            if name != "start" and prev is not None:
+                tot[name] = tot.get(name, 0.0) + prev.elapsed_time(ev)
+            prev = ev
+    brk = {n: v / args.steps for n, v in tot.items()}
+    n_send = sum(sum(c) for _, c in sends)
+    rb = layers[0].row_bytes
+    K, nkb = cfg.topk, d // 128
+    local_rows = sum(int(l.counts.sum().item()) for l in layers)  # routed pairs, all ranks
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    ep_bytes = {
+        # x read (bf16) + the rows written
+        "pack": P * T * d * 2 + n_send * rb,
+        # rows read + the local FP8 rows and kb-major scales written
+        "local_permute": n_send * rb + local_rows * (d + 4 * nkb),
+        # fp32 expert rows read + one fp32 partial row per received row written
+        "partial_combine": local_rows * d * 4 + n_send * d * 4,
+        # shared output + partial rows read (fp32), y written (bf16)
+        "final_combine": P * T * d * 4 + n_send * d * 4 + P * T * d * 2,
+    }
+    passes = {n: {"ms": brk[n], "bytes": b, "gbs": b / (brk[n] / 1e3) / 1e9,
+                  "frac_of_hbm": b / (brk[n] / 1e3) / 1e9 / hbm}
+              for n, b in ep_bytes.items()}
+    top = max(ep_bytes, key=lambda n: brk[n])
+    tok = P * T * args.steps
+    line = {
+        "metric": "ep_emulated_tokens_per_s", "value": tok / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8e4m3/f32", "data": "synthetic",
+        "config": {"workload": "moe_ep_prefill_8_ranks_on_one_gpu", "ranks": P,
+                   "tokens_per_rank": T, "d": d, "n_routed": cfg.n_routed,
+                   "experts_per_rank": cfg.n_routed // P, "topk": K, "inter": cfg.inter,
+                   "exchange": "device copies standing in for the all-to-alls",
+                   "l2": "inputs larger than L2 (11.6 GB of FP8 weights over the ranks)"},
+        "roofline": {"bound": "hbm", "kernel": f"EP {top}", "achieved": passes[top]["gbs"],
+                     "peak": hbm, "unit": "GB/s", "frac": passes[top]["frac_of_hbm"],
+                     "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes_per_launch": ep_bytes[top] / P,
+                     "frac_of_datasheet": passes[top]["gbs"] / DATASHEET["hbm_gbs"]},
+        "ep_passes": passes,
+        "breakdown_ms": brk,
+        "dispatch_rows": n_send, "row_bytes": rb,
+        "rows_per_token": n_send / (P * T),
+        "e2e": None,
+        "gpu_launches": None,
+        "clocks": clk,
+        "device_status": int(sum(int(l.dev_status.item()) for l in layers)),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_redundant(args, world, rank, local):
+    """Redundant experts on the skewed batch (T=16384): after one forward
+    pass, the planner gives 32 extra copies to the hottest experts and the
+    two expert GEMMs run over the copies' groups (each copy a group of the
+    indexed grouped GEMM sharing its expert's weights; the output rows are
+    bit-identical).  Both GEMMs are timed with and without the copies."""
+    import numpy as np
+    import torch
+    import fp8_block_scaled_affinity_b200 as moe
+    import synthetic as S
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg = S.CONFIGS["skewed"]
+    layer, x, off, inp, _ = build_layer(cfg, dev)
+    y = layer.forward(x, logit_offset=off)
+    torch.cuda.synchronize()
+    sh = layer.shape
+    T, d, I, N, K = cfg.T, cfg.d, cfg.inter, cfg.n_routed, cfg.topk
+    R = T * K + T
+    n_extra = 32
+    counts = layer.expert_counts.cpu().numpy()
+    rep, slots = moe.moe_plan_redundant_experts(counts, n_extra)
+    first = np.concatenate([[0], np.cumsum(rep)[:-1]]).astype(np.int32)
+    G = N + n_extra + 1
+    so = torch.empty(G + 1, dtype=torch.int32, device=dev)
+    sw = torch.empty(G, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    todev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    moe.moe_split_groups(sh, layer.expert_offsets, todev(rep), todev(slots), todev(first), n_extra,
+                         so, sw, status)
+    xq = torch.empty((R, d), dtype=torch.uint8, device=dev)
+    xs = torch.empty((d // 128, R), dtype=torch.float32, device=dev)
+    hq = torch.empty((R, I), dtype=torch.uint8, device=dev)
+    hs = torch.empty((I // 128, R), dtype=torch.float32, device=dev)
+    o = torch.empty((R, d), dtype=torch.float32, device=dev)
+    pws = torch.empty((moe.moe_permute_workspace_size(sh),), dtype=torch.uint8, device=dev)
+    moe.moe_quant_permute(sh, x, layer.topk_idx, layer.expert_counts, xq, xs,
+                          layer.expert_offsets, layer.row_of_pair, pws)
+    st = torch.cuda.current_stream()
+
+    def gemms(copies):
+        if copies:
+            moe.moe_grouped_gemm_fp8_indexed(G, so, sw, N + 1, R, xq, xs, d, layer.w13,
+                                             layer.w13_scales, 2 * I, moe.MOE_EPI_SWIGLU_QUANT,
+                                             hq, hs, status)
+            moe.moe_grouped_gemm_fp8_indexed(G, so, sw, N + 1, R, hq, hs, I, layer.w2,
+                                             layer.w2_scales, d, moe.MOE_EPI_F32, o, None,
+                                             status)
+        else:
+            moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, xq, xs, d, layer.w13,
+                                     layer.w13_scales, 2 * I, moe.MOE_EPI_SWIGLU_QUANT, hq, hs,
+                                     status)
+            moe.moe_grouped_gemm_fp8(N + 1, layer.expert_offsets, R, hq, hs, I, layer.w2,
+                                     layer.w2_scales, d, moe.MOE_EPI_F32, o, None, status)
+
+    res = {}
+    for copies in (False, True, False, True):
+        for _ in range(args.warmup):
+            gemms(copies)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(args.steps):
+            gemms(copies)
+        e1.record(st)
+        e1.synchronize()
+        res.setdefault(copies, []).append(e0.elapsed_time(e1) / args.steps)
+    ms_plain, ms_copies = min(res[False]), min(res[True])
+    flops = 2.0 * R * d * 3 * I
+    peaks, peak_src = load_peaks()
+    fp8_peak = float(peaks["bf16_tflops"]) * FP8_PER_BF16
+    tf = flops / (ms_copies / 1e3) / 1e12
+    sizes = np.diff(so.cpu().numpy())[:-1]
+    line = {
+        "metric": "expert_gemm_tflops", "value": tf, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_copies,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8e4m3/f32", "data": "synthetic",
+        "config": {"workload": "redundant_experts_skewed", "T": T, "n_extra": n_extra,
+                   "groups": G, "largest_group_rows": int(sizes.max()),
+                   "largest_expert_rows": int(counts.max()),
+                   "l2": "inputs larger than L2 (11.3 GB of FP8 weights)"},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm (W13 + W2) over the copies",
+                     "achieved": tf, "peak": fp8_peak, "unit": "TFLOP/s", "frac": tf / fp8_peak,
+                     "peak_source": f"{peak_src} bf16 burst x {FP8_PER_BF16:g}", "traffic": None,
+                     "frac_of_datasheet": tf / DATASHEET["fp8_tflops"]},
+        "without_copies": {"ms": ms_plain, "tflops": flops / (ms_plain / 1e3) / 1e12},
+        "with_copies": {"ms": ms_copies, "tflops": tf},
+        "e2e": None,
+        "gpu_launches": 2 * args.steps,
+        "device_status": int(status.item()),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------- GEMM-alone workload
 def run_gemm(args, world, rank, local):
     """The FP8 block-scaled GEMM alone: A [4096, 7168] (1x128 scales) times B
@@ -1162,7 +1383,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="skewed",
                     choices=["tiny", "prefill", "decode", "skewed", "prefill_e16", "gemm",
-                             "route", "permute"])
+                             "route", "permute", "ep", "redundant"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scales", choices=["fp32", "ue8m0"], default="fp32",
                     help="fp32: the pages' recipe (default); ue8m0: the power-of-two scale "
@@ -1185,6 +1406,10 @@ def main(argv=None):
             run_route(args, world, rank, local)
         elif args.workload == "permute":
             run_permute(args, world, rank, local)
+        elif args.workload == "ep":
+            run_ep(args, world, rank, local)
+        elif args.workload == "redundant":
+            run_redundant(args, world, rank, local)
         elif args.which == "backward":
             run_backward(args, world, rank, local)
         else:

@@ -30,6 +30,15 @@ from ._lib import (MOE_EPI_F32, MOE_EPI_SWIGLU_QUANT, make_shape, moe_combine,  
                    fp8_quant_w_128x128)
 
 
+def _mark(marks, name, device):
+    """Append (name, CUDA event recorded on the current stream) when timing."""
+    if marks is not None:
+        import torch
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(torch.cuda.current_stream(device))
+        marks.append((name, ev))
+
+
 class EpMoeLayer:
     """One rank's share of an expert-parallel MoE layer.
 
@@ -80,29 +89,37 @@ class EpMoeLayer:
         fp8_quant_w_128x128(w2, self.w2[j], self.w2_scales[j], stream=stream)
 
     # ---------------------------------------------------------- stages
-    def route_and_pack(self, x, logit_offset=None):
+    def route_and_pack(self, x, logit_offset=None, marks=None):
         """Routing with the (replicated) bias, the dispatch plan and the send
-        rows.  Returns (send_buf, send_counts as a host list)."""
+        rows.  Returns (send_buf, send_counts as a host list).  marks: as in
+        MoeLayer.backward (events after "route", "plan", "pack")."""
         import torch
-        sh = self.shape
+        sh, dev = self.shape, self.device
+        _mark(marks, "start", dev)
         moe_route(sh, x, self.router_w, self.bias, logit_offset, self.topk_idx, self.topk_gate,
                   self.counts, self.route_ws, self.dev_status)
+        _mark(marks, "route", dev)
         ws = torch.empty((moe_ep_workspace_size(sh, self.P, 0),), dtype=torch.uint8,
                          device=self.device)
         moe_ep_dispatch_plan(sh, self.P, self.topk_idx, self.send_counts, self.send_offsets,
                              self.send_row, ws, self.dev_status)
+        _mark(marks, "plan", dev)
         counts = self.send_counts.cpu().tolist()  # split sizes for the exchange
         send_buf = torch.empty((max(sum(counts), 1), self.row_bytes), dtype=torch.uint8,
                                device=self.device)
+        _mark(marks, "counts_to_host", dev)
         moe_ep_pack(sh, self.P, x, self.topk_idx, self.topk_gate, self.send_row, send_buf,
                     self.dev_status)
+        _mark(marks, "pack", dev)
         return send_buf, counts
 
-    def experts(self, recv_buf, n_recv: int):
+    def experts(self, recv_buf, n_recv: int, marks=None):
         """The local experts on the received rows; returns the fp32 partial
-        outputs [n_recv, d] to send back (same row order)."""
+        outputs [n_recv, d] to send back (same row order).  marks: events
+        after "local_permute", "gemm_w13", "gemm_w2", "partial_combine"."""
         import torch
         sh, dev = self.shape, self.device
+        _mark(marks, "start", dev)
         d, I, K = sh.d, sh.inter, sh.topk
         max_rows = max(n_recv * min(K, self.E), 1)
         xq = torch.empty((max_rows, d), dtype=torch.uint8, device=dev)
@@ -113,6 +130,7 @@ class EpMoeLayer:
                          device=dev)
         moe_ep_local_permute(sh, self.P, recv_buf, n_recv, xq, xs, max_rows, off, pair_row, ws,
                              self.dev_status)
+        _mark(marks, "local_permute", dev)
         back = torch.empty((max(n_recv, 1), d), dtype=torch.float32, device=dev)
         if n_recv == 0:
             return back[:0]
@@ -121,17 +139,22 @@ class EpMoeLayer:
         o = torch.empty((max_rows, d), dtype=torch.float32, device=dev)
         moe_grouped_gemm_fp8(self.E, off, max_rows, xq, xs, d, self.w13, self.w13_scales,
                              2 * I, MOE_EPI_SWIGLU_QUANT, hq, hs, self.dev_status)
+        _mark(marks, "gemm_w13", dev)
         moe_grouped_gemm_fp8(self.E, off, max_rows, hq, hs, I, self.w2, self.w2_scales, d,
                              MOE_EPI_F32, o, None, self.dev_status)
+        _mark(marks, "gemm_w2", dev)
         moe_ep_partial_combine(sh, self.P, recv_buf, n_recv, pair_row, o, back,
                                self.dev_status)
+        _mark(marks, "partial_combine", dev)
         return back[:n_recv]
 
-    def shared_and_combine(self, x, back_recv):
+    def shared_and_combine(self, x, back_recv, marks=None):
         """The shared expert on this rank's tokens, then y = its output + the
-        partial outputs of each token's destinations (rank order), bf16."""
+        partial outputs of each token's destinations (rank order), bf16.
+        marks: events after "shared_expert" and "final_combine"."""
         import torch
         sh, dev = self.shape, self.device
+        _mark(marks, "start", dev)
         T, d, I = sh.T, sh.d, sh.inter
         y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
         if T == 0:
@@ -148,8 +171,10 @@ class EpMoeLayer:
                              MOE_EPI_SWIGLU_QUANT, hq, hs, self.dev_status)
         moe_grouped_gemm_fp8(1, off, T, hq, hs, I, self.w2[s:], self.w2_scales[s:], d,
                              MOE_EPI_F32, o, None, self.dev_status)
+        _mark(marks, "shared_expert", dev)
         moe_ep_final_combine(sh, self.P, o, back_recv if back_recv.numel() else None,
                              self.send_row, y, self.dev_status)
+        _mark(marks, "final_combine", dev)
         return y
 
     def update_bias(self, global_counts, total_tokens: int) -> None:
