@@ -495,3 +495,23 @@ def test_layer_wgrad_full_expert_shapes():
     """d = 7168, I = 2048, 16 routed experts: the shared expert and three
     routed ones (the oracle's FP64 weight gradients are 0.35 GB each)."""
     _wgrad_case("prefill_e16", S.CONFIGS["prefill_e16"], experts=[16, 0, 5, 11])
+
+
+def test_layer_backward_empty_batch():
+    """T = 0: every gradient is empty or zero (the weight gradients of every
+    expert, the router's gradient), and nothing faults."""
+    need_gpu()
+    moe = _moe()
+    cfg = S.CONFIGS["tiny"]
+    inp = S.make_layer_inputs_host(cfg, 0)
+    layer = moe.MoeLayer(shape_of(cfg, 0), bf16_dev(inp["router_w"]), to_dev(inp["bias"]),
+                         device=DEV)
+    for e in range(cfg.n_routed + 1):
+        layer.set_expert(e, *expert_bf16(cfg, e))
+    x = bf16_dev(inp["x"][:0])
+    layer.forward_train(x)
+    dx, dE, dW13, dW2 = layer.backward(bf16_dev(inp["x"][:0]), wgrad=True)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert dx.shape == (0, cfg.d)
+    assert not torch.any(dE) and not torch.any(dW13) and not torch.any(dW2)
