@@ -293,10 +293,11 @@ class MoeLayer:
         KP = nb * 128
         xt = torch.empty((d, KP), dtype=u8, device=dev)
         xts = torch.empty((nb, d), dtype=f32, device=dev)
-        moe_wgrad_quant_x(sh, b["x"], pair_scratch, blocks, xt, xts, st, stream)
         dact = torch.empty((2 * I, KP), dtype=u8, device=dev)
         dacts = torch.empty((nb, 2 * I), dtype=f32, device=dev)
-        moe_wgrad_quant_dac(dh, ac, I, blocks, dact, dacts, st, stream)
+        if T > 0:  # with no rows no group has K blocks: the operands are never read
+            moe_wgrad_quant_x(sh, b["x"], pair_scratch, blocks, xt, xts, st, stream)
+            moe_wgrad_quant_dac(dh, ac, I, blocks, dact, dacts, st, stream)
         mark("wgrad_quant_x_dac")
         dW13 = torch.empty((G, 2 * I, d), dtype=f32, device=dev)
         moe_grouped_gemm_wgrad(G, kb_off, nb, dact, dacts, 2 * I, xt, xts, d, dW13, st, stream)
@@ -304,10 +305,12 @@ class MoeLayer:
         del xt, xts, dact, dacts
         dot = torch.empty((d, KP), dtype=u8, device=dev)
         dots = torch.empty((nb, d), dtype=f32, device=dev)
-        moe_wgrad_quant_do(sh, dy, self.topk_gate, pair_scratch, blocks, dot, dots, st, stream)
         ht = torch.empty((I, KP), dtype=u8, device=dev)
         hts = torch.empty((nb, I), dtype=f32, device=dev)
-        moe_wgrad_quant_h(ac, I, blocks, ht, hts, st, stream)
+        if T > 0:
+            moe_wgrad_quant_do(sh, dy, self.topk_gate, pair_scratch, blocks, dot, dots, st,
+                               stream)
+            moe_wgrad_quant_h(ac, I, blocks, ht, hts, st, stream)
         mark("wgrad_quant_do_h")
         dW2 = torch.empty((G, d, I), dtype=f32, device=dev)
         moe_grouped_gemm_wgrad(G, kb_off, nb, dot, dots, d, ht, hts, I, dW2, st, stream)
