@@ -2083,9 +2083,9 @@ int moe::grouped_gemm_fp8(int n_groups, const int32_t* group_offsets, int max_ro
     if (epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_SWIGLU_QUANT)
         return MOE_ERR_ARG;
     if (epilogue == MOE_EPI_SWIGLU_QUANT && n % 256) return MOE_ERR_SHAPE;
-    if (!group_offsets || !w || !w_scales || !out) return MOE_ERR_NULL;
-    if (epilogue == MOE_EPI_SWIGLU_QUANT && !out_scales) return MOE_ERR_NULL;
-    if (max_rows == 0) return MOE_OK;
+    if (!group_offsets || !w || !w_scales) return MOE_ERR_NULL;
+    if (max_rows == 0) return MOE_OK;  // no rows: nothing read or written
+    if (!out || (epilogue == MOE_EPI_SWIGLU_QUANT && !out_scales)) return MOE_ERR_NULL;
     if (!a || !a_scales) return MOE_ERR_NULL;
     if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MOE_ERR_ALIGN;
     if (int64_t(n_weights) * n > INT32_MAX) return MOE_ERR_SHAPE;
@@ -2145,9 +2145,9 @@ extern "C" MOE_API int moe_grouped_gemm_mxfp8(int n_groups, const int32_t* group
         return MOE_ERR_SHAPE;
     if (epilogue != MOE_EPI_F32 && epilogue != MOE_EPI_BF16 && epilogue != MOE_EPI_SWIGLU_QUANT)
         return MOE_ERR_ARG;
-    if (!group_offsets || !w || !w_sf || !out) return MOE_ERR_NULL;
-    if (epilogue == MOE_EPI_SWIGLU_QUANT && !out_sf) return MOE_ERR_NULL;
-    if (max_rows == 0) return MOE_OK;
+    if (!group_offsets || !w || !w_sf) return MOE_ERR_NULL;
+    if (max_rows == 0) return MOE_OK;  // no rows: nothing read or written
+    if (!out || (epilogue == MOE_EPI_SWIGLU_QUANT && !out_sf)) return MOE_ERR_NULL;
     if (!a || !a_sf) return MOE_ERR_NULL;
     if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MOE_ERR_ALIGN;
     if (int64_t(n_groups) * n > INT32_MAX) return MOE_ERR_SHAPE;
