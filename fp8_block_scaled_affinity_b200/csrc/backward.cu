@@ -66,6 +66,21 @@ __global__ void __launch_bounds__(256) combine_backward_quant_kernel(
             const int c = c0 + lane + 32 * j;
             v[j] = c < nvec ? __ldg(dy + int64_t(t) * nvec + c) : make_uint4(0u, 0u, 0u, 0u);
         }
+        // each tile's max |dy| once: for g >= 0, max |fp32(g v)| over a tile
+        // is fp32(g max |v|) (rounding is monotone), so every row's scale
+        // follows from it without another reduction
+        float tmax[PC];
+#pragma unroll
+        for (int j = 0; j < PC; ++j) {
+            const uint4 w = v[j];
+            float a = fmaxf(fmaxf(fabsf(bf16_lo(w.x)), fabsf(bf16_hi(w.x))),
+                            fmaxf(fabsf(bf16_lo(w.y)), fabsf(bf16_hi(w.y))));
+            a = fmaxf(a, fmaxf(fmaxf(fabsf(bf16_lo(w.z)), fabsf(bf16_hi(w.z))),
+                               fmaxf(fabsf(bf16_lo(w.w)), fabsf(bf16_hi(w.w)))));
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            tmax[j] = a;
+        }
         const int tile = c0 / 16 + lane;
         for (int k = 0; k <= K; ++k) {
             const int row = k < K ? __shfl_sync(0xffffffffu, my_row, k) : T * K + t;
@@ -75,19 +90,12 @@ __global__ void __launch_bounds__(256) combine_backward_quant_kernel(
 #pragma unroll
             for (int j = 0; j < PC; ++j) {
                 const uint4 w = v[j];
-                float f[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                              bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    f[i] = __fmul_rn(g, f[i]);
-                    amax = fmaxf(amax, fabsf(f[i]));
-                }
-#pragma unroll
-                for (int o = 8; o >= 1; o >>= 1)
-                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 float scale, inv;
-                scale_from_amax(amax, scale, inv);
+                scale_from_amax(__fmul_rn(fabsf(g), tmax[j]), scale, inv);
+                const float f[8] = {__fmul_rn(g, bf16_lo(w.x)), __fmul_rn(g, bf16_hi(w.x)),
+                                    __fmul_rn(g, bf16_lo(w.y)), __fmul_rn(g, bf16_hi(w.y)),
+                                    __fmul_rn(g, bf16_lo(w.z)), __fmul_rn(g, bf16_hi(w.z)),
+                                    __fmul_rn(g, bf16_lo(w.w)), __fmul_rn(g, bf16_hi(w.w))};
                 const uint32_t a0 = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv));
                 const uint32_t a1 = e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
                 const uint32_t a2 = e4m3x2(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv));
