@@ -524,25 +524,28 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
         // Eight rows at a time: their token indices first, then all their
         // loads, then the arithmetic (a warp keeps eight loads in flight).
         const int fl = f0 + 2 * lane;
-        for (int i0 = 0; i0 < 16; i0 += 8) {
-            float v0[8], v1[8];
+        // rows per batch: all 16 of the warp's rows for the gathered bf16
+        // sources (their token indices, then their loads, all in flight)
+        constexpr int RB = (SRC == kWgX || SRC == kWgDo) ? 16 : 8;
+        for (int i0 = 0; i0 < 16; i0 += RB) {
+            float v0[RB], v1[RB];
             if (SRC == kWgX || SRC == kWgDo) {
-                int tok[8];
-                float g[8];
+                int tok[RB];
+                float g[RB];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < RB; ++i) {
                     const int rr = warp + 8 * (i0 + i);
                     g[i] = 0.0f;
                     tok[i] = rr < blk.y ? wg_token(src, blk.x + rr, g[i]) : -1;
                 }
-                uint32_t w2[8];
+                uint32_t w2[RB];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < RB; ++i)
                     w2[i] = tok[i] >= 0
                                 ? __ldg(reinterpret_cast<const uint32_t*>(src.x + int64_t(tok[i]) * F + fl))
                                 : 0u;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < RB; ++i) {
                     v0[i] = bf16_lo(w2[i]);
                     v1[i] = bf16_hi(w2[i]);
                     if (SRC == kWgDo) {
@@ -596,7 +599,7 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < RB; ++i)
                 *reinterpret_cast<float2*>(&tile[warp + 8 * (i0 + i)][2 * lane]) =
                     make_float2(v0[i], v1[i]);
         }
