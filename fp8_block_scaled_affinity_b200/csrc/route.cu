@@ -32,7 +32,8 @@
 //      in 3 and, when the list is short, for all N_r logits of every listed
 //      token: route_exact_pairs_kernel (a warp per chosen logit) settles
 //      those whose sum provably cannot round, from an exact parallel sum;
-//      route_exact_chain_kernel (a thread per sum) evaluates the rest and
+//      route_exact_chain_kernel (a warp per sum, operands streamed while one
+//      lane adds in order) evaluates the rest and
 //      the listed tokens' rows in ascending k; route_logits_list_kernel
 //      does listed tokens in 64x64 FP64 tiles when the list is long;
 //   5. route_select_kernel (warp per token): exact s and s' of the chosen
@@ -574,77 +575,9 @@ __device__ __forceinline__ void vec_products(const uint4& xv, const uint4& ev, b
     }
 }
 
-// The defining sum when no addition of it can round (sum_is_exact): any
-// order gives the same double, so eight interleaved accumulators shorten
-// the dependent chain eightfold.
-__device__ __forceinline__ float exact_logit_unordered(const uint16_t* __restrict__ xr,
-                                                       const uint16_t* __restrict__ er, int d) {
-    const uint4* xp = reinterpret_cast<const uint4*>(xr);
-    const uint4* ep = reinterpret_cast<const uint4*>(er);
-    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
-    for (int v = 0; v < d / 8; ++v) {
-        const uint4 xv = __ldg(xp + v), ev = __ldg(ep + v);
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-        const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            acc[2 * q] = __fma_rn(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]), acc[2 * q]);
-            acc[2 * q + 1] = __fma_rn(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]), acc[2 * q + 1]);
-        }
-    }
-    const double s = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-    return __double2float_rn(s);
-}
-
-__device__ __forceinline__ float exact_logit(const uint16_t* __restrict__ xr,
-                                             const uint16_t* __restrict__ er, int d,
-                                             bool fp32_products) {
-    // 16-byte vectors (8 k) of both rows stream through a 16-deep register
-    // ring: slot i is consumed, then refilled with the vector 16 further on
-    // (the few threads of this kernel are bound by load latency, so each
-    // keeps 32 loads in flight).
-    // The products of the next vector are formed and widened before the
-    // FP64 adds of the current one, so the conversions overlap the add
-    // chain.  Each product of two bf16 values is exact in FP64 (and in fp32
-    // under fp32_products), so adding it equals the FP64 fma of the
-    // definition.
-    constexpr int kRing = 16;
-    const uint4* xp = reinterpret_cast<const uint4*>(xr);
-    const uint4* ep = reinterpret_cast<const uint4*>(er);
-    const int nv = d / 8;  // a multiple of 16 = kRing
-    uint4 xv[kRing], ev[kRing];
-#pragma unroll
-    for (int i = 0; i < kRing; ++i) {
-        xv[i] = __ldg(xp + i);
-        ev[i] = __ldg(ep + i);
-    }
-    double acc = 0.0;
-    double p[8];
-    vec_products(xv[0], ev[0], fp32_products, p);
-    for (int v0 = 0; v0 < nv; v0 += kRing) {
-#pragma unroll
-        for (int i = 0; i < kRing; ++i) {
-            if (v0 + kRing + i < nv) {
-                xv[i] = __ldg(xp + v0 + kRing + i);
-                ev[i] = __ldg(ep + v0 + kRing + i);
-            }
-            double pn[8];
-            const int ni = (i + 1) % kRing;
-            if (v0 + i + 1 < nv) vec_products(xv[ni], ev[ni], fp32_products, pn);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) acc = __dadd_rn(acc, p[q]);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) p[q] = pn[q];
-        }
-    }
-    return __double2float_rn(acc);
-}
-
 // Chosen logits that the bound did not settle, and every logit of the
-// tokens on the uncertified list, come from one sum per thread
-// while the list holds at most kPairList tokens; longer lists go to the
-// tiled kernel below.
+// tokens on the uncertified list, come from one sum per warp while the list
+// holds at most kPairList tokens; longer lists go to the tiled kernel below.
 constexpr int kPairList = 256;
 
 // Exactness of one row pair's defining sum, decided by a warp.  Every
@@ -789,37 +722,93 @@ __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
     }
 }
 
-// Phase 2, one thread per job: the pair-list jobs phase 1 marked (NaN) and
+// The defining sum of one row pair by a warp, in ascending k: the lanes load
+// the rows 32 vectors (256 k) per chunk, form the exact products and store
+// them in a 4-chunk ring in shared memory, while lane 0 adds the chunk three
+// behind in order.  The additions are the definition's own, one dependent
+// chain; the warp only keeps the operands streaming (a lone thread waited
+// on its loads).  Returns the fp32 result in every lane.
+constexpr int kChainRing = 4;
+__device__ __forceinline__ float warp_chain_logit(const uint16_t* __restrict__ xr,
+                                                  const uint16_t* __restrict__ er, int d,
+                                                  bool fp32_products, int lane,
+                                                  double* __restrict__ ring) {
+    const uint4* xp = reinterpret_cast<const uint4*>(xr);
+    const uint4* ep = reinterpret_cast<const uint4*>(er);
+    const int nv = d / 8;
+    const int nch = (nv + 31) / 32;
+    auto store = [&](int ch, const uint4& xv, const uint4& ev) {
+        double p[8];
+        vec_products(xv, ev, fp32_products, p);
+        double* dst = ring + (ch % kChainRing) * 256 + lane * 8;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = p[q];
+    };
+    for (int ch = 0; ch < kChainRing - 1 && ch < nch; ++ch) {
+        const int v = ch * 32 + lane;
+        if (v < nv) store(ch, __ldg(xp + v), __ldg(ep + v));
+    }
+    __syncwarp();
+    double acc = 0.0;
+    for (int ch = 0; ch < nch; ++ch) {
+        // the loads of the chunk kChainRing - 1 ahead go out before lane 0's adds
+        const int ahead = ch + kChainRing - 1;
+        const int v = ahead * 32 + lane;
+        uint4 xv = make_uint4(0u, 0u, 0u, 0u), ev = xv;
+        if (ahead < nch && v < nv) {
+            xv = __ldg(xp + v);
+            ev = __ldg(ep + v);
+        }
+        if (lane == 0) {
+            const double* src = ring + (ch % kChainRing) * 256;
+            const int n = min(32, nv - ch * 32) * 8;
+            for (int i = 0; i < n; ++i) acc = __dadd_rn(acc, src[i]);
+        }
+        // the slot of chunk `ahead` held chunk ch - 1, summed last round
+        if (ahead < nch && v < nv) store(ahead, xv, ev);
+        __syncwarp();
+    }
+    return __shfl_sync(0xffffffffu, __double2float_rn(acc), 0);
+}
+
+// Phase 2, one warp per job: the pair-list jobs phase 1 marked (NaN) and
 // every logit of the listed uncertified tokens get the defining sum in
-// ascending k, all in parallel (each is one dependent chain of d
-// additions).  Settled results are never NaN: phase 1 settles only finite
-// row pairs.
-__global__ void __launch_bounds__(64) route_exact_chain_kernel(
+// ascending k (a listed logit first tries phase 1's parallel exact sum).
+// Settled results are never NaN: phase 1 settles only finite row pairs.
+constexpr int kChainWarps = 2;
+__global__ void __launch_bounds__(32 * kChainWarps) route_exact_chain_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d, int K,
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
     const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
     const int32_t* __restrict__ list_count, const float* __restrict__ vmax,
-    const float* __restrict__ vmin, const double* __restrict__ l2, const double* __restrict__ lb,
-    float* __restrict__ u_exact, double* __restrict__ uhat, int* dev_status,
-    int32_t* __restrict__ check) {
+    const float* __restrict__ vmin, float* __restrict__ u_exact, double* __restrict__ uhat,
+    int* dev_status, int32_t* __restrict__ check) {
+    __shared__ __align__(16) double ring[kChainWarps][kChainRing * 256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const ExactJobs jobs = exact_jobs(T, N, K, pair_count, list_count, dev_status, check, false);
-    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j < jobs.nA + jobs.nB;
+    const int64_t stride = int64_t(gridDim.x) * kChainWarps;
+    for (int64_t j = int64_t(blockIdx.x) * kChainWarps + warp; j < jobs.nA + jobs.nB;
          j += stride) {
         int t, e, pj;
         if (!exact_job(j, jobs, T, N, K, cand, pair_list, list, t, e, pj)) {
-            if (j >= jobs.nA) route_bad(dev_status, check, 2, int(j));  // phase 1 saw the others
+            if (j >= jobs.nA && lane == 0) route_bad(dev_status, check, 2, int(j));
             continue;
         }
-        if (pj >= 0 && !isnan(u_exact[pj])) continue;  // settled in phase 1
-        const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
-                                   double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
-        const float u =
-            sum_is_exact(t, e, T, l2, lb)
-                ? exact_logit_unordered(x + int64_t(t) * d, E + int64_t(e) * d, d)
-                : exact_logit(x + int64_t(t) * d, E + int64_t(e) * d, d, fp32_products);
-        if (pj >= 0) u_exact[pj] = u;
-        else uhat[int64_t(t) * N + e] = (double)u;
+        if (pj >= 0 && !isnan(u_exact[pj])) continue;  // settled in phase 1 (warp-uniform)
+        const uint16_t* xr = x + int64_t(t) * d;
+        const uint16_t* er = E + int64_t(e) * d;
+        float u = 0.0f;
+        bool done = false;
+        if (pj < 0) done = warp_exact_logit(xr, er, d, lane, u);  // warp-uniform
+        if (!done) {
+            const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
+                                       double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
+            u = warp_chain_logit(xr, er, d, fp32_products, lane, ring[warp]);
+        }
+        if (lane == 0) {
+            if (pj >= 0) u_exact[pj] = u;
+            else uhat[int64_t(t) * N + e] = (double)u;
+        }
     }
 }
 
@@ -1209,14 +1198,15 @@ extern "C" MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x
     if ((rc = check_launch()) != MOE_OK) return rc;
 
     // 4. the defining FP64 sums where they are needed: a warp per job where
-    // the sum provably cannot round, then a thread per remaining job
+    // the sum provably cannot round, then a warp per remaining job (the
+    // ascending-k chain)
     route_exact_pairs_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
         x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
         w.u_exact, w.uhat, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
-    route_exact_chain_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
+    route_exact_chain_kernel<<<unsigned(sms * 8), 32 * kChainWarps, 0, st>>>(
         x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
-        w.vmax, w.vmin, w.l2, w.lb, w.u_exact, w.uhat, dev_status, w.check);
+        w.vmax, w.vmin, w.u_exact, w.uhat, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
     dim3 gl((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
     route_logits_list_kernel<<<gl, kLThreads, 0, st>>>(x, router_w, T, d, N, w.list,
