@@ -33,9 +33,10 @@
 //      token: route_exact_pairs_kernel (a warp per chosen logit) settles
 //      those whose sum provably cannot round, from an exact parallel sum;
 //      route_exact_chain_kernel (a warp per sum, operands streamed while one
-//      lane adds in order) evaluates the rest and
-//      the listed tokens' rows in ascending k; route_logits_list_kernel
-//      does listed tokens in 64x64 FP64 tiles when the list is long;
+//      lane adds in order) evaluates the rest in ascending k;
+//      route_list_rows_kernel (a thread per sum) the listed tokens' rows
+//      while the list is short, route_logits_list_kernel (64x64 FP64
+//      tiles) when it is long;
 //   5. route_select_kernel (warp per token): exact s and s' of the chosen
 //      experts, slot order, gates and histogram for certified tokens; the
 //      full selection on the exact logits for listed ones.
@@ -575,9 +576,10 @@ __device__ __forceinline__ void vec_products(const uint4& xv, const uint4& ev, b
     }
 }
 
-// Chosen logits that the bound did not settle, and every logit of the
-// tokens on the uncertified list, come from one sum per warp while the list
-// holds at most kPairList tokens; longer lists go to the tiled kernel below.
+// Chosen logits that the bound did not settle come from one sum per warp;
+// every logit of the tokens on the uncertified list from one chain per
+// thread while the list holds at most kPairList tokens, from the tiled
+// kernel below for longer lists.
 constexpr int kPairList = 256;
 
 // Exactness of one row pair's defining sum, decided by a warp.  Every
@@ -649,41 +651,31 @@ __device__ __forceinline__ bool warp_exact_logit(const uint16_t* __restrict__ xr
     return true;
 }
 
-// Jobs of the exact-sum kernels: the listed chosen logits (pair list) and,
-// while the list of uncertified tokens is short, every logit of those
-// tokens.  Job j -> token t, expert e and the pair index pj (-1 for a
-// listed token's logit); false (reported) when an index is out of range.
+// Jobs of the exact-sum kernels: the listed chosen logits (pair list).  Job
+// j -> token t, expert e and the pair index pj; false when an index is out
+// of range.
 struct ExactJobs {
-    int64_t nA, nB;
+    int64_t nA;
 };
 
-__device__ __forceinline__ ExactJobs exact_jobs(int T, int N, int K, const int32_t* pair_count,
+__device__ __forceinline__ ExactJobs exact_jobs(int T, int K, const int32_t* pair_count,
                                                 const int32_t* list_count, int* dev_status,
                                                 int32_t* check, bool report) {
     int np = *pair_count, nl = *list_count;
     if (np > T * K || nl > T) {
         if (report) route_bad(dev_status, check, 1, max(np, nl));
         np = min(np, T * K);
-        nl = min(nl, T);
     }
-    return {int64_t(np), nl <= kPairList ? int64_t(nl) * N : 0};
+    return {int64_t(np)};
 }
 
-__device__ __forceinline__ bool exact_job(int64_t j, const ExactJobs& jobs, int T, int N, int K,
+__device__ __forceinline__ bool exact_job(int64_t j, int T, int N, int K,
                                           const int32_t* __restrict__ cand,
-                                          const int32_t* __restrict__ pair_list,
-                                          const int32_t* __restrict__ list, int& t, int& e,
+                                          const int32_t* __restrict__ pair_list, int& t, int& e,
                                           int& pj) {
-    pj = -1;
-    if (j < jobs.nA) {
-        pj = pair_list[j];
-        t = pj / K;
-        e = (pj >= 0 && pj < T * K) ? cand[pj] : -1;
-    } else {
-        const int64_t jj = j - jobs.nA;
-        t = list[jj / N];
-        e = int(jj % N);
-    }
+    pj = pair_list[j];
+    t = pj / K;
+    e = (pj >= 0 && pj < T * K) ? cand[pj] : -1;
     return t >= 0 && t < T && e >= 0 && e < N;
 }
 
@@ -691,23 +683,22 @@ __device__ __forceinline__ bool exact_job(int64_t j, const ExactJobs& jobs, int 
 // whose fp32 rounding was not settled): the warp settles the job by
 // warp_exact_logit when its defining sum cannot round (nearly every row pair
 // of real data) and otherwise marks it with a NaN for phase 2.  The full
-// rows of uncertified tokens go to phase 2 directly: those tokens are
-// uncertified mostly because of values far below their row's maximum, which
-// also fail this test.
+// rows of uncertified tokens skip this test (route_list_rows_kernel): those
+// tokens are uncertified mostly because of values far below their row's
+// maximum, which also fail it.
 __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d, int K,
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
-    const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
-    const int32_t* __restrict__ list_count, float* __restrict__ u_exact,
-    double* __restrict__ uhat, int* dev_status, int32_t* __restrict__ check) {
+    const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list_count,
+    float* __restrict__ u_exact, int* dev_status, int32_t* __restrict__ check) {
     const int lane = threadIdx.x & 31;
-    const ExactJobs jobs = exact_jobs(T, N, K, pair_count, list_count, dev_status, check,
+    const ExactJobs jobs = exact_jobs(T, K, pair_count, list_count, dev_status, check,
                                       blockIdx.x == 0 && threadIdx.x == 0);
     const int64_t stride = int64_t(gridDim.x) * (blockDim.x / 32);
     for (int64_t j = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); j < jobs.nA;
          j += stride) {
         int t, e, pj;
-        if (!exact_job(j, jobs, T, N, K, cand, pair_list, list, t, e, pj)) {
+        if (!exact_job(j, T, N, K, cand, pair_list, t, e, pj)) {
             if (lane == 0) route_bad(dev_status, check, 2, int(j));
             continue;
         }
@@ -715,10 +706,7 @@ __global__ void __launch_bounds__(64) route_exact_pairs_kernel(
         // are warp-uniform
         float u = 0.0f;
         const bool fast = warp_exact_logit(x + int64_t(t) * d, E + int64_t(e) * d, d, lane, u);
-        if (lane == 0) {
-            if (pj >= 0) u_exact[pj] = fast ? u : __int_as_float(0x7FFFFFFF);
-            else uhat[int64_t(t) * N + e] = fast ? (double)u : __longlong_as_double(0x7FF8000000000000ll);
-        }
+        if (lane == 0) u_exact[pj] = fast ? u : __int_as_float(0x7FFFFFFF);
     }
 }
 
@@ -771,45 +759,90 @@ __device__ __forceinline__ float warp_chain_logit(const uint16_t* __restrict__ x
     return __shfl_sync(0xffffffffu, __double2float_rn(acc), 0);
 }
 
-// Phase 2, one warp per job: the pair-list jobs phase 1 marked (NaN) and
-// every logit of the listed uncertified tokens get the defining sum in
-// ascending k (a listed logit first tries phase 1's parallel exact sum).
-// Settled results are never NaN: phase 1 settles only finite row pairs.
+// Phase 2, one warp per job: the pair-list jobs phase 1 marked (NaN) get the
+// defining sum in ascending k.  Settled results are never NaN: phase 1
+// settles only finite row pairs.  (The listed tokens' rows go to
+// route_list_rows_kernel.)
 constexpr int kChainWarps = 2;
 __global__ void __launch_bounds__(32 * kChainWarps) route_exact_chain_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d, int K,
     const int32_t* __restrict__ cand, const int32_t* __restrict__ pair_list,
-    const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list,
-    const int32_t* __restrict__ list_count, const float* __restrict__ vmax,
-    const float* __restrict__ vmin, float* __restrict__ u_exact, double* __restrict__ uhat,
+    const int32_t* __restrict__ pair_count, const int32_t* __restrict__ list_count,
+    const float* __restrict__ vmax, const float* __restrict__ vmin, float* __restrict__ u_exact,
     int* dev_status, int32_t* __restrict__ check) {
     __shared__ __align__(16) double ring[kChainWarps][kChainRing * 256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const ExactJobs jobs = exact_jobs(T, N, K, pair_count, list_count, dev_status, check, false);
+    const ExactJobs jobs = exact_jobs(T, K, pair_count, list_count, dev_status, check, false);
     const int64_t stride = int64_t(gridDim.x) * kChainWarps;
-    for (int64_t j = int64_t(blockIdx.x) * kChainWarps + warp; j < jobs.nA + jobs.nB;
-         j += stride) {
+    for (int64_t j = int64_t(blockIdx.x) * kChainWarps + warp; j < jobs.nA; j += stride) {
         int t, e, pj;
-        if (!exact_job(j, jobs, T, N, K, cand, pair_list, list, t, e, pj)) {
-            if (j >= jobs.nA && lane == 0) route_bad(dev_status, check, 2, int(j));
-            continue;
-        }
-        if (pj >= 0 && !isnan(u_exact[pj])) continue;  // settled in phase 1 (warp-uniform)
-        const uint16_t* xr = x + int64_t(t) * d;
-        const uint16_t* er = E + int64_t(e) * d;
-        float u = 0.0f;
-        bool done = false;
-        if (pj < 0) done = warp_exact_logit(xr, er, d, lane, u);  // warp-uniform
-        if (!done) {
-            const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
-                                       double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
-            u = warp_chain_logit(xr, er, d, fp32_products, lane, ring[warp]);
-        }
-        if (lane == 0) {
-            if (pj >= 0) u_exact[pj] = u;
-            else uhat[int64_t(t) * N + e] = (double)u;
+        // (a bad pair index was reported by phase 1)
+        if (!exact_job(j, T, N, K, cand, pair_list, t, e, pj)) continue;
+        if (!isnan(u_exact[pj])) continue;  // settled in phase 1 (warp-uniform)
+        const bool fp32_products = double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
+                                   double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
+        const float u = warp_chain_logit(x + int64_t(t) * d, E + int64_t(e) * d, d,
+                                         fp32_products, lane, ring[warp]);
+        if (lane == 0) u_exact[pj] = u;
+    }
+}
+
+// Every logit of the listed (uncertified) tokens while the list is short:
+// one thread per (listed token, expert) runs the defining sum in ascending
+// k.  The bf16 x bf16 products are exact in FP64, so each FMA is the
+// definition's addition of one product.  A block takes one listed token and
+// kRowThreads experts: the token's row is read by all its threads at once
+// (one broadcast load), each expert row by its own thread, kRowAhead
+// 16-byte vectors of both in flight.  With a few dozen listed tokens this
+// runs thousands of independent chains side by side; a chain's time is
+// d dependent FP64 additions.
+constexpr int kRowThreads = 64;
+constexpr int kRowAhead = 4;
+__global__ void __launch_bounds__(kRowThreads) route_list_rows_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int d, int n_routed,
+    const int32_t* __restrict__ list, const int32_t* __restrict__ list_count,
+    double* __restrict__ uhat, int* dev_status, int32_t* __restrict__ check) {
+    const int nl = min(*list_count, T);
+    const int l = blockIdx.x;
+    if (nl > kPairList || l >= nl) return;
+    const int t = list[l];
+    if (t < 0 || t >= T) {
+        if (threadIdx.x == 0) route_bad(dev_status, check, 2, t);
+        return;
+    }
+    const int e = blockIdx.y * kRowThreads + threadIdx.x;
+    if (e >= n_routed) return;
+    const uint4* xp = reinterpret_cast<const uint4*>(x + int64_t(t) * d);
+    const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e) * d);
+    const int nv = d / 8;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    uint4 xa[kRowAhead], ea[kRowAhead];
+#pragma unroll
+    for (int i = 0; i < kRowAhead; ++i) {
+        xa[i] = i < nv ? __ldg(xp + i) : zero;
+        ea[i] = i < nv ? __ldg(ep + i) : zero;
+    }
+    double acc = 0.0;
+    for (int v0 = 0; v0 < nv; v0 += kRowAhead) {
+#pragma unroll
+        for (int i = 0; i < kRowAhead; ++i) {
+            const uint32_t xw[4] = {xa[i].x, xa[i].y, xa[i].z, xa[i].w};
+            const uint32_t ew[4] = {ea[i].x, ea[i].y, ea[i].z, ea[i].w};
+            const int vn = v0 + kRowAhead + i;
+            if (vn < nv) {
+                xa[i] = __ldg(xp + vn);
+                ea[i] = __ldg(ep + vn);
+            }
+            if (v0 + i < nv) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fma(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]), acc);
+                    acc = fma(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]), acc);
+                }
+            }
         }
     }
+    uhat[int64_t(t) * n_routed + e] = (double)__double2float_rn(acc);
 }
 
 // The same sums for a long list, in 64 x 64 tiles of (listed token, expert):
@@ -1197,17 +1230,25 @@ extern "C" MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x
         w.pair_list, w.pair_count, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
-    // 4. the defining FP64 sums where they are needed: a warp per job where
-    // the sum provably cannot round, then a warp per remaining job (the
-    // ascending-k chain)
+    // 4. the defining FP64 sums where they are needed: a warp per chosen
+    // logit where the sum provably cannot round, then a warp per remaining
+    // one (the ascending-k chain); the listed tokens' rows a thread per sum
+    // (short list) or in tiles (long list)
     route_exact_pairs_kernel<<<unsigned(sms * 8), 64, 0, st>>>(
-        x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
-        w.u_exact, w.uhat, dev_status, w.check);
+        x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list_count, w.u_exact,
+        dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
     route_exact_chain_kernel<<<unsigned(sms * 8), 32 * kChainWarps, 0, st>>>(
-        x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list, w.list_count,
-        w.vmax, w.vmin, w.u_exact, w.uhat, dev_status, w.check);
+        x, router_w, T, N, d, K, w.cand, w.pair_list, w.pair_count, w.list_count, w.vmax,
+        w.vmin, w.u_exact, dev_status, w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
+    if (T > 0) {
+        dim3 gr(unsigned(std::min(T, kPairList)), unsigned((N + kRowThreads - 1) / kRowThreads));
+        route_list_rows_kernel<<<gr, kRowThreads, 0, st>>>(x, router_w, T, d, N, w.list,
+                                                           w.list_count, w.uhat, dev_status,
+                                                           w.check);
+        if ((rc = check_launch()) != MOE_OK) return rc;
+    }
     dim3 gl((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
     route_logits_list_kernel<<<gl, kLThreads, 0, st>>>(x, router_w, T, d, N, w.list,
                                                        w.list_count, w.uhat, dev_status, w.check);
