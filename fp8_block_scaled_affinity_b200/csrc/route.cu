@@ -112,21 +112,28 @@ __device__ __forceinline__ float warp_max(float v) {
 //   lb[r]  = the lowest bit any value of the row can carry: a bf16 value
 //            in [2^e, 2^(e+1)) has no bit below 2^(e-7) (2^-133 below 2^-126).
 // Block 0 also clears the two list counters and the check words of this call.
-__global__ void __launch_bounds__(256) route_slice_kernel(
+// With `staged`, the first pass keeps the row in the warp's slice of shared
+// memory (d * 2 bytes; the launch provides kSliceWarps of them) and the
+// second reads it from there; otherwise the second pass reads the row again.
+constexpr int kSliceWarps = 4;
+constexpr int kSliceStageMax = 32 * 1024;  // largest row staged per warp (d <= 16384)
+__global__ void __launch_bounds__(kSliceWarps * 32) route_slice_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int N, int d,
-    double nmargin, int8_t* __restrict__ xp, int8_t* __restrict__ ep, double* __restrict__ rsc,
-    int32_t* __restrict__ rex, double* __restrict__ r1, double* __restrict__ l2,
-    float* __restrict__ vmax, float* __restrict__ vmin, double* __restrict__ lb,
-    int32_t* __restrict__ list_count, int32_t* __restrict__ pair_count,
+    double nmargin, int staged, int8_t* __restrict__ xp, int8_t* __restrict__ ep,
+    double* __restrict__ rsc, int32_t* __restrict__ rex, double* __restrict__ r1,
+    double* __restrict__ l2, float* __restrict__ vmax, float* __restrict__ vmin,
+    double* __restrict__ lb, int32_t* __restrict__ list_count, int32_t* __restrict__ pair_count,
     int32_t* __restrict__ check) {
+    extern __shared__ __align__(16) uint4 slice_rows[];
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *list_count = 0;
         *pair_count = 0;
     }
     if (blockIdx.x == 0 && threadIdx.x < kCheckWords) check[threadIdx.x] = 0;
     const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x >> 5);
-    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T + N; r += warps) {
+    const int warps = gridDim.x * kSliceWarps;
+    uint4* const mine = slice_rows + (staged ? (threadIdx.x >> 5) * (d / 8) : 0);
+    for (int r = blockIdx.x * kSliceWarps + (threadIdx.x >> 5); r < T + N; r += warps) {
         const bool is_x = r < T;
         const int rr = is_x ? r : r - T;
         const int nrows = is_x ? T : N;
@@ -134,8 +141,11 @@ __global__ void __launch_bounds__(256) route_slice_kernel(
         int8_t* planes = is_x ? xp : ep;
         float mx = 0.0f, mn = FLT_MAX;
         bool finite = true;
+        __syncwarp();  // the previous row's second pass is done with the slice
+#pragma unroll 4
         for (int v = lane; v < d / 8; v += 32) {
             const uint4 w = __ldg(row + v);
+            if (staged) mine[v] = w;
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -148,14 +158,14 @@ __global__ void __launch_bounds__(256) route_slice_kernel(
         }
         mx = warp_max(mx);
         mn = warp_min(mn);
-        finite = __all_sync(0xffffffffu, finite);
+        finite = __all_sync(0xffffffffu, finite);  // (also orders the slice's stores)
         int sigma = 0;
         if (finite && mx > 0.0f) frexpf(mx, &sigma);  // mx < 2^sigma
         const double unit_inv = ldexp(1.0, 28 - sigma);
         bool exact = finite;
         double s1 = 0.0, s2 = 0.0;
         for (int v = lane; v < d / 8; v += 32) {
-            const uint4 w = __ldg(row + v);
+            const uint4 w = staged ? mine[v] : __ldg(row + v);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
             uint32_t dg[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
 #pragma unroll
@@ -790,59 +800,99 @@ __global__ void __launch_bounds__(32 * kChainWarps) route_exact_chain_kernel(
 // Every logit of the listed (uncertified) tokens while the list is short:
 // one thread per (listed token, expert) runs the defining sum in ascending
 // k.  The bf16 x bf16 products are exact in FP64, so each FMA is the
-// definition's addition of one product.  A block takes one listed token and
-// kRowThreads experts: the token's row is read by all its threads at once
-// (one broadcast load), each expert row by its own thread, kRowAhead
-// 16-byte vectors of both in flight.  With a few dozen listed tokens this
-// runs thousands of independent chains side by side; a chain's time is
-// d dependent FP64 additions.
+// definition's addition of one product; where the rows' ranges keep every
+// product a normal-range fp32 (the test of the chain kernel), the product is
+// formed in fp32, exactly, and one conversion per term replaces two.  A block
+// takes one listed token and kRowThreads experts.  A chain is d dependent
+// FP64 additions, so the operands must arrive well ahead:
+// asynchronous copies keep kRowStages - 1 chunks of 64 k in flight, each
+// thread copying its own expert row into its slot of a shared ring and 8
+// threads the token's row, which the whole block reads.
 constexpr int kRowThreads = 64;
-constexpr int kRowAhead = 4;
+constexpr int kRowStages = 3;
+constexpr int kRowChunk = 8;                    // 16-byte vectors per row and chunk
+constexpr int kRowPitch = kRowChunk * 16 + 16;  // a thread's slot (padded: no bank conflicts)
+
+__device__ __forceinline__ void row_cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void row_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void row_cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __global__ void __launch_bounds__(kRowThreads) route_list_rows_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ E, int T, int d, int n_routed,
     const int32_t* __restrict__ list, const int32_t* __restrict__ list_count,
-    double* __restrict__ uhat, int* dev_status, int32_t* __restrict__ check) {
+    const float* __restrict__ vmax, const float* __restrict__ vmin, double* __restrict__ uhat,
+    int* dev_status, int32_t* __restrict__ check) {
+    __shared__ __align__(16) uint8_t es[kRowStages][kRowThreads * kRowPitch];
+    __shared__ __align__(16) uint4 xs[kRowStages][kRowChunk];
     const int nl = min(*list_count, T);
     const int l = blockIdx.x;
-    if (nl > kPairList || l >= nl) return;
+    if (nl > kPairList || l >= nl) return;  // uniform over the block
     const int t = list[l];
     if (t < 0 || t >= T) {
         if (threadIdx.x == 0) route_bad(dev_status, check, 2, t);
         return;
     }
-    const int e = blockIdx.y * kRowThreads + threadIdx.x;
-    if (e >= n_routed) return;
+    const int tid = threadIdx.x;
+    const int e = blockIdx.y * kRowThreads + tid;
+    const bool e_ok = e < n_routed;  // threads past N copy nothing but keep the barriers
     const uint4* xp = reinterpret_cast<const uint4*>(x + int64_t(t) * d);
-    const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e) * d);
+    const uint4* ep = reinterpret_cast<const uint4*>(E + int64_t(e_ok ? e : 0) * d);
     const int nv = d / 8;
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    uint4 xa[kRowAhead], ea[kRowAhead];
+    const int nch = (nv + kRowChunk - 1) / kRowChunk;
+    const bool fp32_products = e_ok && double(vmin[t]) * double(vmin[T + e]) >= 0x1p-133 &&
+                               double(vmax[t]) * double(vmax[T + e]) < 0x1p127;
+    auto issue = [&](int ch) {
+        if (ch < nch) {
+            const int st = ch % kRowStages, v0 = ch * kRowChunk;
+            if (e_ok) {
 #pragma unroll
-    for (int i = 0; i < kRowAhead; ++i) {
-        xa[i] = i < nv ? __ldg(xp + i) : zero;
-        ea[i] = i < nv ? __ldg(ep + i) : zero;
-    }
-    double acc = 0.0;
-    for (int v0 = 0; v0 < nv; v0 += kRowAhead) {
-#pragma unroll
-        for (int i = 0; i < kRowAhead; ++i) {
-            const uint32_t xw[4] = {xa[i].x, xa[i].y, xa[i].z, xa[i].w};
-            const uint32_t ew[4] = {ea[i].x, ea[i].y, ea[i].z, ea[i].w};
-            const int vn = v0 + kRowAhead + i;
-            if (vn < nv) {
-                xa[i] = __ldg(xp + vn);
-                ea[i] = __ldg(ep + vn);
+                for (int i = 0; i < kRowChunk; ++i)
+                    if (v0 + i < nv) row_cp16(&es[st][tid * kRowPitch + 16 * i], ep + v0 + i);
             }
-            if (v0 + i < nv) {
+            if (tid < kRowChunk && v0 + tid < nv) row_cp16(&xs[st][tid], xp + v0 + tid);
+        }
+        row_cp_commit();  // (an empty group past the row end keeps the count)
+    };
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    acc = fma(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]), acc);
-                    acc = fma(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]), acc);
+    for (int ch = 0; ch < kRowStages - 1; ++ch) issue(ch);
+    double acc = 0.0;
+    for (int ch = 0; ch < nch; ++ch) {
+        row_cp_wait<kRowStages - 2>();  // this thread's copies of chunk ch have landed
+        __syncthreads();                // so have everyone's; chunk ch - 1 is consumed
+        issue(ch + kRowStages - 1);     // into the slot chunk ch - 1 held
+        const int st = ch % kRowStages;
+        const int nvc = min(kRowChunk, nv - ch * kRowChunk);
+#pragma unroll
+        for (int i = 0; i < kRowChunk; ++i) {
+            if (i < nvc) {
+                const uint4 xv = xs[st][i];
+                const uint4 ev = *reinterpret_cast<const uint4*>(&es[st][tid * kRowPitch + 16 * i]);
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+                if (fp32_products) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc = __dadd_rn(acc, (double)__fmul_rn(bf16_lo(xw[q]), bf16_lo(ew[q])));
+                        acc = __dadd_rn(acc, (double)__fmul_rn(bf16_hi(xw[q]), bf16_hi(ew[q])));
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc = fma(bf16_lo_d(xw[q]), bf16_lo_d(ew[q]), acc);
+                        acc = fma(bf16_hi_d(xw[q]), bf16_hi_d(ew[q]), acc);
+                    }
                 }
             }
         }
     }
-    uhat[int64_t(t) * n_routed + e] = (double)__double2float_rn(acc);
+    row_cp_wait<0>();
+    if (e_ok) uhat[int64_t(t) * n_routed + e] = (double)__double2float_rn(acc);
 }
 
 // The same sums for a long list, in 64 x 64 tiles of (listed token, expert):
@@ -1187,10 +1237,16 @@ extern "C" MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x
 
     // 1. digit planes and row statistics (also clears the list counter)
     const double nmargin = 4.0 * (d + 64) * 0x1p-53 + 0x1p-50;
-    route_slice_kernel<<<(T + N + 7) / 8, 256, 0, st>>>(x, router_w, T, N, d, nmargin, w.xp,
-                                                        w.ep, w.rsc, w.rex, w.r1, w.l2, w.vmax,
-                                                        w.vmin, w.lb, w.list_count, w.pair_count,
-                                                        w.check);
+    const int staged = 2 * d <= kSliceStageMax;
+    const size_t slice_smem = staged ? size_t(kSliceWarps) * 2 * d : 0;
+    if (slice_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(route_slice_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(slice_smem)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    route_slice_kernel<<<(T + N + kSliceWarps - 1) / kSliceWarps, kSliceWarps * 32, slice_smem,
+                         st>>>(x, router_w, T, N, d, nmargin, staged, w.xp, w.ep, w.rsc, w.rex,
+                               w.r1, w.l2, w.vmax, w.vmin, w.lb, w.list_count, w.pair_count,
+                               w.check);
     if ((rc = check_launch()) != MOE_OK) return rc;
 
     // 2. integer logits; K is split when the tiles alone leave SMs idle
@@ -1245,8 +1301,8 @@ extern "C" MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x
     if (T > 0) {
         dim3 gr(unsigned(std::min(T, kPairList)), unsigned((N + kRowThreads - 1) / kRowThreads));
         route_list_rows_kernel<<<gr, kRowThreads, 0, st>>>(x, router_w, T, d, N, w.list,
-                                                           w.list_count, w.uhat, dev_status,
-                                                           w.check);
+                                                           w.list_count, w.vmax, w.vmin, w.uhat,
+                                                           dev_status, w.check);
         if ((rc = check_launch()) != MOE_OK) return rc;
     }
     dim3 gl((T + kLT - 1) / kLT, (N + kLE - 1) / kLE);
