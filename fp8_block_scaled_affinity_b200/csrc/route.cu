@@ -377,6 +377,8 @@ __global__ void __launch_bounds__(128, 1) route_imma_kernel(
 // u~ - B and u~ + B round to the same fp32 value; otherwise (t, slot) goes
 // on the pair list, to be summed.
 constexpr int kCertWarps = 8;
+__host__ __device__ constexpr int cert_pitch(int n) { return n + n / 32 + 1; }
+__device__ __forceinline__ int cert_at(int i) { return i + (i >> 5); }
 
 // sum_L 2^(7(6-L)) acc_L = hi * 2^28 + lo, both parts exact in int64.
 __device__ __forceinline__ void level_parts(const int32_t* __restrict__ acc, int64_t plane,
@@ -441,9 +443,12 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
     int32_t* __restrict__ check) {
     extern __shared__ __align__(16) float cert_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* cen = cert_smem + warp * 3 * N;
-    float* lo = cen + N;
-    float* hi = lo + N;
+    // expert i at i + i / 32: the lanes of a group scan (stride ng, often 32)
+    // and of a 32-wide sweep then hit distinct banks
+    const int pitch = cert_pitch(N);
+    float* cen = cert_smem + warp * 3 * pitch;
+    float* lo = cen + pitch;
+    float* hi = lo + pitch;
     const int t = blockIdx.x * kCertWarps + warp;
     if (t >= T) return;  // no block-wide barrier below
     const int64_t plane = int64_t(T) * N;
@@ -457,9 +462,9 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
         const double c = 1.0 / (1.0 + exp(-(u + off))) + b;
         const double delta = 0.25 * Bp + 0x1p-23 + 0x1p-24 * fabs(b) + 1e-14;
         fin = fin && rex[T + i] >= 0 && isfinite(c) && isfinite(delta);
-        cen[i] = __double2float_rn(c);
-        lo[i] = __double2float_rd(c - delta);
-        hi[i] = __double2float_ru(c + delta);
+        cen[cert_at(i)] = __double2float_rn(c);
+        lo[cert_at(i)] = __double2float_rd(c - delta);
+        hi[cert_at(i)] = __double2float_ru(c + delta);
     }
     fin = __all_sync(0xffffffffu, fin);
     __syncwarp();
@@ -471,9 +476,9 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
     if (lane < n_groups) {
         for (int j = 0; j < ng; ++j) {
             const int i = lane * ng + j;
-            gv = fmaxf(gv, cen[i]);
-            glo = fmaxf(glo, lo[i]);
-            ghi = fmaxf(ghi, hi[i]);
+            gv = fmaxf(gv, cen[cert_at(i)]);
+            glo = fmaxf(glo, lo[cert_at(i)]);
+            ghi = fmaxf(ghi, hi[cert_at(i)]);
         }
         gi = lane;
     }
@@ -506,8 +511,8 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
         for (int j = 0, i = lane; i < N; ++j, i += 32) {
             if ((taken >> j) & 1u) continue;
             if (!((gmask >> (i / ng)) & 1u)) continue;
-            if (better(cen[i], i, bv, bi)) {
-                bv = cen[i];
+            if (better(cen[cert_at(i)], i, bv, bi)) {
+                bv = cen[cert_at(i)];
                 bi = i;
             }
         }
@@ -517,12 +522,12 @@ __global__ void __launch_bounds__(kCertWarps * 32) route_certify_kernel(
         if (lane == r) my_idx = bi;
     }
     {
-        const float chosen_lo = warp_min((lane < topk && my_idx < N) ? lo[my_idx] : INFINITY);
+        const float chosen_lo = warp_min((lane < topk && my_idx < N) ? lo[cert_at(my_idx)] : INFINITY);
         float rej_hi = -INFINITY;
         for (int j = 0, i = lane; i < N; ++j, i += 32) {
             if ((taken >> j) & 1u) continue;
             if (!((gmask >> (i / ng)) & 1u)) continue;
-            rej_hi = fmaxf(rej_hi, hi[i]);
+            rej_hi = fmaxf(rej_hi, hi[cert_at(i)]);
         }
         rej_hi = warp_max(rej_hi);
         const bool all_chosen = __all_sync(0xffffffffu, lane >= topk || my_idx < N);
@@ -1275,7 +1280,7 @@ extern "C" MOE_API int moe_route_scores(const MoeShape* shape, const uint16_t* x
     // 3. certify the choice of every token; gamma_d of FP64 bounds the
     // defining sum's rounding: |u_def - sum| <= gamma_d ||x|| ||E||
     const double gamma64 = (double(d) * 0x1p-53 / (1.0 - double(d) * 0x1p-53)) * (1.0 + 0x1p-20);
-    const size_t csmem = sizeof(float) * 3 * size_t(N) * kCertWarps;
+    const size_t csmem = sizeof(float) * 3 * size_t(cert_pitch(N)) * kCertWarps;
     if (csmem > 48 * 1024 &&
         cudaFuncSetAttribute(route_certify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(csmem)) != cudaSuccess)
