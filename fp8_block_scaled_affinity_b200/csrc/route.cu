@@ -167,25 +167,31 @@ __global__ void __launch_bounds__(kSliceWarps * 32) route_slice_kernel(
         for (int v = lane; v < d / 8; v += 32) {
             const uint4 w = staged ? mine[v] : __ldg(row + v);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-            uint32_t dg[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
+            // digit s of X is sign(X) * ((|X| >> 7(3-s)) & 127) (the truncating
+            // base-128 digits: all share X's sign); four values' digits are
+            // packed as magnitudes, then the negative ones negated bytewise
+            uint32_t dg[4][2];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float f = (q & 1) ? bf16_hi(ws[q >> 1]) : bf16_lo(ws[q >> 1]);
-                s2 = fma((double)f, (double)f, s2);
-                const double xd = finite ? (double)f * unit_inv : 0.0;
-                const int X = __double2int_rz(xd);  // |X| < 2^28
-                exact = exact && (double)X == xd;
-                s1 += fabs(xd - (double)X);  // exact: a remainder below one unit
-                const int x0 = X / (1 << 21);
-                int rem = X - x0 * (1 << 21);
-                const int x1 = rem / (1 << 14);
-                rem -= x1 * (1 << 14);
-                const int x2 = rem / (1 << 7);
-                const int x3 = rem - x2 * (1 << 7);
-                const int digit[4] = {x0, x1, x2, x3};
+            for (int h = 0; h < 2; ++h) {
+                uint32_t mag[4] = {0u, 0u, 0u, 0u}, neg = 0u;
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    dg[s][q >> 2] |= (uint32_t(digit[s]) & 0xFFu) << (8 * (q & 3));
+                for (int j = 0; j < 4; ++j) {
+                    const int q = 4 * h + j;
+                    const float f = (q & 1) ? bf16_hi(ws[q >> 1]) : bf16_lo(ws[q >> 1]);
+                    s2 = fma((double)f, (double)f, s2);
+                    const double xd = finite ? (double)f * unit_inv : 0.0;
+                    const int X = __double2int_rz(xd);  // |X| < 2^28
+                    exact = exact && (double)X == xd;
+                    s1 += fabs(xd - (double)X);  // exact: a remainder below one unit
+                    const uint32_t a = uint32_t(abs(X));
+                    if (X < 0) neg |= 0xFFu << (8 * j);
+                    mag[0] |= (a >> 21) << (8 * j);
+                    mag[1] |= ((a >> 14) & 0x7Fu) << (8 * j);
+                    mag[2] |= ((a >> 7) & 0x7Fu) << (8 * j);
+                    mag[3] |= (a & 0x7Fu) << (8 * j);
+                }
+#pragma unroll
+                for (int s = 0; s < 4; ++s) dg[s][h] = __vsub4(mag[s] ^ neg, neg);
             }
 #pragma unroll
             for (int s = 0; s < 4; ++s)

@@ -255,6 +255,26 @@ def test_near_tied_scores_bit_exact(N, G, M, K, d):
     assert np.sum((gap >= 1) & (gap <= 2)) >= T // 20
 
 
+@pytest.mark.parametrize("T", [3, 200])
+def test_near_tied_short_list(T):
+    """Few tokens, all near ties: the uncertified list stays short, so every
+    logit of a listed token is summed by one thread in ascending k (fp32
+    products where the rows allow, FP64 otherwise), at the full width."""
+    import fp8_block_scaled_affinity_b200 as moe
+    need_gpu()
+    N, G, M, K, d = 256, 8, 4, 8, 7168
+    rng = np.random.default_rng(T + 17)
+    E = _near_tie_router(N, d, rng)
+    x = S.host_normal_bf16(rng, (T, d), 1.0)
+    bias = np.zeros(N, np.float32)
+    shape = moe.make_shape(T, d, N, G, M, K, 256, 0.001)
+    idx, gate, counts = gpu_route(shape, x, E, bias)
+    ref = oracle.route(x, E, bias, G, M, K)
+    assert np.array_equal(idx, ref["topk_idx"])
+    assert np.array_equal(gate.view(np.uint32), ref["topk_gate"].view(np.uint32))
+    assert np.array_equal(counts, ref["counts"])
+
+
 def test_near_tied_scores_with_offsets_and_biases():
     """The same near-tied router with a logit offset and biases that differ
     by single ulps."""
