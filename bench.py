@@ -443,7 +443,7 @@ def run_route(args, world, rank, local):
         "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": x.numel() * 2,
                 "d2h_bytes_per_step": idx.numel() * 4 + gate.numel() * 4},
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": 8 * args.steps,  # the router's kernels
         "clocks": clk,
         "device_status": int(status.item()),
     }
@@ -1217,8 +1217,8 @@ def run_ours(args, world, rank, local):
                  "unpipelined_value": tokens_total / (e2e[False] / 1e3),
                  "unpipelined_api": "moe_layer_forward_host, one call per step"}
                 if e2e else None),
-        # route 6, quant+permute 4, GEMMs 2, combine 1, bias update 1
-        "gpu_launches": 15 * args.steps,
+        # route 8, quant+permute 4, GEMMs 2, combine 1, bias update 1
+        "gpu_launches": 16 * args.steps,
         "clocks": clk,
         "device_status": status,
     }
