@@ -513,13 +513,26 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
     uint8_t* __restrict__ qt, float* __restrict__ st) {
     __shared__ __align__(16) float tile[128][68];
     __shared__ float red[4][64];
+    __shared__ int tok_s[128];    // gathered sources: token of each row of the block
+    __shared__ float gate_s[128]; // and the gate its gradient carries
     const int fchunks = F / 64;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int64_t u = blockIdx.x; u < int64_t(n_blocks) * fchunks; u += gridDim.x) {
-        const int b = int(u / fchunks);
-        const int f0 = int(u - int64_t(b) * fchunks) * 64;
+    const int n_units = n_blocks * fchunks;  // < 2^31 (checked by the launch)
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int b = u / fchunks;
+        const int f0 = (u - b * fchunks) * 64;
         const int2 blk = blocks[b];
-        if (blk.y <= 0) continue;  // past the last expert's rows: never read
+        if (blk.y <= 0) continue;  // past the last expert's rows: never read (uniform)
+        if (SRC == kWgX || SRC == kWgDo) {
+            // the block's tokens once, not once per lane and row
+            if (threadIdx.x < 128) {
+                float g = 0.0f;
+                tok_s[threadIdx.x] =
+                    int(threadIdx.x) < blk.y ? wg_token(src, blk.x + int(threadIdx.x), g) : -1;
+                gate_s[threadIdx.x] = g;
+            }
+            __syncthreads();
+        }
         // ---- load: warp w, rows w, w + 8, ...; lane: features f0 + 2 lane, +1.
         // Eight rows at a time: their token indices first, then all their
         // loads, then the arithmetic (a warp keeps eight loads in flight).
@@ -535,8 +548,8 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
 #pragma unroll
                 for (int i = 0; i < RB; ++i) {
                     const int rr = warp + 8 * (i0 + i);
-                    g[i] = 0.0f;
-                    tok[i] = rr < blk.y ? wg_token(src, blk.x + rr, g[i]) : -1;
+                    tok[i] = tok_s[rr];
+                    g[i] = gate_s[rr];
                 }
                 uint32_t w2[RB];
 #pragma unroll
@@ -849,6 +862,7 @@ int launch_wgrad_quant(const WgSrc& src, const int32_t* blocks, int n_blocks, in
     if (!blocks || !qt || !st) return MOE_ERR_NULL;
     if (!aligned16(qt)) return MOE_ERR_ALIGN;
     const int64_t units = int64_t(n_blocks) * (F / 64);
+    if (units > INT32_MAX) return MOE_ERR_SHAPE;
     const int grid = int(std::min<int64_t>(units, int64_t(sm_count()) * 8));
     wgrad_quant_kernel<SRC><<<grid, 256, 0, as_stream(stream)>>>(
         src, reinterpret_cast<const int2*>(blocks), n_blocks, F, int64_t(n_blocks) * 128, qt, st);
