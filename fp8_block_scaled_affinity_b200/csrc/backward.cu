@@ -502,7 +502,9 @@ __device__ __forceinline__ int wg_token(const WgSrc& s, int r, float& g) {
     return p / s.K;
 }
 
-__device__ __forceinline__ float wg_sigmoid(float a) { return 1.0f / (1.0f + expf(-a)); }
+// sigmoid with the fast exponential and a correctly rounded reciprocal (a few
+// ulps, as in the forward SwiGLU epilogue; e^-a = inf gives 0)
+__device__ __forceinline__ float wg_sigmoid(float a) { return __frcp_rn(1.0f + __expf(-a)); }
 
 // A CTA per (128-row block, 64 output features): the block's values in
 // shared memory, one amax per feature over the block's rows, codes written
@@ -580,8 +582,8 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    v0[i] = a[i].x / (1.0f + expf(-a[i].x)) * c[i].x;
-                    v1[i] = a[i].y / (1.0f + expf(-a[i].y)) * c[i].y;
+                    v0[i] = a[i].x * wg_sigmoid(a[i].x) * c[i].x;
+                    v1[i] = a[i].y * wg_sigmoid(a[i].y) * c[i].y;
                 }
             } else {  // [da | dc]
                 const bool is_da = fl < src.I;
