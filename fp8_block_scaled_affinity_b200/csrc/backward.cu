@@ -111,6 +111,10 @@ __global__ void __launch_bounds__(256) combine_backward_quant_kernel(
 }
 
 // ------------------------------------------- 4. SwiGLU backward, quantised
+// sigmoid with the fast exponential and a correctly rounded reciprocal (a few
+// ulps, as in the forward SwiGLU epilogue; e^-a = inf gives 0)
+__device__ __forceinline__ float fast_sigmoid(float a) { return __frcp_rn(1.0f + __expf(-a)); }
+
 // A warp per (row, piece of 2P tiles of the 2I-wide row [da | dc]).
 template <int PC>
 __global__ void __launch_bounds__(256) swiglu_backward_quant_kernel(
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(256) swiglu_backward_quant_kernel(
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float a = av[i];
-                    const float sg = 1.0f / (1.0f + expf(-a));
+                    const float sg = fast_sigmoid(a);
                     f[i] = is_da ? hv[i] * cv[i] * sg * (1.0f + a * (1.0f - sg)) : hv[i] * a * sg;
                 }
             }
@@ -502,9 +506,7 @@ __device__ __forceinline__ int wg_token(const WgSrc& s, int r, float& g) {
     return p / s.K;
 }
 
-// sigmoid with the fast exponential and a correctly rounded reciprocal (a few
-// ulps, as in the forward SwiGLU epilogue; e^-a = inf gives 0)
-__device__ __forceinline__ float wg_sigmoid(float a) { return __frcp_rn(1.0f + __expf(-a)); }
+
 
 // A CTA per (128-row block, 64 output features): the block's values in
 // shared memory, one amax per feature over the block's rows, codes written
@@ -582,8 +584,8 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    v0[i] = a[i].x * wg_sigmoid(a[i].x) * c[i].x;
-                    v1[i] = a[i].y * wg_sigmoid(a[i].y) * c[i].y;
+                    v0[i] = a[i].x * fast_sigmoid(a[i].x) * c[i].x;
+                    v1[i] = a[i].y * fast_sigmoid(a[i].y) * c[i].y;
                 }
             } else {  // [da | dc]
                 const bool is_da = fl < src.I;
@@ -603,7 +605,7 @@ __global__ void __launch_bounds__(256) wgrad_quant_kernel(
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float sg0 = wg_sigmoid(a[i].x), sg1 = wg_sigmoid(a[i].y);
+                    const float sg0 = fast_sigmoid(a[i].x), sg1 = fast_sigmoid(a[i].y);
                     if (is_da) {
                         v0[i] = h[i].x * c[i].x * sg0 * (1.0f + a[i].x * (1.0f - sg0));
                         v1[i] = h[i].y * c[i].y * sg1 * (1.0f + a[i].y * (1.0f - sg1));
